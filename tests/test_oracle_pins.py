@@ -1,0 +1,312 @@
+"""Pins of the fp64 oracle against facts that do not come from the oracle itself.
+
+Each test fixes one part of the oracle with something independent of its code:
+closed forms on constructed inputs, brute-force enumeration on tiny inputs,
+invariants the method must satisfy, a library attention routine
+(torch scaled_dot_product_attention in fp64) in the cases where the sparse
+step reduces to dense causal attention, and the constants the pages print
+(tests/golden/page_constants.json).  A plausible slip in the oracle (a dropped
+causal mask, a wrong tie order, a transposed page layout, a missing scale, a
+local block leaking into the remote slots) fails at least one of them.
+"""
+import itertools
+import json
+import os
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import workloads
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden", "page_constants.json")
+
+
+def bf16(x):
+    return torch.as_tensor(x, dtype=torch.float32).to(torch.bfloat16)
+
+
+# ----------------------------------------------------------------------------- page constants
+def test_page_constants_match_oracle():
+    g = json.load(open(GOLDEN))
+    assert oracle.BLOCK == g["sparse_block_size"]["value"]
+    assert oracle.N_LOCAL == g["sparse_local_block"]["value"]
+    assert oracle.N_REMOTE == g["dash_topk_blocks"]["value"]
+    assert oracle.N_SEL == g["sparse_topk_blocks"]["value"]
+    assert oracle.N_LOCAL * oracle.BLOCK == g["sliding_window_size"]["value"]
+    assert oracle.N_SEL * oracle.BLOCK == g["read_set_tokens"]["value"]
+    assert oracle.HEADS == g["num_attention_heads"]["value"]
+    assert oracle.HEAD_DIM == g["head_dim"]["value"]
+    assert oracle.IDX_DIM == g["indexer_dim"]["value"]
+    frac = g["read_set_tokens"]["value"] / g["read_fraction_at_128k_below"]["context"]
+    assert frac < g["read_fraction_at_128k_below"]["value"]
+    # K and V, bf16, all layers at 128K: same order as the page's estimate (within 10 %).
+    kv = g["num_layers"]["value"] * 131072 * oracle.HEADS * oracle.HEAD_DIM * 2 * 2 / 1e9
+    assert abs(kv - g["kv_cache_128k_gb_estimate"]["value"]) / kv < 0.10
+
+
+# ----------------------------------------------------------------------------- block scores
+def _ramp_case(n_blocks, sign=1.0, d_idx=128):
+    """idx_q = e_0, idx_k[t][0] = sign * t/64 (exact in bf16 for t < 256), everything else 0."""
+    qi = torch.zeros(d_idx)
+    qi[0] = 1.0
+    ki = torch.zeros(n_blocks * 32, d_idx)
+    ki[:, 0] = sign * torch.arange(n_blocks * 32, dtype=torch.float32) / 64.0
+    assert torch.equal(bf16(ki).float(), ki)
+    return bf16(qi), bf16(ki).view(n_blocks, 32, d_idx)
+
+
+@pytest.mark.parametrize("p", [255, 200, 31, 0, 32, 100])
+def test_scores_closed_form_increasing(p):
+    qi, pages = _ramp_case(8)
+    s = oracle.block_scores(qi, pages, np.arange(8), p)
+    nb = p // 32 + 1
+    want = [min(32 * j + 31, p) / 64.0 for j in range(nb)]
+    assert s.shape == (nb,)
+    assert s.tolist() == want
+
+
+def test_scores_closed_form_decreasing():
+    qi, pages = _ramp_case(8, sign=-1.0)
+    s = oracle.block_scores(qi, pages, np.arange(8), 255)
+    assert s.tolist() == [-(32 * j) / 64.0 for j in range(8)]
+
+
+def test_scores_use_the_block_table():
+    qi, pages = _ramp_case(8)
+    perm = np.array([5, 2, 7, 0, 1, 6, 3, 4])
+    shuffled = torch.empty_like(pages)
+    shuffled[perm] = pages                    # logical block j lives at physical page perm[j]
+    s = oracle.block_scores(qi, shuffled, perm, 255)
+    assert s.tolist() == [(32 * j + 31) / 64.0 for j in range(8)]
+
+
+def test_scores_brute_force_random():
+    g = torch.Generator().manual_seed(7)
+    qi = bf16(torch.randn(128, generator=g))
+    pages = bf16(torch.randn(5, 32, 128, generator=g))
+    for p in [0, 17, 63, 64, 159]:
+        s = oracle.block_scores(qi, pages, np.arange(5), p)
+        dots = pages.double().reshape(-1, 128)[: p + 1] @ qi.double()
+        want = [dots[32 * j: 32 * j + 32].max().item() for j in range((p // 32) + 1)]
+        np.testing.assert_allclose(s, want, rtol=0, atol=1e-12)
+
+
+# ----------------------------------------------------------------------------- selection
+def _brute_force_select(s, nb, n_local, n_remote):
+    """All subsets of the remote candidates of size min(n_remote, n_cand); keep the
+    maximum-sum ones; the chosen one is the lexicographically smallest of them."""
+    n_cand = max(nb - n_local, 0)
+    k = min(n_remote, n_cand)
+    best, best_sets = None, []
+    for comb in itertools.combinations(range(n_cand), k):
+        tot = sum(s[j] for j in comb)
+        if best is None or tot > best:
+            best, best_sets = tot, [comb]
+        elif tot == best:
+            best_sets.append(comb)
+    chosen = sorted(min(best_sets)) + list(range(max(nb - n_local, 0), nb))
+    return sorted(chosen), len(best_sets)
+
+
+@pytest.mark.parametrize("seed", range(40))
+def test_select_brute_force_with_ties(seed):
+    rng = np.random.default_rng(seed)
+    nb = int(rng.integers(0, 13))
+    n_local = int(rng.integers(0, 5))
+    n_remote = int(rng.integers(0, 6))
+    s = rng.integers(-3, 4, size=max(nb, 1)).astype(np.float64)  # small integers: exact sums, many ties
+    sel, tie = oracle.select(s, nb, n_local, n_remote, tie_eps=0.5)
+    want, n_opt = _brute_force_select(s, nb, n_local, n_remote)
+    assert sel.tolist() == want + [-1] * (n_local + n_remote - len(want))
+    # With integer scores and eps = 0.5 the near-tie flag means "more than one optimal set".
+    n_cand = max(nb - n_local, 0)
+    assert tie == (n_cand > n_remote and n_opt > 1)
+
+
+def test_select_small_context_takes_everything():
+    for nb in range(0, 17):
+        sel, tie = oracle.select(np.random.default_rng(nb).standard_normal(max(nb, 1)), nb)
+        assert sel.tolist() == list(range(nb)) + [-1] * (16 - nb)
+        assert not tie
+
+
+def test_select_remote_never_in_local_window():
+    rng = np.random.default_rng(3)
+    for nb in [17, 40, 100]:
+        s = rng.standard_normal(nb)
+        s[nb - 4:] = 1e9                      # local blocks score highest: they still take no remote slot
+        sel, _ = oracle.select(s, nb)
+        assert list(sel[-4:]) == list(range(nb - 4, nb))
+        remote = sel[:12]
+        assert (remote < nb - 4).all() and len(set(remote.tolist())) == 12
+        top = np.argsort(-s[: nb - 4], kind="stable")[:12]
+        assert sorted(top.tolist()) == remote.tolist()
+
+
+def _oracle_sel(case, **kw):
+    return oracle.run(case.q, case.idx_q, case.k_pool, case.v_pool, case.idx_k_pool,
+                      case.block_table, case.q_seq, case.q_pos, want_out=False, **kw)
+
+
+def test_local_window_invariant_on_keys():
+    """Whatever the local blocks' indexer keys hold, they are selected and the remote set does not move."""
+    case = workloads.make_case([32 * 40 - 5, 32 * 21], heads=1, seed=11)
+    base = _oracle_sel(case)["sel"]
+    for fill in (+40.0, -40.0):
+        ikp = case.idx_k_pool.clone()
+        for b in range(2):
+            nb = (int(case.seq_lens[b]) + 31) // 32
+            for j in range(nb - 4, nb):
+                page = int(case.block_table[b, j])
+                ikp[page] = bf16(fill * case.idx_q[b].float()).expand(32, -1)
+        alt = oracle.run(case.q, case.idx_q, case.k_pool, case.v_pool, ikp, case.block_table,
+                         case.q_seq, case.q_pos, want_out=False)["sel"]
+        assert np.array_equal(base, alt)
+
+
+def test_planted_references_are_recovered():
+    case = workloads.make_case([32768, 32768, 32 * 300], heads=1, planted_blocks=12, seed=0)
+    r = _oracle_sel(case)
+    for b in range(3):
+        nb = (int(case.seq_lens[b]) + 31) // 32
+        assert sorted(case.planted[b]) == r["sel"][b, :12].tolist()
+        assert r["sel"][b, 12:].tolist() == list(range(nb - 4, nb))
+        assert not r["near_tie"][b]
+
+
+def test_selection_is_scale_invariant():
+    case = workloads.make_case([32 * 64, 32 * 50 + 7], heads=1, seed=5)
+    base = _oracle_sel(case)["sel"]
+    doubled = (case.idx_q.float() * 2).to(torch.bfloat16)   # exact in bf16
+    alt = oracle.run(case.q, doubled, case.k_pool, case.v_pool, case.idx_k_pool, case.block_table,
+                     case.q_seq, case.q_pos, want_out=False)["sel"]
+    assert np.array_equal(base, alt)
+
+
+# ----------------------------------------------------------------------------- attention
+def _dense_sdpa(case, b, p):
+    """Dense causal attention of the query at p over tokens 0..p (torch SDPA, fp64, CPU)."""
+    nb = p // 32 + 1
+    pages = case.block_table[b, :nb].long()
+    k = case.k_pool[pages].double().permute(1, 0, 2, 3).reshape(case.k_pool.shape[1], -1, 128)[:, : p + 1]
+    v = case.v_pool[pages].double().permute(1, 0, 2, 3).reshape(case.v_pool.shape[1], -1, 128)[:, : p + 1]
+    qi = [i for i in range(case.n_q) if int(case.q_seq[i]) == b and int(case.q_pos[i]) == p][0]
+    q = case.q[qi].double().unsqueeze(1)                     # [H, 1, D]
+    return torch.nn.functional.scaled_dot_product_attention(q, k, v).squeeze(1).numpy()
+
+
+def test_dense_equivalence_when_everything_fits():
+    """With at most 16 causal blocks every block is selected: the step is dense causal attention."""
+    lens = [1, 31, 32, 33, 200, 512]
+    case = workloads.make_case(lens, heads=3, shuffle=True, seed=2)
+    r = oracle.run(case.q, case.idx_q, case.k_pool, case.v_pool, case.idx_k_pool, case.block_table,
+                   case.q_seq, case.q_pos)
+    for b, L in enumerate(lens):
+        np.testing.assert_allclose(r["out"][b], _dense_sdpa(case, b, L - 1), rtol=0, atol=1e-12)
+
+
+def test_dense_equivalence_with_wide_topk_and_prefill_positions():
+    """Parametrised oracle: n_remote >= candidates reduces to dense causal attention at any p."""
+    case = workloads.make_case([32 * 30], heads=2, q_seq=[0] * 5, q_pos=[0, 45, 511, 700, 959], seed=4)
+    r = oracle.run(case.q, case.idx_q, case.k_pool, case.v_pool, case.idx_k_pool, case.block_table,
+                   case.q_seq, case.q_pos, n_remote=40)
+    for i, p in enumerate([0, 45, 511, 700, 959]):
+        np.testing.assert_allclose(r["out"][i], _dense_sdpa(case, 0, p), rtol=0, atol=1e-12)
+
+
+def test_sparse_differs_from_dense_on_long_context():
+    """Sanity: with 40 blocks the 16-block selection is not dense attention (the mask matters)."""
+    case = workloads.make_case([32 * 40], heads=2, seed=4)
+    r = oracle.run(case.q, case.idx_q, case.k_pool, case.v_pool, case.idx_k_pool, case.block_table,
+                   case.q_seq, case.q_pos)
+    assert np.abs(r["out"][0] - _dense_sdpa(case, 0, 32 * 40 - 1)).max() > 1e-3
+
+
+def test_constant_values_give_constant_output():
+    case = workloads.make_case([32 * 30 + 9], heads=2, seed=8)
+    v = torch.full_like(case.v_pool, 0.0)
+    v[..., :] = bf16(torch.linspace(-2, 2, 128))
+    r = oracle.run(case.q, case.idx_q, case.k_pool, v, case.idx_k_pool, case.block_table,
+                   case.q_seq, case.q_pos)
+    np.testing.assert_allclose(r["out"][0], np.broadcast_to(bf16(torch.linspace(-2, 2, 128)).double().numpy(), (2, 128)),
+                               rtol=0, atol=1e-12)
+
+
+def test_zero_query_gives_mean_of_selected_values():
+    case = workloads.make_case([32 * 30 + 9], heads=2, seed=9)
+    q0 = torch.zeros_like(case.q)
+    r = oracle.run(q0, case.idx_q, case.k_pool, case.v_pool, case.idx_k_pool, case.block_table,
+                   case.q_seq, case.q_pos)
+    p = int(case.q_pos[0])
+    rows = []
+    for j in r["sel"][0]:
+        if j < 0:
+            continue
+        page = int(case.block_table[0, j])
+        n = min(32, p + 1 - 32 * j)
+        rows.append(case.v_pool[page, :, :n].double())
+    mean = torch.cat(rows, dim=1).mean(dim=1).numpy()
+    np.testing.assert_allclose(r["out"][0], mean, rtol=0, atol=1e-12)
+
+
+def test_output_is_a_convex_combination():
+    case = workloads.make_case([32 * 50 + 3, 32 * 19], heads=3, seed=10)
+    r = oracle.run(case.q, case.idx_q, case.k_pool, case.v_pool, case.idx_k_pool, case.block_table,
+                   case.q_seq, case.q_pos)
+    vmin = case.v_pool.float().amin(dim=(0, 2)).double().numpy()
+    vmax = case.v_pool.float().amax(dim=(0, 2)).double().numpy()
+    assert (r["out"] >= vmin - 1e-12).all() and (r["out"] <= vmax + 1e-12).all()
+
+
+def test_scale_argument_is_applied():
+    """scale -> 0 turns the softmax uniform: the output becomes the mean of the selected values."""
+    case = workloads.make_case([32 * 20], heads=1, seed=12)
+    r0 = oracle.run(case.q, case.idx_q, case.k_pool, case.v_pool, case.idx_k_pool, case.block_table,
+                    case.q_seq, case.q_pos, scale=0.0)
+    rq = oracle.run(torch.zeros_like(case.q), case.idx_q, case.k_pool, case.v_pool, case.idx_k_pool,
+                    case.block_table, case.q_seq, case.q_pos)
+    np.testing.assert_allclose(r0["out"], rq["out"], rtol=0, atol=1e-14)
+    r1 = oracle.run(case.q, case.idx_q, case.k_pool, case.v_pool, case.idx_k_pool, case.block_table,
+                    case.q_seq, case.q_pos)
+    assert np.abs(r1["out"] - r0["out"]).max() > 1e-2
+
+
+def test_paging_invariance():
+    lens = [32 * 70 + 5, 32 * 33, 32 * 18 + 31]
+    a = workloads.make_case(lens, heads=2, shuffle=False, seed=21)
+    # same logical content, pages scattered over the pool in another order
+    perm = torch.randperm(a.num_pages, generator=torch.Generator().manual_seed(99))
+    inv = torch.empty_like(perm)
+    inv[perm] = torch.arange(a.num_pages)
+    kp, vp, ikp = (torch.empty_like(t) for t in (a.k_pool, a.v_pool, a.idx_k_pool))
+    kp[inv], vp[inv], ikp[inv] = a.k_pool, a.v_pool, a.idx_k_pool
+    bt = a.block_table.clone()
+    valid = bt >= 0
+    bt[valid] = inv[bt[valid].long()].to(torch.int32)
+    ra = oracle.run(a.q, a.idx_q, a.k_pool, a.v_pool, a.idx_k_pool, a.block_table, a.q_seq, a.q_pos)
+    rb = oracle.run(a.q, a.idx_q, kp, vp, ikp, bt, a.q_seq, a.q_pos)
+    assert np.array_equal(ra["sel"], rb["sel"])
+    assert np.array_equal(ra["out"], rb["out"])
+    assert np.array_equal(ra["scores"], rb["scores"])
+
+
+def test_attention_over_given_selection_matches_attend():
+    case = workloads.make_case([32 * 40 + 1], heads=2, seed=13)
+    r = oracle.run(case.q, case.idx_q, case.k_pool, case.v_pool, case.idx_k_pool, case.block_table,
+                   case.q_seq, case.q_pos)
+    other = np.array([[0, 3, 5, 7, 9, 11, 13, 15, 17, 19, 21, 23, 37, 38, 39, 40]], dtype=np.int32)
+    r2 = oracle.run(case.q, case.idx_q, case.k_pool, case.v_pool, case.idx_k_pool, case.block_table,
+                    case.q_seq, case.q_pos, sel_in=other)
+    direct = oracle.attend(case.q[0], case.k_pool, case.v_pool, case.block_table[0], other[0], int(case.q_pos[0]))
+    np.testing.assert_array_equal(r2["out"][0], direct)
+    assert np.abs(r2["out"][0] - r["out"][0]).max() > 1e-3
+
+
+def test_empty_query_gives_zero_output():
+    case = workloads.make_case([32], heads=1, seed=1)
+    r = oracle.run(case.q, case.idx_q, case.k_pool, case.v_pool, case.idx_k_pool, case.block_table,
+                   case.q_seq, torch.tensor([-1], dtype=torch.int32))
+    assert (r["sel"] == -1).all() and (r["out"] == 0).all()
+    assert np.isneginf(r["scores"]).all()
