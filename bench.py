@@ -1,0 +1,444 @@
+#!/usr/bin/env python
+"""Benchmark of the SR-SWA / DASH block-sparse decode step on B200.
+
+    python bench.py [--gpus N --steps K --warmup W] [--workload long_decode|batched_decode|
+                    tiny_decode|ragged_paged_decode] [--impl uocr|reference]
+
+Default workload: long-context decode, batch 16, context 131072 (4096 blocks
+of 32 tokens), 12 independent layer caches (126 GiB resident in HBM).  One
+step = the decode of every sequence through all 12 layers = 12 calls of
+``uocr_sparse_decode`` (scan -> top-k -> split-K attention -> combine).
+Metric: decode queries/s per layer (= 16 * 12 / step time) and achieved HBM
+bandwidth on the algorithmic bytes (256 B of indexer key per causal token +
+512 tokens x 10 heads x 128 dims x 2 B x (K and V) per query).
+
+Prints ONE JSON line on rank 0.  Under torchrun each rank runs its own shard
+of sequences (weak scaling, no collective on the data path).
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import workloads  # noqa: E402
+from block_sparse_long_uocr_b200 import dist as udist  # noqa: E402
+
+METRIC = "sparse-attn decode queries/s per layer @128K ctx; achieved HBM GB/s vs peak"
+UNIT = "queries/s per layer"
+KV_BYTES_PER_QUERY = 16 * 32 * 10 * 128 * 2 * 2      # 512 gathered tokens x 10 heads x 128 x bf16 x (K,V)
+NOMINAL_HBM_GBS = 8000.0
+FALLBACK_HBM_GBS = 6650.0
+
+# DRAM traffic of the dominant kernel from one ncu capture (dram__bytes_read.sum +
+# dram__bytes_write.sum), per launch of the default workload, and the hash of the
+# kernel source it was taken on.  Reported as null once the source has changed.
+NCU_TRAFFIC = {}
+
+
+def kernel_source_hash(name: str) -> str:
+    path = os.path.join(ROOT, "block_sparse_long_uocr_b200", "csrc", name)
+    return hashlib.sha256(open(path, "rb").read()).hexdigest()[:16]
+
+
+def measured_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        try:
+            return json.load(open(path)), "measured"
+        except Exception:
+            pass
+    return {"hbm_gbs": FALLBACK_HBM_GBS}, "fallback"
+
+
+# --------------------------------------------------------------------------- clocks
+class ClockSampler:
+    """nvidia-smi samples (200 ms) of SM clock and throttle reasons while the timed region runs."""
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                                          "-lms", "200", "-i", str(self.gpu)],
+                                         stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except Exception:
+            self.proc = None
+        return self
+
+    def __exit__(self, *exc):
+        self.lines = []
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                out, _ = self.proc.communicate(timeout=5)
+            except Exception:
+                self.proc.kill()
+                out, _ = self.proc.communicate()
+            self.lines = [l for l in out.splitlines() if l.strip()]
+        return False
+
+    def summary(self):
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for l in getattr(self, "lines", []):
+            f = [x.strip() for x in l.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                sm.append(float(f[1]))
+                mx = float(f[2])
+            except ValueError:
+                continue
+            for n, v in zip(names, f[5:9]):
+                if v.lower().startswith("active"):
+                    reasons.add(n)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": mx, "reasons": [], "samples": 0}
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx, "reasons": sorted(reasons), "samples": len(sm)}
+
+
+def physical_gpu(local_rank: int) -> str:
+    """nvidia-smi id of this process's GPU (honours CUDA_VISIBLE_DEVICES indices or UUIDs)."""
+    vis = os.environ.get("CUDA_VISIBLE_DEVICES", "").strip()
+    if vis:
+        ids = [v.strip() for v in vis.split(",") if v.strip()]
+        if local_rank < len(ids):
+            return ids[local_rank]
+    return str(local_rank)
+
+
+# --------------------------------------------------------------------------- workloads
+def build_workload(name: str, device, seed: int):
+    if name == "long_decode":
+        return workloads.long_decode(device=device, seed=seed)
+    if name == "batched_decode":
+        return workloads.batched_decode(device=device, seed=seed)
+    if name == "tiny_decode":
+        return workloads.tiny_decode(device=device, seed=seed)
+    if name == "ragged_paged_decode":
+        return workloads.ragged_paged_decode(device=device, seed=seed)
+    raise SystemExit(f"unknown workload {name}")
+
+
+def algorithmic_bytes(case) -> tuple[int, int]:
+    """(bytes per decode call over all queries, indexer-scan bytes of those queries)."""
+    lens = case.seq_lens.cpu().tolist()
+    scan = sum(256 * L for L in lens)
+    return scan + KV_BYTES_PER_QUERY * len(lens), scan
+
+
+# --------------------------------------------------------------------------- our arm
+def run_uocr(args):
+    rank, local_rank, world = udist.env_rank_world()
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    if world > 1:
+        import datetime
+        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                             device_id=dev)
+    import block_sparse_long_uocr_b200 as uocr
+
+    case = build_workload(args.workload, dev, udist.shard_seed(args.seed, rank))
+    n_layers = len(case.layers)
+    B, H, mb = case.n_q, case.q.shape[1], case.max_blocks
+    bytes_call, scan_bytes_call = algorithmic_bytes(case)
+    ws = uocr.alloc_workspace(B, H, mb, dev)
+    outs = [torch.empty_like(case.q) for _ in range(n_layers)]
+    sels = [torch.empty((B, 16), dtype=torch.int32, device=dev) for _ in range(n_layers)]
+    stream = torch.cuda.current_stream()
+    l2 = torch.cuda.get_device_properties(dev).L2_cache_size
+    flush = bytes_call * n_layers < 4 * l2
+    flush_buf = torch.empty(2 * l2 if flush else 1, dtype=torch.uint8, device=dev)
+
+    def step():
+        for l in range(n_layers):
+            q, qi = case.q_layers[l]
+            kp, vp, ikp = case.layers[l]
+            uocr.sparse_decode(q, kp, vp, qi, ikp, case.block_table, case.seq_lens, out=outs[l], sel=sels[l],
+                               workspace=ws, stream=stream)
+
+    def barrier():
+        if world > 1:
+            torch.distributed.barrier(device_ids=[local_rank])
+
+    for _ in range(args.warmup):
+        if flush:
+            flush_buf.zero_()
+        step()
+    torch.cuda.synchronize()
+    barrier()
+    torch.cuda.synchronize()
+
+    with ClockSampler(physical_gpu(local_rank)) as clk:
+        if flush:
+            # L2 flushed between steps; each step timed on its own
+            times = []
+            for _ in range(args.steps):
+                flush_buf.zero_()
+                e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                e0.record(stream)
+                step()
+                e1.record(stream)
+                times.append((e0, e1))
+            torch.cuda.synchronize()
+            elapsed_ms = sum(a.elapsed_time(b) for a, b in times)
+        else:
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            for _ in range(args.steps):
+                step()
+            e1.record(stream)
+            torch.cuda.synchronize()
+            elapsed_ms = e0.elapsed_time(e1)
+    barrier()
+    torch.cuda.synchronize()
+    max_ms = udist.max_over_ranks(elapsed_ms, dev)
+    ms_per_step = max_ms / args.steps
+    queries_per_step = B * n_layers
+    value = world * queries_per_step * args.steps / (max_ms / 1e3) / n_layers
+
+    # ---- dominant kernel (indexer scan) timed on its own launches, same inputs and stream
+    scores = torch.empty((B, mb), dtype=torch.float32, device=dev)
+    n_rep = max(3, min(args.steps * n_layers, 48))
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(n_rep)]
+    for r in range(n_rep):
+        l = r % n_layers
+        if flush:
+            flush_buf.zero_()
+        ev[r][0].record(stream)
+        uocr.index_score(case.q_layers[l][1], case.layers[l][2], case.block_table, case.seq_lens,
+                         scores=scores, stream=stream)
+        ev[r][1].record(stream)
+    torch.cuda.synchronize()
+    scan_ms = statistics.mean(a.elapsed_time(b) for a, b in ev)
+    peaks, peak_kind = measured_peaks()
+    peak = float(peaks.get("hbm_gbs", FALLBACK_HBM_GBS))
+    scan_gbs = scan_bytes_call / (scan_ms / 1e3) / 1e9
+    step_gbs = bytes_call * n_layers / (ms_per_step / 1e3) / 1e9
+    tr = NCU_TRAFFIC.get(args.workload)
+    traffic = tr["bytes"] if tr and tr.get("src") == kernel_source_hash("index_scan.cu") else None
+
+    # ---- end to end through the public API: pinned host inputs in, results out, every step
+    e2e = run_e2e(args, uocr, case, ws, outs, sels, stream, world, dev)
+
+    clocks = clk.summary()
+    result = {
+        "metric": METRIC, "value": round(value, 1), "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": round(ms_per_step, 4), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": case.name, "batch_per_gpu": B, "context": int(case.seq_lens.max().item()),
+                   "layers": n_layers, "heads": H, "head_dim": 128, "block": 32, "local_blocks": 4,
+                   "remote_blocks": 12, "max_blocks": mb,
+                   "l2": "flushed between steps" if flush else "inputs larger than L2 (no flush)",
+                   "parallelism": f"dp{world} (independent sequence shards)"},
+        "roofline": {"bound": "hbm", "kernel": "index_scan_kernel", "achieved": round(scan_gbs, 1),
+                     "peak": peak, "unit": "GB/s", "frac": round(scan_gbs / peak, 4), "traffic": traffic,
+                     "peak_kind": f"{peak_kind} hbm copy", "bytes_per_launch": scan_bytes_call,
+                     "avg_launch_ms": round(scan_ms, 5), "frac_of_8tbs": round(scan_gbs / NOMINAL_HBM_GBS, 4)},
+        "step_roofline": {"bound": "hbm", "achieved": round(step_gbs, 1), "peak": peak, "unit": "GB/s",
+                          "frac": round(step_gbs / peak, 4), "frac_of_8tbs": round(step_gbs / NOMINAL_HBM_GBS, 4),
+                          "bytes_per_step": bytes_call * n_layers},
+        "e2e": e2e,
+        "gpu_launches": args.steps * n_layers * 4,
+        "clocks": clocks,
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        result["cpu_baseline"] = cpu_baseline(case, budget_s=args.cpu_budget)
+    if world > 1:
+        torch.distributed.destroy_process_group()
+    if rank == 0:
+        print(json.dumps(result), flush=True)
+
+
+def run_e2e(args, uocr, case, ws, outs, sels, stream, world, dev):
+    """Same metric through sparse_decode with the step's per-query inputs copied in from pinned
+    host memory and the outputs copied back, inside the timed region.  The KV / indexer caches
+    stay resident on the device (they are the decode state, not a per-step input)."""
+    n_layers = len(case.layers)
+    h_q = [case.q_layers[l][0].cpu().pin_memory() for l in range(n_layers)]
+    h_qi = [case.q_layers[l][1].cpu().pin_memory() for l in range(n_layers)]
+    h_bt = case.block_table.cpu().pin_memory()
+    h_sl = case.seq_lens.cpu().pin_memory()
+    d_q = [torch.empty_like(case.q_layers[l][0]) for l in range(n_layers)]
+    d_qi = [torch.empty_like(case.q_layers[l][1]) for l in range(n_layers)]
+    d_bt, d_sl = torch.empty_like(case.block_table), torch.empty_like(case.seq_lens)
+    h_out = [torch.empty(outs[0].shape, dtype=outs[0].dtype).pin_memory() for _ in range(n_layers)]
+    h_sel = [torch.empty(sels[0].shape, dtype=sels[0].dtype).pin_memory() for _ in range(n_layers)]
+    h2d = sum(t.numel() * t.element_size() for t in h_q + h_qi + [h_bt, h_sl])
+    d2h = sum(t.numel() * t.element_size() for t in h_out + h_sel)
+
+    def step():
+        d_bt.copy_(h_bt, non_blocking=True)
+        d_sl.copy_(h_sl, non_blocking=True)
+        for l in range(n_layers):
+            d_q[l].copy_(h_q[l], non_blocking=True)
+            d_qi[l].copy_(h_qi[l], non_blocking=True)
+            kp, vp, ikp = case.layers[l]
+            uocr.sparse_decode(d_q[l], kp, vp, d_qi[l], ikp, d_bt, d_sl, out=outs[l], sel=sels[l],
+                               workspace=ws, stream=stream)
+            h_out[l].copy_(outs[l], non_blocking=True)
+            h_sel[l].copy_(sels[l], non_blocking=True)
+
+    for _ in range(max(1, args.warmup)):
+        step()
+    torch.cuda.synchronize()
+    steps = max(1, args.steps)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(steps):
+        step()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    ms = udist.max_over_ranks(e0.elapsed_time(e1), dev)
+    value = world * case.n_q * n_layers * steps / (ms / 1e3) / n_layers
+    return {"value": round(value, 1), "unit": UNIT, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+            "ms_per_step": round(ms / steps, 4)}
+
+
+# --------------------------------------------------------------------------- oracle timing
+def _gather_for_oracle(case, layer, queries):
+    """Host copies of what the oracle reads for `queries`: their indexer pages and queries."""
+    import numpy as np
+    q, qi = case.q_layers[layer]
+    ikp = case.layers[layer][2]
+    pages, bt_rows, pos = [], [], []
+    off = 0
+    mb = case.max_blocks
+    for i in queries:
+        b, p = int(case.q_seq[i]), int(case.q_pos[i])
+        nb = p // 32 + 1
+        pages.append(case.block_table[b, :nb].long())
+        row = np.full(mb, -1, np.int32)
+        row[:nb] = np.arange(off, off + nb)
+        bt_rows.append(row)
+        pos.append(p)
+        off += nb
+    pidx = torch.cat(pages)
+    mini_idx = ikp[pidx].cpu()
+    return (q[list(queries)].cpu(), qi[list(queries)].cpu(), mini_idx, np.stack(bt_rows),
+            np.arange(len(queries), dtype=np.int32), np.array(pos, np.int32))
+
+
+def _gather_kv(case, layer, queries, sel):
+    import numpy as np
+    kp, vp, _ = case.layers[layer]
+    rows, pages = [], []
+    off = 0
+    for n, i in enumerate(queries):
+        b = int(case.q_seq[i])
+        row = np.full(case.max_blocks, -1, np.int32)
+        for j in sel[n]:
+            if j >= 0:
+                row[j] = off
+                pages.append(int(case.block_table[b, j]))
+                off += 1
+        rows.append(row)
+    pidx = torch.tensor(pages, dtype=torch.long, device=kp.device)
+    return kp[pidx].cpu(), vp[pidx].cpu(), np.stack(rows)
+
+
+def oracle_time_queries(case, layer, queries, threads=0):
+    """Seconds of oracle work (scores + selection, then attention) for `queries` of one layer."""
+    import numpy as np
+    import oracle
+    q, qi, mini_idx, bt, qs, qp = _gather_for_oracle(case, layer, queries)
+    H = q.shape[1]
+    dummy = torch.zeros((1, H, 32, 128), dtype=torch.bfloat16)
+    t0 = time.perf_counter()
+    r = oracle.run(q, qi, dummy, dummy, mini_idx, bt, qs, qp, want_out=False, want_scores=False, threads=threads)
+    t1 = time.perf_counter()
+    kp, vp, bt2 = _gather_kv(case, layer, queries, r["sel"])
+    t2 = time.perf_counter()
+    r2 = oracle.run(q, qi, kp, vp, mini_idx[:1], bt2, qs, qp, sel_in=r["sel"], threads=threads)
+    t3 = time.perf_counter()
+    return (t1 - t0) + (t3 - t2), r["threads"], r2
+
+
+def cpu_baseline(case, budget_s: float = 15.0):
+    """The oracle as it stands, on this host's cores, on a bounded sample of the same workload."""
+    n_layers = len(case.layers)
+    done, secs, threads = 0, 0.0, 1
+    layer = 0
+    while secs < budget_s and layer < n_layers:
+        t, threads, _ = oracle_time_queries(case, layer, list(range(case.n_q)))
+        secs += t
+        done += case.n_q
+        layer += 1
+    return {"value": round(done / secs, 2), "unit": UNIT, "cores": threads, "kind": "oracle",
+            "sample": f"{done} queries ({layer} of {n_layers} layers x {case.n_q} sequences) of {case.name}, "
+                      f"fp64, {secs:.1f} s of oracle time (host reads excluded)",
+            "host_cpus": os.cpu_count()}
+
+
+# --------------------------------------------------------------------------- reference arm
+def run_reference(args):
+    """The oracle as the reference arm: same metric / unit / workload, on host cores."""
+    rank, local_rank, world = udist.env_rank_world()
+    if rank != 0:
+        return
+    dev = torch.device("cuda", local_rank) if torch.cuda.is_available() else torch.device("cpu")
+    if dev.type == "cuda":
+        torch.cuda.set_device(dev)
+    name = args.workload
+    if name == "long_decode":
+        case = workloads.long_decode(device=dev, seed=args.seed, n_layers=1)
+    else:
+        case = build_workload(name, dev, args.seed)
+    queries = list(range(case.n_q))
+    for _ in range(args.warmup):
+        oracle_time_queries(case, 0, queries[:1])
+    secs, threads = [], 1
+    for _ in range(args.steps):
+        t, threads, _ = oracle_time_queries(case, 0, queries)
+        secs.append(t)
+    total = sum(secs)
+    value = len(queries) * args.steps / total
+    full_name = "long_decode_b16_ctx131072_layers12" if name == "long_decode" else case.name
+    res = {"impl": "reference", "metric": METRIC, "value": round(value, 2), "unit": UNIT, "n_gpus": 1,
+           "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(1e3 * total / args.steps, 2),
+           "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+           "config": {"workload": full_name, "sample_per_step": f"{len(queries)} queries of one layer"},
+           "cpu_baseline": {"value": round(value, 2), "unit": UNIT, "cores": threads, "kind": "oracle",
+                            "sample": f"{len(queries)} queries x {args.steps} steps of {case.name}"},
+           "e2e": {"value": round(value, 2), "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(res), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="uocr", choices=["uocr", "reference"])
+    ap.add_argument("--workload", default="long_decode",
+                    choices=["long_decode", "batched_decode", "tiny_decode", "ragged_paged_decode"])
+    ap.add_argument("--seed", type=int, default=0)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-budget", type=float, default=15.0)
+    args = ap.parse_args()
+    if args.warmup < 3 and args.impl == "uocr":
+        print("note: fewer than 3 warm-up steps", file=sys.stderr)
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_uocr(args)
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,192 @@
+"""Python binding of libuocr.so, the B200 (sm_100a) SR-SWA / DASH block-sparse attention step.
+
+Argument marshalling only: every step of the computation runs in the CUDA
+kernels behind the C ABI declared in ``include/uocr.h``.  PyTorch provides the
+device memory and the stream; there is no CPU fallback, and importing this
+package fails loudly when ``libuocr.so`` has not been built
+(``python -m block_sparse_long_uocr_b200.build``).
+
+Entry points (same names as the C ABI, without the ``uocr_`` prefix):
+
+* :func:`index_score`  -- block scores of the 1-head x 128 Lightning Indexer;
+* :func:`block_topk`   -- 4 local + top-12 remote block selection;
+* :func:`sparse_attn`  -- exact 10-head attention over the selected 512 tokens;
+* :func:`sparse_decode` -- the three fused into one decode call;
+* :func:`workspace_bytes`.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libuocr.so")
+
+BLOCK = 32
+N_LOCAL = 4
+N_REMOTE = 12
+N_SEL = 16
+HEAD_DIM = 128
+IDX_DIM = 128
+
+STATUS = {0: "UOCR_OK", 1: "UOCR_ERR_INVALID_ARG", 2: "UOCR_ERR_UNSUPPORTED",
+          3: "UOCR_ERR_WORKSPACE", 4: "UOCR_ERR_CUDA"}
+DEVERR_PAGE, DEVERR_POS, DEVERR_SEL = 1, 2, 4
+
+
+class UocrError(RuntimeError):
+    def __init__(self, fn: str, status: int, msg: str):
+        super().__init__(f"{fn} failed: {msg}")
+        self.status = status
+
+
+def _load() -> ctypes.CDLL:
+    if not os.path.exists(LIB_PATH):
+        raise ImportError(f"{LIB_PATH} is missing: build it with `python -m block_sparse_long_uocr_b200.build` "
+                          "(there is no CPU fallback)")
+    lib = ctypes.CDLL(LIB_PATH)
+    P, I, F, Z = ctypes.c_void_p, ctypes.c_int, ctypes.c_float, ctypes.c_size_t
+    lib.uocr_status_string.argtypes = [I]
+    lib.uocr_status_string.restype = ctypes.c_char_p
+    lib.uocr_abi_version.argtypes = []
+    lib.uocr_abi_version.restype = I
+    lib.uocr_workspace_bytes.argtypes = [I, I, I]
+    lib.uocr_workspace_bytes.restype = Z
+    lib.uocr_index_score.argtypes = [P, P, P, P, P, P, I, I, I, I, P, P, P]
+    lib.uocr_index_score.restype = I
+    lib.uocr_block_topk.argtypes = [P, P, P, P, I, I, I, P, P, P]
+    lib.uocr_block_topk.restype = I
+    lib.uocr_sparse_attn.argtypes = [P, P, P, P, P, P, P, P, I, I, I, I, I, F, P, P, Z, P, P]
+    lib.uocr_sparse_attn.restype = I
+    lib.uocr_sparse_decode.argtypes = [P, P, P, P, P, P, P, I, I, I, I, P, P, P, Z, P, P]
+    lib.uocr_sparse_decode.restype = I
+    return lib
+
+
+lib = _load()
+
+
+# --------------------------------------------------------------------------- helpers
+def _check(fn: str, st: int):
+    if st != 0:
+        raise UocrError(fn, st, lib.uocr_status_string(st).decode())
+
+
+def _ptr(t: torch.Tensor | None):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _dev(t: torch.Tensor, name: str, dtype: torch.dtype, ndim: int | None = None) -> torch.Tensor:
+    if not isinstance(t, torch.Tensor):
+        raise TypeError(f"{name} must be a torch.Tensor")
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be on a CUDA device (no CPU path)")
+    if t.dtype != dtype:
+        raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
+    if ndim is not None and t.dim() != ndim:
+        raise ValueError(f"{name} must have {ndim} dims, got shape {tuple(t.shape)}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    return t
+
+
+def _opt_i32(t, name):
+    return None if t is None else _dev(t, name, torch.int32, 1)
+
+
+def _stream(stream) -> ctypes.c_void_p:
+    s = torch.cuda.current_stream() if stream is None else stream
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def workspace_bytes(n_q: int, heads: int, max_blocks: int) -> int:
+    return int(lib.uocr_workspace_bytes(int(n_q), int(heads), int(max_blocks)))
+
+
+def alloc_workspace(n_q: int, heads: int, max_blocks: int, device) -> torch.Tensor:
+    """A uint8 tensor of workspace_bytes(...) bytes (torch allocations are 256-byte aligned)."""
+    return torch.empty(max(workspace_bytes(n_q, heads, max_blocks), 1), dtype=torch.uint8, device=device)
+
+
+# --------------------------------------------------------------------------- entry points
+def index_score(idx_q, idx_k_cache, block_table, seq_lens, q_seq=None, q_pos=None, *,
+                scores=None, dev_err=None, stream=None) -> torch.Tensor:
+    """fp32 [n_q, max_blocks] block scores (entries past a query's causal blocks untouched)."""
+    _dev(idx_q, "idx_q", torch.bfloat16, 2)
+    _dev(idx_k_cache, "idx_k_cache", torch.bfloat16, 3)
+    _dev(block_table, "block_table", torch.int32, 2)
+    _dev(seq_lens, "seq_lens", torch.int32, 1)
+    n_q, B, mb = idx_q.shape[0], block_table.shape[0], block_table.shape[1]
+    if scores is None:
+        scores = torch.full((n_q, mb), float("-inf"), dtype=torch.float32, device=idx_q.device)
+    _dev(scores, "scores", torch.float32, 2)
+    _check("uocr_index_score", lib.uocr_index_score(
+        _ptr(idx_q), _ptr(idx_k_cache), _ptr(block_table), _ptr(seq_lens), _ptr(_opt_i32(q_seq, "q_seq")),
+        _ptr(_opt_i32(q_pos, "q_pos")), n_q, B, mb, idx_k_cache.shape[0], _ptr(scores),
+        _ptr(dev_err), _stream(stream)))
+    return scores
+
+
+def block_topk(scores, seq_lens, q_seq=None, q_pos=None, *, sel=None, dev_err=None, stream=None) -> torch.Tensor:
+    """int32 [n_q, 16] selected logical blocks (ascending, -1 padded)."""
+    _dev(scores, "scores", torch.float32, 2)
+    _dev(seq_lens, "seq_lens", torch.int32, 1)
+    n_q, mb = scores.shape
+    if sel is None:
+        sel = torch.empty((n_q, N_SEL), dtype=torch.int32, device=scores.device)
+    _dev(sel, "sel", torch.int32, 2)
+    _check("uocr_block_topk", lib.uocr_block_topk(
+        _ptr(scores), _ptr(seq_lens), _ptr(_opt_i32(q_seq, "q_seq")), _ptr(_opt_i32(q_pos, "q_pos")),
+        n_q, seq_lens.shape[0], mb, _ptr(sel), _ptr(dev_err), _stream(stream)))
+    return sel
+
+
+def sparse_attn(q, k_cache, v_cache, block_table, seq_lens, sel, q_seq=None, q_pos=None, *,
+                scale: float | None = None, out=None, workspace=None, dev_err=None, stream=None) -> torch.Tensor:
+    """bf16 [n_q, H, 128] attention output over the selected blocks."""
+    _dev(q, "q", torch.bfloat16, 3)
+    _dev(k_cache, "k_cache", torch.bfloat16, 4)
+    _dev(v_cache, "v_cache", torch.bfloat16, 4)
+    _dev(block_table, "block_table", torch.int32, 2)
+    _dev(seq_lens, "seq_lens", torch.int32, 1)
+    _dev(sel, "sel", torch.int32, 2)
+    n_q, H = q.shape[0], q.shape[1]
+    B, mb = block_table.shape
+    if out is None:
+        out = torch.empty_like(q)
+    if workspace is None:
+        workspace = alloc_workspace(n_q, H, mb, q.device)
+    sc = float(scale) if scale is not None else HEAD_DIM ** -0.5
+    _check("uocr_sparse_attn", lib.uocr_sparse_attn(
+        _ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(block_table), _ptr(seq_lens),
+        _ptr(_opt_i32(q_seq, "q_seq")), _ptr(_opt_i32(q_pos, "q_pos")), _ptr(sel), n_q, B, H, mb,
+        k_cache.shape[0], ctypes.c_float(sc), _ptr(out), _ptr(workspace), workspace.numel(),
+        _ptr(dev_err), _stream(stream)))
+    return out
+
+
+def sparse_decode(q, k_cache, v_cache, idx_q, idx_k_cache, block_table, seq_lens, *,
+                  out=None, sel=None, workspace=None, dev_err=None, stream=None):
+    """One decode query per sequence at p = seq_len - 1.  Returns (out [B,H,128] bf16, sel [B,16] int32)."""
+    _dev(q, "q", torch.bfloat16, 3)
+    _dev(k_cache, "k_cache", torch.bfloat16, 4)
+    _dev(v_cache, "v_cache", torch.bfloat16, 4)
+    _dev(idx_q, "idx_q", torch.bfloat16, 2)
+    _dev(idx_k_cache, "idx_k_cache", torch.bfloat16, 3)
+    _dev(block_table, "block_table", torch.int32, 2)
+    _dev(seq_lens, "seq_lens", torch.int32, 1)
+    B, H = q.shape[0], q.shape[1]
+    mb = block_table.shape[1]
+    if out is None:
+        out = torch.empty_like(q)
+    if sel is None:
+        sel = torch.empty((B, N_SEL), dtype=torch.int32, device=q.device)
+    if workspace is None:
+        workspace = alloc_workspace(B, H, mb, q.device)
+    _check("uocr_sparse_decode", lib.uocr_sparse_decode(
+        _ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(idx_q), _ptr(idx_k_cache), _ptr(block_table),
+        _ptr(seq_lens), B, H, mb, k_cache.shape[0], _ptr(out), _ptr(sel), _ptr(workspace),
+        workspace.numel(), _ptr(dev_err), _stream(stream)))
+    return out, sel

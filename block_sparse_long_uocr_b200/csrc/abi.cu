@@ -1,0 +1,182 @@
+// abi.cu -- the extern "C" entry points of libuocr.so (declared in include/uocr.h).
+//
+// Host side only: argument validation, workspace carving, device attribute
+// lookup and the launches on the caller's stream.  No allocation, no
+// synchronisation, no state kept between calls.
+#include <cuda_runtime.h>
+#include <math.h>
+#include <stdint.h>
+
+#include "common.cuh"
+#include "kernels.h"
+#include "uocr.h"
+
+namespace {
+
+constexpr size_t kWsAlign = 256;
+
+inline size_t round_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+inline bool aligned(const void *p, size_t a) { return ((uintptr_t)p % a) == 0; }
+
+struct WsLayout {
+    size_t scores_off, acc_off, ml_off, total;
+};
+
+inline WsLayout ws_layout(int n_q, int H, int max_blocks) {
+    WsLayout w{};
+    const size_t splits = (size_t)uocr::attn_splits(n_q, H);
+    w.scores_off = 0;
+    w.acc_off = round_up((size_t)n_q * max_blocks * sizeof(float), kWsAlign);
+    w.ml_off = w.acc_off + round_up((size_t)n_q * H * splits * uocr::kD * sizeof(float), kWsAlign);
+    w.total = w.ml_off + round_up((size_t)n_q * H * splits * 2 * sizeof(float), kWsAlign);
+    return w;
+}
+
+inline uocr_status_t make_ctx(uocr_stream_t stream, bool pdl, uocr::LaunchCtx &c) {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return UOCR_ERR_CUDA;
+    int sms = 0;
+    if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+        return UOCR_ERR_CUDA;
+    c.stream = (cudaStream_t)stream;
+    c.num_sms = sms;
+    c.pdl = pdl;
+    return UOCR_OK;
+}
+
+inline uocr_status_t cuda_status(cudaError_t e) {
+    if (e == cudaSuccess) return UOCR_OK;
+    (void)cudaGetLastError();   // clear the sticky-free launch error so later calls are clean
+    return UOCR_ERR_CUDA;
+}
+
+// Common shape checks shared by every compute entry point.
+inline uocr_status_t check_common(int n_q, int B, int max_blocks, int num_pages,
+                                  const int32_t *block_table, const int32_t *seq_lens,
+                                  const int32_t *q_seq, const int32_t *q_pos, const int32_t *dev_err) {
+    if (n_q < 0 || B < 1 || max_blocks < 1 || num_pages < 1) return UOCR_ERR_INVALID_ARG;
+    if (!block_table || !seq_lens) return UOCR_ERR_INVALID_ARG;
+    if (!aligned(block_table, 4) || !aligned(seq_lens, 4)) return UOCR_ERR_INVALID_ARG;
+    if ((q_seq && !aligned(q_seq, 4)) || (q_pos && !aligned(q_pos, 4))) return UOCR_ERR_INVALID_ARG;
+    if (dev_err && !aligned(dev_err, 4)) return UOCR_ERR_INVALID_ARG;
+    if ((long long)max_blocks * UOCR_BLOCK > 0x7fffffffLL) return UOCR_ERR_UNSUPPORTED;
+    return UOCR_OK;
+}
+
+inline bool bf16_ok(const void *p) { return p && aligned(p, 16); }
+
+}  // namespace
+
+extern "C" {
+
+const char *uocr_status_string(uocr_status_t status) {
+    switch (status) {
+        case UOCR_OK: return "UOCR_OK";
+        case UOCR_ERR_INVALID_ARG: return "UOCR_ERR_INVALID_ARG: NULL pointer, bad size or misaligned pointer";
+        case UOCR_ERR_UNSUPPORTED: return "UOCR_ERR_UNSUPPORTED: shape outside what the kernels implement";
+        case UOCR_ERR_WORKSPACE: return "UOCR_ERR_WORKSPACE: workspace NULL, misaligned or too small";
+        case UOCR_ERR_CUDA: return "UOCR_ERR_CUDA: a CUDA launch or attribute query failed";
+    }
+    return "UOCR_ERR_UNKNOWN";
+}
+
+int uocr_abi_version(void) { return 1; }
+
+size_t uocr_workspace_bytes(int n_q, int H, int max_blocks) {
+    if (n_q <= 0 || H <= 0 || max_blocks <= 0) return 0;
+    return ws_layout(n_q, H, max_blocks).total;
+}
+
+uocr_status_t uocr_index_score(const void *idx_q, const void *idx_k_cache,
+                               const int32_t *block_table, const int32_t *seq_lens,
+                               const int32_t *q_seq, const int32_t *q_pos, int n_q, int B,
+                               int max_blocks, int num_pages, float *scores, int32_t *dev_err,
+                               uocr_stream_t stream) {
+    uocr_status_t st = check_common(n_q, B, max_blocks, num_pages, block_table, seq_lens, q_seq,
+                                    q_pos, dev_err);
+    if (st != UOCR_OK) return st;
+    if (!bf16_ok(idx_q) || !bf16_ok(idx_k_cache) || !scores || !aligned(scores, 4))
+        return UOCR_ERR_INVALID_ARG;
+    if (n_q == 0) return UOCR_OK;
+    uocr::LaunchCtx c;
+    if ((st = make_ctx(stream, false, c)) != UOCR_OK) return st;
+    return cuda_status(uocr::launch_index_scan(c, idx_q, idx_k_cache, block_table, seq_lens, q_seq,
+                                               q_pos, n_q, B, max_blocks, num_pages, scores, dev_err));
+}
+
+uocr_status_t uocr_block_topk(const float *scores, const int32_t *seq_lens, const int32_t *q_seq,
+                              const int32_t *q_pos, int n_q, int B, int max_blocks, int32_t *sel,
+                              int32_t *dev_err, uocr_stream_t stream) {
+    if (n_q < 0 || B < 1 || max_blocks < 1) return UOCR_ERR_INVALID_ARG;
+    if (!scores || !seq_lens || !sel) return UOCR_ERR_INVALID_ARG;
+    if (!aligned(scores, 4) || !aligned(seq_lens, 4) || !aligned(sel, 4)) return UOCR_ERR_INVALID_ARG;
+    if ((q_seq && !aligned(q_seq, 4)) || (q_pos && !aligned(q_pos, 4))) return UOCR_ERR_INVALID_ARG;
+    if (dev_err && !aligned(dev_err, 4)) return UOCR_ERR_INVALID_ARG;
+    if (n_q == 0) return UOCR_OK;
+    uocr::LaunchCtx c;
+    uocr_status_t st;
+    if ((st = make_ctx(stream, false, c)) != UOCR_OK) return st;
+    return cuda_status(uocr::launch_block_topk(c, scores, seq_lens, q_seq, q_pos, n_q, B, max_blocks,
+                                               sel, dev_err));
+}
+
+uocr_status_t uocr_sparse_attn(const void *q, const void *k_cache, const void *v_cache,
+                               const int32_t *block_table, const int32_t *seq_lens,
+                               const int32_t *q_seq, const int32_t *q_pos, const int32_t *sel,
+                               int n_q, int B, int H, int max_blocks, int num_pages, float scale,
+                               void *out, void *workspace, size_t workspace_bytes,
+                               int32_t *dev_err, uocr_stream_t stream) {
+    uocr_status_t st = check_common(n_q, B, max_blocks, num_pages, block_table, seq_lens, q_seq,
+                                    q_pos, dev_err);
+    if (st != UOCR_OK) return st;
+    if (!bf16_ok(q) || !bf16_ok(k_cache) || !bf16_ok(v_cache) || !bf16_ok(out)) return UOCR_ERR_INVALID_ARG;
+    if (!sel || !aligned(sel, 4)) return UOCR_ERR_INVALID_ARG;
+    if (H < 1 || H > UOCR_MAX_HEADS) return UOCR_ERR_UNSUPPORTED;
+    if (!isfinite(scale)) return UOCR_ERR_INVALID_ARG;
+    if (n_q == 0) return UOCR_OK;
+    const WsLayout w = ws_layout(n_q, H, max_blocks);
+    if (!workspace || !aligned(workspace, kWsAlign) || workspace_bytes < w.total) return UOCR_ERR_WORKSPACE;
+    uocr::LaunchCtx c;
+    if ((st = make_ctx(stream, false, c)) != UOCR_OK) return st;
+    char *ws = (char *)workspace;
+    return cuda_status(uocr::launch_sparse_attn(c, q, k_cache, v_cache, block_table, seq_lens, q_seq,
+                                                q_pos, sel, n_q, B, H, max_blocks, num_pages, scale,
+                                                out, (float *)(ws + w.acc_off),
+                                                (float *)(ws + w.ml_off), dev_err));
+}
+
+uocr_status_t uocr_sparse_decode(const void *q, const void *k_cache, const void *v_cache,
+                                 const void *idx_q, const void *idx_k_cache,
+                                 const int32_t *block_table, const int32_t *seq_lens, int B, int H,
+                                 int max_blocks, int num_pages, void *out, int32_t *sel_out,
+                                 void *workspace, size_t workspace_bytes, int32_t *dev_err,
+                                 uocr_stream_t stream) {
+    uocr_status_t st = check_common(B, B, max_blocks, num_pages, block_table, seq_lens, nullptr,
+                                    nullptr, dev_err);
+    if (st != UOCR_OK) return st;
+    if (!bf16_ok(q) || !bf16_ok(k_cache) || !bf16_ok(v_cache) || !bf16_ok(out) || !bf16_ok(idx_q) ||
+        !bf16_ok(idx_k_cache))
+        return UOCR_ERR_INVALID_ARG;
+    if (!sel_out || !aligned(sel_out, 4)) return UOCR_ERR_INVALID_ARG;
+    if (H < 1 || H > UOCR_MAX_HEADS) return UOCR_ERR_UNSUPPORTED;
+    const WsLayout w = ws_layout(B, H, max_blocks);
+    if (!workspace || !aligned(workspace, kWsAlign) || workspace_bytes < w.total) return UOCR_ERR_WORKSPACE;
+    uocr::LaunchCtx c;
+    if ((st = make_ctx(stream, false, c)) != UOCR_OK) return st;
+    char *ws = (char *)workspace;
+    float *scores = (float *)(ws + w.scores_off);
+    cudaError_t e = uocr::launch_index_scan(c, idx_q, idx_k_cache, block_table, seq_lens, nullptr,
+                                            nullptr, B, B, max_blocks, num_pages, scores, dev_err);
+    if (e != cudaSuccess) return cuda_status(e);
+    c.pdl = true;
+    e = uocr::launch_block_topk(c, scores, seq_lens, nullptr, nullptr, B, B, max_blocks, sel_out, dev_err);
+    if (e != cudaSuccess) return cuda_status(e);
+    const float scale = 1.0f / sqrtf((float)UOCR_HEAD_DIM);
+    e = uocr::launch_sparse_attn(c, q, k_cache, v_cache, block_table, seq_lens, nullptr, nullptr, sel_out,
+                                 B, B, H, max_blocks, num_pages, scale, out, (float *)(ws + w.acc_off),
+                                 (float *)(ws + w.ml_off), dev_err);
+    return cuda_status(e);
+}
+
+}  // extern "C"

@@ -1,0 +1,127 @@
+// common.cuh -- device helpers shared by the libuocr kernels (sm_100a).
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "uocr.h"
+
+namespace uocr {
+
+constexpr int kBlock = UOCR_BLOCK;        // tokens per KV block / page
+constexpr int kLocal = UOCR_N_LOCAL;
+constexpr int kRemote = UOCR_N_REMOTE;
+constexpr int kSel = UOCR_N_SEL;
+constexpr int kD = UOCR_HEAD_DIM;
+constexpr int kDIdx = UOCR_IDX_DIM;
+constexpr int kPageElems = kBlock * kD;   // elements of one (page, head) tile: 4096 bf16 = 8 KiB
+constexpr float kLog2e = 1.4426950408889634f;
+
+// Query position and sequence for query i, with the device-side checks the
+// ABI documents.  Returns false (and flags dev_err) when the query is invalid;
+// p < 0 (empty sequence) is valid and means "no visible token".
+struct QueryRef {
+    int b;
+    int p;
+    int nb;
+};
+
+__device__ __forceinline__ void flag_error(int32_t *dev_err, uint32_t bits) {
+    if (dev_err) atomicOr(reinterpret_cast<unsigned int *>(dev_err), bits);
+}
+
+__device__ __forceinline__ bool resolve_query(int i, const int32_t *seq_lens, const int32_t *q_seq,
+                                              const int32_t *q_pos, int B, int max_blocks,
+                                              int32_t *dev_err, bool report, QueryRef &r) {
+    int b = q_seq ? __ldg(q_seq + i) : i;
+    if (b < 0 || b >= B) {
+        if (report) flag_error(dev_err, UOCR_DEVERR_POS);
+        return false;
+    }
+    int len = __ldg(seq_lens + b);
+    int p = q_pos ? __ldg(q_pos + i) : len - 1;
+    if (p >= len || len > max_blocks * kBlock) {
+        if (report) flag_error(dev_err, UOCR_DEVERR_POS);
+        return false;
+    }
+    r.b = b;
+    r.p = p;
+    r.nb = p < 0 ? 0 : p / kBlock + 1;
+    return true;
+}
+
+// 8 bf16 packed in a uint4 -> 8 floats (exact: bf16 is the top half of fp32).
+__device__ __forceinline__ void bf16x8_to_f32(const uint4 &v, float (&f)[8]) {
+    const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+        f[2 * k] = __uint_as_float(w[k] << 16);
+        f[2 * k + 1] = __uint_as_float(w[k] & 0xffff0000u);
+    }
+}
+
+// Streaming 16-byte load that bypasses L1 allocation (each byte is read once).
+__device__ __forceinline__ uint4 ld_stream(const uint4 *p) {
+    uint4 v;
+    asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0,%1,%2,%3}, [%4];"
+                 : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+                 : "l"(p));
+    return v;
+}
+
+__device__ __forceinline__ float warp_max(float v) {
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
+    return v;
+}
+
+__device__ __forceinline__ float warp_sum(float v) {
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+    return v;
+}
+
+// Transposed reduction of 16 partial sums over the 16 lanes of a half-warp.
+// On entry lane l holds v[0..15], partial over its own slice of the reduced
+// dimension; on exit v[0] of lane l is the full sum of index (l & 15).
+// 8 + 4 + 2 + 1 = 15 shuffles instead of 16 x 4.
+__device__ __forceinline__ float half_warp_transpose_sum16(float (&v)[16], int lane) {
+#pragma unroll
+    for (int k = 0; k < 8; ++k) {
+        const bool hi = lane & 8;
+        float send = hi ? v[k] : v[k + 8];
+        float keep = hi ? v[k + 8] : v[k];
+        v[k] = keep + __shfl_xor_sync(0xffffffffu, send, 8);
+    }
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+        const bool hi = lane & 4;
+        float send = hi ? v[k] : v[k + 4];
+        float keep = hi ? v[k + 4] : v[k];
+        v[k] = keep + __shfl_xor_sync(0xffffffffu, send, 4);
+    }
+#pragma unroll
+    for (int k = 0; k < 2; ++k) {
+        const bool hi = lane & 2;
+        float send = hi ? v[k] : v[k + 2];
+        float keep = hi ? v[k + 2] : v[k];
+        v[k] = keep + __shfl_xor_sync(0xffffffffu, send, 2);
+    }
+    {
+        const bool hi = lane & 1;
+        float send = hi ? v[0] : v[1];
+        float keep = hi ? v[1] : v[0];
+        v[0] = keep + __shfl_xor_sync(0xffffffffu, send, 1);
+    }
+    return v[0];
+}
+
+// Programmatic dependent launch: wait for the preceding grid's memory, and
+// allow the next grid to begin launching.  Both are no-ops when the kernel was
+// launched without the programmatic-serialization attribute.
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_launch_dependents() {
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
+}  // namespace uocr

@@ -1,0 +1,34 @@
+// kernels.h -- internal launchers of libuocr (not part of the public ABI).
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+namespace uocr {
+
+struct LaunchCtx {
+    cudaStream_t stream;
+    int num_sms;
+    bool pdl;   // launch with programmatic stream serialization
+};
+
+// Number of split-K partitions the attention uses for n_q queries of H heads.
+int attn_splits(int n_q, int H);
+
+cudaError_t launch_index_scan(const LaunchCtx &c, const void *idx_q, const void *idx_k,
+                              const int32_t *bt, const int32_t *seq_lens, const int32_t *q_seq,
+                              const int32_t *q_pos, int n_q, int B, int max_blocks, int num_pages,
+                              float *scores, int32_t *dev_err);
+
+cudaError_t launch_block_topk(const LaunchCtx &c, const float *scores, const int32_t *seq_lens,
+                              const int32_t *q_seq, const int32_t *q_pos, int n_q, int B,
+                              int max_blocks, int32_t *sel, int32_t *dev_err);
+
+cudaError_t launch_sparse_attn(const LaunchCtx &c, const void *q, const void *k, const void *v,
+                               const int32_t *bt, const int32_t *seq_lens, const int32_t *q_seq,
+                               const int32_t *q_pos, const int32_t *sel, int n_q, int B, int H,
+                               int max_blocks, int num_pages, float scale, void *out,
+                               float *part_acc, float *part_ml, int32_t *dev_err);
+
+}  // namespace uocr

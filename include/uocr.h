@@ -1,0 +1,172 @@
+/*
+ * uocr.h -- C ABI of libuocr.so: the SR-SWA / DASH block-sparse attention step
+ * of Unlimited-OCR-2 on NVIDIA B200 (sm_100a).
+ *
+ * What the step computes (cited by page and section):
+ *   [rkmt]  Unlimited-OCR-2 walk-through, news.rkmt.cn/news/25027, section 五
+ *           ("SR-SWA: block-level sparse attention"): keys are cut into 32-token
+ *           blocks (step 1); a 1-head x 128-dim Lightning Indexer scores every
+ *           block for every query, the block score being the maximum over the
+ *           block's tokens (step 2); each query keeps 16 blocks, 4 local blocks
+ *           (the 128-token sliding window) plus 12 remote blocks (step 3); exact
+ *           attention runs over the selected blocks only (step 4).  Section 三:
+ *           10 attention heads, 10 KV heads (MHA), head dim 128.
+ *   [lqnn]  Unlimited-OCR-2-8bit page, www.lqnn.cn/news/271890, section
+ *           显存账本: top-12 remote + 4 local = 16 blocks x 32 = 512 tokens.
+ *   [leheaven] release report, leheavengame.com (Unlimited OCR 2 open-source),
+ *           section 三: chunked prefill materialises a [tokens, context/32]
+ *           block-score tensor.
+ *
+ * Readings where the pages are open (the same in the CPU oracle):
+ *   - block score = max over tokens t <= p of the raw dot product q_idx . k_idx
+ *     (no ReLU, no weight, no scale);
+ *   - a query at position p sees tokens 0..p; nb = p/32 + 1 causal blocks;
+ *     local = the last 4 causal blocks, remote candidates = blocks [0, nb-4);
+ *   - remote ranking: score descending, then lower block id; with no more than
+ *     12 candidates all of them are taken;
+ *   - the decode query is the last cached token: p = seq_len - 1.
+ *
+ * Conventions for every entry point:
+ *   - All tensor pointers are DEVICE pointers owned by the caller; the library
+ *     never allocates, frees or keeps device memory and holds no global state.
+ *   - bf16 tensors are passed as void* (IEEE bfloat16 bit patterns), must be
+ *     16-byte aligned and densely packed in the layouts given below.
+ *   - Every call is asynchronous on `stream` (NULL = the legacy default stream)
+ *     and performs no host/device synchronisation.
+ *   - Host-side argument checks run before any launch; a failed check returns
+ *     UOCR_ERR_INVALID_ARG / UOCR_ERR_UNSUPPORTED / UOCR_ERR_WORKSPACE and
+ *     launches nothing.  A failed launch returns UOCR_ERR_CUDA.
+ *   - Data-dependent checks run on the device: a block-table entry outside
+ *     [0, num_pages), a query position at or past its sequence length, a
+ *     sequence index outside [0, B), or more causal blocks than max_blocks make
+ *     the kernel skip the offending block / query (its outputs are -inf scores,
+ *     -1 selections, zero attention output) and, when `dev_err` is not NULL,
+ *     OR a UOCR_DEVERR_* bit into *dev_err.  Kernels never trap.
+ *
+ * Layouts (P = num_pages, B = sequences, n_q = queries, H = heads):
+ *   q            bf16  [n_q][H][128]
+ *   k_cache      bf16  [P][H][32][128]   one (page, head) tile = 8 KiB contiguous
+ *   v_cache      bf16  [P][H][32][128]
+ *   idx_q        bf16  [n_q][128]
+ *   idx_k_cache  bf16  [P][32][128]      one page = 8 KiB contiguous
+ *   block_table  int32 [B][max_blocks]   logical block j of sequence b -> page
+ *   seq_lens     int32 [B]               cached tokens of each sequence
+ *   q_seq        int32 [n_q]             sequence of each query (NULL: query i -> sequence i)
+ *   q_pos        int32 [n_q]             token position p of each query (NULL: seq_len - 1)
+ *   scores       fp32  [n_q][max_blocks] block scores; entries j >= nb are not written
+ *   sel          int32 [n_q][16]         selected logical blocks, ascending, -1 padded
+ *   out          bf16  [n_q][H][128]
+ */
+#ifndef UOCR_H
+#define UOCR_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Same handle as cudaStream_t / CUstream. */
+typedef struct CUstream_st *uocr_stream_t;
+
+typedef enum {
+    UOCR_OK = 0,
+    UOCR_ERR_INVALID_ARG = 1,   /* NULL pointer, bad size, misaligned pointer */
+    UOCR_ERR_UNSUPPORTED = 2,   /* shape outside what the kernels implement */
+    UOCR_ERR_WORKSPACE = 3,     /* workspace NULL, misaligned or too small */
+    UOCR_ERR_CUDA = 4           /* a CUDA launch or attribute call failed */
+} uocr_status_t;
+
+/* Method constants ([rkmt 五], [lqnn 显存账本]). */
+#define UOCR_BLOCK 32
+#define UOCR_N_LOCAL 4
+#define UOCR_N_REMOTE 12
+#define UOCR_N_SEL 16
+#define UOCR_HEAD_DIM 128
+#define UOCR_IDX_DIM 128
+#define UOCR_MAX_HEADS 64
+
+/* Bits OR-ed into *dev_err by the kernels. */
+#define UOCR_DEVERR_PAGE 1u   /* block-table entry outside [0, num_pages) */
+#define UOCR_DEVERR_POS 2u    /* q_pos >= seq_len, q_seq outside [0, B), or nb > max_blocks */
+#define UOCR_DEVERR_SEL 4u    /* a selected block outside the query's causal blocks */
+
+/* Human-readable name of a status code (static storage; never NULL). */
+const char *uocr_status_string(uocr_status_t status);
+
+/* ABI version of this header; bumped on any signature change. */
+int uocr_abi_version(void);
+
+/*
+ * Workspace bytes that uocr_sparse_attn, uocr_sparse_decode and
+ * uocr_sparse_prefill need for n_q queries of H heads over max_blocks blocks.
+ * A pure function of the shapes (0 for a non-positive argument).  The
+ * workspace holds the fp32 block scores [n_q][max_blocks] and the split-K
+ * partial softmax states; callers may reuse it across calls on one stream.
+ */
+size_t uocr_workspace_bytes(int n_q, int H, int max_blocks);
+
+/*
+ * Indexer scan, [rkmt 五 steps 1-2]:
+ *   scores[i][j] = max_{t in block j, t <= p_i} sum_{d<128} idx_q[i][d] * idx_k[t][d]
+ * for every causal block j < nb_i of query i, in fp32 from bf16 inputs.
+ * HBM-bound: reads every causal indexer page of the query's sequence once.
+ * Errors: INVALID_ARG for NULL idx_q / idx_k_cache / block_table / seq_lens /
+ * scores, n_q < 0, B < 1, max_blocks < 1, num_pages < 1, or misalignment.
+ */
+uocr_status_t uocr_index_score(const void *idx_q, const void *idx_k_cache,
+                               const int32_t *block_table, const int32_t *seq_lens,
+                               const int32_t *q_seq, const int32_t *q_pos,
+                               int n_q, int B, int max_blocks, int num_pages,
+                               float *scores, int32_t *dev_err, uocr_stream_t stream);
+
+/*
+ * Block selection, [rkmt 五 step 3]: for each query, the local blocks
+ * {nb-4, ..., nb-1} (clipped at 0) and the 12 highest-scoring remote
+ * candidates in [0, nb-4), ranked by (score desc, block id asc); all
+ * candidates when there are at most 12.  sel[i] = the union, ascending, -1
+ * padded to 16.  Reads scores[i][0 .. nb-5] only.
+ */
+uocr_status_t uocr_block_topk(const float *scores, const int32_t *seq_lens,
+                              const int32_t *q_seq, const int32_t *q_pos,
+                              int n_q, int B, int max_blocks, int32_t *sel,
+                              int32_t *dev_err, uocr_stream_t stream);
+
+/*
+ * Gathered exact attention, [rkmt 五 step 4]: per query i and head h,
+ *   z_t = scale * q[i][h] . k[h][t]  over the tokens t <= p_i of the blocks in sel[i],
+ *   out[i][h] = sum_t softmax(z)_t v[h][t]    (fp32 softmax and accumulation, bf16 out).
+ * Entries of sel < 0 are skipped; a query with no visible token gets zeros.
+ * Split-K over the 16 blocks with a flash-decoding combine through the
+ * workspace (uocr_workspace_bytes(n_q, H, max_blocks) bytes, 256-byte aligned).
+ * H in [1, UOCR_MAX_HEADS] (the model uses 10); head dim fixed at 128.
+ */
+uocr_status_t uocr_sparse_attn(const void *q, const void *k_cache, const void *v_cache,
+                               const int32_t *block_table, const int32_t *seq_lens,
+                               const int32_t *q_seq, const int32_t *q_pos,
+                               const int32_t *sel, int n_q, int B, int H,
+                               int max_blocks, int num_pages, float scale, void *out,
+                               void *workspace, size_t workspace_bytes,
+                               int32_t *dev_err, uocr_stream_t stream);
+
+/*
+ * The whole decode step for B sequences, one query each at p = seq_len - 1:
+ * uocr_index_score -> uocr_block_topk -> uocr_sparse_attn with
+ * scale = 1/sqrt(128), launched back to back on `stream` (programmatic
+ * dependent launch, no host synchronisation).  sel_out [B][16] receives the
+ * selection and must not be NULL.  Workspace: uocr_workspace_bytes(B, H, max_blocks).
+ */
+uocr_status_t uocr_sparse_decode(const void *q, const void *k_cache, const void *v_cache,
+                                 const void *idx_q, const void *idx_k_cache,
+                                 const int32_t *block_table, const int32_t *seq_lens,
+                                 int B, int H, int max_blocks, int num_pages,
+                                 void *out, int32_t *sel_out,
+                                 void *workspace, size_t workspace_bytes,
+                                 int32_t *dev_err, uocr_stream_t stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* UOCR_H */

@@ -1,0 +1,175 @@
+"""Host-side checks of the C ABI: the library loads, exports every declared
+symbol, and rejects bad arguments before launching anything.
+
+These run without a GPU.  Calls with fake pointers are made only on hosts
+with no CUDA device, and every one of them carries an argument that the host
+validation rejects before any CUDA call.
+"""
+import ctypes
+import os
+import re
+import subprocess
+
+import pytest
+import torch
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "uocr.h")
+
+
+@pytest.fixture(scope="module")
+def pkg():
+    from block_sparse_long_uocr_b200 import build
+    build.build()
+    import block_sparse_long_uocr_b200 as m
+    return m
+
+
+def declared_functions():
+    src = open(HEADER).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"\b(uocr_[a-z0-9_]+)\s*\(", src)))
+
+
+def test_header_declares_the_entry_points():
+    names = declared_functions()
+    for n in ["uocr_index_score", "uocr_block_topk", "uocr_sparse_attn", "uocr_sparse_decode",
+              "uocr_workspace_bytes", "uocr_status_string", "uocr_abi_version"]:
+        assert n in names
+
+
+def test_library_exports_every_declared_symbol(pkg):
+    out = subprocess.run(["nm", "-D", "--defined-only", pkg.LIB_PATH], capture_output=True, text=True,
+                         check=True).stdout
+    exported = set(re.findall(r"\bT (uocr_[a-z0-9_]+)\b", out))
+    missing = [n for n in declared_functions() if n not in exported]
+    assert not missing, f"declared but not exported: {missing}"
+    for n in declared_functions():
+        assert hasattr(pkg.lib, n)
+
+
+def test_status_strings_and_version(pkg):
+    for code in range(5):
+        s = pkg.lib.uocr_status_string(code).decode()
+        assert s.startswith(pkg.STATUS[code])
+    assert pkg.lib.uocr_status_string(99).decode() == "UOCR_ERR_UNKNOWN"
+    assert pkg.lib.uocr_abi_version() == 1
+
+
+def test_workspace_is_a_pure_function_of_shapes(pkg):
+    ws = pkg.workspace_bytes
+    assert ws(0, 10, 64) == 0 and ws(4, 0, 64) == 0 and ws(4, 10, 0) == 0
+    a = ws(16, 10, 4096)
+    assert a == ws(16, 10, 4096) and a % 256 == 0
+    assert a >= 16 * 4096 * 4                       # block-score scratch
+    assert ws(32, 10, 4096) > a and ws(16, 10, 8192) > a
+    # independent of data: same answer regardless of sequence lengths (none are passed)
+
+
+# --------------------------------------------------------------------------- host fault injection
+no_gpu = pytest.mark.skipif(torch.cuda.is_available(),
+                            reason="fake-pointer calls run only on hosts without a CUDA device")
+FAKE = 1 << 20          # 16-byte aligned, never dereferenced: every call below fails validation first
+MIS = FAKE + 2          # misaligned for bf16 / int32
+
+
+def _score_args(**over):
+    a = dict(idx_q=FAKE, idx_k=FAKE, bt=FAKE, sl=FAKE, qs=None, qp=None, n_q=4, B=4, mb=64, P=256,
+             scores=FAKE, err=None)
+    a.update(over)
+    return a
+
+
+def _call_score(lib, a):
+    return lib.uocr_index_score(a["idx_q"], a["idx_k"], a["bt"], a["sl"], a["qs"], a["qp"], a["n_q"], a["B"],
+                                a["mb"], a["P"], a["scores"], a["err"], None)
+
+
+@no_gpu
+@pytest.mark.parametrize("over", [dict(idx_q=None), dict(idx_k=None), dict(bt=None), dict(sl=None),
+                                  dict(scores=None), dict(n_q=-1), dict(B=0), dict(mb=0), dict(P=0),
+                                  dict(idx_q=MIS), dict(idx_k=FAKE + 8), dict(bt=MIS), dict(scores=MIS),
+                                  dict(qs=MIS), dict(qp=MIS), dict(err=MIS)])
+def test_index_score_rejects(pkg, over):
+    assert _call_score(pkg.lib, _score_args(**over)) == 1
+
+
+@no_gpu
+def test_index_score_rejects_huge_block_count(pkg):
+    assert _call_score(pkg.lib, _score_args(mb=1 << 27)) == 2
+
+
+@no_gpu
+def test_zero_queries_is_a_no_op(pkg):
+    # n_q == 0 returns before touching the device
+    assert _call_score(pkg.lib, _score_args(n_q=0)) == 0
+    assert pkg.lib.uocr_block_topk(FAKE, FAKE, None, None, 0, 4, 64, FAKE, None, None) == 0
+
+
+@no_gpu
+@pytest.mark.parametrize("args", [
+    (None, FAKE, None, None, 4, 4, 64, FAKE),     # scores NULL
+    (FAKE, None, None, None, 4, 4, 64, FAKE),     # seq_lens NULL
+    (FAKE, FAKE, None, None, 4, 4, 64, None),     # sel NULL
+    (FAKE, FAKE, None, None, 4, 0, 64, FAKE),     # B < 1
+    (FAKE, FAKE, None, None, 4, 4, 0, FAKE),      # max_blocks < 1
+    (MIS, FAKE, None, None, 4, 4, 64, FAKE),      # misaligned scores
+    (FAKE, FAKE, None, None, 4, 4, 64, MIS),      # misaligned sel
+])
+def test_block_topk_rejects(pkg, args):
+    assert pkg.lib.uocr_block_topk(*args, None, None) == 1
+
+
+def _call_attn(lib, **over):
+    a = dict(q=FAKE, k=FAKE, v=FAKE, bt=FAKE, sl=FAKE, sel=FAKE, n_q=4, B=4, H=10, mb=64, P=256,
+             scale=0.088, out=FAKE, ws=FAKE, wsb=1 << 30)
+    a.update(over)
+    return lib.uocr_sparse_attn(a["q"], a["k"], a["v"], a["bt"], a["sl"], None, None, a["sel"], a["n_q"],
+                                a["B"], a["H"], a["mb"], a["P"], ctypes.c_float(a["scale"]), a["out"], a["ws"],
+                                a["wsb"], None, None)
+
+
+@no_gpu
+@pytest.mark.parametrize("over,code", [
+    (dict(q=None), 1), (dict(k=MIS), 1), (dict(v=None), 1), (dict(out=FAKE + 4), 1), (dict(sel=None), 1),
+    (dict(H=0), 2), (dict(H=65), 2), (dict(scale=float("nan")), 1), (dict(scale=float("inf")), 1),
+    (dict(ws=None), 3), (dict(ws=FAKE + 16), 3), (dict(wsb=1024), 3),
+])
+def test_sparse_attn_rejects(pkg, over, code):
+    assert _call_attn(pkg.lib, **over) == code
+
+
+@no_gpu
+def test_sparse_attn_workspace_boundary(pkg):
+    need = pkg.workspace_bytes(4, 10, 64)
+    assert _call_attn(pkg.lib, wsb=need - 1) == 3
+
+
+@no_gpu
+@pytest.mark.parametrize("over,code", [
+    (dict(sel=None), 1), (dict(idx_q=None), 1), (dict(idx_k=MIS), 1), (dict(H=0), 2),
+    (dict(wsb=0), 3), (dict(ws=None), 3), (dict(B=0), 1), (dict(mb=0), 1),
+])
+def test_sparse_decode_rejects(pkg, over, code):
+    a = dict(q=FAKE, k=FAKE, v=FAKE, idx_q=FAKE, idx_k=FAKE, bt=FAKE, sl=FAKE, B=4, H=10, mb=64, P=256,
+             out=FAKE, sel=FAKE, ws=FAKE, wsb=1 << 30)
+    a.update(over)
+    st = pkg.lib.uocr_sparse_decode(a["q"], a["k"], a["v"], a["idx_q"], a["idx_k"], a["bt"], a["sl"], a["B"],
+                                    a["H"], a["mb"], a["P"], a["out"], a["sel"], a["ws"], a["wsb"], None, None)
+    assert st == code
+
+
+def test_python_binding_refuses_cpu_tensors(pkg):
+    x = torch.zeros(2, 128, dtype=torch.bfloat16)
+    with pytest.raises(ValueError, match="CUDA"):
+        pkg.index_score(x, torch.zeros(4, 32, 128, dtype=torch.bfloat16), torch.zeros(2, 4, dtype=torch.int32),
+                        torch.ones(2, dtype=torch.int32))
+
+
+def test_product_package_does_not_import_the_oracle():
+    pkg_dir = os.path.join(ROOT, "block_sparse_long_uocr_b200")
+    for dirpath, _, files in os.walk(pkg_dir):
+        for f in files:
+            if f.endswith((".py", ".cu", ".cuh", ".h", ".c", ".cpp")):
+                src = open(os.path.join(dirpath, f)).read()
+                assert not re.search(r"\boracle\b", src.replace("oracle-free", "")), f"{f} mentions the oracle"
