@@ -43,7 +43,11 @@ FALLBACK_HBM_GBS = 6650.0
 # DRAM traffic of the dominant kernel from one ncu capture (dram__bytes_read.sum +
 # dram__bytes_write.sum), per launch of the default workload, and the hash of the
 # kernel source it was taken on.  Reported as null once the source has changed.
-NCU_TRAFFIC = {}
+NCU_TRAFFIC = {
+    # ncu --set full on long_decode batch 4 (1 layer), one launch: 134,301,184 B read +
+    # 3,638,272 B written (the write-back of the bench's L2 flush), scaled x4 to 16 queries.
+    "long_decode": {"bytes": 4 * (134301184 + 3638272), "src": "f7c4636027d893b4"},
+}
 
 
 def kernel_source_hash(name: str) -> str:
@@ -63,40 +67,83 @@ def measured_peaks():
 
 # --------------------------------------------------------------------------- clocks
 class ClockSampler:
-    """nvidia-smi samples (200 ms) of SM clock and throttle reasons while the timed region runs."""
+    """nvidia-smi samples (every 100 ms) of SM clock and throttle reasons.
+
+    start() launches the sampler and waits for its first sample; mark() brackets the
+    timed region; stop() waits for one sample after the region and ends the sampler.
+    The summary keeps the samples taken inside the region, or, when the region is
+    shorter than the sampling period, the one just before and the one just after it.
+    """
     FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
               "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
 
-    def __init__(self, gpu_index: int):
+    def __init__(self, gpu_index):
+        import threading
         self.gpu = gpu_index
         self.proc = None
+        self.samples = []          # (time, line)
+        self.lock = threading.Lock()
+        self.t0 = self.t1 = None
+        self.raw_error = None
 
-    def __enter__(self):
+    def _reader(self):
+        for line in self.proc.stdout:
+            if line.strip():
+                with self.lock:
+                    self.samples.append((time.perf_counter(), line.strip()))
+
+    def start(self):
+        import threading
         try:
             self.proc = subprocess.Popen(["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
-                                          "-lms", "200", "-i", str(self.gpu)],
-                                         stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
-        except Exception:
-            self.proc = None
+                                          "-lms", "100", "-i", str(self.gpu)],
+                                         stdout=subprocess.PIPE, stderr=subprocess.PIPE, text=True)
+        except Exception as e:
+            self.raw_error = repr(e)
+            return self
+        threading.Thread(target=self._reader, daemon=True).start()
+        deadline = time.perf_counter() + 10
+        while time.perf_counter() < deadline and not self.samples and self.proc.poll() is None:
+            time.sleep(0.02)
         return self
 
-    def __exit__(self, *exc):
-        self.lines = []
-        if self.proc is not None:
-            self.proc.terminate()
-            try:
-                out, _ = self.proc.communicate(timeout=5)
-            except Exception:
-                self.proc.kill()
-                out, _ = self.proc.communicate()
-            self.lines = [l for l in out.splitlines() if l.strip()]
-        return False
+    def mark_start(self):
+        self.t0 = time.perf_counter()
+
+    def mark_end(self):
+        self.t1 = time.perf_counter()
+
+    def stop(self):
+        if self.proc is None:
+            return
+        deadline = time.perf_counter() + 2
+        while time.perf_counter() < deadline and self.proc.poll() is None:
+            with self.lock:
+                if self.samples and self.samples[-1][0] > (self.t1 or 0):
+                    break
+            time.sleep(0.02)
+        self.proc.terminate()
+        try:
+            _, err = self.proc.communicate(timeout=5)
+            if not self.samples and err:
+                self.raw_error = err.strip()[:200]
+        except Exception:
+            self.proc.kill()
 
     def summary(self):
         sm, mx, reasons = [], None, set()
         names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        for l in getattr(self, "lines", []):
+        with self.lock:
+            samples = list(self.samples)
+        inside = [l for t, l in samples if self.t0 is not None and self.t0 <= t <= (self.t1 or t)]
+        where = "inside the timed region"
+        if not inside:
+            before = [l for t, l in samples if self.t0 is not None and t < self.t0][-1:]
+            after = [l for t, l in samples if self.t1 is not None and t > self.t1][:1]
+            inside = before + after
+            where = "bracketing the timed region (shorter than the 100 ms sampling period)"
+        for l in inside:
             f = [x.strip() for x in l.split(",")]
             if len(f) < 9:
                 continue
@@ -109,8 +156,9 @@ class ClockSampler:
                 if v.lower().startswith("active"):
                     reasons.add(n)
         if not sm:
-            return {"sm_mhz": None, "sm_max_mhz": mx, "reasons": [], "samples": 0}
-        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx, "reasons": sorted(reasons), "samples": len(sm)}
+            return {"sm_mhz": None, "sm_max_mhz": mx, "reasons": [], "samples": 0, "error": self.raw_error}
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx, "reasons": sorted(reasons), "samples": len(sm),
+                "where": where}
 
 
 def physical_gpu(local_rank: int) -> str:
@@ -124,9 +172,9 @@ def physical_gpu(local_rank: int) -> str:
 
 
 # --------------------------------------------------------------------------- workloads
-def build_workload(name: str, device, seed: int):
+def build_workload(name: str, device, seed: int, batch=None, layers=None):
     if name == "long_decode":
-        return workloads.long_decode(device=device, seed=seed)
+        return workloads.long_decode(device=device, seed=seed, B=batch or 16, n_layers=layers or 12)
     if name == "batched_decode":
         return workloads.batched_decode(device=device, seed=seed)
     if name == "tiny_decode":
@@ -154,7 +202,7 @@ def run_uocr(args):
                                              device_id=dev)
     import block_sparse_long_uocr_b200 as uocr
 
-    case = build_workload(args.workload, dev, udist.shard_seed(args.seed, rank))
+    case = build_workload(args.workload, dev, udist.shard_seed(args.seed, rank), args.batch, args.layers)
     n_layers = len(case.layers)
     B, H, mb = case.n_q, case.q.shape[1], case.max_blocks
     bytes_call, scan_bytes_call = algorithmic_bytes(case)
@@ -177,6 +225,7 @@ def run_uocr(args):
         if world > 1:
             torch.distributed.barrier(device_ids=[local_rank])
 
+    clk = ClockSampler(physical_gpu(local_rank)).start()
     for _ in range(args.warmup):
         if flush:
             flush_buf.zero_()
@@ -185,33 +234,36 @@ def run_uocr(args):
     barrier()
     torch.cuda.synchronize()
 
-    with ClockSampler(physical_gpu(local_rank)) as clk:
-        if flush:
-            # L2 flushed between steps; each step timed on its own
-            times = []
-            for _ in range(args.steps):
-                flush_buf.zero_()
-                e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-                e0.record(stream)
-                step()
-                e1.record(stream)
-                times.append((e0, e1))
-            torch.cuda.synchronize()
-            elapsed_ms = sum(a.elapsed_time(b) for a, b in times)
-        else:
+    clk.mark_start()
+    if flush:
+        # L2 flushed between steps; each step timed on its own
+        times = []
+        for _ in range(args.steps):
+            flush_buf.zero_()
             e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
             e0.record(stream)
-            for _ in range(args.steps):
-                step()
+            step()
             e1.record(stream)
-            torch.cuda.synchronize()
-            elapsed_ms = e0.elapsed_time(e1)
+            times.append((e0, e1))
+        torch.cuda.synchronize()
+        elapsed_ms = sum(a.elapsed_time(b) for a, b in times)
+    else:
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(args.steps):
+            step()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        elapsed_ms = e0.elapsed_time(e1)
+    clk.mark_end()
+    clk.stop()
     barrier()
     torch.cuda.synchronize()
     max_ms = udist.max_over_ranks(elapsed_ms, dev)
     ms_per_step = max_ms / args.steps
     queries_per_step = B * n_layers
-    value = world * queries_per_step * args.steps / (max_ms / 1e3) / n_layers
+    # queries/s per layer: each layer call decodes B queries; a step makes n_layers calls
+    value = world * queries_per_step * args.steps / (max_ms / 1e3)
 
     # ---- dominant kernel (indexer scan) timed on its own launches, same inputs and stream
     scores = torch.empty((B, mb), dtype=torch.float32, device=dev)
@@ -231,7 +283,7 @@ def run_uocr(args):
     peak = float(peaks.get("hbm_gbs", FALLBACK_HBM_GBS))
     scan_gbs = scan_bytes_call / (scan_ms / 1e3) / 1e9
     step_gbs = bytes_call * n_layers / (ms_per_step / 1e3) / 1e9
-    tr = NCU_TRAFFIC.get(args.workload)
+    tr = NCU_TRAFFIC.get(args.workload) if (args.workload != "long_decode" or B == 16) else None
     traffic = tr["bytes"] if tr and tr.get("src") == kernel_source_hash("index_scan.cu") else None
 
     # ---- end to end through the public API: pinned host inputs in, results out, every step
@@ -306,7 +358,7 @@ def run_e2e(args, uocr, case, ws, outs, sels, stream, world, dev):
     e1.record(stream)
     torch.cuda.synchronize()
     ms = udist.max_over_ranks(e0.elapsed_time(e1), dev)
-    value = world * case.n_q * n_layers * steps / (ms / 1e3) / n_layers
+    value = world * case.n_q * n_layers * steps / (ms / 1e3)
     return {"value": round(value, 1), "unit": UNIT, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
             "ms_per_step": round(ms / steps, 4)}
 
@@ -370,18 +422,18 @@ def oracle_time_queries(case, layer, queries, threads=0):
     return (t1 - t0) + (t3 - t2), r["threads"], r2
 
 
-def cpu_baseline(case, budget_s: float = 15.0):
-    """The oracle as it stands, on this host's cores, on a bounded sample of the same workload."""
+def cpu_baseline(case, budget_s: float = 10.0, max_passes: int = 4):
+    """The oracle as it stands, on this host's cores, on a bounded sample of the same workload:
+    whole layers of queries, cycling over the layers, until about budget_s seconds of oracle time."""
     n_layers = len(case.layers)
-    done, secs, threads = 0, 0.0, 1
-    layer = 0
-    while secs < budget_s and layer < n_layers:
-        t, threads, _ = oracle_time_queries(case, layer, list(range(case.n_q)))
+    done, secs, threads, calls = 0, 0.0, 1, 0
+    while secs < budget_s and calls < max_passes * n_layers:
+        t, threads, _ = oracle_time_queries(case, calls % n_layers, list(range(case.n_q)))
         secs += t
         done += case.n_q
-        layer += 1
+        calls += 1
     return {"value": round(done / secs, 2), "unit": UNIT, "cores": threads, "kind": "oracle",
-            "sample": f"{done} queries ({layer} of {n_layers} layers x {case.n_q} sequences) of {case.name}, "
+            "sample": f"{done} queries ({calls} layer calls of {case.n_q} sequences) of {case.name}, "
                       f"fp64, {secs:.1f} s of oracle time (host reads excluded)",
             "host_cpus": os.cpu_count()}
 
@@ -423,14 +475,16 @@ def run_reference(args):
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=20)
-    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", default="uocr", choices=["uocr", "reference"])
     ap.add_argument("--workload", default="long_decode",
                     choices=["long_decode", "batched_decode", "tiny_decode", "ragged_paged_decode"])
     ap.add_argument("--seed", type=int, default=0)
+    ap.add_argument("--batch", type=int, default=None, help="long_decode only: sequences (default 16)")
+    ap.add_argument("--layers", type=int, default=None, help="long_decode only: layer caches (default 12)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--cpu-budget", type=float, default=15.0)
+    ap.add_argument("--cpu-budget", type=float, default=10.0)
     args = ap.parse_args()
     if args.warmup < 3 and args.impl == "uocr":
         print("note: fewer than 3 warm-up steps", file=sys.stderr)
