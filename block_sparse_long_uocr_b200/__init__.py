@@ -2,9 +2,10 @@
 
 Argument marshalling only: every step of the computation runs in the CUDA
 kernels behind the C ABI declared in ``include/uocr.h``.  PyTorch provides the
-device memory and the stream; there is no CPU fallback, and importing this
-package fails loudly when ``libuocr.so`` has not been built
-(``python -m block_sparse_long_uocr_b200.build``).
+device memory and the stream; there is no CPU fallback: the first call (or
+any access to ``lib``) raises ``ImportError`` when ``libuocr.so`` has not been
+built (``python -m block_sparse_long_uocr_b200.build``).  The library is loaded
+on first use so that the build module can be imported before it exists.
 
 Entry points (same names as the C ABI, without the ``uocr_`` prefix):
 
@@ -12,6 +13,8 @@ Entry points (same names as the C ABI, without the ``uocr_`` prefix):
 * :func:`block_topk`   -- 4 local + top-12 remote block selection;
 * :func:`sparse_attn`  -- exact 10-head attention over the selected 512 tokens;
 * :func:`sparse_decode` -- the three fused into one decode call;
+* :func:`sparse_decode_static` -- the same decode call for callers that cannot
+  allocate device memory (scratch held inside the library);
 * :func:`workspace_bytes`.
 """
 from __future__ import annotations
@@ -62,16 +65,31 @@ def _load() -> ctypes.CDLL:
     lib.uocr_sparse_attn.restype = I
     lib.uocr_sparse_decode.argtypes = [P, P, P, P, P, P, P, I, I, I, I, P, P, P, Z, P, P]
     lib.uocr_sparse_decode.restype = I
+    lib.uocr_sparse_decode_static.argtypes = [P, P, P, P, P, P, P, I, I, I, I, P, P, P, P]
+    lib.uocr_sparse_decode_static.restype = I
     return lib
 
 
-lib = _load()
+_LIB = None
+
+
+def _lib() -> ctypes.CDLL:
+    global _LIB
+    if _LIB is None:
+        _LIB = _load()
+    return _LIB
+
+
+def __getattr__(name):
+    if name == "lib":
+        return _lib()
+    raise AttributeError(name)
 
 
 # --------------------------------------------------------------------------- helpers
 def _check(fn: str, st: int):
     if st != 0:
-        raise UocrError(fn, st, lib.uocr_status_string(st).decode())
+        raise UocrError(fn, st, _lib().uocr_status_string(st).decode())
 
 
 def _ptr(t: torch.Tensor | None):
@@ -102,7 +120,7 @@ def _stream(stream) -> ctypes.c_void_p:
 
 
 def workspace_bytes(n_q: int, heads: int, max_blocks: int) -> int:
-    return int(lib.uocr_workspace_bytes(int(n_q), int(heads), int(max_blocks)))
+    return int(_lib().uocr_workspace_bytes(int(n_q), int(heads), int(max_blocks)))
 
 
 def alloc_workspace(n_q: int, heads: int, max_blocks: int, device) -> torch.Tensor:
@@ -122,7 +140,7 @@ def index_score(idx_q, idx_k_cache, block_table, seq_lens, q_seq=None, q_pos=Non
     if scores is None:
         scores = torch.full((n_q, mb), float("-inf"), dtype=torch.float32, device=idx_q.device)
     _dev(scores, "scores", torch.float32, 2)
-    _check("uocr_index_score", lib.uocr_index_score(
+    _check("uocr_index_score", _lib().uocr_index_score(
         _ptr(idx_q), _ptr(idx_k_cache), _ptr(block_table), _ptr(seq_lens), _ptr(_opt_i32(q_seq, "q_seq")),
         _ptr(_opt_i32(q_pos, "q_pos")), n_q, B, mb, idx_k_cache.shape[0], _ptr(scores),
         _ptr(dev_err), _stream(stream)))
@@ -137,7 +155,7 @@ def block_topk(scores, seq_lens, q_seq=None, q_pos=None, *, sel=None, dev_err=No
     if sel is None:
         sel = torch.empty((n_q, N_SEL), dtype=torch.int32, device=scores.device)
     _dev(sel, "sel", torch.int32, 2)
-    _check("uocr_block_topk", lib.uocr_block_topk(
+    _check("uocr_block_topk", _lib().uocr_block_topk(
         _ptr(scores), _ptr(seq_lens), _ptr(_opt_i32(q_seq, "q_seq")), _ptr(_opt_i32(q_pos, "q_pos")),
         n_q, seq_lens.shape[0], mb, _ptr(sel), _ptr(dev_err), _stream(stream)))
     return sel
@@ -159,7 +177,7 @@ def sparse_attn(q, k_cache, v_cache, block_table, seq_lens, sel, q_seq=None, q_p
     if workspace is None:
         workspace = alloc_workspace(n_q, H, mb, q.device)
     sc = float(scale) if scale is not None else HEAD_DIM ** -0.5
-    _check("uocr_sparse_attn", lib.uocr_sparse_attn(
+    _check("uocr_sparse_attn", _lib().uocr_sparse_attn(
         _ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(block_table), _ptr(seq_lens),
         _ptr(_opt_i32(q_seq, "q_seq")), _ptr(_opt_i32(q_pos, "q_pos")), _ptr(sel), n_q, B, H, mb,
         k_cache.shape[0], ctypes.c_float(sc), _ptr(out), _ptr(workspace), workspace.numel(),
@@ -185,8 +203,36 @@ def sparse_decode(q, k_cache, v_cache, idx_q, idx_k_cache, block_table, seq_lens
         sel = torch.empty((B, N_SEL), dtype=torch.int32, device=q.device)
     if workspace is None:
         workspace = alloc_workspace(B, H, mb, q.device)
-    _check("uocr_sparse_decode", lib.uocr_sparse_decode(
+    _check("uocr_sparse_decode", _lib().uocr_sparse_decode(
         _ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(idx_q), _ptr(idx_k_cache), _ptr(block_table),
         _ptr(seq_lens), B, H, mb, k_cache.shape[0], _ptr(out), _ptr(sel), _ptr(workspace),
         workspace.numel(), _ptr(dev_err), _stream(stream)))
+    return out, sel
+
+
+STATIC_SCRATCH_BYTES = 8 << 20   # UOCR_STATIC_SCRATCH_BYTES
+
+
+def sparse_decode_static(q, k_cache, v_cache, idx_q, idx_k_cache, block_table, seq_lens, *,
+                         out, sel, dev_err=None, stream=None):
+    """Decode without a workspace, for callers that cannot allocate device memory.
+
+    The caller passes the outputs (`out` [B,H,128] bf16, `sel` [B,16] int32); the scratch
+    lives in one fixed-size device array inside libuocr.so, shared by every call on the
+    device (calls that overlap on the GPU race on it), so nothing is allocated here or in
+    the library.  Raises UocrError (UOCR_ERR_WORKSPACE) when the shapes need more scratch
+    than STATIC_SCRATCH_BYTES.  The first call on a device looks the array up; make it
+    before any stream capture.
+    """
+    for t, n, dt, nd in ((q, "q", torch.bfloat16, 3), (k_cache, "k_cache", torch.bfloat16, 4),
+                         (v_cache, "v_cache", torch.bfloat16, 4), (idx_q, "idx_q", torch.bfloat16, 2),
+                         (idx_k_cache, "idx_k_cache", torch.bfloat16, 3), (block_table, "block_table", torch.int32, 2),
+                         (seq_lens, "seq_lens", torch.int32, 1), (out, "out", torch.bfloat16, 3),
+                         (sel, "sel", torch.int32, 2)):
+        _dev(t, n, dt, nd)
+    B, H = q.shape[0], q.shape[1]
+    _check("uocr_sparse_decode_static", _lib().uocr_sparse_decode_static(
+        _ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(idx_q), _ptr(idx_k_cache), _ptr(block_table),
+        _ptr(seq_lens), B, H, block_table.shape[1], k_cache.shape[0], _ptr(out), _ptr(sel),
+        _ptr(dev_err), _stream(stream)))
     return out, sel

@@ -28,7 +28,9 @@
  *
  * Conventions for every entry point:
  *   - All tensor pointers are DEVICE pointers owned by the caller; the library
- *     never allocates, frees or keeps device memory and holds no global state.
+ *     never allocates or frees device memory and, apart from the one fixed
+ *     scratch array of uocr_sparse_decode_static (see its declaration), keeps
+ *     no device memory and no global state.
  *   - bf16 tensors are passed as void* (IEEE bfloat16 bit patterns), must be
  *     16-byte aligned and densely packed in the layouts given below.
  *   - Every call is asynchronous on `stream` (NULL = the legacy default stream)
@@ -164,6 +166,37 @@ uocr_status_t uocr_sparse_decode(const void *q, const void *k_cache, const void 
                                  void *out, int32_t *sel_out,
                                  void *workspace, size_t workspace_bytes,
                                  int32_t *dev_err, uocr_stream_t stream);
+
+/*
+ * uocr_sparse_decode_static -- uocr_sparse_decode for callers that cannot
+ * allocate device memory (for example a plugin inside a host engine that owns
+ * every device allocation, or a decode loop where a cudaMalloc, which may
+ * synchronise the device, is not allowed).  The paper has no counterpart: this
+ * is a packaging variant, not a step of the method.
+ *
+ * Same arguments, layouts, checks and results as uocr_sparse_decode, without
+ * the workspace: the scratch lives in one device array of
+ * UOCR_STATIC_SCRATCH_BYTES inside the library, which every GPU that loads the
+ * library keeps until the process exits.  Nothing is allocated or freed.
+ *   - Returns UOCR_ERR_WORKSPACE, launching nothing, when
+ *     uocr_workspace_bytes(B, H, max_blocks) > UOCR_STATIC_SCRATCH_BYTES
+ *     (e.g. B = 64 sequences of 10 heads fit up to max_blocks = 27568).
+ *   - The first call on a device (with that device current) looks up the
+ *     array's device address and caches it; make that first call before any
+ *     stream capture on that device.
+ *   - All calls on a device share the array and it keeps the last call's
+ *     contents (no part of it needs to start at zero).  Calls whose kernels
+ *     overlap on the GPU -- several streams, or several host threads -- race
+ *     on it: serialise them.
+ */
+#define UOCR_STATIC_SCRATCH_BYTES (8u << 20)
+
+uocr_status_t uocr_sparse_decode_static(const void *q, const void *k_cache, const void *v_cache,
+                                        const void *idx_q, const void *idx_k_cache,
+                                        const int32_t *block_table, const int32_t *seq_lens,
+                                        int B, int H, int max_blocks, int num_pages,
+                                        void *out, int32_t *sel_out,
+                                        int32_t *dev_err, uocr_stream_t stream);
 
 #ifdef __cplusplus
 }
