@@ -36,7 +36,7 @@ IDX_DIM = 128
 
 STATUS = {0: "UOCR_OK", 1: "UOCR_ERR_INVALID_ARG", 2: "UOCR_ERR_UNSUPPORTED",
           3: "UOCR_ERR_WORKSPACE", 4: "UOCR_ERR_CUDA"}
-DEVERR_PAGE, DEVERR_POS, DEVERR_SEL = 1, 2, 4
+DEVERR_PAGE, DEVERR_POS, DEVERR_SEL, DEVERR_TIMEOUT = 1, 2, 4, 8
 
 
 class UocrError(RuntimeError):
@@ -61,7 +61,7 @@ def _load() -> ctypes.CDLL:
     lib.uocr_index_score.restype = I
     lib.uocr_block_topk.argtypes = [P, P, P, P, I, I, I, P, P, P]
     lib.uocr_block_topk.restype = I
-    lib.uocr_sparse_attn.argtypes = [P, P, P, P, P, P, P, P, I, I, I, I, I, F, P, P, Z, P, P]
+    lib.uocr_sparse_attn.argtypes = [P, P, P, P, P, P, P, P, I, I, I, I, I, F, P, P, P]
     lib.uocr_sparse_attn.restype = I
     lib.uocr_sparse_decode.argtypes = [P, P, P, P, P, P, P, I, I, I, I, P, P, P, Z, P, P]
     lib.uocr_sparse_decode.restype = I
@@ -162,7 +162,7 @@ def block_topk(scores, seq_lens, q_seq=None, q_pos=None, *, sel=None, dev_err=No
 
 
 def sparse_attn(q, k_cache, v_cache, block_table, seq_lens, sel, q_seq=None, q_pos=None, *,
-                scale: float | None = None, out=None, workspace=None, dev_err=None, stream=None) -> torch.Tensor:
+                scale: float | None = None, out=None, dev_err=None, stream=None) -> torch.Tensor:
     """bf16 [n_q, H, 128] attention output over the selected blocks."""
     _dev(q, "q", torch.bfloat16, 3)
     _dev(k_cache, "k_cache", torch.bfloat16, 4)
@@ -174,14 +174,11 @@ def sparse_attn(q, k_cache, v_cache, block_table, seq_lens, sel, q_seq=None, q_p
     B, mb = block_table.shape
     if out is None:
         out = torch.empty_like(q)
-    if workspace is None:
-        workspace = alloc_workspace(n_q, H, mb, q.device)
     sc = float(scale) if scale is not None else HEAD_DIM ** -0.5
     _check("uocr_sparse_attn", _lib().uocr_sparse_attn(
         _ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(block_table), _ptr(seq_lens),
         _ptr(_opt_i32(q_seq, "q_seq")), _ptr(_opt_i32(q_pos, "q_pos")), _ptr(sel), n_q, B, H, mb,
-        k_cache.shape[0], ctypes.c_float(sc), _ptr(out), _ptr(workspace), workspace.numel(),
-        _ptr(dev_err), _stream(stream)))
+        k_cache.shape[0], ctypes.c_float(sc), _ptr(out), _ptr(dev_err), _stream(stream)))
     return out
 
 

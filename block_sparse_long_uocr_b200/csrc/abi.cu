@@ -20,16 +20,15 @@ inline size_t round_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 inline bool aligned(const void *p, size_t a) { return ((uintptr_t)p % a) == 0; }
 
 struct WsLayout {
-    size_t scores_off, acc_off, ml_off, total;
+    size_t scores_off, total;
 };
 
-inline WsLayout ws_layout(int n_q, int H, int max_blocks) {
+// The workspace holds the block scores [n_q][max_blocks] f32 (the attention merges its
+// split-K partials on chip, so it needs none).
+inline WsLayout ws_layout(int n_q, int /*H*/, int max_blocks) {
     WsLayout w{};
-    const size_t splits = (size_t)uocr::attn_splits(n_q, H);
     w.scores_off = 0;
-    w.acc_off = round_up((size_t)n_q * max_blocks * sizeof(float), kWsAlign);
-    w.ml_off = w.acc_off + round_up((size_t)n_q * H * splits * uocr::kD * sizeof(float), kWsAlign);
-    w.total = w.ml_off + round_up((size_t)n_q * H * splits * 2 * sizeof(float), kWsAlign);
+    w.total = round_up((size_t)n_q * max_blocks * sizeof(float), kWsAlign);
     return w;
 }
 
@@ -81,7 +80,7 @@ const char *uocr_status_string(uocr_status_t status) {
     return "UOCR_ERR_UNKNOWN";
 }
 
-int uocr_abi_version(void) { return 1; }
+int uocr_abi_version(void) { return 2; }
 
 size_t uocr_workspace_bytes(int n_q, int H, int max_blocks) {
     if (n_q <= 0 || H <= 0 || max_blocks <= 0) return 0;
@@ -125,8 +124,7 @@ uocr_status_t uocr_sparse_attn(const void *q, const void *k_cache, const void *v
                                const int32_t *block_table, const int32_t *seq_lens,
                                const int32_t *q_seq, const int32_t *q_pos, const int32_t *sel,
                                int n_q, int B, int H, int max_blocks, int num_pages, float scale,
-                               void *out, void *workspace, size_t workspace_bytes,
-                               int32_t *dev_err, uocr_stream_t stream) {
+                               void *out, int32_t *dev_err, uocr_stream_t stream) {
     uocr_status_t st = check_common(n_q, B, max_blocks, num_pages, block_table, seq_lens, q_seq,
                                     q_pos, dev_err);
     if (st != UOCR_OK) return st;
@@ -135,15 +133,11 @@ uocr_status_t uocr_sparse_attn(const void *q, const void *k_cache, const void *v
     if (H < 1 || H > UOCR_MAX_HEADS) return UOCR_ERR_UNSUPPORTED;
     if (!isfinite(scale)) return UOCR_ERR_INVALID_ARG;
     if (n_q == 0) return UOCR_OK;
-    const WsLayout w = ws_layout(n_q, H, max_blocks);
-    if (!workspace || !aligned(workspace, kWsAlign) || workspace_bytes < w.total) return UOCR_ERR_WORKSPACE;
     uocr::LaunchCtx c;
     if ((st = make_ctx(stream, false, c)) != UOCR_OK) return st;
-    char *ws = (char *)workspace;
     return cuda_status(uocr::launch_sparse_attn(c, q, k_cache, v_cache, block_table, seq_lens, q_seq,
                                                 q_pos, sel, n_q, B, H, max_blocks, num_pages, scale,
-                                                out, (float *)(ws + w.acc_off),
-                                                (float *)(ws + w.ml_off), dev_err));
+                                                out, false, dev_err));
 }
 
 uocr_status_t uocr_sparse_decode(const void *q, const void *k_cache, const void *v_cache,
@@ -174,8 +168,7 @@ uocr_status_t uocr_sparse_decode(const void *q, const void *k_cache, const void 
     if (e != cudaSuccess) return cuda_status(e);
     const float scale = 1.0f / sqrtf((float)UOCR_HEAD_DIM);
     e = uocr::launch_sparse_attn(c, q, k_cache, v_cache, block_table, seq_lens, nullptr, nullptr, sel_out,
-                                 B, B, H, max_blocks, num_pages, scale, out, (float *)(ws + w.acc_off),
-                                 (float *)(ws + w.ml_off), dev_err);
+                                 B, B, H, max_blocks, num_pages, scale, out, true, dev_err);
     return cuda_status(e);
 }
 

@@ -5,11 +5,22 @@
 // window) and the 12 remote blocks with the highest indexer score; inference
 // uses a hard top-k.  Ranking: score descending, then lower block id.
 //
-// One CTA per query.  The 12th-largest score is found exactly by a 4-pass,
-// 8-bit radix select on order-preserving fp32 keys (shared-memory histograms),
-// then one ordered pass over contiguous per-thread id ranges emits the chosen
-// remote ids in ascending order, taking the lowest ids among keys equal to the
-// threshold.  Cost is ~5 reads of the candidate scores from L2 per query.
+// One CTA of 512 threads per query; every candidate's ranking key is the
+// 64-bit composite (order-preserving fp32 key << 32 | ~id): distinct, larger
+// for a higher score and, among equal scores, for the lower id.
+//   1. The candidates' scores are read once from L2 (the scan just wrote them)
+//      into shared memory as order-preserving keys.
+//   2. Threshold: the 12th largest of the 16 warp maxima.  Those 12 maxima are
+//      12 distinct candidates at or above it, so every member of the top 12 is
+//      at or above it too.
+//   3. Survivors (keys >= threshold; typically a few dozen) are appended to a
+//      shared list; each survivor's rank is the number of survivors with a
+//      larger composite, and ranks 0..11 are the answer.
+//   4. One warp writes the 12 ids in ascending order plus the 4 local blocks.
+// If the survivors overflow their list (heavily tied scores) the CTA falls
+// back to an exact two-level extraction: every warp takes its top 12 by 12
+// rounds of a warp-wide max, then one warp takes the top 12 of those.
+// Rows longer than the shared-memory budget are read from L2 instead of staged.
 #include <math.h>
 
 #include "common.cuh"
@@ -17,51 +28,105 @@
 
 namespace uocr {
 
-constexpr int kTopkThreads = 256;
+constexpr int kTopkThreads = 512;
+constexpr int kTopkWarps = kTopkThreads / 32;
+constexpr int kTopkSmemKeys = 48 * 1024;    // stage rows up to 48K candidates (192 KiB of keys)
+constexpr int kSurvivorCap = 2048;          // survivor list capacity (16 KiB)
 
-// Larger key <=> larger float (total order on non-NaN values, -0 < +0).
+// Larger key <=> larger float; -0 and +0 map to the same key (they compare equal).
 __device__ __forceinline__ uint32_t order_key(float f) {
-    const uint32_t u = __float_as_uint(f);
+    const uint32_t u = (f == 0.0f) ? 0u : __float_as_uint(f);
     return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
 }
 
-// Exclusive prefix sum over the CTA; also returns the total through *total.
-__device__ __forceinline__ int cta_exclusive_scan(int x, int *warp_buf, int *total) {
-    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-    int incl = x;
+__device__ __forceinline__ uint64_t composite(uint32_t key, int j) {
+    return ((uint64_t)key << 32) | (uint32_t)(~(uint32_t)j);
+}
+
+__device__ __forceinline__ uint64_t warp_max_u64(uint64_t v) {
 #pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-        const int n = __shfl_up_sync(0xffffffffu, incl, o);
-        if (lane >= o) incl += n;
+    for (int o = 16; o > 0; o >>= 1) {
+        const uint64_t w = __shfl_xor_sync(0xffffffffu, v, o);
+        v = w > v ? w : v;
     }
-    if (lane == 31) warp_buf[warp] = incl;
+    return v;
+}
+
+// Keys of one query's candidates: staged in shared memory, or read from the scores row.
+struct KeySource {
+    const uint32_t *smem;
+    const float *row;
+    __device__ __forceinline__ uint32_t operator()(int j) const {
+        return smem ? smem[j] : order_key(__ldcg(row + j));
+    }
+};
+
+// Largest composite strictly below `cap` among candidates j = first, first + stride, ... < n
+// (0 when there is none; a real composite is never 0 because ~j != 0 for j < 2^31 - 1).
+__device__ __forceinline__ uint64_t best_below(const KeySource &key, int first, int stride, int n,
+                                               uint64_t cap) {
+    uint64_t best = 0;
+    for (int j = first; j < n; j += stride) {
+        const uint64_t c = composite(key(j), j);
+        if (c < cap && c > best) best = c;
+    }
+    return best;
+}
+
+// Exact fallback: the top kRemote composites of candidates [0, nc) into out_c[0..11].
+// Called by every thread of the CTA.
+__device__ void topk_two_level(const KeySource &key, int nc, uint64_t *s_cand, uint64_t *out_c) {
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    uint64_t cap = ~0ull;
+    uint64_t mine = best_below(key, tid, kTopkThreads, nc, cap);
+#pragma unroll 1
+    for (int k = 0; k < kRemote; ++k) {
+        const uint64_t w = warp_max_u64(mine);
+        if (lane == 0) s_cand[warp * kRemote + k] = w;   // 0 when the warp ran out of candidates
+        if (mine == w && w != 0) {
+            cap = mine;
+            mine = best_below(key, tid, kTopkThreads, nc, cap);
+        }
+    }
     __syncthreads();
     if (warp == 0) {
-        int w = lane < kTopkThreads / 32 ? warp_buf[lane] : 0;
-        int wi = w;
+        constexpr int kPer = kTopkWarps * kRemote / 32;   // survivors per lane
+        uint64_t c[kPer];
 #pragma unroll
-        for (int o = 1; o < 32; o <<= 1) {
-            const int n = __shfl_up_sync(0xffffffffu, wi, o);
-            if (lane >= o) wi += n;
+        for (int e = 0; e < kPer; ++e) c[e] = s_cand[lane * kPer + e];
+#pragma unroll 1
+        for (int k = 0; k < kRemote; ++k) {
+            uint64_t best = 0;
+            int at = -1;
+#pragma unroll
+            for (int e = 0; e < kPer; ++e)
+                if (c[e] > best) {
+                    best = c[e];
+                    at = e;
+                }
+            const uint64_t w = warp_max_u64(best);
+            if (best == w && at >= 0) {
+#pragma unroll
+                for (int e = 0; e < kPer; ++e)
+                    if (e == at) c[e] = 0;
+            }
+            if (lane == 0) out_c[k] = w;
         }
-        if (lane < kTopkThreads / 32) warp_buf[lane] = wi - w;
-        if (lane == kTopkThreads / 32 - 1) warp_buf[kTopkThreads / 32] = wi;
     }
     __syncthreads();
-    const int res = warp_buf[warp] + incl - x;
-    *total = warp_buf[kTopkThreads / 32];
-    __syncthreads();
-    return res;
 }
 
 __global__ void __launch_bounds__(kTopkThreads)
 block_topk_kernel(const float *__restrict__ scores, const int32_t *__restrict__ seq_lens,
                   const int32_t *__restrict__ q_seq, const int32_t *__restrict__ q_pos, int B,
-                  int max_blocks, int32_t *__restrict__ sel, int32_t *dev_err) {
-    __shared__ int hist[256];
-    __shared__ int warp_buf[kTopkThreads / 32 + 1];
-    __shared__ uint32_t s_prefix;
-    __shared__ int s_need;
+                  int max_blocks, int32_t *__restrict__ sel, int32_t *dev_err, int staged) {
+    extern __shared__ uint32_t s_keys[];
+    __shared__ uint64_t s_surv[kSurvivorCap];
+    __shared__ uint64_t s_cand[kTopkWarps * kRemote];
+    __shared__ uint64_t s_top[kRemote];
+    __shared__ uint32_t s_wmax[kTopkWarps];
+    __shared__ uint32_t s_thr;
+    __shared__ int s_n;
 
     const int i = blockIdx.x;
     const int tid = threadIdx.x;
@@ -69,6 +134,9 @@ block_topk_kernel(const float *__restrict__ scores, const int32_t *__restrict__ 
     int32_t *out = sel + (size_t)i * kSel;
 
     pdl_wait();
+    // the attention kernel of a decode call may start its prologue while this runs
+    pdl_launch_dependents();
+
     QueryRef r;
     if (!resolve_query(i, seq_lens, q_seq, q_pos, B, max_blocks, dev_err, tid == 0, r)) {
         if (tid < kSel) out[tid] = -1;
@@ -81,99 +149,105 @@ block_topk_kernel(const float *__restrict__ scores, const int32_t *__restrict__ 
         if (tid < kSel) out[tid] = tid < nb ? tid : -1;
         return;
     }
-    const float *s = scores + (size_t)i * max_blocks;
+    const float *row = scores + (size_t)i * max_blocks;
+    KeySource key{nullptr, row};
+    if (tid == 0) s_n = 0;
 
-    // ---- radix select of the kRemote-th largest key
-    uint32_t prefix = 0, mask = 0;
-    int need = kRemote;
-#pragma unroll 1
-    for (int shift = 24; shift >= 0; shift -= 8) {
-        for (int b = tid; b < 256; b += kTopkThreads) hist[b] = 0;
-        __syncthreads();
+    // ---- 1. stage keys, 2. per-thread then per-warp maximum
+    uint32_t tmax = 0;
+    if (staged) {
+#pragma unroll 8
         for (int j = tid; j < nc; j += kTopkThreads) {
-            const uint32_t key = order_key(s[j]);
-            if ((key & mask) == prefix) atomicAdd(&hist[(key >> shift) & 255u], 1);
+            const uint32_t k = order_key(__ldcg(row + j));
+            s_keys[j] = k;
+            tmax = k > tmax ? k : tmax;
         }
-        __syncthreads();
-        if (warp == 0) {
-            // lane L owns bins 255-8L .. 248-8L (descending); find the bin holding rank `need`
-            int c[8], tot = 0;
-#pragma unroll
-            for (int k = 0; k < 8; ++k) {
-                c[k] = hist[255 - 8 * lane - k];
-                tot += c[k];
-            }
-            int incl = tot;
-#pragma unroll
-            for (int o = 1; o < 32; o <<= 1) {
-                const int n = __shfl_up_sync(0xffffffffu, incl, o);
-                if (lane >= o) incl += n;
-            }
-            const int excl = incl - tot;
-            const unsigned owner = __ballot_sync(0xffffffffu, excl < need && need <= incl);
-            if (lane == __ffs(owner) - 1) {
-                int run = excl;
-#pragma unroll
-                for (int k = 0; k < 8; ++k) {
-                    if (run + c[k] >= need) {
-                        s_prefix = prefix | ((uint32_t)(255 - 8 * lane - k) << shift);
-                        s_need = need - run;
-                        break;
-                    }
-                    run += c[k];
-                }
-            }
+        key.smem = s_keys;
+    } else {
+        for (int j = tid; j < nc; j += kTopkThreads) {
+            const uint32_t k = key(j);
+            tmax = k > tmax ? k : tmax;
         }
-        __syncthreads();
-        prefix = s_prefix;
-        need = s_need;
-        mask |= 255u << shift;
-        __syncthreads();
     }
-    const uint32_t thr = prefix;   // key of the kRemote-th ranked candidate
-    // `need` = how many candidates equal to thr are taken (the lowest ids among them)
+    const uint32_t wmax = __reduce_max_sync(0xffffffffu, tmax);
+    if (lane == 0) s_wmax[warp] = wmax;
+    __syncthreads();
 
-    // ---- ordered emission over contiguous id ranges
-    const int per = (nc + kTopkThreads - 1) / kTopkThreads;
-    const int lo = tid * per;
-    const int hi = lo + per < nc ? lo + per : nc;
-    int n_eq = 0;
-    for (int j = lo; j < hi; ++j) n_eq += order_key(s[j]) == thr;
-    int total;
-    const int eq_base = cta_exclusive_scan(n_eq, warp_buf, &total);
-    int n_take = 0;
-    {
-        int seen = eq_base;
-        for (int j = lo; j < hi; ++j) {
-            const uint32_t key = order_key(s[j]);
-            const bool eq = key == thr;
-            n_take += (key > thr) || (eq && seen < need);
-            seen += eq;
+    // ---- threshold = the kRemote-th largest warp maximum (with multiplicity)
+    if (warp == 0) {
+        const uint32_t v = lane < kTopkWarps ? s_wmax[lane] : 0u;
+        int gt = 0, ge = 0;
+#pragma unroll
+        for (int w = 0; w < kTopkWarps; ++w) {
+            const uint32_t o = s_wmax[w];
+            gt += o > v;
+            ge += o >= v;
+        }
+        const bool is_thr = lane < kTopkWarps && gt <= kRemote - 1 && kRemote - 1 < ge;
+        const unsigned who = __ballot_sync(0xffffffffu, is_thr);
+        if (lane == __ffs(who) - 1) s_thr = v;
+    }
+    __syncthreads();
+    const uint32_t thr = s_thr;
+
+    // ---- 3. survivors: every candidate at or above the threshold
+    for (int j0 = 0; j0 < nc; j0 += kTopkThreads) {
+        const int j = j0 + tid;
+        const uint32_t k = j < nc ? key(j) : 0u;
+        const bool keep = j < nc && k >= thr;
+        const unsigned m = __ballot_sync(0xffffffffu, keep);
+        if (m) {
+            const int leader = __ffs(m) - 1;
+            int base = 0;
+            if (lane == leader) base = atomicAdd(&s_n, __popc(m));
+            base = __shfl_sync(0xffffffffu, base, leader);
+            const int slot = base + __popc(m & ((1u << lane) - 1u));
+            if (keep && slot < kSurvivorCap) s_surv[slot] = composite(k, j);
         }
     }
-    const int pos0 = cta_exclusive_scan(n_take, warp_buf, &total);
-    {
-        int seen = eq_base, pos = pos0;
-        for (int j = lo; j < hi; ++j) {
-            const uint32_t key = order_key(s[j]);
-            const bool eq = key == thr;
-            if ((key > thr) || (eq && seen < need)) {
-                if (pos < kRemote) out[pos] = j;
-                ++pos;
-            }
-            seen += eq;
+    __syncthreads();
+    const int n = s_n;
+    if (n <= kSurvivorCap) {
+        for (int a = tid; a < n; a += kTopkThreads) {
+            const uint64_t c = s_surv[a];
+            int rank = 0;
+            for (int b = 0; b < n; ++b) rank += s_surv[b] > c;
+            if (rank < kRemote) s_top[rank] = c;
         }
+        __syncthreads();
+    } else {
+        topk_two_level(key, nc, s_cand, s_top);
     }
-    if (tid < kLocal) out[kRemote + tid] = nb - kLocal + tid;
-    pdl_launch_dependents();
+
+    // ---- 4. the 12 remote ids ascending, then the 4 local blocks
+    if (warp == 0) {
+        const int id = lane < kRemote ? (int)~(uint32_t)(s_top[lane] & 0xffffffffu) : 0x7fffffff;
+        int rank = 0;
+#pragma unroll
+        for (int k = 0; k < kRemote; ++k) {
+            const int other = __shfl_sync(0xffffffffu, id, k);
+            rank += other < id;
+        }
+        if (lane < kRemote) out[rank] = id;
+        if (lane < kLocal) out[kRemote + lane] = nb - kLocal + lane;
+    }
 }
 
 cudaError_t launch_block_topk(const LaunchCtx &c, const float *scores, const int32_t *seq_lens,
                               const int32_t *q_seq, const int32_t *q_pos, int n_q, int B,
                               int max_blocks, int32_t *sel, int32_t *dev_err) {
+    const int staged = max_blocks <= kTopkSmemKeys;
+    const size_t smem = staged ? (size_t)max_blocks * sizeof(uint32_t) : 0;
+    if (smem > 16 * 1024) {
+        // the static shared memory (~19 KiB) plus the staged keys may pass the 48 KiB default
+        cudaError_t e = cudaFuncSetAttribute(block_topk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                             (int)smem);
+        if (e != cudaSuccess) return e;
+    }
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3((unsigned)n_q);
     cfg.blockDim = dim3(kTopkThreads);
+    cfg.dynamicSmemBytes = smem;
     cfg.stream = c.stream;
     cudaLaunchAttribute attr[1];
     attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
@@ -181,7 +255,7 @@ cudaError_t launch_block_topk(const LaunchCtx &c, const float *scores, const int
     cfg.attrs = attr;
     cfg.numAttrs = c.pdl ? 1 : 0;
     return cudaLaunchKernelEx(&cfg, block_topk_kernel, scores, seq_lens, q_seq, q_pos, B, max_blocks,
-                              sel, dev_err);
+                              sel, dev_err, staged);
 }
 
 }  // namespace uocr

@@ -13,7 +13,7 @@ struct LaunchCtx {
     bool pdl;   // launch with programmatic stream serialization
 };
 
-// Number of split-K partitions the attention uses for n_q queries of H heads.
+// CTAs (split-K partitions, one thread-block cluster) per (query, head) in the attention.
 int attn_splits(int n_q, int H);
 
 cudaError_t launch_index_scan(const LaunchCtx &c, const void *idx_q, const void *idx_k,
@@ -29,6 +29,6 @@ cudaError_t launch_sparse_attn(const LaunchCtx &c, const void *q, const void *k,
                                const int32_t *bt, const int32_t *seq_lens, const int32_t *q_seq,
                                const int32_t *q_pos, const int32_t *sel, int n_q, int B, int H,
                                int max_blocks, int num_pages, float scale, void *out,
-                               float *part_acc, float *part_ml, int32_t *dev_err);
+                               bool implicit_local, int32_t *dev_err);
 
 }  // namespace uocr

@@ -93,6 +93,7 @@ typedef enum {
 #define UOCR_DEVERR_PAGE 1u   /* block-table entry outside [0, num_pages) */
 #define UOCR_DEVERR_POS 2u    /* q_pos >= seq_len, q_seq outside [0, B), or nb > max_blocks */
 #define UOCR_DEVERR_SEL 4u    /* a selected block outside the query's causal blocks */
+#define UOCR_DEVERR_TIMEOUT 8u /* a bounded wait on an asynchronous copy gave up (block skipped) */
 
 /* Human-readable name of a status code (static storage; never NULL). */
 const char *uocr_status_string(uocr_status_t status);
@@ -101,11 +102,11 @@ const char *uocr_status_string(uocr_status_t status);
 int uocr_abi_version(void);
 
 /*
- * Workspace bytes that uocr_sparse_attn, uocr_sparse_decode and
- * uocr_sparse_prefill need for n_q queries of H heads over max_blocks blocks.
- * A pure function of the shapes (0 for a non-positive argument).  The
- * workspace holds the fp32 block scores [n_q][max_blocks] and the split-K
- * partial softmax states; callers may reuse it across calls on one stream.
+ * Workspace bytes that uocr_sparse_decode needs for B = n_q queries over
+ * max_blocks blocks: the fp32 block scores [n_q][max_blocks], rounded up to
+ * 256 bytes.  A pure function of the shapes (0 for a non-positive argument);
+ * H is accepted for symmetry with the other entry points and does not change
+ * the result.  Callers may reuse one workspace across calls on one stream.
  */
 size_t uocr_workspace_bytes(int n_q, int H, int max_blocks);
 
@@ -140,8 +141,8 @@ uocr_status_t uocr_block_topk(const float *scores, const int32_t *seq_lens,
  *   z_t = scale * q[i][h] . k[h][t]  over the tokens t <= p_i of the blocks in sel[i],
  *   out[i][h] = sum_t softmax(z)_t v[h][t]    (fp32 softmax and accumulation, bf16 out).
  * Entries of sel < 0 are skipped; a query with no visible token gets zeros.
- * Split-K over the 16 blocks with a flash-decoding combine through the
- * workspace (uocr_workspace_bytes(n_q, H, max_blocks) bytes, 256-byte aligned).
+ * Split-K over the 16 blocks (one thread-block cluster of 4 CTAs per query
+ * and head) with the flash-decoding merge done on chip: no workspace.
  * H in [1, UOCR_MAX_HEADS] (the model uses 10); head dim fixed at 128.
  */
 uocr_status_t uocr_sparse_attn(const void *q, const void *k_cache, const void *v_cache,
@@ -149,7 +150,6 @@ uocr_status_t uocr_sparse_attn(const void *q, const void *k_cache, const void *v
                                const int32_t *q_seq, const int32_t *q_pos,
                                const int32_t *sel, int n_q, int B, int H,
                                int max_blocks, int num_pages, float scale, void *out,
-                               void *workspace, size_t workspace_bytes,
                                int32_t *dev_err, uocr_stream_t stream);
 
 /*
@@ -180,7 +180,7 @@ uocr_status_t uocr_sparse_decode(const void *q, const void *k_cache, const void 
  * library keeps until the process exits.  Nothing is allocated or freed.
  *   - Returns UOCR_ERR_WORKSPACE, launching nothing, when
  *     uocr_workspace_bytes(B, H, max_blocks) > UOCR_STATIC_SCRATCH_BYTES
- *     (e.g. B = 64 sequences of 10 heads fit up to max_blocks = 27568).
+ *     (e.g. B = 64 sequences fit up to max_blocks = 32768, 1M tokens each).
  *   - The first call on a device (with that device current) looks up the
  *     array's device address and caches it; make that first call before any
  *     stream capture on that device.

@@ -53,7 +53,7 @@ def test_status_strings_and_version(pkg):
         s = pkg.lib.uocr_status_string(code).decode()
         assert s.startswith(pkg.STATUS[code])
     assert pkg.lib.uocr_status_string(99).decode() == "UOCR_ERR_UNKNOWN"
-    assert pkg.lib.uocr_abi_version() == 1
+    assert pkg.lib.uocr_abi_version() == 2
 
 
 def test_workspace_is_a_pure_function_of_shapes(pkg):
@@ -61,9 +61,10 @@ def test_workspace_is_a_pure_function_of_shapes(pkg):
     assert ws(0, 10, 64) == 0 and ws(4, 0, 64) == 0 and ws(4, 10, 0) == 0
     a = ws(16, 10, 4096)
     assert a == ws(16, 10, 4096) and a % 256 == 0
-    assert a >= 16 * 4096 * 4                       # block-score scratch
+    assert a == 16 * 4096 * 4                       # the block-score scratch, nothing else
     assert ws(32, 10, 4096) > a and ws(16, 10, 8192) > a
-    # independent of data: same answer regardless of sequence lengths (none are passed)
+    assert ws(16, 1, 4096) == a                     # heads do not change it (attention merges on chip)
+    assert ws(3, 10, 5) == 256                      # rounded up to 256 bytes
 
 
 # --------------------------------------------------------------------------- host fault injection
@@ -122,27 +123,28 @@ def test_block_topk_rejects(pkg, args):
 
 def _call_attn(lib, **over):
     a = dict(q=FAKE, k=FAKE, v=FAKE, bt=FAKE, sl=FAKE, sel=FAKE, n_q=4, B=4, H=10, mb=64, P=256,
-             scale=0.088, out=FAKE, ws=FAKE, wsb=1 << 30)
+             scale=0.088, out=FAKE)
     a.update(over)
     return lib.uocr_sparse_attn(a["q"], a["k"], a["v"], a["bt"], a["sl"], None, None, a["sel"], a["n_q"],
-                                a["B"], a["H"], a["mb"], a["P"], ctypes.c_float(a["scale"]), a["out"], a["ws"],
-                                a["wsb"], None, None)
+                                a["B"], a["H"], a["mb"], a["P"], ctypes.c_float(a["scale"]), a["out"], None, None)
 
 
 @no_gpu
 @pytest.mark.parametrize("over,code", [
     (dict(q=None), 1), (dict(k=MIS), 1), (dict(v=None), 1), (dict(out=FAKE + 4), 1), (dict(sel=None), 1),
     (dict(H=0), 2), (dict(H=65), 2), (dict(scale=float("nan")), 1), (dict(scale=float("inf")), 1),
-    (dict(ws=None), 3), (dict(ws=FAKE + 16), 3), (dict(wsb=1024), 3),
+    (dict(sel=MIS), 1), (dict(bt=None), 1), (dict(P=0), 1),
 ])
 def test_sparse_attn_rejects(pkg, over, code):
     assert _call_attn(pkg.lib, **over) == code
 
 
 @no_gpu
-def test_sparse_attn_workspace_boundary(pkg):
+def test_sparse_decode_workspace_boundary(pkg):
     need = pkg.workspace_bytes(4, 10, 64)
-    assert _call_attn(pkg.lib, wsb=need - 1) == 3
+    a = [FAKE] * 7 + [4, 10, 64, 256, FAKE, FAKE, FAKE]
+    assert pkg.lib.uocr_sparse_decode(*a, need - 1, None, None) == 3
+    assert pkg.lib.uocr_sparse_decode(*a[:13], FAKE + 128, need, None, None) == 3   # misaligned workspace
 
 
 @no_gpu
