@@ -13,6 +13,8 @@ Entry points (same names as the C ABI, without the ``uocr_`` prefix):
 * :func:`block_topk`   -- 4 local + top-12 remote block selection;
 * :func:`sparse_attn`  -- exact 10-head attention over the selected 512 tokens;
 * :func:`sparse_decode` -- the three fused into one decode call;
+* :func:`prefill_index_score` -- the block scores of a prefill chunk on the tcgen05 tensor cores;
+* :func:`sparse_prefill` -- tensor-core scoring, selection and attention for a prefill chunk;
 * :func:`sparse_decode_static` -- the same decode call for callers that cannot
   allocate device memory (scratch held inside the library);
 * :func:`workspace_bytes`.
@@ -65,6 +67,10 @@ def _load() -> ctypes.CDLL:
     lib.uocr_sparse_attn.restype = I
     lib.uocr_sparse_decode.argtypes = [P, P, P, P, P, P, P, I, I, I, I, P, P, P, Z, P, P]
     lib.uocr_sparse_decode.restype = I
+    lib.uocr_prefill_index_score.argtypes = [P, P, P, P, I, P, I, I, I, I, P, P, P]
+    lib.uocr_prefill_index_score.restype = I
+    lib.uocr_sparse_prefill.argtypes = [P, P, P, P, P, P, P, I, P, I, I, I, I, I, P, P, P, Z, P, P]
+    lib.uocr_sparse_prefill.restype = I
     lib.uocr_sparse_decode_static.argtypes = [P, P, P, P, P, P, P, I, I, I, I, P, P, P, P]
     lib.uocr_sparse_decode_static.restype = I
     return lib
@@ -203,6 +209,47 @@ def sparse_decode(q, k_cache, v_cache, idx_q, idx_k_cache, block_table, seq_lens
     _check("uocr_sparse_decode", _lib().uocr_sparse_decode(
         _ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(idx_q), _ptr(idx_k_cache), _ptr(block_table),
         _ptr(seq_lens), B, H, mb, k_cache.shape[0], _ptr(out), _ptr(sel), _ptr(workspace),
+        workspace.numel(), _ptr(dev_err), _stream(stream)))
+    return out, sel
+
+
+def prefill_index_score(idx_q, idx_k_cache, block_table, seq_lens, seq: int, q_pos, *,
+                        scores=None, dev_err=None, stream=None) -> torch.Tensor:
+    """fp32 [n_q, max_blocks] block scores of n_q queries of sequence `seq` (tcgen05 GEMM)."""
+    _dev(idx_q, "idx_q", torch.bfloat16, 2)
+    _dev(idx_k_cache, "idx_k_cache", torch.bfloat16, 3)
+    _dev(block_table, "block_table", torch.int32, 2)
+    _dev(seq_lens, "seq_lens", torch.int32, 1)
+    _dev(q_pos, "q_pos", torch.int32, 1)
+    n_q, B, mb = idx_q.shape[0], block_table.shape[0], block_table.shape[1]
+    if scores is None:
+        scores = torch.full((n_q, mb), float("-inf"), dtype=torch.float32, device=idx_q.device)
+    _dev(scores, "scores", torch.float32, 2)
+    _check("uocr_prefill_index_score", _lib().uocr_prefill_index_score(
+        _ptr(idx_q), _ptr(idx_k_cache), _ptr(block_table), _ptr(seq_lens), int(seq), _ptr(q_pos), n_q, B, mb,
+        idx_k_cache.shape[0], _ptr(scores), _ptr(dev_err), _stream(stream)))
+    return scores
+
+
+def sparse_prefill(q, k_cache, v_cache, idx_q, idx_k_cache, block_table, seq_lens, seq: int, q_pos, *,
+                   out=None, sel=None, workspace=None, dev_err=None, stream=None):
+    """Prefill chunk of sequence `seq`.  Returns (out [n_q,H,128] bf16, sel [n_q,16] int32)."""
+    for t, n, dt, nd in ((q, "q", torch.bfloat16, 3), (k_cache, "k_cache", torch.bfloat16, 4),
+                         (v_cache, "v_cache", torch.bfloat16, 4), (idx_q, "idx_q", torch.bfloat16, 2),
+                         (idx_k_cache, "idx_k_cache", torch.bfloat16, 3), (block_table, "block_table", torch.int32, 2),
+                         (seq_lens, "seq_lens", torch.int32, 1), (q_pos, "q_pos", torch.int32, 1)):
+        _dev(t, n, dt, nd)
+    n_q, H = q.shape[0], q.shape[1]
+    B, mb = block_table.shape
+    if out is None:
+        out = torch.empty_like(q)
+    if sel is None:
+        sel = torch.empty((n_q, N_SEL), dtype=torch.int32, device=q.device)
+    if workspace is None:
+        workspace = alloc_workspace(n_q, H, mb, q.device)
+    _check("uocr_sparse_prefill", _lib().uocr_sparse_prefill(
+        _ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(idx_q), _ptr(idx_k_cache), _ptr(block_table), _ptr(seq_lens),
+        int(seq), _ptr(q_pos), n_q, B, H, mb, k_cache.shape[0], _ptr(out), _ptr(sel), _ptr(workspace),
         workspace.numel(), _ptr(dev_err), _stream(stream)))
     return out, sel
 

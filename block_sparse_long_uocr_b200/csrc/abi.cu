@@ -137,7 +137,7 @@ uocr_status_t uocr_sparse_attn(const void *q, const void *k_cache, const void *v
     if ((st = make_ctx(stream, false, c)) != UOCR_OK) return st;
     return cuda_status(uocr::launch_sparse_attn(c, q, k_cache, v_cache, block_table, seq_lens, q_seq,
                                                 q_pos, sel, n_q, B, H, max_blocks, num_pages, scale,
-                                                out, false, dev_err));
+                                                out, false, -1, false, dev_err));
 }
 
 uocr_status_t uocr_sparse_decode(const void *q, const void *k_cache, const void *v_cache,
@@ -168,7 +168,56 @@ uocr_status_t uocr_sparse_decode(const void *q, const void *k_cache, const void 
     if (e != cudaSuccess) return cuda_status(e);
     const float scale = 1.0f / sqrtf((float)UOCR_HEAD_DIM);
     e = uocr::launch_sparse_attn(c, q, k_cache, v_cache, block_table, seq_lens, nullptr, nullptr, sel_out,
-                                 B, B, H, max_blocks, num_pages, scale, out, true, dev_err);
+                                 B, B, H, max_blocks, num_pages, scale, out, true, -1, false, dev_err);
+    return cuda_status(e);
+}
+
+uocr_status_t uocr_prefill_index_score(const void *idx_q, const void *idx_k_cache, const int32_t *block_table,
+                                       const int32_t *seq_lens, int seq, const int32_t *q_pos, int n_q, int B,
+                                       int max_blocks, int num_pages, float *scores, int32_t *dev_err,
+                                       uocr_stream_t stream) {
+    uocr_status_t st = check_common(n_q, B, max_blocks, num_pages, block_table, seq_lens, nullptr, q_pos, dev_err);
+    if (st != UOCR_OK) return st;
+    if (!bf16_ok(idx_q) || !bf16_ok(idx_k_cache) || !q_pos || !scores || !aligned(scores, 4))
+        return UOCR_ERR_INVALID_ARG;
+    if (seq < 0 || seq >= B) return UOCR_ERR_INVALID_ARG;
+    if (n_q == 0) return UOCR_OK;
+    uocr::LaunchCtx c;
+    if ((st = make_ctx(stream, false, c)) != UOCR_OK) return st;
+    return cuda_status(uocr::launch_prefill_index_gemm(c, idx_q, idx_k_cache, block_table + (size_t)seq * max_blocks,
+                                                       seq_lens + seq, q_pos, n_q, max_blocks, num_pages, scores,
+                                                       dev_err));
+}
+
+uocr_status_t uocr_sparse_prefill(const void *q, const void *k_cache, const void *v_cache, const void *idx_q,
+                                  const void *idx_k_cache, const int32_t *block_table, const int32_t *seq_lens,
+                                  int seq, const int32_t *q_pos, int n_q, int B, int H, int max_blocks,
+                                  int num_pages, void *out, int32_t *sel_out, void *workspace,
+                                  size_t workspace_bytes, int32_t *dev_err, uocr_stream_t stream) {
+    uocr_status_t st = check_common(n_q, B, max_blocks, num_pages, block_table, seq_lens, nullptr, q_pos, dev_err);
+    if (st != UOCR_OK) return st;
+    if (!bf16_ok(q) || !bf16_ok(k_cache) || !bf16_ok(v_cache) || !bf16_ok(out) || !bf16_ok(idx_q) ||
+        !bf16_ok(idx_k_cache) || !q_pos)
+        return UOCR_ERR_INVALID_ARG;
+    if (!sel_out || !aligned(sel_out, 4)) return UOCR_ERR_INVALID_ARG;
+    if (seq < 0 || seq >= B) return UOCR_ERR_INVALID_ARG;
+    if (H < 1 || H > UOCR_MAX_HEADS) return UOCR_ERR_UNSUPPORTED;
+    if (n_q == 0) return UOCR_OK;
+    const WsLayout w = ws_layout(n_q, H, max_blocks);
+    if (!workspace || !aligned(workspace, kWsAlign) || workspace_bytes < w.total) return UOCR_ERR_WORKSPACE;
+    uocr::LaunchCtx c;
+    if ((st = make_ctx(stream, false, c)) != UOCR_OK) return st;
+    float *scores = (float *)((char *)workspace + w.scores_off);
+    cudaError_t e = uocr::launch_prefill_index_gemm(c, idx_q, idx_k_cache, block_table + (size_t)seq * max_blocks,
+                                                    seq_lens + seq, q_pos, n_q, max_blocks, num_pages, scores,
+                                                    dev_err);
+    if (e != cudaSuccess) return cuda_status(e);
+    c.pdl = true;
+    e = uocr::launch_block_topk(c, scores, seq_lens, nullptr, q_pos, n_q, B, max_blocks, sel_out, dev_err, seq);
+    if (e != cudaSuccess) return cuda_status(e);
+    const float scale = 1.0f / sqrtf((float)UOCR_HEAD_DIM);
+    e = uocr::launch_sparse_attn(c, q, k_cache, v_cache, block_table, seq_lens, nullptr, q_pos, sel_out, n_q, B, H,
+                                 max_blocks, num_pages, scale, out, true, seq, true, dev_err);
     return cuda_status(e);
 }
 

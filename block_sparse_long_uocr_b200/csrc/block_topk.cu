@@ -119,7 +119,7 @@ __device__ void topk_two_level(const KeySource &key, int nc, uint64_t *s_cand, u
 __global__ void __launch_bounds__(kTopkThreads)
 block_topk_kernel(const float *__restrict__ scores, const int32_t *__restrict__ seq_lens,
                   const int32_t *__restrict__ q_seq, const int32_t *__restrict__ q_pos, int B,
-                  int max_blocks, int32_t *__restrict__ sel, int32_t *dev_err, int staged) {
+                  int max_blocks, int32_t *__restrict__ sel, int32_t *dev_err, int staged, int fixed_seq) {
     extern __shared__ uint32_t s_keys[];
     __shared__ uint64_t s_surv[kSurvivorCap];
     __shared__ uint64_t s_cand[kTopkWarps * kRemote];
@@ -138,7 +138,7 @@ block_topk_kernel(const float *__restrict__ scores, const int32_t *__restrict__ 
     pdl_launch_dependents();
 
     QueryRef r;
-    if (!resolve_query(i, seq_lens, q_seq, q_pos, B, max_blocks, dev_err, tid == 0, r)) {
+    if (!resolve_query(i, seq_lens, q_seq, q_pos, B, max_blocks, dev_err, tid == 0, r, fixed_seq)) {
         if (tid < kSel) out[tid] = -1;
         return;
     }
@@ -235,7 +235,7 @@ block_topk_kernel(const float *__restrict__ scores, const int32_t *__restrict__ 
 
 cudaError_t launch_block_topk(const LaunchCtx &c, const float *scores, const int32_t *seq_lens,
                               const int32_t *q_seq, const int32_t *q_pos, int n_q, int B,
-                              int max_blocks, int32_t *sel, int32_t *dev_err) {
+                              int max_blocks, int32_t *sel, int32_t *dev_err, int fixed_seq) {
     const int staged = max_blocks <= kTopkSmemKeys;
     const size_t smem = staged ? (size_t)max_blocks * sizeof(uint32_t) : 0;
     if (smem > 16 * 1024) {
@@ -255,7 +255,7 @@ cudaError_t launch_block_topk(const LaunchCtx &c, const float *scores, const int
     cfg.attrs = attr;
     cfg.numAttrs = c.pdl ? 1 : 0;
     return cudaLaunchKernelEx(&cfg, block_topk_kernel, scores, seq_lens, q_seq, q_pos, B, max_blocks,
-                              sel, dev_err, staged);
+                              sel, dev_err, staged, fixed_seq);
 }
 
 }  // namespace uocr

@@ -30,10 +30,13 @@ __device__ __forceinline__ void flag_error(int32_t *dev_err, uint32_t bits) {
     if (dev_err) atomicOr(reinterpret_cast<unsigned int *>(dev_err), bits);
 }
 
+// fixed_seq >= 0 puts every query in that sequence (a prefill chunk); otherwise
+// query i belongs to q_seq[i], or to sequence i when q_seq is NULL.
 __device__ __forceinline__ bool resolve_query(int i, const int32_t *seq_lens, const int32_t *q_seq,
                                               const int32_t *q_pos, int B, int max_blocks,
-                                              int32_t *dev_err, bool report, QueryRef &r) {
-    int b = q_seq ? __ldg(q_seq + i) : i;
+                                              int32_t *dev_err, bool report, QueryRef &r,
+                                              int fixed_seq = -1) {
+    int b = fixed_seq >= 0 ? fixed_seq : (q_seq ? __ldg(q_seq + i) : i);
     if (b < 0 || b >= B) {
         if (report) flag_error(dev_err, UOCR_DEVERR_POS);
         return false;
@@ -161,6 +164,28 @@ __device__ __forceinline__ bool mbar_wait_bounded(uint64_t *bar, uint32_t parity
     for (int it = 0; it < max_tries; ++it)
         if (mbar_try_wait(bar, parity)) return true;
     return false;
+}
+
+__device__ __forceinline__ uint64_t global_timer_ns() {
+    uint64_t t;
+    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+    return t;
+}
+
+// Wait on phase `parity` of `bar` for at most `timeout_ns` of wall time, giving up early
+// when *abort becomes non-zero.  Returns true when the phase completed.
+__device__ __forceinline__ bool mbar_wait_timed(uint64_t *bar, uint32_t parity, uint64_t timeout_ns,
+                                                const volatile int *abort) {
+    if (mbar_try_wait(bar, parity)) return true;
+    const uint64_t t0 = global_timer_ns();
+    for (uint32_t it = 1;; ++it) {
+        if (mbar_try_wait(bar, parity)) return true;
+        if ((it & 63u) == 0) {
+            if (abort && *abort) return false;
+            if (global_timer_ns() - t0 > timeout_ns) return false;
+            if (it > (1u << 30)) return false;   // in case the timer does not advance
+        }
+    }
 }
 
 // Programmatic dependent launch: wait for the preceding grid's memory, and

@@ -23,12 +23,18 @@ cudaError_t launch_index_scan(const LaunchCtx &c, const void *idx_q, const void 
 
 cudaError_t launch_block_topk(const LaunchCtx &c, const float *scores, const int32_t *seq_lens,
                               const int32_t *q_seq, const int32_t *q_pos, int n_q, int B,
-                              int max_blocks, int32_t *sel, int32_t *dev_err);
+                              int max_blocks, int32_t *sel, int32_t *dev_err, int fixed_seq = -1);
 
 cudaError_t launch_sparse_attn(const LaunchCtx &c, const void *q, const void *k, const void *v,
                                const int32_t *bt, const int32_t *seq_lens, const int32_t *q_seq,
                                const int32_t *q_pos, const int32_t *sel, int n_q, int B, int H,
                                int max_blocks, int num_pages, float scale, void *out,
-                               bool implicit_local, int32_t *dev_err);
+                               bool implicit_local, int fixed_seq, bool head_major, int32_t *dev_err);
+
+// tcgen05 block scoring of n_q queries of one sequence (block table row bt_row,
+// length *seq_len_ptr) into scores [n_q][max_blocks].
+cudaError_t launch_prefill_index_gemm(const LaunchCtx &c, const void *idx_q, const void *idx_k,
+                                      const int32_t *bt_row, const int32_t *seq_len_ptr, const int32_t *q_pos,
+                                      int n_q, int max_blocks, int num_pages, float *scores, int32_t *dev_err);
 
 }  // namespace uocr

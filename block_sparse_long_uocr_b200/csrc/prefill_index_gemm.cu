@@ -1,0 +1,386 @@
+// prefill_index_gemm.cu -- chunked-prefill block scoring on the tcgen05 tensor cores.
+//
+// Unlimited-OCR-2 release report (leheavengame.com, "百度OCR-2开源", section 三): a
+// prefill chunk of `tokens` queries builds a [tokens, context/32] block-score
+// tensor.  With many queries per sequence the indexer scan becomes a dense
+// contraction, S = Qi [n_q x 128] . Ki^T [128 x tokens], followed by the block
+// maximum of the walk-through (news.rkmt.cn/news/25027, section 五 step 2):
+//   scores[i][j] = max_{t in block j, t <= p_i} S[i][t].
+//
+// Kernel (persistent, one CTA per SM, 192 threads, warp-specialised):
+//   warp 4  TMA producer: per work unit the 128-query A tile (two 64-dim halves,
+//           128-byte swizzle) into a 2-deep ring, and per 256-token N tile the
+//           8 pages' indexer keys (16 boxes of 32 tokens x 64 dims, gathered
+//           through the block table) into a 2-stage ring;
+//   warp 5  MMA issuer: allocates 512 TMEM columns (two 128 x 256 fp32
+//           accumulators) and issues 8 tcgen05.mma (M=128, N=256, K=16) per tile;
+//   warps 0-3 epilogue: tcgen05.ld of the accumulator (warp w owns rows
+//           32w .. 32w+31 = TMEM lanes), causal mask, max over each 32-column
+//           block, fp32 scores to global memory.
+// Work unit = (128-query tile, chunk of 4 N tiles); units whose tokens all lie
+// past the tile's last query are skipped.  Every mbarrier wait is bounded in
+// wall time: on timeout the CTA reports UOCR_DEVERR_TIMEOUT, every role stops
+// issuing, waits (bounded) for what it issued, and the TMEM is freed.
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <math.h>
+
+#include "common.cuh"
+#include "kernels.h"
+#include "tcgen05.cuh"
+
+namespace uocr {
+
+namespace {
+
+constexpr int kBM = 128;                  // queries per tile (TMEM lanes)
+constexpr int kBN = 256;                  // tokens per N tile (8 pages)
+constexpr int kPagesPerTile = kBN / kBlock;
+constexpr int kTilesPerUnit = 4;
+constexpr int kStagesB = 2;
+constexpr int kStagesA = 2;
+constexpr int kHalfBytesA = kBM * 128;    // one 64-dim half of an A tile: 16 KiB
+constexpr int kHalfBytesB = kBN * 128;    // one 64-dim half of a B tile: 32 KiB
+constexpr int kBoxBytesB = kBlock * 128;  // one page x 64 dims: 4 KiB
+constexpr int kThreads = 192;
+constexpr int kEpiWarps = 4;
+constexpr int kProducerWarp = 4;
+constexpr int kMmaWarp = 5;
+constexpr uint64_t kTimeoutNs = 2000000000ull;   // 2 s: far above any legitimate wait
+
+struct __align__(1024) Smem {
+    uint8_t a[kStagesA][2][kHalfBytesA];      // 64 KiB
+    uint8_t b[kStagesB][2][kHalfBytesB];      // 128 KiB
+    uint64_t a_full[kStagesA], a_empty[kStagesA];
+    uint64_t b_full[kStagesB], b_empty[kStagesB];
+    uint64_t acc_full[2], acc_empty[2];
+    uint64_t mma_done;
+    uint32_t tmem_base;
+    int abort_flag;
+};
+
+struct UnitInfo {
+    int m0;       // first query of the tile
+    int t0;       // first N tile
+    int ntiles;   // tiles to compute (0: skip)
+    int nb_max;   // causal blocks of the tile's last valid query
+};
+
+// Position of query `row`, or -1 when it has no visible token or is invalid.
+__device__ __forceinline__ int row_pos(const int32_t *q_pos, int row, int n_q, int seq_len) {
+    if (row >= n_q) return -1;
+    const int p = __ldg(q_pos + row);
+    return p < seq_len ? p : -1;
+}
+
+// Same answer in every role: the unit's tile range, from the queries' positions.
+__device__ __forceinline__ UnitInfo unit_info(int u, int n_chunks, const int32_t *q_pos, int n_q, int seq_len,
+                                              int lane) {
+    UnitInfo w;
+    w.m0 = (u / n_chunks) * kBM;
+    w.t0 = (u % n_chunks) * kTilesPerUnit;
+    int pmax = -1;
+#pragma unroll
+    for (int k = 0; k < kBM / 32; ++k) pmax = max(pmax, row_pos(q_pos, w.m0 + k * 32 + lane, n_q, seq_len));
+    pmax = __reduce_max_sync(0xffffffffu, pmax);
+    w.nb_max = pmax < 0 ? 0 : pmax / kBlock + 1;
+    const int tiles_needed = (w.nb_max + kPagesPerTile - 1) / kPagesPerTile;
+    w.ntiles = max(0, min(kTilesPerUnit, tiles_needed - w.t0));
+    return w;
+}
+
+// Lane 0 waits; the verdict is broadcast so the whole warp leaves its loops together.
+__device__ __forceinline__ bool warp_wait(uint64_t *bar, uint32_t parity, Smem &s, int32_t *dev_err, int lane) {
+    int ok = 1;
+    if (lane == 0) {
+        ok = mbar_wait_timed(bar, parity, kTimeoutNs, &s.abort_flag);
+        if (!ok) {
+            if (!*(volatile int *)&s.abort_flag) flag_error(dev_err, UOCR_DEVERR_TIMEOUT);
+            atomicExch(&s.abort_flag, 1);
+        }
+    }
+    return __shfl_sync(0xffffffffu, ok, 0) != 0;
+}
+
+__device__ __forceinline__ bool aborted(Smem &s) { return *(volatile int *)&s.abort_flag != 0; }
+
+}  // namespace
+
+__global__ void __launch_bounds__(kThreads, 1)
+prefill_index_gemm_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__ CUtensorMap map_k,
+                          const int32_t *__restrict__ bt_row, const int32_t *__restrict__ seq_len_ptr,
+                          const int32_t *__restrict__ q_pos, int n_q, int a_box_rows, int num_pages,
+                          int max_blocks, int n_chunks, int n_units, float *__restrict__ scores,
+                          int32_t *dev_err) {
+    extern __shared__ uint8_t smem_raw[];
+    Smem &s = *reinterpret_cast<Smem *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    const int warp = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31;
+
+    if (threadIdx.x == 0) {
+        for (int k = 0; k < kStagesA; ++k) {
+            mbar_init(&s.a_full[k], 1);
+            mbar_init(&s.a_empty[k], 1);
+        }
+        for (int k = 0; k < kStagesB; ++k) {
+            mbar_init(&s.b_full[k], 1);
+            mbar_init(&s.b_empty[k], 1);
+        }
+        for (int k = 0; k < 2; ++k) {
+            mbar_init(&s.acc_full[k], 1);
+            mbar_init(&s.acc_empty[k], kEpiWarps);
+        }
+        mbar_init(&s.mma_done, 1);
+        s.abort_flag = 0;
+        fence_mbar_init();
+    }
+    if (warp == kMmaWarp) {
+        tc::tmem_alloc(&s.tmem_base, 512);
+        tc::tmem_relinquish();
+    }
+    if (warp == kProducerWarp && lane == 0) {
+        tc::prefetch_tensormap(&map_q);
+        tc::prefetch_tensormap(&map_k);
+    }
+    tc::fence_before_sync();
+    __syncthreads();
+    tc::fence_after_sync();
+    const uint32_t tmem = s.tmem_base;
+
+    pdl_wait();   // inputs may come from the preceding kernel in the stream
+    const int seq_len = __ldg(seq_len_ptr);
+    if (threadIdx.x == 0 && seq_len > max_blocks * kBlock) flag_error(dev_err, UOCR_DEVERR_POS);
+    const int seq_len_ok = min(seq_len, max_blocks * kBlock);
+
+    if (warp == kProducerWarp) {
+        // ------------------------------------------------------------ TMA producer
+        int it = 0, uc = 0;
+        int b_fills[kStagesB] = {0, 0};
+        int a_fills[kStagesA] = {0, 0};
+        bool stop = false;
+        for (int u = blockIdx.x; u < n_units && !stop; u += gridDim.x) {
+            const UnitInfo w = unit_info(u, n_chunks, q_pos, n_q, seq_len_ok, lane);
+            if (w.ntiles == 0) continue;
+            const int sa = uc % kStagesA;
+            if (!warp_wait(&s.a_empty[sa], ((uc / kStagesA) & 1) ^ 1, s, dev_err, lane)) break;
+            if (lane == 0) {
+                mbar_arrive_expect_tx(&s.a_full[sa], 2u * a_box_rows * 128u);
+                tc::tma_load_2d(s.a[sa][0], &map_q, 0, w.m0, &s.a_full[sa]);
+                tc::tma_load_2d(s.a[sa][1], &map_q, 64, w.m0, &s.a_full[sa]);
+            }
+            ++a_fills[sa];
+            ++uc;
+            for (int t = 0; t < w.ntiles; ++t, ++it) {
+                const int st = it % kStagesB;
+                const int tile = w.t0 + t;
+                int page = -1;   // lanes 0..7 look up the tile's pages
+                if (lane < kPagesPerTile) {
+                    const int j = tile * kPagesPerTile + lane;
+                    if (j < w.nb_max) {
+                        page = __ldg(bt_row + j);
+                        if ((unsigned)page >= (unsigned)num_pages) {
+                            flag_error(dev_err, UOCR_DEVERR_PAGE);
+                            page = -1;
+                        }
+                    }
+                }
+                const unsigned valid = __ballot_sync(0xffffffffu, page >= 0);
+                if (!warp_wait(&s.b_empty[st], ((it / kStagesB) & 1) ^ 1, s, dev_err, lane)) {
+                    stop = true;
+                    break;
+                }
+                if (lane == 0) mbar_arrive_expect_tx(&s.b_full[st], (uint32_t)__popc(valid) * 2u * kBoxBytesB);
+                __syncwarp();
+                if (page >= 0) {   // lane k issues page k's two boxes
+                    tc::tma_load_2d(s.b[st][0] + lane * kBoxBytesB, &map_k, 0, page * kBlock, &s.b_full[st]);
+                    tc::tma_load_2d(s.b[st][1] + lane * kBoxBytesB, &map_k, 64, page * kBlock, &s.b_full[st]);
+                }
+                ++b_fills[st];
+                if (aborted(s)) {
+                    stop = true;
+                    break;
+                }
+            }
+        }
+        // drain: every buffer this warp filled must have landed before the CTA exits
+        if (lane == 0) {
+            for (int k = 0; k < kStagesB; ++k)
+                if (b_fills[k] > 0) mbar_wait_timed(&s.b_full[k], (b_fills[k] - 1) & 1, kTimeoutNs, nullptr);
+            for (int k = 0; k < kStagesA; ++k)
+                if (a_fills[k] > 0) mbar_wait_timed(&s.a_full[k], (a_fills[k] - 1) & 1, kTimeoutNs, nullptr);
+        }
+    } else if (warp == kMmaWarp) {
+        // ------------------------------------------------------------ MMA issuer
+        constexpr uint32_t idesc = tc::idesc_bf16_f32(kBM, kBN);
+        int it = 0, uc = 0;
+        bool issued = false, stop = false;
+        for (int u = blockIdx.x; u < n_units && !stop; u += gridDim.x) {
+            const UnitInfo w = unit_info(u, n_chunks, q_pos, n_q, seq_len_ok, lane);
+            if (w.ntiles == 0) continue;
+            const int sa = uc % kStagesA;
+            if (!warp_wait(&s.a_full[sa], (uc / kStagesA) & 1, s, dev_err, lane)) break;
+            ++uc;
+            const uint32_t a0 = smem_addr(s.a[sa][0]), a1 = smem_addr(s.a[sa][1]);
+            for (int t = 0; t < w.ntiles; ++t, ++it) {
+                const int st = it % kStagesB;
+                const int acc = it & 1;
+                if (!warp_wait(&s.b_full[st], (it / kStagesB) & 1, s, dev_err, lane) ||
+                    !warp_wait(&s.acc_empty[acc], ((it >> 1) & 1) ^ 1, s, dev_err, lane)) {
+                    stop = true;
+                    break;
+                }
+                if (lane == 0) {
+                    tc::fence_after_sync();
+                    const uint32_t b0 = smem_addr(s.b[st][0]), b1 = smem_addr(s.b[st][1]);
+#pragma unroll
+                    for (int k = 0; k < 8; ++k) {
+                        const uint32_t koff = (k & 3) * 32;   // 16 bf16 = 32 bytes inside the swizzle atom
+                        const uint64_t ad = tc::smem_desc_k_sw128((k < 4 ? a0 : a1) + koff);
+                        const uint64_t bd = tc::smem_desc_k_sw128((k < 4 ? b0 : b1) + koff);
+                        tc::mma_bf16(tmem + acc * kBN, ad, bd, idesc, k > 0 ? 1u : 0u);
+                    }
+                    tc::commit(&s.b_empty[st]);
+                    tc::commit(&s.acc_full[acc]);
+                }
+                issued = true;
+                __syncwarp();
+            }
+            if (lane == 0) tc::commit(&s.a_empty[sa]);   // the A tile is free once its MMAs complete
+            __syncwarp();
+            if (aborted(s)) break;
+        }
+        // drain: every MMA this thread issued has completed before TMEM is freed
+        if (lane == 0 && issued) {
+            tc::commit(&s.mma_done);
+            mbar_wait_timed(&s.mma_done, 0, kTimeoutNs, nullptr);
+        }
+        __syncwarp();
+    } else {
+        // ------------------------------------------------------------ epilogue, warps 0..3
+        int it = 0;
+        bool stop = false;
+        for (int u = blockIdx.x; u < n_units && !stop; u += gridDim.x) {
+            const UnitInfo w = unit_info(u, n_chunks, q_pos, n_q, seq_len_ok, lane);
+            if (w.ntiles == 0) continue;
+            const int row = w.m0 + warp * 32 + lane;
+            if (row < n_q) {
+                const int p_raw = __ldg(q_pos + row);
+                if (p_raw >= seq_len && w.t0 == 0) flag_error(dev_err, UOCR_DEVERR_POS);
+            }
+            const int p = row_pos(q_pos, row, n_q, seq_len_ok);
+            const int nb_row = p < 0 ? 0 : p / kBlock + 1;
+            float *srow = scores + (size_t)(row < n_q ? row : 0) * max_blocks;
+            for (int t = 0; t < w.ntiles; ++t, ++it) {
+                const int acc = it & 1;
+                if (!warp_wait(&s.acc_full[acc], (it >> 1) & 1, s, dev_err, lane)) {
+                    stop = true;
+                    break;
+                }
+                tc::fence_after_sync();
+                const int tile = w.t0 + t;
+                float best[kPagesPerTile];
+                const uint32_t tbase = tmem + ((uint32_t)(warp * 32) << 16) + (uint32_t)(acc * kBN);
+#pragma unroll
+                for (int k = 0; k < kPagesPerTile; ++k) {
+                    float v[32];
+                    tc::tmem_ld_32x32b_x32(tbase + k * 32, v);
+                    tc::tmem_ld_wait();
+                    const int tok0 = (tile * kPagesPerTile + k) * kBlock;
+                    float m = -INFINITY;
+#pragma unroll
+                    for (int c = 0; c < 32; ++c) m = (tok0 + c <= p) ? fmaxf(m, v[c]) : m;
+                    best[k] = m;
+                }
+                tc::fence_before_sync();
+                __syncwarp();
+                if (lane == 0)
+                    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_addr(&s.acc_empty[acc]))
+                                 : "memory");
+                // a block whose page is not in the pool scores -inf; blocks past the row's
+                // causal range are not written
+                const int j0 = tile * kPagesPerTile;
+#pragma unroll
+                for (int k = 0; k < kPagesPerTile; ++k) {
+                    const int j = j0 + k;
+                    if (j < nb_row) {
+                        const int page = __ldg(bt_row + j);
+                        srow[j] = ((unsigned)page < (unsigned)num_pages) ? best[k] : -INFINITY;
+                    }
+                }
+            }
+        }
+    }
+
+    tc::fence_before_sync();
+    __syncthreads();
+    if (warp == kMmaWarp) {
+        tc::fence_after_sync();
+        tc::tmem_dealloc(tmem, 512);
+    }
+}
+
+// ---------------------------------------------------------------- host side
+namespace {
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *, const cuuint64_t *,
+                                  const cuuint64_t *, const cuuint32_t *, const cuuint32_t *, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn get_encode() {
+    void *p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) != cudaSuccess ||
+        q != cudaDriverEntryPointSuccess)
+        return nullptr;
+    return reinterpret_cast<EncodeTiledFn>(p);
+}
+
+// 2-D bf16 tensor of `rows` x 128 (row stride 256 B), boxes of 64 x box_rows, 128-byte swizzle.
+bool make_map(CUtensorMap *m, const void *base, uint64_t rows, uint32_t box_rows) {
+    EncodeTiledFn enc = get_encode();
+    if (!enc) return false;
+    const cuuint64_t dims[2] = {128, rows};
+    const cuuint64_t strides[1] = {256};
+    const cuuint32_t box[2] = {64, box_rows};
+    const cuuint32_t estr[2] = {1, 1};
+    return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(base), dims, strides, box, estr,
+               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+}  // namespace
+
+size_t prefill_index_gemm_smem() { return sizeof(Smem) + 1024; }
+
+cudaError_t launch_prefill_index_gemm(const LaunchCtx &c, const void *idx_q, const void *idx_k,
+                                      const int32_t *bt_row, const int32_t *seq_len_ptr, const int32_t *q_pos,
+                                      int n_q, int max_blocks, int num_pages, float *scores, int32_t *dev_err) {
+    const int a_box_rows = n_q < kBM ? n_q : kBM;
+    CUtensorMap map_q, map_k;
+    if (!make_map(&map_q, idx_q, (uint64_t)n_q, (uint32_t)a_box_rows)) return cudaErrorInvalidValue;
+    if (!make_map(&map_k, idx_k, (uint64_t)num_pages * kBlock, kBlock)) return cudaErrorInvalidValue;
+    const int m_tiles = (n_q + kBM - 1) / kBM;
+    const int n_tiles = (max_blocks + kPagesPerTile - 1) / kPagesPerTile;
+    const int n_chunks = (n_tiles + kTilesPerUnit - 1) / kTilesPerUnit;
+    const long long units = (long long)m_tiles * n_chunks;
+    if (units > 0x7fffffffLL) return cudaErrorInvalidConfiguration;
+    const int grid = (int)(units < c.num_sms ? units : c.num_sms);
+    const size_t smem = prefill_index_gemm_smem();
+    cudaError_t e = cudaFuncSetAttribute(prefill_index_gemm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)smem);
+    if (e != cudaSuccess) return e;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)grid);
+    cfg.blockDim = dim3(kThreads);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = c.stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = c.pdl ? 1 : 0;
+    return cudaLaunchKernelEx(&cfg, prefill_index_gemm_kernel, map_q, map_k, bt_row, seq_len_ptr, q_pos, n_q,
+                              a_box_rows, num_pages, max_blocks, n_chunks, (int)units, scores, dev_err);
+}
+
+}  // namespace uocr

@@ -68,8 +68,8 @@ sparse_attn_kernel(const uint4 *__restrict__ q, const uint4 *__restrict__ kc, co
                    const int32_t *__restrict__ bt, const int32_t *__restrict__ seq_lens,
                    const int32_t *__restrict__ q_seq, const int32_t *__restrict__ q_pos,
                    const int32_t *__restrict__ sel, int B, int H, int max_blocks, int num_pages,
-                   float scale_log2, int implicit_local, __nv_bfloat16 *__restrict__ out,
-                   int32_t *dev_err) {
+                   float scale_log2, int implicit_local, int fixed_seq, int head_major, int n_q,
+                   __nv_bfloat16 *__restrict__ out, int32_t *dev_err) {
     __shared__ float s_m[kAttnWarps], s_l[kAttnWarps];
     __shared__ float s_acc[kAttnWarps][kD];
     __shared__ float s_cta_ml[2];
@@ -77,10 +77,13 @@ sparse_attn_kernel(const uint4 *__restrict__ q, const uint4 *__restrict__ kc, co
     __shared__ __align__(8) uint64_t s_bar[kAttnWarps];
     __shared__ __align__(128) uint4 s_v[kAttnWarps][kPageElems / 8];   // one V tile per warp
 
-    const int ih = blockIdx.x / kAttnCluster;
+    const int cl = blockIdx.x / kAttnCluster;
     const int split = (int)cluster_ctarank();    // == blockIdx.x % kAttnCluster
-    const int h = ih % H;
-    const int i = ih / H;
+    // head-major order (all queries of head 0 first) keeps one head's K/V hot in L2
+    // when many queries share a sequence (prefill); query-major otherwise
+    const int h = head_major ? cl / n_q : cl % H;
+    const int i = head_major ? cl % n_q : cl / H;
+    const int ih = i * H + h;
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
     const int slot = split * kAttnWarps + warp;
@@ -94,7 +97,7 @@ sparse_attn_kernel(const uint4 *__restrict__ q, const uint4 *__restrict__ kc, co
     // outputs of the preceding kernel, so they are read before the dependency wait
     QueryRef r;
     const bool ok = resolve_query(i, seq_lens, q_seq, q_pos, B, max_blocks, dev_err,
-                                  threadIdx.x == 0 && split == 0 && h == 0, r);
+                                  threadIdx.x == 0 && split == 0 && h == 0, r, fixed_seq);
     int j = ok && implicit_local ? implicit_slot(slot, r.nb) : -2;
     if (j == -2) {
         pdl_wait();
@@ -230,7 +233,7 @@ cudaError_t launch_sparse_attn(const LaunchCtx &c, const void *q, const void *k,
                                const int32_t *bt, const int32_t *seq_lens, const int32_t *q_seq,
                                const int32_t *q_pos, const int32_t *sel, int n_q, int B, int H,
                                int max_blocks, int num_pages, float scale, void *out,
-                               bool implicit_local, int32_t *dev_err) {
+                               bool implicit_local, int fixed_seq, bool head_major, int32_t *dev_err) {
     const long long grid = (long long)n_q * H * kAttnCluster;
     if (grid > 0x7fffffffLL) return cudaErrorInvalidConfiguration;
     cudaLaunchAttribute attr[2];
@@ -249,7 +252,8 @@ cudaError_t launch_sparse_attn(const LaunchCtx &c, const void *q, const void *k,
     cfg.numAttrs = c.pdl ? 2 : 1;
     return cudaLaunchKernelEx(&cfg, sparse_attn_kernel, (const uint4 *)q, (const uint4 *)k, (const uint4 *)v, bt,
                               seq_lens, q_seq, q_pos, sel, B, H, max_blocks, num_pages, scale * kLog2e,
-                              implicit_local ? 1 : 0, (__nv_bfloat16 *)out, dev_err);
+                              implicit_local ? 1 : 0, fixed_seq, head_major ? 1 : 0, n_q, (__nv_bfloat16 *)out,
+                              dev_err);
 }
 
 }  // namespace uocr

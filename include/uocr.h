@@ -102,7 +102,7 @@ const char *uocr_status_string(uocr_status_t status);
 int uocr_abi_version(void);
 
 /*
- * Workspace bytes that uocr_sparse_decode needs for B = n_q queries over
+ * Workspace bytes that uocr_sparse_decode and uocr_sparse_prefill need for n_q queries over
  * max_blocks blocks: the fp32 block scores [n_q][max_blocks], rounded up to
  * 256 bytes.  A pure function of the shapes (0 for a non-positive argument);
  * H is accepted for symmetry with the other entry points and does not change
@@ -166,6 +166,39 @@ uocr_status_t uocr_sparse_decode(const void *q, const void *k_cache, const void 
                                  void *out, int32_t *sel_out,
                                  void *workspace, size_t workspace_bytes,
                                  int32_t *dev_err, uocr_stream_t stream);
+
+/*
+ * Chunked-prefill block scores on the tensor cores, [leheaven 三] with the
+ * scoring rule of [rkmt 五 step 2]: the same scores as uocr_index_score for
+ * n_q queries that all belong to sequence `seq`, at positions q_pos[i]
+ * (required; a position at or past seq_lens[seq] flags UOCR_DEVERR_POS and
+ * scores nothing), computed as S = idx_q . idx_k^T on tcgen05 (bf16 inputs,
+ * fp32 accumulation in TMEM) with the causal mask and the per-block maximum
+ * applied while the accumulator is read back.  scores [n_q][max_blocks];
+ * entries j >= nb_i are not written.  Needs an sm_100a device; one persistent
+ * CTA per SM holds ~193 KiB of shared memory and 512 TMEM columns.
+ */
+uocr_status_t uocr_prefill_index_score(const void *idx_q, const void *idx_k_cache,
+                                       const int32_t *block_table, const int32_t *seq_lens,
+                                       int seq, const int32_t *q_pos, int n_q, int B,
+                                       int max_blocks, int num_pages, float *scores,
+                                       int32_t *dev_err, uocr_stream_t stream);
+
+/*
+ * The whole chunked-prefill step for n_q queries of sequence `seq` at
+ * positions q_pos (their K/V and indexer keys already cached):
+ * uocr_prefill_index_score -> uocr_block_topk -> uocr_sparse_attn with
+ * scale = 1/sqrt(128), launched back to back on `stream`.  Each query selects
+ * its own 4 local + 12 remote blocks over its causal prefix.  out [n_q][H][128]
+ * bf16, sel_out [n_q][16].  Workspace: uocr_workspace_bytes(n_q, H, max_blocks).
+ */
+uocr_status_t uocr_sparse_prefill(const void *q, const void *k_cache, const void *v_cache,
+                                  const void *idx_q, const void *idx_k_cache,
+                                  const int32_t *block_table, const int32_t *seq_lens,
+                                  int seq, const int32_t *q_pos, int n_q, int B, int H,
+                                  int max_blocks, int num_pages, void *out, int32_t *sel_out,
+                                  void *workspace, size_t workspace_bytes,
+                                  int32_t *dev_err, uocr_stream_t stream);
 
 /*
  * uocr_sparse_decode_static -- uocr_sparse_decode for callers that cannot

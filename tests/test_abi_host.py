@@ -175,3 +175,31 @@ def test_product_package_does_not_import_the_oracle():
             if f.endswith((".py", ".cu", ".cuh", ".h", ".c", ".cpp")):
                 src = open(os.path.join(dirpath, f)).read()
                 assert not re.search(r"\boracle\b", src.replace("oracle-free", "")), f"{f} mentions the oracle"
+
+
+@no_gpu
+@pytest.mark.parametrize("over,code", [
+    (dict(q_pos=None), 1), (dict(seq=-1), 1), (dict(seq=4), 1), (dict(idx_q=MIS), 1), (dict(scores=None), 1),
+    (dict(B=0), 1), (dict(mb=0), 1), (dict(P=0), 1), (dict(idx_k=None), 1),
+])
+def test_prefill_index_score_rejects(pkg, over, code):
+    a = dict(idx_q=FAKE, idx_k=FAKE, bt=FAKE, sl=FAKE, seq=0, q_pos=FAKE, n_q=4, B=4, mb=64, P=256, scores=FAKE)
+    a.update(over)
+    st = pkg.lib.uocr_prefill_index_score(a["idx_q"], a["idx_k"], a["bt"], a["sl"], a["seq"], a["q_pos"], a["n_q"],
+                                          a["B"], a["mb"], a["P"], a["scores"], None, None)
+    assert st == code
+
+
+@no_gpu
+@pytest.mark.parametrize("over,code", [
+    (dict(q_pos=None), 1), (dict(seq=5), 1), (dict(sel=None), 1), (dict(out=MIS), 1), (dict(H=0), 2),
+    (dict(ws=None), 3), (dict(wsb=16), 3), (dict(ws=FAKE + 64), 3),
+])
+def test_sparse_prefill_rejects(pkg, over, code):
+    a = dict(q=FAKE, k=FAKE, v=FAKE, idx_q=FAKE, idx_k=FAKE, bt=FAKE, sl=FAKE, seq=0, q_pos=FAKE, n_q=4, B=4, H=10,
+             mb=64, P=256, out=FAKE, sel=FAKE, ws=FAKE, wsb=1 << 30)
+    a.update(over)
+    st = pkg.lib.uocr_sparse_prefill(a["q"], a["k"], a["v"], a["idx_q"], a["idx_k"], a["bt"], a["sl"], a["seq"],
+                                     a["q_pos"], a["n_q"], a["B"], a["H"], a["mb"], a["P"], a["out"], a["sel"],
+                                     a["ws"], a["wsb"], None, None)
+    assert st == code

@@ -1,0 +1,108 @@
+"""Parity of the chunked-prefill path (tcgen05 block scoring, selection, attention)
+with the fp64 oracle, through the C ABI.
+
+Small cases check every query and every block score; they span several
+128-query and 256-token tiles with ragged tails (n_q not a multiple of 128,
+contexts not a multiple of 256, shuffled pages).  The full chunked-prefill
+workload (2048 queries over 65536 tokens) is checked on sampled queries.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import workloads
+from parity_util import check_queries
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def uocr(cuda_device):
+    import block_sparse_long_uocr_b200 as m
+    return m
+
+
+def _prefill_case(total, n_new, extra_pos=(), seed=0, shuffle=True, device="cpu", heads=10):
+    pos = list(range(total - n_new, total)) + list(extra_pos)
+    return workloads.make_case([total], q_seq=[0] * len(pos), q_pos=pos, shuffle=shuffle, seed=seed,
+                               device=device, heads=heads)
+
+
+@pytest.mark.parametrize("total,n_new,extra", [
+    (300, 1, ()),                                  # one query, one partial N tile
+    (1000, 5, (0, 31, 32, 255, 256, 257)),         # n_q < 128: shrunk A box
+    (4096 + 17, 300, (0, 1, 4000)),                # 3 M tiles (ragged), 17 N tiles (ragged)
+    (2048, 128, ()),                               # exactly one M tile
+    (2048, 129, ()),                               # one query over
+])
+def test_prefill_scores_match_oracle(uocr, cuda_device, total, n_new, extra):
+    case = _prefill_case(total, n_new, extra, seed=total + n_new, device=cuda_device, heads=1)
+    sc = uocr.prefill_index_score(case.idx_q, case.idx_k_pool, case.block_table, case.seq_lens, 0, case.q_pos)
+    torch.cuda.synchronize()
+    r = oracle.run(case.q, case.idx_q, case.k_pool, case.v_pool, case.idx_k_pool, case.block_table,
+                   case.q_seq, case.q_pos, want_out=False)
+    got = sc.cpu().double().numpy()
+    for i in range(case.n_q):
+        nb = int(case.q_pos[i]) // 32 + 1
+        np.testing.assert_allclose(got[i, :nb], r["scores"][i, :nb], rtol=0, atol=1e-3, err_msg=f"query {i}")
+        assert np.isneginf(got[i, nb:]).all()          # not written past the causal blocks
+
+
+def test_prefill_scores_agree_with_the_scan_kernel(uocr, cuda_device):
+    case = _prefill_case(32 * 700 + 9, 260, seed=11, device=cuda_device, heads=1)
+    a = uocr.prefill_index_score(case.idx_q, case.idx_k_pool, case.block_table, case.seq_lens, 0, case.q_pos)
+    b = uocr.index_score(case.idx_q, case.idx_k_pool, case.block_table, case.seq_lens, case.q_seq, case.q_pos)
+    torch.cuda.synchronize()
+    fin = torch.isfinite(b)
+    assert torch.equal(fin, torch.isfinite(a))
+    assert (a[fin] - b[fin]).abs().max().item() <= 1e-3
+
+
+def test_sparse_prefill_matches_oracle(uocr, cuda_device):
+    case = _prefill_case(4096, 300, (0, 31, 100, 511, 512, 513), seed=5, device=cuda_device)
+    out, sel = uocr.sparse_prefill(case.q, case.k_pool, case.v_pool, case.idx_q, case.idx_k_pool, case.block_table,
+                                   case.seq_lens, 0, case.q_pos)
+    torch.cuda.synchronize()
+    check_queries(case, range(case.n_q), out, sel)
+
+
+def test_sparse_prefill_second_sequence_and_paging(uocr, cuda_device):
+    """Queries of sequence 1 of a 3-sequence batch with shuffled pages."""
+    lens = [32 * 40, 32 * 90 + 3, 700]
+    pos = list(range(lens[1] - 150, lens[1]))
+    case = workloads.make_case(lens, q_seq=[1] * len(pos), q_pos=pos, shuffle=True, seed=9, device=cuda_device)
+    out, sel = uocr.sparse_prefill(case.q, case.k_pool, case.v_pool, case.idx_q, case.idx_k_pool, case.block_table,
+                                   case.seq_lens, 1, case.q_pos)
+    torch.cuda.synchronize()
+    check_queries(case, range(case.n_q), out, sel)
+
+
+def test_prefill_flags_bad_positions_and_pages(uocr, cuda_device):
+    case = _prefill_case(2000, 40, seed=3, device=cuda_device, heads=1)
+    err = torch.zeros(1, dtype=torch.int32, device=cuda_device)
+    bad_pos = case.q_pos.clone()
+    bad_pos[3] = 2000                                    # at the sequence length: invalid
+    sc = uocr.prefill_index_score(case.idx_q, case.idx_k_pool, case.block_table, case.seq_lens, 0, bad_pos,
+                                  dev_err=err)
+    torch.cuda.synchronize()
+    assert int(err.item()) & uocr.DEVERR_POS
+    assert torch.isneginf(sc[3]).all()                   # nothing written for the invalid query
+    err.zero_()
+    bt = case.block_table.clone()
+    bt[0, 7] = case.num_pages + 3
+    sc = uocr.prefill_index_score(case.idx_q, case.idx_k_pool, bt, case.seq_lens, 0, case.q_pos, dev_err=err)
+    torch.cuda.synchronize()
+    assert int(err.item()) & uocr.DEVERR_PAGE
+    assert torch.isneginf(sc[:, 7]).all() and torch.isfinite(sc[:, 6]).all()
+
+
+@pytest.mark.slow
+def test_chunked_prefill_workload_sampled(uocr, cuda_device):
+    case = workloads.chunked_prefill(device=cuda_device)
+    ws = uocr.alloc_workspace(case.n_q, 10, case.max_blocks, cuda_device)
+    out, sel = uocr.sparse_prefill(case.q, case.k_pool, case.v_pool, case.idx_q, case.idx_k_pool, case.block_table,
+                                   case.seq_lens, 0, case.q_pos, workspace=ws)
+    torch.cuda.synchronize()
+    scores = ws[: case.n_q * case.max_blocks * 4].view(torch.float32).view(case.n_q, case.max_blocks)
+    check_queries(case, [0, 1, 127, 128, 1000, 2046, 2047], out, sel, scores)
