@@ -181,6 +181,8 @@ def build_workload(name: str, device, seed: int, batch=None, layers=None):
         return workloads.tiny_decode(device=device, seed=seed)
     if name == "ragged_paged_decode":
         return workloads.ragged_paged_decode(device=device, seed=seed)
+    if name == "chunked_prefill":
+        return workloads.chunked_prefill(device=device, seed=seed)
     raise SystemExit(f"unknown workload {name}")
 
 
@@ -361,6 +363,143 @@ def run_uocr(args):
         print(json.dumps(result), flush=True)
 
 
+def graph_time_fn(fn, stream, n_rep, flush_buf=None):
+    """Device ms per call of fn(stream) from n_rep calls captured in one CUDA graph
+    (minus the captured L2 flushes between them, when flush_buf is given)."""
+    side = torch.cuda.Stream()
+    side.wait_stream(stream)
+    with torch.cuda.stream(side):
+        fn(side)
+    side.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=side):
+        for _ in range(n_rep):
+            if flush_buf is not None:
+                flush_buf.zero_()
+            fn(side)
+    fg = None
+    if flush_buf is not None:
+        fg = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(fg, stream=side):
+            for _ in range(n_rep):
+                flush_buf.zero_()
+    g.replay()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    g.replay()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    ms = e0.elapsed_time(e1)
+    if fg is not None:
+        fg.replay()
+        torch.cuda.synchronize()
+        e0.record(stream)
+        fg.replay()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        ms -= e0.elapsed_time(e1)
+    return ms / n_rep
+
+
+def run_prefill(args):
+    """Chunked prefill: one uocr_sparse_prefill call of 2048 queries over a 65536-token sequence per step."""
+    rank, local_rank, world = udist.env_rank_world()
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    if world > 1:
+        import datetime
+        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
+    import block_sparse_long_uocr_b200 as uocr
+
+    case = workloads.chunked_prefill(device=dev, seed=udist.shard_seed(args.seed, rank))
+    n_q, H, mb = case.n_q, case.q.shape[1], case.max_blocks
+    ws = uocr.alloc_prefill_workspace(n_q, H, mb, dev)
+    out = torch.empty_like(case.q)
+    sel = torch.empty((n_q, 16), dtype=torch.int32, device=dev)
+    scores = ws[: n_q * mb * 4].view(torch.float32).view(n_q, mb)
+    stream = torch.cuda.current_stream()
+    l2 = torch.cuda.get_device_properties(dev).L2_cache_size
+    flush_buf = torch.empty(2 * l2, dtype=torch.uint8, device=dev)
+
+    def step(st=None):
+        uocr.sparse_prefill(case.q, case.k_pool, case.v_pool, case.idx_q, case.idx_k_pool, case.block_table,
+                            case.seq_lens, 0, case.q_pos, out=out, sel=sel, workspace=ws, stream=st or stream)
+
+    def barrier():
+        if world > 1:
+            torch.distributed.barrier(device_ids=[local_rank])
+
+    clk = ClockSampler(physical_gpu(local_rank)).start()
+    for _ in range(args.warmup):
+        flush_buf.zero_()
+        step()
+    torch.cuda.synchronize()
+    barrier()
+    clk.mark_start()
+    times = []
+    for _ in range(args.steps):
+        flush_buf.zero_()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        step()
+        e1.record(stream)
+        times.append((e0, e1))
+    torch.cuda.synchronize()
+    clk.mark_end()
+    clk.stop()
+    elapsed_ms = sum(a.elapsed_time(b) for a, b in times)
+    barrier()
+    max_ms = udist.max_over_ranks(elapsed_ms, dev)
+    ms_per_step = max_ms / args.steps
+    value = world * n_q * args.steps / (max_ms / 1e3)
+
+    n_rep = 10
+    gemm_ms = graph_time_fn(lambda st: uocr.prefill_index_score(case.idx_q, case.idx_k_pool, case.block_table,
+                                                                case.seq_lens, 0, case.q_pos, scores=scores,
+                                                                stream=st), stream, n_rep, flush_buf)
+    topk_ms = graph_time_fn(lambda st: uocr.block_topk(scores, case.seq_lens, case.q_seq, case.q_pos, sel=sel,
+                                                       stream=st), stream, n_rep, flush_buf)
+    attn_ms = graph_time_fn(lambda st: uocr.sparse_attn(case.q, case.k_pool, case.v_pool, case.block_table,
+                                                        case.seq_lens, sel, case.q_seq, case.q_pos, out=out,
+                                                        stream=st), stream, n_rep, flush_buf)
+    call_ms = graph_time_fn(lambda st: step(st), stream, n_rep, flush_buf)
+    pos = case.q_pos.cpu().long()
+    idx_flops = float(((pos + 1) * 128 * 2).sum())                 # causal q_idx . k_idx products
+    attn_flops = float(n_q * H * 16 * 32 * 128 * 4)                 # QK and PV over 512 tokens
+    peaks, peak_kind = measured_peaks()
+    tc_peak = float(peaks.get("bf16_tflops", 1590.0))
+    tc_sust = float(peaks.get("bf16_tflops_sustained", 1400.0))
+    hbm_peak = float(peaks.get("hbm_gbs", FALLBACK_HBM_GBS))
+    gemm_tflops = idx_flops / (gemm_ms / 1e3) / 1e12
+    kv_union = case.num_pages * H * 32 * 128 * 2 * 2               # every page is selected by some query
+    step_bytes = kv_union + case.num_pages * 32 * 128 * 2 + 2 * n_q * mb * 4 + 2 * n_q * H * 128 * 2
+    result = {
+        "metric": "chunked-prefill queries/s per layer; tensor-core TFLOP/s of the scoring GEMM vs peak",
+        "value": round(value, 1), "unit": "queries/s per layer", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": round(ms_per_step, 4), "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": case.name, "queries": n_q, "context": int(case.seq_lens[0]), "heads": H,
+                   "max_blocks": mb, "l2": "flushed between steps", "parallelism": f"dp{world}"},
+        "roofline": {"bound": "tensor", "kernel": "prefill_index_gemm_kernel", "achieved": round(gemm_tflops, 1),
+                     "peak": tc_peak, "unit": "TFLOP/s", "frac": round(gemm_tflops / tc_peak, 4), "traffic": None,
+                     "peak_kind": f"{peak_kind} bf16 burst", "frac_of_sustained": round(gemm_tflops / tc_sust, 4),
+                     "flops_per_launch": idx_flops, "avg_launch_ms": round(gemm_ms, 5)},
+        "step_roofline": {"bound": "hbm", "achieved": round(step_bytes / (call_ms / 1e3) / 1e9, 1),
+                          "peak": hbm_peak, "unit": "GB/s",
+                          "frac": round(step_bytes / (call_ms / 1e3) / 1e9 / hbm_peak, 4),
+                          "bytes_per_step": step_bytes, "flops_per_step": idx_flops + attn_flops},
+        "breakdown_us": {"prefill_index_gemm": round(1e3 * gemm_ms, 2), "block_topk": round(1e3 * topk_ms, 2),
+                         "sparse_attn": round(1e3 * attn_ms, 2), "prefill_call_graph": round(1e3 * call_ms, 2)},
+        "gpu_launches": args.steps * 3,
+        "clocks": clk.summary(),
+    }
+    if world > 1:
+        torch.distributed.destroy_process_group()
+    if rank == 0:
+        print(json.dumps(result), flush=True)
+
+
 def run_e2e(args, uocr, case, ws, outs, sels, stream, world, dev):
     """Same metric through sparse_decode with the step's per-query inputs copied in from pinned
     host memory and the outputs copied back, inside the timed region.  The KV / indexer caches
@@ -408,26 +547,27 @@ def run_e2e(args, uocr, case, ws, outs, sels, stream, world, dev):
 
 # --------------------------------------------------------------------------- oracle timing
 def _gather_for_oracle(case, layer, queries):
-    """Host copies of what the oracle reads for `queries`: their indexer pages and queries."""
+    """Host copies of what the oracle reads for `queries`: their queries and, once per
+    sequence, that sequence's indexer pages (a small pool with its own block table)."""
     import numpy as np
     q, qi = case.q_layers[layer]
     ikp = case.layers[layer][2]
-    pages, bt_rows, pos = [], [], []
-    off = 0
     mb = case.max_blocks
-    for i in queries:
-        b, p = int(case.q_seq[i]), int(case.q_pos[i])
-        nb = p // 32 + 1
+    seqs = sorted({int(case.q_seq[i]) for i in queries})
+    need = {b: max(int(case.q_pos[i]) // 32 + 1 for i in queries if int(case.q_seq[i]) == b) for b in seqs}
+    pages, rows, where, off = [], [], {}, 0
+    for b in seqs:
+        nb = need[b]
         pages.append(case.block_table[b, :nb].long())
         row = np.full(mb, -1, np.int32)
         row[:nb] = np.arange(off, off + nb)
-        bt_rows.append(row)
-        pos.append(p)
+        where[b] = len(rows)
+        rows.append(row)
         off += nb
-    pidx = torch.cat(pages)
-    mini_idx = ikp[pidx].cpu()
-    return (q[list(queries)].cpu(), qi[list(queries)].cpu(), mini_idx, np.stack(bt_rows),
-            np.arange(len(queries), dtype=np.int32), np.array(pos, np.int32))
+    mini_idx = ikp[torch.cat(pages)].cpu()
+    qs = np.array([where[int(case.q_seq[i])] for i in queries], np.int32)
+    pos = np.array([int(case.q_pos[i]) for i in queries], np.int32)
+    return q[list(queries)].cpu(), qi[list(queries)].cpu(), mini_idx, np.stack(rows), qs, pos
 
 
 def _gather_kv(case, layer, queries, sel):
@@ -460,7 +600,8 @@ def oracle_time_queries(case, layer, queries, threads=0):
     t1 = time.perf_counter()
     kp, vp, bt2 = _gather_kv(case, layer, queries, r["sel"])
     t2 = time.perf_counter()
-    r2 = oracle.run(q, qi, kp, vp, mini_idx[:1], bt2, qs, qp, sel_in=r["sel"], threads=threads)
+    own_row = np.arange(len(queries), dtype=np.int32)     # bt2 has one row per query
+    r2 = oracle.run(q, qi, kp, vp, mini_idx[:1], bt2, own_row, qp, sel_in=r["sel"], threads=threads)
     t3 = time.perf_counter()
     return (t1 - t0) + (t3 - t2), r["threads"], r2
 
@@ -495,7 +636,7 @@ def run_reference(args):
         case = workloads.long_decode(device=dev, seed=args.seed, n_layers=1)
     else:
         case = build_workload(name, dev, args.seed)
-    queries = list(range(case.n_q))
+    queries = list(range(min(case.n_q, 128)))     # a bounded sample per step
     for _ in range(args.warmup):
         oracle_time_queries(case, 0, queries[:1])
     secs, threads = [], 1
@@ -522,7 +663,8 @@ def main():
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", default="uocr", choices=["uocr", "reference"])
     ap.add_argument("--workload", default="long_decode",
-                    choices=["long_decode", "batched_decode", "tiny_decode", "ragged_paged_decode"])
+                    choices=["long_decode", "batched_decode", "tiny_decode", "ragged_paged_decode",
+                             "chunked_prefill"])
     ap.add_argument("--seed", type=int, default=0)
     ap.add_argument("--batch", type=int, default=None, help="long_decode only: sequences (default 16)")
     ap.add_argument("--layers", type=int, default=None, help="long_decode only: layer caches (default 12)")
@@ -533,6 +675,8 @@ def main():
         print("note: fewer than 3 warm-up steps", file=sys.stderr)
     if args.impl == "reference":
         run_reference(args)
+    elif args.workload == "chunked_prefill":
+        run_prefill(args)
     else:
         run_uocr(args)
 

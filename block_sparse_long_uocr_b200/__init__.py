@@ -67,6 +67,8 @@ def _load() -> ctypes.CDLL:
     lib.uocr_sparse_attn.restype = I
     lib.uocr_sparse_decode.argtypes = [P, P, P, P, P, P, P, I, I, I, I, P, P, P, Z, P, P]
     lib.uocr_sparse_decode.restype = I
+    lib.uocr_prefill_workspace_bytes.argtypes = [I, I, I]
+    lib.uocr_prefill_workspace_bytes.restype = Z
     lib.uocr_prefill_index_score.argtypes = [P, P, P, P, I, P, I, I, I, I, P, P, P]
     lib.uocr_prefill_index_score.restype = I
     lib.uocr_sparse_prefill.argtypes = [P, P, P, P, P, P, P, I, P, I, I, I, I, I, P, P, P, Z, P, P]
@@ -127,6 +129,15 @@ def _stream(stream) -> ctypes.c_void_p:
 
 def workspace_bytes(n_q: int, heads: int, max_blocks: int) -> int:
     return int(_lib().uocr_workspace_bytes(int(n_q), int(heads), int(max_blocks)))
+
+
+def prefill_workspace_bytes(n_q: int, heads: int, max_blocks: int) -> int:
+    return int(_lib().uocr_prefill_workspace_bytes(int(n_q), int(heads), int(max_blocks)))
+
+
+def alloc_prefill_workspace(n_q: int, heads: int, max_blocks: int, device) -> torch.Tensor:
+    """uint8 workspace for sparse_prefill; its first n_q*max_blocks*4 bytes hold the block scores."""
+    return torch.empty(max(prefill_workspace_bytes(n_q, heads, max_blocks), 1), dtype=torch.uint8, device=device)
 
 
 def alloc_workspace(n_q: int, heads: int, max_blocks: int, device) -> torch.Tensor:
@@ -246,7 +257,7 @@ def sparse_prefill(q, k_cache, v_cache, idx_q, idx_k_cache, block_table, seq_len
     if sel is None:
         sel = torch.empty((n_q, N_SEL), dtype=torch.int32, device=q.device)
     if workspace is None:
-        workspace = alloc_workspace(n_q, H, mb, q.device)
+        workspace = alloc_prefill_workspace(n_q, H, mb, q.device)
     _check("uocr_sparse_prefill", _lib().uocr_sparse_prefill(
         _ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(idx_q), _ptr(idx_k_cache), _ptr(block_table), _ptr(seq_lens),
         int(seq), _ptr(q_pos), n_q, B, H, mb, k_cache.shape[0], _ptr(out), _ptr(sel), _ptr(workspace),

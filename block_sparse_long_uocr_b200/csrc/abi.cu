@@ -189,6 +189,11 @@ uocr_status_t uocr_prefill_index_score(const void *idx_q, const void *idx_k_cach
                                                        dev_err));
 }
 
+size_t uocr_prefill_workspace_bytes(int n_q, int H, int max_blocks) {
+    if (n_q <= 0 || H <= 0 || max_blocks <= 0) return 0;
+    return ws_layout(n_q, H, max_blocks).total + uocr::prefill_attn_workspace(n_q, H, max_blocks, nullptr);
+}
+
 uocr_status_t uocr_sparse_prefill(const void *q, const void *k_cache, const void *v_cache, const void *idx_q,
                                   const void *idx_k_cache, const int32_t *block_table, const int32_t *seq_lens,
                                   int seq, const int32_t *q_pos, int n_q, int B, int H, int max_blocks,
@@ -203,21 +208,28 @@ uocr_status_t uocr_sparse_prefill(const void *q, const void *k_cache, const void
     if (seq < 0 || seq >= B) return UOCR_ERR_INVALID_ARG;
     if (H < 1 || H > UOCR_MAX_HEADS) return UOCR_ERR_UNSUPPORTED;
     if (n_q == 0) return UOCR_OK;
+    if ((long long)n_q * UOCR_N_SEL > 0x7fffffffLL || (long long)n_q * H > 0x7fffffffLL) return UOCR_ERR_UNSUPPORTED;
     const WsLayout w = ws_layout(n_q, H, max_blocks);
-    if (!workspace || !aligned(workspace, kWsAlign) || workspace_bytes < w.total) return UOCR_ERR_WORKSPACE;
+    if (!workspace || !aligned(workspace, kWsAlign) || workspace_bytes < uocr_prefill_workspace_bytes(n_q, H, max_blocks))
+        return UOCR_ERR_WORKSPACE;
     uocr::LaunchCtx c;
     if ((st = make_ctx(stream, false, c)) != UOCR_OK) return st;
     float *scores = (float *)((char *)workspace + w.scores_off);
-    cudaError_t e = uocr::launch_prefill_index_gemm(c, idx_q, idx_k_cache, block_table + (size_t)seq * max_blocks,
-                                                    seq_lens + seq, q_pos, n_q, max_blocks, num_pages, scores,
-                                                    dev_err);
+    char *attn_ws = (char *)workspace + w.total;
+    uocr::PrefillAttnWs aw;
+    uocr::prefill_attn_workspace(n_q, H, max_blocks, &aw);
+    cudaError_t e = cudaMemsetAsync(attn_ws + aw.counts_off, 0, (size_t)max_blocks * sizeof(int32_t), c.stream);
+    if (e != cudaSuccess) return cuda_status(e);
+    const int32_t *bt_row = block_table + (size_t)seq * max_blocks;
+    e = uocr::launch_prefill_index_gemm(c, idx_q, idx_k_cache, bt_row, seq_lens + seq, q_pos, n_q, max_blocks,
+                                        num_pages, scores, dev_err);
     if (e != cudaSuccess) return cuda_status(e);
     c.pdl = true;
     e = uocr::launch_block_topk(c, scores, seq_lens, nullptr, q_pos, n_q, B, max_blocks, sel_out, dev_err, seq);
     if (e != cudaSuccess) return cuda_status(e);
     const float scale = 1.0f / sqrtf((float)UOCR_HEAD_DIM);
-    e = uocr::launch_sparse_attn(c, q, k_cache, v_cache, block_table, seq_lens, nullptr, q_pos, sel_out, n_q, B, H,
-                                 max_blocks, num_pages, scale, out, true, seq, true, dev_err);
+    e = uocr::launch_prefill_attn(c, q, k_cache, v_cache, bt_row, q_pos, sel_out, n_q, H, max_blocks, num_pages,
+                                  scale, out, attn_ws, dev_err);
     return cuda_status(e);
 }
 

@@ -37,4 +37,16 @@ cudaError_t launch_prefill_index_gemm(const LaunchCtx &c, const void *idx_q, con
                                       const int32_t *bt_row, const int32_t *seq_len_ptr, const int32_t *q_pos,
                                       int n_q, int max_blocks, int num_pages, float *scores, int32_t *dev_err);
 
+// Block-centric prefill attention (selection inverted per block, one CTA per (block, head),
+// per-slot partials merged per (query, head)).  Workspace regions, 256-byte aligned.
+struct PrefillAttnWs {
+    size_t counts_off, offsets_off, cursor_off, list_off, ml_off, acc_off;
+};
+size_t prefill_attn_workspace(int n_q, int H, int max_blocks, PrefillAttnWs *w);
+// `ws` must start with max_blocks zeroed int32 counts (the caller clears them).
+cudaError_t launch_prefill_attn(const LaunchCtx &c, const void *q, const void *k, const void *v,
+                                const int32_t *bt_row, const int32_t *q_pos, const int32_t *sel, int n_q, int H,
+                                int max_blocks, int num_pages, float scale, void *out, void *ws,
+                                int32_t *dev_err);
+
 }  // namespace uocr

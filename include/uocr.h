@@ -190,8 +190,15 @@ uocr_status_t uocr_prefill_index_score(const void *idx_q, const void *idx_k_cach
  * uocr_prefill_index_score -> uocr_block_topk -> uocr_sparse_attn with
  * scale = 1/sqrt(128), launched back to back on `stream`.  Each query selects
  * its own 4 local + 12 remote blocks over its causal prefix.  out [n_q][H][128]
- * bf16, sel_out [n_q][16].  Workspace: uocr_workspace_bytes(n_q, H, max_blocks).
+ * bf16, sel_out [n_q][16].  The attention is block-centric: the selection is
+ * inverted per block and every selected (block, head) K/V tile is read once
+ * for all the queries that chose it, with per-slot partial softmax states
+ * merged per query.  Workspace: uocr_prefill_workspace_bytes(n_q, H, max_blocks)
+ * bytes (the block scores first, then the inverted index and the partials).
  */
+/* Workspace bytes uocr_sparse_prefill needs; a pure function of the shapes. */
+size_t uocr_prefill_workspace_bytes(int n_q, int H, int max_blocks);
+
 uocr_status_t uocr_sparse_prefill(const void *q, const void *k_cache, const void *v_cache,
                                   const void *idx_q, const void *idx_k_cache,
                                   const int32_t *block_table, const int32_t *seq_lens,

@@ -203,3 +203,13 @@ def test_sparse_prefill_rejects(pkg, over, code):
                                      a["q_pos"], a["n_q"], a["B"], a["H"], a["mb"], a["P"], a["out"], a["sel"],
                                      a["ws"], a["wsb"], None, None)
     assert st == code
+
+
+def test_prefill_workspace_is_a_pure_function_of_shapes(pkg):
+    pw, ws = pkg.prefill_workspace_bytes, pkg.workspace_bytes
+    assert pw(0, 10, 64) == 0 and pw(4, 0, 64) == 0 and pw(4, 10, 0) == 0
+    a = pw(2048, 10, 2048)
+    assert a == pw(2048, 10, 2048) and a % 256 == 0
+    # scores, then the inverted index (3 x max_blocks + 16 n_q ints) and 16 partial states per (query, head)
+    assert a >= ws(2048, 10, 2048) + 2048 * 10 * 16 * 130 * 4 + 2048 * 16 * 4 + 3 * 2048 * 4
+    assert pw(2048, 1, 2048) < a and pw(4096, 10, 2048) > a

@@ -100,7 +100,7 @@ def test_prefill_flags_bad_positions_and_pages(uocr, cuda_device):
 @pytest.mark.slow
 def test_chunked_prefill_workload_sampled(uocr, cuda_device):
     case = workloads.chunked_prefill(device=cuda_device)
-    ws = uocr.alloc_workspace(case.n_q, 10, case.max_blocks, cuda_device)
+    ws = uocr.alloc_prefill_workspace(case.n_q, 10, case.max_blocks, cuda_device)
     out, sel = uocr.sparse_prefill(case.q, case.k_pool, case.v_pool, case.idx_q, case.idx_k_pool, case.block_table,
                                    case.seq_lens, 0, case.q_pos, workspace=ws)
     torch.cuda.synchronize()
