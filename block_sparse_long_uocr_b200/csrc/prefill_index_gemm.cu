@@ -7,16 +7,18 @@
 // maximum of the walk-through (news.rkmt.cn/news/25027, section 五 step 2):
 //   scores[i][j] = max_{t in block j, t <= p_i} S[i][t].
 //
-// Kernel (persistent, one CTA per SM, 192 threads, warp-specialised):
-//   warp 4  TMA producer: per work unit the 128-query A tile (two 64-dim halves,
+// Kernel (persistent, one CTA per SM, 320 threads, warp-specialised):
+//   warp 8  TMA producer: per work unit the 128-query A tile (two 64-dim halves,
 //           128-byte swizzle) into a 2-deep ring, and per 256-token N tile the
 //           8 pages' indexer keys (16 boxes of 32 tokens x 64 dims, gathered
 //           through the block table) into a 2-stage ring;
-//   warp 5  MMA issuer: allocates 512 TMEM columns (two 128 x 256 fp32
+//   warp 9  MMA issuer: allocates 512 TMEM columns (two 128 x 256 fp32
 //           accumulators) and issues 8 tcgen05.mma (M=128, N=256, K=16) per tile;
-//   warps 0-3 epilogue: tcgen05.ld of the accumulator (warp w owns rows
-//           32w .. 32w+31 = TMEM lanes), causal mask, max over each 32-column
-//           block, fp32 scores to global memory.
+//   warps 0-7 epilogue: tcgen05.ld of the accumulator (warp w owns rows
+//           32(w%4) .. +31 = its TMEM lane quarter, and blocks 4(w/4) .. +3 of
+//           the tile), max over each 32-column block (the causal mask only on
+//           tiles that reach past the row's position), fp32 scores to global
+//           memory, four at a time.
 // Work unit = (128-query tile, chunk of 4 N tiles); units whose tokens all lie
 // past the tile's last query are skipped.  Every mbarrier wait is bounded in
 // wall time: on timeout the CTA reports UOCR_DEVERR_TIMEOUT, every role stops
@@ -42,10 +44,10 @@ constexpr int kStagesA = 2;
 constexpr int kHalfBytesA = kBM * 128;    // one 64-dim half of an A tile: 16 KiB
 constexpr int kHalfBytesB = kBN * 128;    // one 64-dim half of a B tile: 32 KiB
 constexpr int kBoxBytesB = kBlock * 128;  // one page x 64 dims: 4 KiB
-constexpr int kThreads = 192;
-constexpr int kEpiWarps = 4;
-constexpr int kProducerWarp = 4;
-constexpr int kMmaWarp = 5;
+constexpr int kEpiWarps = 8;             // two warps per TMEM lane quarter, 4 blocks of a tile each
+constexpr int kProducerWarp = 8;
+constexpr int kMmaWarp = 9;
+constexpr int kThreads = 320;
 constexpr uint64_t kTimeoutNs = 2000000000ull;   // 2 s: far above any legitimate wait
 
 struct __align__(1024) Smem {
@@ -256,14 +258,16 @@ prefill_index_gemm_kernel(const __grid_constant__ CUtensorMap map_q, const __gri
         }
         __syncwarp();
     } else {
-        // ------------------------------------------------------------ epilogue, warps 0..3
+        // ------------------------------------------------------------ epilogue, warps 0..7
+        const int quarter = warp & 3;            // TMEM lane quarter = rows 32q .. 32q+31
+        const int half = warp >> 2;              // blocks 4*half .. 4*half+3 of each tile
         int it = 0;
         bool stop = false;
         for (int u = blockIdx.x; u < n_units && !stop; u += gridDim.x) {
             const UnitInfo w = unit_info(u, n_chunks, q_pos, n_q, seq_len_ok, lane);
             if (w.ntiles == 0) continue;
-            const int row = w.m0 + warp * 32 + lane;
-            if (row < n_q) {
+            const int row = w.m0 + quarter * 32 + lane;
+            if (row < n_q && half == 0) {
                 const int p_raw = __ldg(q_pos + row);
                 if (p_raw >= seq_len && w.t0 == 0) flag_error(dev_err, UOCR_DEVERR_POS);
             }
@@ -278,18 +282,39 @@ prefill_index_gemm_kernel(const __grid_constant__ CUtensorMap map_q, const __gri
                 }
                 tc::fence_after_sync();
                 const int tile = w.t0 + t;
-                float best[kPagesPerTile];
-                const uint32_t tbase = tmem + ((uint32_t)(warp * 32) << 16) + (uint32_t)(acc * kBN);
+                const int j0 = tile * kPagesPerTile + half * 4;          // first block of this warp
+                const bool interior = (j0 + 4) * kBlock - 1 <= p;        // no masking needed
+                float best[4];
+                const uint32_t tbase =
+                    tmem + ((uint32_t)(quarter * 32) << 16) + (uint32_t)(acc * kBN + half * 4 * kBlock);
 #pragma unroll
-                for (int k = 0; k < kPagesPerTile; ++k) {
-                    float v[32];
-                    tc::tmem_ld_32x32b_x32(tbase + k * 32, v);
+                for (int k = 0; k < 4; k += 2) {
+                    float v0[32], v1[32];
+                    tc::tmem_ld_32x32b_x32(tbase + k * 32, v0);
+                    tc::tmem_ld_32x32b_x32(tbase + (k + 1) * 32, v1);
                     tc::tmem_ld_wait();
-                    const int tok0 = (tile * kPagesPerTile + k) * kBlock;
-                    float m = -INFINITY;
+                    if (interior) {
 #pragma unroll
-                    for (int c = 0; c < 32; ++c) m = (tok0 + c <= p) ? fmaxf(m, v[c]) : m;
-                    best[k] = m;
+                        for (int c = 16; c > 0; c >>= 1) {
+#pragma unroll
+                            for (int x = 0; x < c; ++x) {
+                                v0[x] = fmaxf(v0[x], v0[x + c]);
+                                v1[x] = fmaxf(v1[x], v1[x + c]);
+                            }
+                        }
+                        best[k] = v0[0];
+                        best[k + 1] = v1[0];
+                    } else {
+                        const int t0 = (j0 + k) * kBlock, t1 = t0 + kBlock;
+                        float m0 = -INFINITY, m1 = -INFINITY;
+#pragma unroll
+                        for (int c = 0; c < 32; ++c) {
+                            m0 = (t0 + c <= p) ? fmaxf(m0, v0[c]) : m0;
+                            m1 = (t1 + c <= p) ? fmaxf(m1, v1[c]) : m1;
+                        }
+                        best[k] = m0;
+                        best[k + 1] = m1;
+                    }
                 }
                 tc::fence_before_sync();
                 __syncwarp();
@@ -298,14 +323,18 @@ prefill_index_gemm_kernel(const __grid_constant__ CUtensorMap map_q, const __gri
                                  : "memory");
                 // a block whose page is not in the pool scores -inf; blocks past the row's
                 // causal range are not written
-                const int j0 = tile * kPagesPerTile;
+                int pg[4];
 #pragma unroll
-                for (int k = 0; k < kPagesPerTile; ++k) {
-                    const int j = j0 + k;
-                    if (j < nb_row) {
-                        const int page = __ldg(bt_row + j);
-                        srow[j] = ((unsigned)page < (unsigned)num_pages) ? best[k] : -INFINITY;
-                    }
+                for (int k = 0; k < 4; ++k) pg[k] = (j0 + k < nb_row) ? __ldg(bt_row + j0 + k) : -1;
+#pragma unroll
+                for (int k = 0; k < 4; ++k)
+                    if ((unsigned)pg[k] >= (unsigned)num_pages) best[k] = -INFINITY;
+                if (j0 + 4 <= nb_row && (reinterpret_cast<uintptr_t>(srow + j0) & 15u) == 0) {
+                    *reinterpret_cast<float4 *>(srow + j0) = make_float4(best[0], best[1], best[2], best[3]);
+                } else {
+#pragma unroll
+                    for (int k = 0; k < 4; ++k)
+                        if (j0 + k < nb_row) srow[j0 + k] = best[k];
                 }
             }
         }
