@@ -319,6 +319,27 @@ def run_uocr(args):
                                                             case.layers[l][1], case.q_layers[l][1],
                                                             case.layers[l][2], case.block_table, case.seq_lens,
                                                             out=outs[l], sel=sels[l], workspace=ws, stream=st))
+    comparators = None
+    if args.workload == "long_decode" and not args.no_comparators:
+        # the baselines the pages quote per decode step: full causal attention, and R-SWA read as a
+        # reference prefix of 80 % of the context plus the 128-token window (the pages' 7.0x / 5.6x
+        # ratios imply R-SWA reads 5.6 / 7.0 = 0.8 of what full attention reads)
+        dws = torch.empty(uocr.dense_workspace_bytes(B, H, mb), dtype=torch.uint8, device=dev)
+        ref_blocks = int(0.8 * mb)
+        full_ms = graph_time(lambda l, st: uocr.dense_decode(case.q_layers[l][0], case.layers[l][0], case.layers[l][1],
+                                                             case.block_table, case.seq_lens, out=outs[l],
+                                                             workspace=dws, stream=st))
+        rswa_ms = graph_time(lambda l, st: uocr.dense_decode(case.q_layers[l][0], case.layers[l][0], case.layers[l][1],
+                                                             case.block_table, case.seq_lens, ref_blocks=ref_blocks,
+                                                             out=outs[l], workspace=dws, stream=st))
+        comparators = {"full_attention_us": round(1e3 * full_ms, 2), "rswa_us": round(1e3 * rswa_ms, 2),
+                       "sparse_decode_us": round(1e3 * decode_ms, 2),
+                       "speedup_vs_full": round(full_ms / decode_ms, 2), "speedup_vs_rswa": round(rswa_ms / decode_ms, 2),
+                       "pages_claim": {"vs_full": 7.0, "vs_rswa": 5.6},
+                       "rswa_reading": f"reference prefix {ref_blocks} of {mb} blocks + 4-block window",
+                       "full_gbs": round(B * 5120 * int(case.seq_lens[0]) / (full_ms / 1e3) / 1e9, 1)}
+        for o in outs:
+            o.zero_()
     peaks, peak_kind = measured_peaks()
     peak = float(peaks.get("hbm_gbs", FALLBACK_HBM_GBS))
     scan_gbs = scan_bytes_call / (scan_ms / 1e3) / 1e9
@@ -351,6 +372,7 @@ def run_uocr(args):
                          "decode_call_eager": round(1e3 * ms_per_step / n_layers, 2),
                          "note": "device time per launch from CUDA-graph replays of each entry point alone; "
                                  "the decode call chains the three with programmatic dependent launch"},
+        "comparators": comparators,
         "e2e": e2e,
         "gpu_launches": args.steps * n_layers * 3,
         "clocks": clocks,
@@ -669,6 +691,7 @@ def main():
     ap.add_argument("--batch", type=int, default=None, help="long_decode only: sequences (default 16)")
     ap.add_argument("--layers", type=int, default=None, help="long_decode only: layer caches (default 12)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-comparators", action="store_true", help="skip the full-attention / R-SWA timings")
     ap.add_argument("--cpu-budget", type=float, default=10.0)
     args = ap.parse_args()
     if args.warmup < 3 and args.impl == "uocr":

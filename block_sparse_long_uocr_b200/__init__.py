@@ -15,6 +15,8 @@ Entry points (same names as the C ABI, without the ``uocr_`` prefix):
 * :func:`sparse_decode` -- the three fused into one decode call;
 * :func:`prefill_index_score` -- the block scores of a prefill chunk on the tcgen05 tensor cores;
 * :func:`sparse_prefill` -- tensor-core scoring, selection and attention for a prefill chunk;
+* :func:`dense_decode` -- comparator: full causal attention, or an R-SWA-style reference
+  prefix plus the 128-token window (the baselines the sparse step is measured against);
 * :func:`sparse_decode_static` -- the same decode call for callers that cannot
   allocate device memory (scratch held inside the library);
 * :func:`workspace_bytes`.
@@ -67,6 +69,10 @@ def _load() -> ctypes.CDLL:
     lib.uocr_sparse_attn.restype = I
     lib.uocr_sparse_decode.argtypes = [P, P, P, P, P, P, P, I, I, I, I, P, P, P, Z, P, P]
     lib.uocr_sparse_decode.restype = I
+    lib.uocr_dense_workspace_bytes.argtypes = [I, I, I]
+    lib.uocr_dense_workspace_bytes.restype = Z
+    lib.uocr_dense_decode.argtypes = [P, P, P, P, P, I, I, I, I, I, P, P, Z, P, P]
+    lib.uocr_dense_decode.restype = I
     lib.uocr_prefill_workspace_bytes.argtypes = [I, I, I]
     lib.uocr_prefill_workspace_bytes.restype = Z
     lib.uocr_prefill_index_score.argtypes = [P, P, P, P, I, P, I, I, I, I, P, P, P]
@@ -263,6 +269,31 @@ def sparse_prefill(q, k_cache, v_cache, idx_q, idx_k_cache, block_table, seq_len
         int(seq), _ptr(q_pos), n_q, B, H, mb, k_cache.shape[0], _ptr(out), _ptr(sel), _ptr(workspace),
         workspace.numel(), _ptr(dev_err), _stream(stream)))
     return out, sel
+
+
+def dense_workspace_bytes(n_q: int, heads: int, max_blocks: int) -> int:
+    return int(_lib().uocr_dense_workspace_bytes(int(n_q), int(heads), int(max_blocks)))
+
+
+def dense_decode(q, k_cache, v_cache, block_table, seq_lens, *, ref_blocks: int | None = None,
+                 out=None, workspace=None, dev_err=None, stream=None) -> torch.Tensor:
+    """Decode attention over blocks [0, ref_blocks) plus the 4-block local window (all blocks when
+    ref_blocks is None: full causal attention).  Returns out [B,H,128] bf16."""
+    for t, n, dt, nd in ((q, "q", torch.bfloat16, 3), (k_cache, "k_cache", torch.bfloat16, 4),
+                         (v_cache, "v_cache", torch.bfloat16, 4), (block_table, "block_table", torch.int32, 2),
+                         (seq_lens, "seq_lens", torch.int32, 1)):
+        _dev(t, n, dt, nd)
+    B, H = q.shape[0], q.shape[1]
+    mb = block_table.shape[1]
+    rb = mb if ref_blocks is None else int(ref_blocks)
+    if out is None:
+        out = torch.empty_like(q)
+    if workspace is None:
+        workspace = torch.empty(max(dense_workspace_bytes(B, H, mb), 1), dtype=torch.uint8, device=q.device)
+    _check("uocr_dense_decode", _lib().uocr_dense_decode(
+        _ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(block_table), _ptr(seq_lens), rb, B, H, mb, k_cache.shape[0],
+        _ptr(out), _ptr(workspace), workspace.numel(), _ptr(dev_err), _stream(stream)))
+    return out
 
 
 STATIC_SCRATCH_BYTES = 8 << 20   # UOCR_STATIC_SCRATCH_BYTES

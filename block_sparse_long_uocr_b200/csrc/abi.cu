@@ -233,4 +233,27 @@ uocr_status_t uocr_sparse_prefill(const void *q, const void *k_cache, const void
     return cuda_status(e);
 }
 
+size_t uocr_dense_workspace_bytes(int B, int H, int max_blocks) {
+    if (B <= 0 || H <= 0 || max_blocks <= 0) return 0;
+    return uocr::dense_attn_workspace(B, H, max_blocks);
+}
+
+uocr_status_t uocr_dense_decode(const void *q, const void *k_cache, const void *v_cache, const int32_t *block_table,
+                                const int32_t *seq_lens, int ref_blocks, int B, int H, int max_blocks, int num_pages,
+                                void *out, void *workspace, size_t workspace_bytes, int32_t *dev_err,
+                                uocr_stream_t stream) {
+    uocr_status_t st = check_common(B, B, max_blocks, num_pages, block_table, seq_lens, nullptr, nullptr, dev_err);
+    if (st != UOCR_OK) return st;
+    if (!bf16_ok(q) || !bf16_ok(k_cache) || !bf16_ok(v_cache) || !bf16_ok(out)) return UOCR_ERR_INVALID_ARG;
+    if (ref_blocks < 0) return UOCR_ERR_INVALID_ARG;
+    if (H < 1 || H > UOCR_MAX_HEADS) return UOCR_ERR_UNSUPPORTED;
+    if (!workspace || !aligned(workspace, kWsAlign) || workspace_bytes < uocr_dense_workspace_bytes(B, H, max_blocks))
+        return UOCR_ERR_WORKSPACE;
+    uocr::LaunchCtx c;
+    if ((st = make_ctx(stream, false, c)) != UOCR_OK) return st;
+    const float scale = 1.0f / sqrtf((float)UOCR_HEAD_DIM);
+    return cuda_status(uocr::launch_dense_attn(c, q, k_cache, v_cache, block_table, seq_lens, B, H, max_blocks,
+                                               num_pages, ref_blocks, scale, out, workspace, dev_err));
+}
+
 }  // extern "C"

@@ -49,4 +49,11 @@ cudaError_t launch_prefill_attn(const LaunchCtx &c, const void *q, const void *k
                                 int max_blocks, int num_pages, float scale, void *out, void *ws,
                                 int32_t *dev_err);
 
+// Comparator decode attention over [0, min(ref_blocks, nb)) U the 4-block local window.
+int dense_chunks(int max_blocks);
+size_t dense_attn_workspace(int n_q, int H, int max_blocks);
+cudaError_t launch_dense_attn(const LaunchCtx &c, const void *q, const void *k, const void *v, const int32_t *bt,
+                              const int32_t *seq_lens, int B, int H, int max_blocks, int num_pages, int ref_blocks,
+                              float scale, void *out, void *ws, int32_t *dev_err);
+
 }  // namespace uocr

@@ -208,6 +208,24 @@ uocr_status_t uocr_sparse_prefill(const void *q, const void *k_cache, const void
                                   int32_t *dev_err, uocr_stream_t stream);
 
 /*
+ * Comparator decode attention (baselines the pages quote the sparse step
+ * against: full attention and R-SWA; release report, leheavengame.com, section
+ * 一: 7.0x and 5.6x; R-SWA: Unlimited OCR v1 article, chenxutan.com/d/4261.html,
+ * section 2.3.2).  For each sequence's decode query (p = seq_len - 1), exact
+ * softmax attention (scale 1/sqrt(128)) over the tokens t <= p of the blocks
+ *   [0, min(ref_blocks, nb))  U  [max(nb - 4, 0), nb)
+ * i.e. a reference prefix plus the 128-token local window; ref_blocks >=
+ * max_blocks gives full causal attention.  Split-K over 16-block chunks with a
+ * merge kernel.  Workspace: uocr_dense_workspace_bytes(B, H, max_blocks).
+ */
+size_t uocr_dense_workspace_bytes(int B, int H, int max_blocks);
+uocr_status_t uocr_dense_decode(const void *q, const void *k_cache, const void *v_cache,
+                                const int32_t *block_table, const int32_t *seq_lens, int ref_blocks,
+                                int B, int H, int max_blocks, int num_pages, void *out,
+                                void *workspace, size_t workspace_bytes, int32_t *dev_err,
+                                uocr_stream_t stream);
+
+/*
  * uocr_sparse_decode_static -- uocr_sparse_decode for callers that cannot
  * allocate device memory (for example a plugin inside a host engine that owns
  * every device allocation, or a decode loop where a cudaMalloc, which may
