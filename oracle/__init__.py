@@ -14,7 +14,11 @@ cites the page section its C function follows:
 * [rkmt 五 step 3], [lqnn 显存账本] 4 local blocks + top-12 remote blocks
   (www.lqnn.cn/news/271890, section 显存账本);
 * [rkmt 五 step 4], [chenxutan 2.3.2] exact softmax attention over the selected
-  tokens (chenxutan.com/d/4261.html, section 2.3.2, scaled dot product).
+  tokens (chenxutan.com/d/4261.html, section 2.3.2, scaled dot product);
+* [rkmt 四], [rkmt 六] page2d rotary embedding (63 frequency pairs on the in-page
+  token offset, theta 10000, resampled over the full spectrum; 1 pair on the
+  page coordinate page % 2, theta 256) applied before the new token's keys are
+  appended to the paged caches.
 
 Parity status: pinned (tests/test_oracle_pins.py).
 """
@@ -42,6 +46,11 @@ HEADS = 10          # num_attention_heads = num_key_value_heads (MHA)
 HEAD_DIM = 128
 IDX_DIM = 128       # one indexer head of 128 dims
 TIE_EPS = 1e-3      # near-tie band on the 12th/13th remote score gap
+# page2d rotary embedding ([rkmt 四], [rkmt 六]): 1 of the 64 frequency pairs on the page axis
+ROPE_PAGE_PAIRS = 1     # sparse_rope_page_pairs
+ROPE_THETA_TOK = 10000.0
+ROPE_THETA_PAGE = 256.0
+ROPE_PAGE_MOD = 2       # sparse_rope_page_mod: page coordinate = page % 2
 
 
 def build(force: bool = False) -> str:
@@ -76,6 +85,9 @@ def _load():
         lib.uocr_oracle_run.argtypes = ([I, P, P, P, P, P, P, P, P] + [I] * 7
                                         + [Dd, Dd, P, P, P, P, P, I])
         lib.uocr_oracle_run.restype = I
+        L = ctypes.c_longlong
+        lib.uocr_oracle_rope_page2d.argtypes = [P, I, I, Dd, Dd, I, L, L, P]
+        lib.uocr_oracle_rope_page2d.restype = None
         _lib = lib
     return _lib
 
@@ -189,3 +201,50 @@ def run(q, idx_q, k_pool, v_pool, idx_k_pool, block_table, q_seq, q_pos, *,
         sc, float(tie_eps), _ptr(si), _ptr(scores), _ptr(sel), _ptr(tie), _ptr(out), int(threads))
     return {"scores": scores, "sel": sel, "near_tie": None if tie is None else tie.astype(bool),
             "out": out, "threads": int(used)}
+
+
+# --------------------------------------------------------------------------- page2d rotary + cache append
+def rope_page2d(x, tok: int, page: int, *, page_pairs: int = ROPE_PAGE_PAIRS, theta_tok: float = ROPE_THETA_TOK,
+                theta_page: float = ROPE_THETA_PAGE, page_mod: int = ROPE_PAGE_MOD) -> np.ndarray:
+    """[rkmt 四] fp64 page2d rotation of one bf16 vector (last dim = 2 * pairs) -> float64 array."""
+    xb = bits(x).reshape(-1)
+    n_pairs = xb.shape[0] // 2
+    out = np.empty(2 * n_pairs, dtype=np.float64)
+    _load().uocr_oracle_rope_page2d(_ptr(xb), int(n_pairs), int(page_pairs), float(theta_tok), float(theta_page),
+                                    int(page_mod), int(tok), int(page), _ptr(out))
+    return out
+
+
+def rope_append(q, idx_q, k_new, v_new, idx_k_new, tok_pos, page_pos, seqs, positions, block_table,
+                k_cache, v_cache, idx_k_cache):
+    """The step before the scan, for n new tokens: rotate q, idx_q, k_new, idx_k_new with page2d and
+    write k, v, idx_k of token i into the caches at (sequence seqs[i], position positions[i]).
+    Returns (q_rot, idx_q_rot, k_cache, v_cache, idx_k_cache) as float64 arrays (caches copied)."""
+    qb, qib = bits(q), bits(idx_q)
+    kb, vb, ikb = bits(k_new), bits(v_new), bits(idx_k_new)
+    tp, pp = ints(tok_pos).reshape(-1), ints(page_pos).reshape(-1)
+    sq, ps = ints(seqs).reshape(-1), ints(positions).reshape(-1)
+    bt = ints(block_table)
+    kc = bits(k_cache).astype(np.uint32)
+    n, H = qb.shape[0], qb.shape[1]
+    blk = kc.shape[2]
+
+    def widen(a):
+        return (a.astype(np.uint32) << 16).view(np.float32).astype(np.float64)
+
+    kcache, vcache, icache = widen(bits(k_cache)), widen(bits(v_cache)), widen(bits(idx_k_cache))
+    q_rot = np.empty(qb.shape, np.float64)
+    qi_rot = np.empty(qib.shape, np.float64)
+    for i in range(n):
+        t, g = int(tp[i]), int(pp[i])
+        for h in range(H):
+            q_rot[i, h] = rope_page2d(qb[i, h], t, g)
+        qi_rot[i] = rope_page2d(qib[i], t, g)
+        page = int(bt[sq[i], ps[i] // blk])
+        row = int(ps[i]) % blk
+        for h in range(H):
+            kcache[page, h, row] = rope_page2d(kb[i, h], t, g)
+            vcache[page, h, row] = widen(vb[i, h])
+        icache[page, row] = rope_page2d(ikb[i], t, g)
+    del kc
+    return q_rot, qi_rot, kcache, vcache, icache

@@ -257,3 +257,34 @@ int uocr_oracle_run(int n_q, const int32_t *q_seq, const int32_t *q_pos,
     }
     return used;
 }
+
+/*
+ * [rkmt 四 (page2d), 六] page2d rotary position embedding of one head vector
+ * (dim = 2 * n_pairs, rotate-half layout: pair i = dims i and i + n_pairs).
+ * The n_pairs frequency pairs are split between two axes: the first
+ * n_pairs - page_pairs pairs rotate by the in-page token offset `tok`, the
+ * last page_pairs pairs by the page coordinate (page mod page_mod):
+ *   angle_i = tok  * theta_tok ^ (-i / n_tok)          i <  n_tok = n_pairs - page_pairs
+ *   angle_i = pg   * theta_page^(-(i - n_tok) / page_pairs)   i >= n_tok, pg = page mod page_mod
+ *   out[i]           = x[i] cos(angle_i) - x[i + n_pairs] sin(angle_i)
+ *   out[i + n_pairs] = x[i + n_pairs] cos(angle_i) + x[i] sin(angle_i)
+ * ("resample": the n_tok token frequencies are spread over the whole spectrum
+ * of a standard rotary table of n_tok pairs.)
+ */
+void uocr_oracle_rope_page2d(const uint16_t *x, int n_pairs, int page_pairs, double theta_tok,
+                             double theta_page, int page_mod, long long tok, long long page, double *out)
+{
+    int n_tok = n_pairs - page_pairs;
+    long long pg = page_mod > 0 ? ((page % page_mod) + page_mod) % page_mod : page;
+    for (int i = 0; i < n_pairs; ++i) {
+        double angle;
+        if (i < n_tok)
+            angle = (double)tok * pow(theta_tok, -(double)i / (double)n_tok);
+        else
+            angle = (double)pg * pow(theta_page, -(double)(i - n_tok) / (double)page_pairs);
+        double c = cos(angle), s = sin(angle);
+        double a = bf16_bits_to_double(x[i]), b = bf16_bits_to_double(x[i + n_pairs]);
+        out[i] = a * c - b * s;
+        out[i + n_pairs] = b * c + a * s;
+    }
+}

@@ -310,3 +310,105 @@ def test_empty_query_gives_zero_output():
                    case.q_seq, torch.tensor([-1], dtype=torch.int32))
     assert (r["sel"] == -1).all() and (r["out"] == 0).all()
     assert np.isneginf(r["scores"]).all()
+
+
+# ----------------------------------------------------------------------------- page2d rotary
+def _rand_vec(seed, n=128):
+    return bf16(torch.randn(n, generator=torch.Generator().manual_seed(seed)))
+
+
+def test_rope_constants_match_pages():
+    g = json.load(open(GOLDEN))
+    assert oracle.ROPE_PAGE_PAIRS == g["sparse_rope_page_pairs"]["value"]
+    assert oracle.ROPE_PAGE_MOD == g["sparse_rope_page_mod"]["value"]
+    assert oracle.ROPE_THETA_TOK == g["rope_theta_token_axis"]["value"]
+    assert oracle.ROPE_THETA_PAGE == g["rope_theta_page_axis"]["value"]
+
+
+def test_rope_identity_at_origin_and_even_pages():
+    x = _rand_vec(1)
+    for page in (0, 2, 10, -4):
+        np.testing.assert_array_equal(oracle.rope_page2d(x, 0, page), x.double().numpy())
+
+
+def test_rope_is_a_rotation_of_each_pair():
+    x = _rand_vec(2).double().numpy()
+    for tok, page in [(1, 0), (37, 1), (1000, 3), (131071, 0)]:
+        y = oracle.rope_page2d(bf16(x), tok, page)
+        np.testing.assert_allclose(y[:64] ** 2 + y[64:] ** 2, x[:64] ** 2 + x[64:] ** 2, rtol=1e-12, atol=1e-12)
+
+
+def test_rope_dot_products_depend_only_on_the_token_offset():
+    """Relative-position property: <R(t1) q, R(t2) k> is unchanged when both move by the same shift."""
+    q, k = _rand_vec(3), _rand_vec(4)
+    for page in (0, 1):
+        base = oracle.rope_page2d(q, 5, page) @ oracle.rope_page2d(k, 12, page)
+        for shift in (1, 17, 300, 40000):
+            moved = oracle.rope_page2d(q, 5 + shift, page) @ oracle.rope_page2d(k, 12 + shift, page)
+            assert abs(moved - base) < 1e-9
+
+
+def test_rope_page_axis_is_page_parity():
+    x = _rand_vec(5)
+    for tok in (0, 9, 512):
+        np.testing.assert_allclose(oracle.rope_page2d(x, tok, 1), oracle.rope_page2d(x, tok, 3), rtol=0, atol=0)
+        np.testing.assert_allclose(oracle.rope_page2d(x, tok, 0), oracle.rope_page2d(x, tok, 8), rtol=0, atol=0)
+    # same page parity, different token: differ; same token, other parity: differ only in the page pair
+    a, b = oracle.rope_page2d(x, 9, 0), oracle.rope_page2d(x, 9, 1)
+    diff = np.nonzero(np.abs(a - b) > 0)[0].tolist()
+    assert diff and set(diff) <= {63, 127}
+
+
+def test_rope_highest_frequencies():
+    """Both axes start their spectrum at one radian per unit (theta ** 0): the token axis' first pair
+    turns by `tok` radians, the page pair by (page % 2) radians."""
+    e0 = torch.zeros(128)
+    e0[0] = 1.0
+    y = oracle.rope_page2d(bf16(e0), 1, 0)
+    np.testing.assert_allclose([y[0], y[64]], [np.cos(1.0), np.sin(1.0)], rtol=0, atol=1e-15)
+    e63 = torch.zeros(128)
+    e63[63] = 1.0
+    y = oracle.rope_page2d(bf16(e63), 12345, 1)
+    np.testing.assert_allclose([y[63], y[127]], [np.cos(1.0), np.sin(1.0)], rtol=0, atol=1e-15)
+
+
+def test_rope_token_spectrum_spans_theta():
+    """'resample': 63 token frequencies spread over the whole spectrum from 1 down towards 1/theta.
+    The angle of pair i after one step is recovered from the rotation of e_i and must fall
+    monotonically from 1 to between 1/theta and its 63rd root above it."""
+    angles = []
+    for i in range(63):
+        e = torch.zeros(128)
+        e[i] = 1.0
+        y = oracle.rope_page2d(bf16(e), 1, 0)
+        angles.append(np.arctan2(y[i + 64], y[i]))
+    angles = np.array(angles)
+    assert angles[0] == pytest.approx(1.0, abs=1e-15)
+    assert (np.diff(angles) < 0).all()
+    assert 1e-4 < angles[-1] <= 1e-4 * 10000 ** (1 / 63) * (1 + 1e-12)
+    ratios = angles[1:] / angles[:-1]
+    np.testing.assert_allclose(ratios, ratios[0], rtol=1e-9)        # a geometric spectrum
+
+
+def test_rope_append_writes_rotated_keys_and_raw_values():
+    case = workloads.make_case([40, 70], heads=2, shuffle=True, seed=14)
+    n, H = 2, 2
+    g = torch.Generator().manual_seed(15)
+    qn, kn, vn = (bf16(torch.randn(n, H, 128, generator=g)) for _ in range(3))
+    qin, kin = (bf16(torch.randn(n, 128, generator=g)) for _ in range(2))
+    tok, page, pos = np.array([3, 70]), np.array([0, 5]), np.array([39, 69])
+    qr, qir, kc, vc, ic = oracle.rope_append(qn, qin, kn, vn, kin, tok, page, np.array([0, 1]), pos,
+                                             case.block_table, case.k_pool, case.v_pool, case.idx_k_pool)
+    for i in range(n):
+        pg = int(case.block_table[i, pos[i] // 32])
+        r = pos[i] % 32
+        for h in range(H):
+            np.testing.assert_array_equal(kc[pg, h, r], oracle.rope_page2d(kn[i, h], tok[i], page[i]))
+            np.testing.assert_array_equal(vc[pg, h, r], vn[i, h].double().numpy())
+            np.testing.assert_array_equal(qr[i, h], oracle.rope_page2d(qn[i, h], tok[i], page[i]))
+        np.testing.assert_array_equal(ic[pg, r], oracle.rope_page2d(kin[i], tok[i], page[i]))
+    # every other cache row is untouched
+    untouched = np.ones(kc.shape[:3], bool)
+    for i in range(n):
+        untouched[int(case.block_table[i, pos[i] // 32]), :, pos[i] % 32] = False
+    np.testing.assert_array_equal(kc[untouched], case.k_pool.double().numpy()[untouched])
