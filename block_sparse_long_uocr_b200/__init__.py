@@ -15,6 +15,7 @@ Entry points (same names as the C ABI, without the ``uocr_`` prefix):
 * :func:`sparse_decode` -- the three fused into one decode call;
 * :func:`prefill_index_score` -- the block scores of a prefill chunk on the tcgen05 tensor cores;
 * :func:`sparse_prefill` -- tensor-core scoring, selection and attention for a prefill chunk;
+* :func:`rope_append` -- page2d rotary embedding of new tokens and their append to the caches;
 * :func:`dense_decode` -- comparator: full causal attention, or an R-SWA-style reference
   prefix plus the 128-token window (the baselines the sparse step is measured against);
 * :func:`sparse_decode_static` -- the same decode call for callers that cannot
@@ -69,6 +70,8 @@ def _load() -> ctypes.CDLL:
     lib.uocr_sparse_attn.restype = I
     lib.uocr_sparse_decode.argtypes = [P, P, P, P, P, P, P, I, I, I, I, P, P, P, Z, P, P]
     lib.uocr_sparse_decode.restype = I
+    lib.uocr_rope_append.argtypes = [P, P, P, P, P, P, P, P, P, P, P, I, I, I, I, I, P, P, P, P, P]
+    lib.uocr_rope_append.restype = I
     lib.uocr_dense_workspace_bytes.argtypes = [I, I, I]
     lib.uocr_dense_workspace_bytes.restype = Z
     lib.uocr_dense_decode.argtypes = [P, P, P, P, P, I, I, I, I, I, P, P, Z, P, P]
@@ -269,6 +272,27 @@ def sparse_prefill(q, k_cache, v_cache, idx_q, idx_k_cache, block_table, seq_len
         int(seq), _ptr(q_pos), n_q, B, H, mb, k_cache.shape[0], _ptr(out), _ptr(sel), _ptr(workspace),
         workspace.numel(), _ptr(dev_err), _stream(stream)))
     return out, sel
+
+
+def rope_append(q, idx_q, k_new, v_new, idx_k_new, tok_pos, page_pos, block_table, seq_lens,
+                k_cache, v_cache, idx_k_cache, q_seq=None, q_pos=None, *, dev_err=None, stream=None):
+    """Rotate q / idx_q in place (page2d) and write the new tokens' rotated k / idx_k and raw v into the
+    caches at each token's position (default: its sequence's last cached position)."""
+    for t, n, dt, nd in ((q, "q", torch.bfloat16, 3), (idx_q, "idx_q", torch.bfloat16, 2),
+                         (k_new, "k_new", torch.bfloat16, 3), (v_new, "v_new", torch.bfloat16, 3),
+                         (idx_k_new, "idx_k_new", torch.bfloat16, 2), (tok_pos, "tok_pos", torch.int32, 1),
+                         (page_pos, "page_pos", torch.int32, 1), (block_table, "block_table", torch.int32, 2),
+                         (seq_lens, "seq_lens", torch.int32, 1), (k_cache, "k_cache", torch.bfloat16, 4),
+                         (v_cache, "v_cache", torch.bfloat16, 4), (idx_k_cache, "idx_k_cache", torch.bfloat16, 3)):
+        _dev(t, n, dt, nd)
+    n, H = q.shape[0], q.shape[1]
+    B, mb = block_table.shape
+    _check("uocr_rope_append", _lib().uocr_rope_append(
+        _ptr(q), _ptr(idx_q), _ptr(k_new), _ptr(v_new), _ptr(idx_k_new), _ptr(tok_pos), _ptr(page_pos),
+        _ptr(_opt_i32(q_seq, "q_seq")), _ptr(_opt_i32(q_pos, "q_pos")), _ptr(block_table), _ptr(seq_lens),
+        n, B, H, mb, k_cache.shape[0], _ptr(k_cache), _ptr(v_cache), _ptr(idx_k_cache), _ptr(dev_err),
+        _stream(stream)))
+    return q, idx_q
 
 
 def dense_workspace_bytes(n_q: int, heads: int, max_blocks: int) -> int:

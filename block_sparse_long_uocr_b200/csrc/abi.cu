@@ -256,4 +256,24 @@ uocr_status_t uocr_dense_decode(const void *q, const void *k_cache, const void *
                                                num_pages, ref_blocks, scale, out, workspace, dev_err));
 }
 
+uocr_status_t uocr_rope_append(void *q, void *idx_q, const void *k_new, const void *v_new, const void *idx_k_new,
+                               const int32_t *tok_pos, const int32_t *page_pos, const int32_t *q_seq,
+                               const int32_t *q_pos, const int32_t *block_table, const int32_t *seq_lens, int n,
+                               int B, int H, int max_blocks, int num_pages, void *k_cache, void *v_cache,
+                               void *idx_k_cache, int32_t *dev_err, uocr_stream_t stream) {
+    uocr_status_t st = check_common(n, B, max_blocks, num_pages, block_table, seq_lens, q_seq, q_pos, dev_err);
+    if (st != UOCR_OK) return st;
+    if (!bf16_ok(q) || !bf16_ok(idx_q) || !bf16_ok(k_new) || !bf16_ok(v_new) || !bf16_ok(idx_k_new) ||
+        !bf16_ok(k_cache) || !bf16_ok(v_cache) || !bf16_ok(idx_k_cache))
+        return UOCR_ERR_INVALID_ARG;
+    if (!tok_pos || !page_pos || !aligned(tok_pos, 4) || !aligned(page_pos, 4)) return UOCR_ERR_INVALID_ARG;
+    if (H < 1 || H > UOCR_MAX_HEADS) return UOCR_ERR_UNSUPPORTED;
+    if (n == 0) return UOCR_OK;
+    uocr::LaunchCtx c;
+    if ((st = make_ctx(stream, false, c)) != UOCR_OK) return st;
+    return cuda_status(uocr::launch_rope_append(c, q, idx_q, k_new, v_new, idx_k_new, tok_pos, page_pos, q_seq,
+                                                q_pos, block_table, seq_lens, n, B, H, max_blocks, num_pages,
+                                                k_cache, v_cache, idx_k_cache, dev_err));
+}
+
 }  // extern "C"

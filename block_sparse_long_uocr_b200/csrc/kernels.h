@@ -5,6 +5,8 @@
 #include <stddef.h>
 #include <stdint.h>
 
+#include "uocr.h"
+
 namespace uocr {
 
 struct LaunchCtx {
@@ -55,5 +57,16 @@ size_t dense_attn_workspace(int n_q, int H, int max_blocks);
 cudaError_t launch_dense_attn(const LaunchCtx &c, const void *q, const void *k, const void *v, const int32_t *bt,
                               const int32_t *seq_lens, int B, int H, int max_blocks, int num_pages, int ref_blocks,
                               float scale, void *out, void *ws, int32_t *dev_err);
+
+// page2d rotary embedding + cache append of new tokens.
+struct RopeFreqs {
+    double inv[UOCR_HEAD_DIM / 2];   // per frequency pair: radians per unit of its coordinate
+};
+RopeFreqs rope_freqs();
+cudaError_t launch_rope_append(const LaunchCtx &c, void *q, void *idx_q, const void *k_new, const void *v_new,
+                               const void *idx_k_new, const int32_t *tok_pos, const int32_t *page_pos,
+                               const int32_t *q_seq, const int32_t *q_pos, const int32_t *bt,
+                               const int32_t *seq_lens, int n, int B, int H, int max_blocks, int num_pages,
+                               void *k_cache, void *v_cache, void *idx_k_cache, int32_t *dev_err);
 
 }  // namespace uocr

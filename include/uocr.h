@@ -88,6 +88,11 @@ typedef enum {
 #define UOCR_HEAD_DIM 128
 #define UOCR_IDX_DIM 128
 #define UOCR_MAX_HEADS 64
+/* page2d rotary embedding ([rkmt 四], [rkmt 六]). */
+#define UOCR_ROPE_PAGE_PAIRS 1      /* frequency pairs on the page axis (of 64) */
+#define UOCR_ROPE_PAGE_MOD 2        /* page coordinate = page % 2 */
+#define UOCR_ROPE_THETA_TOKEN 10000.0
+#define UOCR_ROPE_THETA_PAGE 256.0
 
 /* Bits OR-ed into *dev_err by the kernels. */
 #define UOCR_DEVERR_PAGE 1u   /* block-table entry outside [0, num_pages) */
@@ -206,6 +211,30 @@ uocr_status_t uocr_sparse_prefill(const void *q, const void *k_cache, const void
                                   int max_blocks, int num_pages, void *out, int32_t *sel_out,
                                   void *workspace, size_t workspace_bytes,
                                   int32_t *dev_err, uocr_stream_t stream);
+
+/*
+ * page2d rotary embedding + cache append for n new tokens, the step before the
+ * indexer scan of a decode call ([rkmt 四 page2d], [rkmt 六]).  Token i has
+ * in-page offset tok_pos[i] and page number page_pos[i]; of the 64 frequency
+ * pairs of a 128-dim head, pairs 0..62 rotate by tok * 10000^(-i/63) and pair 63
+ * by (page % 2) * 256^0, rotate-half layout (pair i = dims i and i + 64).
+ *   q [n][H][128], idx_q [n][128]      rotated in place;
+ *   k_new, v_new [n][H][128], idx_k_new [n][128]
+ *                                      rotated k / idx_k and raw v are written to
+ *                                      row p % 32 of page block_table[b][p / 32]
+ *                                      of k_cache, idx_k_cache and v_cache,
+ * for token i of sequence b = q_seq[i] (NULL: i) at position p = q_pos[i]
+ * (NULL: seq_lens[b] - 1, i.e. seq_lens already counts the new token).
+ * Angles are formed in fp64 and reduced before an fp32 sincos; outputs are
+ * rounded to bf16.  Two new tokens must not target the same cache row.
+ */
+uocr_status_t uocr_rope_append(void *q, void *idx_q, const void *k_new, const void *v_new,
+                               const void *idx_k_new, const int32_t *tok_pos, const int32_t *page_pos,
+                               const int32_t *q_seq, const int32_t *q_pos,
+                               const int32_t *block_table, const int32_t *seq_lens,
+                               int n, int B, int H, int max_blocks, int num_pages,
+                               void *k_cache, void *v_cache, void *idx_k_cache,
+                               int32_t *dev_err, uocr_stream_t stream);
 
 /*
  * Comparator decode attention (baselines the pages quote the sparse step
