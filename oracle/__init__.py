@@ -18,7 +18,9 @@ cites the page section its C function follows:
 * [rkmt 四], [rkmt 六] page2d rotary embedding (63 frequency pairs on the in-page
   token offset, theta 10000, resampled over the full spectrum; 1 pair on the
   page coordinate page % 2, theta 256) applied before the new token's keys are
-  appended to the paged caches.
+  appended to the paged caches;
+* [lqnn 显存账本], [leheaven 二] block-summary scoring (one summary vector per block)
+  and the mean-key summary; [rkmt 五] selection under a page-aware candidate mask.
 
 Parity status: pinned (tests/test_oracle_pins.py).
 """
@@ -88,6 +90,12 @@ def _load():
         L = ctypes.c_longlong
         lib.uocr_oracle_rope_page2d.argtypes = [P, I, I, Dd, Dd, I, L, L, P]
         lib.uocr_oracle_rope_page2d.restype = None
+        lib.uocr_oracle_summary_scores.argtypes = [P, P, P, I, I, I, P]
+        lib.uocr_oracle_summary_scores.restype = I
+        lib.uocr_oracle_block_mean.argtypes = [P, I, I, I, P]
+        lib.uocr_oracle_block_mean.restype = None
+        lib.uocr_oracle_select_masked.argtypes = [P, I, I, I, P, Dd, P, P]
+        lib.uocr_oracle_select_masked.restype = I
         _lib = lib
     return _lib
 
@@ -248,3 +256,36 @@ def rope_append(q, idx_q, k_new, v_new, idx_k_new, tok_pos, page_pos, seqs, posi
         icache[page, row] = rope_page2d(ikb[i], t, g)
     del kc
     return q_rot, qi_rot, kcache, vcache, icache
+
+
+# --------------------------------------------------------------------------- summary scoring, masked selection
+def summary_scores(idx_q_row, summary_pool, bt_row, p: int, blk: int = BLOCK) -> np.ndarray:
+    """fp64 scores of the causal blocks from one summary vector per page ([P, d_idx] bf16)."""
+    qi = bits(idx_q_row).reshape(-1)
+    sp = bits(summary_pool)
+    bt = ints(bt_row).reshape(-1)
+    nb = num_causal_blocks(p, blk)
+    s = np.empty(max(nb, 1), dtype=np.float64)
+    _load().uocr_oracle_summary_scores(_ptr(qi), _ptr(sp), _ptr(bt), int(p), int(blk), int(qi.shape[0]), _ptr(s))
+    return s[:nb]
+
+
+def block_mean(idx_k_pool, page: int) -> np.ndarray:
+    kp = bits(idx_k_pool)
+    blk, d_idx = kp.shape[1], kp.shape[2]
+    out = np.empty(d_idx, dtype=np.float64)
+    _load().uocr_oracle_block_mean(_ptr(kp), int(page), int(blk), int(d_idx), _ptr(out))
+    return out
+
+
+def select_masked(scores, nb: int, mask_words, n_local: int = N_LOCAL, n_remote: int = N_REMOTE,
+                  tie_eps: float = TIE_EPS):
+    """Selection where only remote candidates with their mask bit set may be picked."""
+    s = np.ascontiguousarray(np.asarray(scores, dtype=np.float64).reshape(-1))
+    m = np.ascontiguousarray(np.asarray(mask_words, dtype=np.uint32).reshape(-1))
+    sel = np.empty(n_local + n_remote, dtype=np.int32)
+    tie = ctypes.c_int(0)
+    _load().uocr_oracle_select_masked(_ptr(s if s.size else np.zeros(1)), int(nb), int(n_local), int(n_remote),
+                                      _ptr(m if m.size else np.zeros(1, np.uint32)), float(tie_eps), _ptr(sel),
+                                      ctypes.byref(tie))
+    return sel, bool(tie.value)

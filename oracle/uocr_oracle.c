@@ -288,3 +288,63 @@ void uocr_oracle_rope_page2d(const uint16_t *x, int n_pairs, int page_pairs, dou
         out[i + n_pairs] = b * c + a * s;
     }
 }
+
+/*
+ * [lqnn 显存账本], [leheaven 二 Token Sieve] Block-summary scoring: each KV block
+ * carries one summary vector ("learnable summary vectors" / a block's "brief
+ * representation"); the score of causal block j < nb is the raw dot product
+ *   s[j] = sum_d idx_q[d] * summary[bt_row[j]][d]
+ * (one vector per block instead of the maximum over its tokens).  Returns nb.
+ */
+int uocr_oracle_summary_scores(const uint16_t *idx_q, const uint16_t *summary_pool, const int32_t *bt_row,
+                               int p, int blk, int d_idx, double *s)
+{
+    int nb = uocr_oracle_num_causal_blocks(p, blk);
+    for (int j = 0; j < nb; ++j) {
+        const uint16_t *v = summary_pool + (size_t)bt_row[j] * d_idx;
+        double dot = 0.0;
+        for (int d = 0; d < d_idx; ++d) dot += bf16_bits_to_double(idx_q[d]) * bf16_bits_to_double(v[d]);
+        s[j] = dot;
+    }
+    return nb;
+}
+
+/* The mean of a page's blk indexer keys (one summary vector that needs no training). */
+void uocr_oracle_block_mean(const uint16_t *idx_k_pool, int page, int blk, int d_idx, double *out)
+{
+    for (int d = 0; d < d_idx; ++d) {
+        double acc = 0.0;
+        for (int r = 0; r < blk; ++r) acc += bf16_bits_to_double(idx_k_pool[((size_t)page * blk + r) * d_idx + d]);
+        out[d] = acc / blk;
+    }
+}
+
+/*
+ * [rkmt 五 page-aware candidates, image_bucket_constraint] Selection with a
+ * candidate constraint: only remote candidates j in [0, nb - n_local) whose bit
+ * (mask[j / 32] >> (j % 32)) & 1 is set may be picked; the local window is kept
+ * unconditionally.  Otherwise as uocr_oracle_select (score desc, id asc; all
+ * allowed candidates when there are no more than n_remote).
+ */
+int uocr_oracle_select_masked(const double *s, int nb, int n_local, int n_remote, const uint32_t *mask,
+                              double tie_eps, int32_t *sel, int *near_tie)
+{
+    int n_sel = n_local + n_remote;
+    int n_cand = nb - n_local > 0 ? nb - n_local : 0;
+    ranked_t *r = (ranked_t *)malloc(sizeof(ranked_t) * (size_t)(n_cand > 0 ? n_cand : 1));
+    int m = 0;
+    for (int j = 0; j < n_cand; ++j)
+        if ((mask[j / 32] >> (j % 32)) & 1u) { r[m].s = s[j]; r[m].j = j; ++m; }
+    qsort(r, (size_t)m, sizeof(ranked_t), rank_cmp);
+    int n_take = m < n_remote ? m : n_remote;
+    int *chosen = (int *)malloc(sizeof(int) * (size_t)(n_sel > 0 ? n_sel : 1));
+    int count = 0;
+    for (int k = 0; k < n_take; ++k) chosen[count++] = r[k].j;
+    if (near_tie) *near_tie = (m > n_remote && n_remote > 0) ? (r[n_remote - 1].s - r[n_remote].s) < tie_eps : 0;
+    for (int j = (nb - n_local > 0 ? nb - n_local : 0); j < nb; ++j) chosen[count++] = j;
+    qsort(chosen, (size_t)count, sizeof(int), int_cmp);
+    for (int k = 0; k < n_sel; ++k) sel[k] = (k < count) ? chosen[k] : -1;
+    free(chosen);
+    free(r);
+    return count;
+}

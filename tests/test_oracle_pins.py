@@ -412,3 +412,68 @@ def test_rope_append_writes_rotated_keys_and_raw_values():
     for i in range(n):
         untouched[int(case.block_table[i, pos[i] // 32]), :, pos[i] % 32] = False
     np.testing.assert_array_equal(kc[untouched], case.k_pool.double().numpy()[untouched])
+
+
+# ----------------------------------------------------------------------------- summary scoring, masked selection
+def test_summary_scores_brute_force():
+    g = torch.Generator().manual_seed(21)
+    qi = bf16(torch.randn(128, generator=g))
+    summ = bf16(torch.randn(6, 128, generator=g))
+    perm = np.array([3, 0, 5, 1, 4, 2])
+    for p in [0, 31, 32, 100, 191]:
+        s = oracle.summary_scores(qi, summ, perm, p)
+        want = (summ.double()[perm[: p // 32 + 1]] @ qi.double()).numpy()
+        np.testing.assert_allclose(s, want, rtol=0, atol=1e-12)
+
+
+def test_mean_summary_score_is_the_mean_token_score():
+    """Linearity: q . mean_t(k_t) = mean_t(q . k_t) -- ties the summary path to the per-token dots."""
+    g = torch.Generator().manual_seed(22)
+    qi = bf16(torch.randn(128, generator=g))
+    pages = bf16(torch.randn(4, 32, 128, generator=g))
+    for page in range(4):
+        mean = oracle.block_mean(pages, page)
+        dots = (pages[page].double() @ qi.double()).numpy()
+        assert abs(mean @ qi.double().numpy() - dots.mean()) < 1e-10
+        np.testing.assert_allclose(mean, pages[page].double().mean(0).numpy(), rtol=0, atol=1e-15)
+
+
+def test_summary_of_a_constant_block_is_its_row():
+    row = bf16(torch.linspace(-3, 3, 128))
+    pages = row.expand(2, 32, 128).clone()
+    np.testing.assert_array_equal(oracle.block_mean(pages, 1), row.double().numpy())
+
+
+@pytest.mark.parametrize("seed", range(30))
+def test_masked_select_brute_force(seed):
+    rng = np.random.default_rng(100 + seed)
+    nb = int(rng.integers(0, 14))
+    n_local, n_remote = int(rng.integers(0, 5)), int(rng.integers(0, 6))
+    s = rng.integers(-3, 4, size=max(nb, 1)).astype(np.float64)
+    allowed = rng.random(max(nb, 1)) < 0.6
+    mask = np.zeros(1, np.uint32)
+    for j in range(nb):
+        if allowed[j]:
+            mask[0] |= np.uint32(1 << j)
+    sel, _ = oracle.select_masked(s, nb, mask, n_local, n_remote, tie_eps=0.5)
+    cand = [j for j in range(max(nb - n_local, 0)) if allowed[j]]
+    k = min(n_remote, len(cand))
+    best, sets = None, []
+    for comb in itertools.combinations(cand, k):
+        tot = sum(s[j] for j in comb)
+        if best is None or tot > best:
+            best, sets = tot, [comb]
+        elif tot == best:
+            sets.append(comb)
+    want = sorted(list(min(sets)) + list(range(max(nb - n_local, 0), nb)))
+    assert sel.tolist() == want + [-1] * (n_local + n_remote - len(want))
+
+
+def test_full_mask_equals_unmasked_selection():
+    rng = np.random.default_rng(5)
+    for nb in [0, 5, 16, 17, 40, 200]:
+        s = rng.standard_normal(max(nb, 1))
+        full = np.full((nb + 31) // 32 + 1, 0xFFFFFFFF, np.uint32)
+        a, ta = oracle.select(s, nb)
+        b, tb = oracle.select_masked(s, nb, full)
+        assert np.array_equal(a, b) and ta == tb
