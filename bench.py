@@ -338,6 +338,24 @@ def run_uocr(args):
                        "pages_claim": {"vs_full": 7.0, "vs_rswa": 5.6},
                        "rswa_reading": f"reference prefix {ref_blocks} of {mb} blocks + 4-block window",
                        "full_gbs": round(B * 5120 * int(case.seq_lens[0]) / (full_ms / 1e3) / 1e9, 1)}
+        # the next-step variants on the same inputs: block-summary scoring (mean-key summaries,
+        # one 256-byte vector per page) and selection under a page-aware candidate mask
+        summ = [uocr.block_summary_mean(case.layers[l][2]) for l in range(n_layers)]
+        summary_ms = graph_time(lambda l, st: uocr.sparse_decode_summary(
+            case.q_layers[l][0], case.layers[l][0], case.layers[l][1], case.q_layers[l][1], summ[l],
+            case.block_table, case.seq_lens, out=outs[l], sel=sels[l], workspace=ws, stream=st))
+        words = (mb + 31) // 32
+        mask = torch.randint(-2 ** 31, 2 ** 31 - 1, (B, words), dtype=torch.int32, device=dev,
+                             generator=torch.Generator(device=dev).manual_seed(1))
+        masked_topk_ms = graph_time(lambda l, st: uocr.block_topk_masked(scores, case.seq_lens, mask, sel=sels[l],
+                                                                         stream=st))
+        summary_bytes = B * (256 * mb + KV_BYTES_PER_QUERY)     # one 256-byte summary per causal block
+        comparators["variants"] = {
+            "summary_decode_us": round(1e3 * summary_ms, 2),
+            "summary_decode_gbs": round(summary_bytes / (summary_ms / 1e3) / 1e9, 1),
+            "summary_speedup_vs_token_scan": round(decode_ms / summary_ms, 2),
+            "masked_topk_us": round(1e3 * masked_topk_ms, 2), "topk_us": round(1e3 * topk_ms, 2)}
+        del summ
         for o in outs:
             o.zero_()
     peaks, peak_kind = measured_peaks()

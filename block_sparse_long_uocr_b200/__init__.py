@@ -15,6 +15,9 @@ Entry points (same names as the C ABI, without the ``uocr_`` prefix):
 * :func:`sparse_decode` -- the three fused into one decode call;
 * :func:`prefill_index_score` -- the block scores of a prefill chunk on the tcgen05 tensor cores;
 * :func:`sparse_prefill` -- tensor-core scoring, selection and attention for a prefill chunk;
+* :func:`summary_score`, :func:`block_summary_mean`, :func:`sparse_decode_summary` -- block-summary
+  scoring (one vector per block) and the decode step built on it;
+* :func:`block_topk_masked` -- selection under a page-aware candidate bitmap;
 * :func:`rope_append` -- page2d rotary embedding of new tokens and their append to the caches;
 * :func:`dense_decode` -- comparator: full causal attention, or an R-SWA-style reference
   prefix plus the 128-token window (the baselines the sparse step is measured against);
@@ -70,6 +73,14 @@ def _load() -> ctypes.CDLL:
     lib.uocr_sparse_attn.restype = I
     lib.uocr_sparse_decode.argtypes = [P, P, P, P, P, P, P, I, I, I, I, P, P, P, Z, P, P]
     lib.uocr_sparse_decode.restype = I
+    lib.uocr_summary_score.argtypes = [P, P, P, P, P, P, I, I, I, I, P, P, P]
+    lib.uocr_summary_score.restype = I
+    lib.uocr_block_summary_mean.argtypes = [P, P, I, I, P, P, P]
+    lib.uocr_block_summary_mean.restype = I
+    lib.uocr_sparse_decode_summary.argtypes = [P, P, P, P, P, P, P, I, I, I, I, P, P, P, Z, P, P]
+    lib.uocr_sparse_decode_summary.restype = I
+    lib.uocr_block_topk_masked.argtypes = [P, P, P, P, P, I, I, I, I, P, P, P]
+    lib.uocr_block_topk_masked.restype = I
     lib.uocr_rope_append.argtypes = [P, P, P, P, P, P, P, P, P, P, P, I, I, I, I, I, P, P, P, P, P]
     lib.uocr_rope_append.restype = I
     lib.uocr_dense_workspace_bytes.argtypes = [I, I, I]
@@ -272,6 +283,74 @@ def sparse_prefill(q, k_cache, v_cache, idx_q, idx_k_cache, block_table, seq_len
         int(seq), _ptr(q_pos), n_q, B, H, mb, k_cache.shape[0], _ptr(out), _ptr(sel), _ptr(workspace),
         workspace.numel(), _ptr(dev_err), _stream(stream)))
     return out, sel
+
+
+def summary_score(idx_q, summary_cache, block_table, seq_lens, q_seq=None, q_pos=None, *,
+                  scores=None, dev_err=None, stream=None) -> torch.Tensor:
+    """fp32 [n_q, max_blocks]: idx_q . summary of each causal block's page."""
+    _dev(idx_q, "idx_q", torch.bfloat16, 2)
+    _dev(summary_cache, "summary_cache", torch.bfloat16, 2)
+    _dev(block_table, "block_table", torch.int32, 2)
+    _dev(seq_lens, "seq_lens", torch.int32, 1)
+    n_q, B, mb = idx_q.shape[0], block_table.shape[0], block_table.shape[1]
+    if scores is None:
+        scores = torch.full((n_q, mb), float("-inf"), dtype=torch.float32, device=idx_q.device)
+    _check("uocr_summary_score", _lib().uocr_summary_score(
+        _ptr(idx_q), _ptr(summary_cache), _ptr(block_table), _ptr(seq_lens), _ptr(_opt_i32(q_seq, "q_seq")),
+        _ptr(_opt_i32(q_pos, "q_pos")), n_q, B, mb, summary_cache.shape[0], _ptr(scores), _ptr(dev_err),
+        _stream(stream)))
+    return scores
+
+
+def block_summary_mean(idx_k_cache, summary_cache=None, pages=None, *, dev_err=None, stream=None) -> torch.Tensor:
+    """bf16 [P, 128]: the mean of each (listed) page's indexer keys."""
+    _dev(idx_k_cache, "idx_k_cache", torch.bfloat16, 3)
+    P = idx_k_cache.shape[0]
+    if summary_cache is None:
+        summary_cache = torch.zeros((P, IDX_DIM), dtype=torch.bfloat16, device=idx_k_cache.device)
+    _dev(summary_cache, "summary_cache", torch.bfloat16, 2)
+    n = P if pages is None else _dev(pages, "pages", torch.int32, 1).shape[0]
+    _check("uocr_block_summary_mean", _lib().uocr_block_summary_mean(
+        _ptr(idx_k_cache), _ptr(pages), n, P, _ptr(summary_cache), _ptr(dev_err), _stream(stream)))
+    return summary_cache
+
+
+def sparse_decode_summary(q, k_cache, v_cache, idx_q, summary_cache, block_table, seq_lens, *,
+                          out=None, sel=None, workspace=None, dev_err=None, stream=None):
+    """sparse_decode with block-summary scoring.  Returns (out, sel)."""
+    for t, n, dt, nd in ((q, "q", torch.bfloat16, 3), (k_cache, "k_cache", torch.bfloat16, 4),
+                         (v_cache, "v_cache", torch.bfloat16, 4), (idx_q, "idx_q", torch.bfloat16, 2),
+                         (summary_cache, "summary_cache", torch.bfloat16, 2), (block_table, "block_table", torch.int32, 2),
+                         (seq_lens, "seq_lens", torch.int32, 1)):
+        _dev(t, n, dt, nd)
+    B, H = q.shape[0], q.shape[1]
+    mb = block_table.shape[1]
+    if out is None:
+        out = torch.empty_like(q)
+    if sel is None:
+        sel = torch.empty((B, N_SEL), dtype=torch.int32, device=q.device)
+    if workspace is None:
+        workspace = alloc_workspace(B, H, mb, q.device)
+    _check("uocr_sparse_decode_summary", _lib().uocr_sparse_decode_summary(
+        _ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(idx_q), _ptr(summary_cache), _ptr(block_table), _ptr(seq_lens),
+        B, H, mb, k_cache.shape[0], _ptr(out), _ptr(sel), _ptr(workspace), workspace.numel(), _ptr(dev_err),
+        _stream(stream)))
+    return out, sel
+
+
+def block_topk_masked(scores, seq_lens, cand_mask, q_seq=None, q_pos=None, *, sel=None, dev_err=None,
+                      stream=None) -> torch.Tensor:
+    """Selection where remote candidate j of sequence b needs bit j of cand_mask[b] (int32 words)."""
+    _dev(scores, "scores", torch.float32, 2)
+    _dev(seq_lens, "seq_lens", torch.int32, 1)
+    _dev(cand_mask, "cand_mask", torch.int32, 2)
+    n_q, mb = scores.shape
+    if sel is None:
+        sel = torch.empty((n_q, N_SEL), dtype=torch.int32, device=scores.device)
+    _check("uocr_block_topk_masked", _lib().uocr_block_topk_masked(
+        _ptr(scores), _ptr(seq_lens), _ptr(_opt_i32(q_seq, "q_seq")), _ptr(_opt_i32(q_pos, "q_pos")),
+        _ptr(cand_mask), cand_mask.shape[1], n_q, seq_lens.shape[0], mb, _ptr(sel), _ptr(dev_err), _stream(stream)))
+    return sel
 
 
 def rope_append(q, idx_q, k_new, v_new, idx_k_new, tok_pos, page_pos, block_table, seq_lens,

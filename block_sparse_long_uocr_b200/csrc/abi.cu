@@ -276,4 +276,76 @@ uocr_status_t uocr_rope_append(void *q, void *idx_q, const void *k_new, const vo
                                                 k_cache, v_cache, idx_k_cache, dev_err));
 }
 
+uocr_status_t uocr_summary_score(const void *idx_q, const void *summary_cache, const int32_t *block_table,
+                                 const int32_t *seq_lens, const int32_t *q_seq, const int32_t *q_pos, int n_q, int B,
+                                 int max_blocks, int num_pages, float *scores, int32_t *dev_err,
+                                 uocr_stream_t stream) {
+    uocr_status_t st = check_common(n_q, B, max_blocks, num_pages, block_table, seq_lens, q_seq, q_pos, dev_err);
+    if (st != UOCR_OK) return st;
+    if (!bf16_ok(idx_q) || !bf16_ok(summary_cache) || !scores || !aligned(scores, 4)) return UOCR_ERR_INVALID_ARG;
+    if (n_q == 0) return UOCR_OK;
+    uocr::LaunchCtx c;
+    if ((st = make_ctx(stream, false, c)) != UOCR_OK) return st;
+    return cuda_status(uocr::launch_summary_scan(c, idx_q, summary_cache, block_table, seq_lens, q_seq, q_pos, n_q,
+                                                 B, max_blocks, num_pages, scores, dev_err));
+}
+
+uocr_status_t uocr_block_summary_mean(const void *idx_k_cache, const int32_t *pages, int n_pages, int num_pages,
+                                      void *summary_cache, int32_t *dev_err, uocr_stream_t stream) {
+    if (!bf16_ok(idx_k_cache) || !bf16_ok(summary_cache) || n_pages < 0 || num_pages < 1) return UOCR_ERR_INVALID_ARG;
+    if ((pages && !aligned(pages, 4)) || (dev_err && !aligned(dev_err, 4))) return UOCR_ERR_INVALID_ARG;
+    if (n_pages == 0) return UOCR_OK;
+    uocr::LaunchCtx c;
+    uocr_status_t st;
+    if ((st = make_ctx(stream, false, c)) != UOCR_OK) return st;
+    return cuda_status(uocr::launch_block_mean(c, idx_k_cache, pages, n_pages, num_pages, summary_cache, dev_err));
+}
+
+uocr_status_t uocr_sparse_decode_summary(const void *q, const void *k_cache, const void *v_cache, const void *idx_q,
+                                         const void *summary_cache, const int32_t *block_table,
+                                         const int32_t *seq_lens, int B, int H, int max_blocks, int num_pages,
+                                         void *out, int32_t *sel_out, void *workspace, size_t workspace_bytes,
+                                         int32_t *dev_err, uocr_stream_t stream) {
+    uocr_status_t st = check_common(B, B, max_blocks, num_pages, block_table, seq_lens, nullptr, nullptr, dev_err);
+    if (st != UOCR_OK) return st;
+    if (!bf16_ok(q) || !bf16_ok(k_cache) || !bf16_ok(v_cache) || !bf16_ok(out) || !bf16_ok(idx_q) ||
+        !bf16_ok(summary_cache))
+        return UOCR_ERR_INVALID_ARG;
+    if (!sel_out || !aligned(sel_out, 4)) return UOCR_ERR_INVALID_ARG;
+    if (H < 1 || H > UOCR_MAX_HEADS) return UOCR_ERR_UNSUPPORTED;
+    const WsLayout w = ws_layout(B, H, max_blocks);
+    if (!workspace || !aligned(workspace, kWsAlign) || workspace_bytes < w.total) return UOCR_ERR_WORKSPACE;
+    uocr::LaunchCtx c;
+    if ((st = make_ctx(stream, false, c)) != UOCR_OK) return st;
+    float *scores = (float *)((char *)workspace + w.scores_off);
+    cudaError_t e = uocr::launch_summary_scan(c, idx_q, summary_cache, block_table, seq_lens, nullptr, nullptr, B, B,
+                                              max_blocks, num_pages, scores, dev_err);
+    if (e != cudaSuccess) return cuda_status(e);
+    c.pdl = true;
+    e = uocr::launch_block_topk(c, scores, seq_lens, nullptr, nullptr, B, B, max_blocks, sel_out, dev_err);
+    if (e != cudaSuccess) return cuda_status(e);
+    const float scale = 1.0f / sqrtf((float)UOCR_HEAD_DIM);
+    e = uocr::launch_sparse_attn(c, q, k_cache, v_cache, block_table, seq_lens, nullptr, nullptr, sel_out, B, B, H,
+                                 max_blocks, num_pages, scale, out, true, -1, false, dev_err);
+    return cuda_status(e);
+}
+
+uocr_status_t uocr_block_topk_masked(const float *scores, const int32_t *seq_lens, const int32_t *q_seq,
+                                     const int32_t *q_pos, const uint32_t *cand_mask, int mask_words, int n_q, int B,
+                                     int max_blocks, int32_t *sel, int32_t *dev_err, uocr_stream_t stream) {
+    if (n_q < 0 || B < 1 || max_blocks < 1) return UOCR_ERR_INVALID_ARG;
+    if (!scores || !seq_lens || !sel || !cand_mask) return UOCR_ERR_INVALID_ARG;
+    if (!aligned(scores, 4) || !aligned(seq_lens, 4) || !aligned(sel, 4) || !aligned(cand_mask, 4))
+        return UOCR_ERR_INVALID_ARG;
+    if ((q_seq && !aligned(q_seq, 4)) || (q_pos && !aligned(q_pos, 4))) return UOCR_ERR_INVALID_ARG;
+    if (dev_err && !aligned(dev_err, 4)) return UOCR_ERR_INVALID_ARG;
+    if ((long long)mask_words * 32 < (long long)max_blocks) return UOCR_ERR_INVALID_ARG;
+    if (n_q == 0) return UOCR_OK;
+    uocr::LaunchCtx c;
+    uocr_status_t st;
+    if ((st = make_ctx(stream, false, c)) != UOCR_OK) return st;
+    return cuda_status(uocr::launch_block_topk(c, scores, seq_lens, q_seq, q_pos, n_q, B, max_blocks, sel, dev_err,
+                                               -1, cand_mask, mask_words));
+}
+
 }  // extern "C"

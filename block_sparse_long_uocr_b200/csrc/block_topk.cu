@@ -21,6 +21,9 @@
 // back to an exact two-level extraction: every warp takes its top 12 by 12
 // rounds of a warp-wide max, then one warp takes the top 12 of those.
 // Rows longer than the shared-memory budget are read from L2 instead of staged.
+// An optional per-sequence candidate bitmap (the walk-through's page-aware
+// candidate constraint, section 五 image_bucket_constraint) excludes remote
+// candidates before the ranking; the local window is always kept.
 #include <math.h>
 
 #include "common.cuh"
@@ -53,12 +56,17 @@ __device__ __forceinline__ uint64_t warp_max_u64(uint64_t v) {
 }
 
 // Keys of one query's candidates: staged in shared memory, or read from the scores row.
+// A candidate that the optional candidate mask excludes gets key 0, below every real key
+// (order_key never returns 0 for a non-NaN score).
 struct KeySource {
     const uint32_t *smem;
     const float *row;
-    __device__ __forceinline__ uint32_t operator()(int j) const {
-        return smem ? smem[j] : order_key(__ldcg(row + j));
+    const uint32_t *mask;   // this sequence's candidate bitmap, or NULL
+    __device__ __forceinline__ uint32_t raw(int j) const {
+        if (mask && !((__ldg(mask + (j >> 5)) >> (j & 31)) & 1u)) return 0u;
+        return order_key(__ldcg(row + j));
     }
+    __device__ __forceinline__ uint32_t operator()(int j) const { return smem ? smem[j] : raw(j); }
 };
 
 // Largest composite strictly below `cap` among candidates j = first, first + stride, ... < n
@@ -119,7 +127,8 @@ __device__ void topk_two_level(const KeySource &key, int nc, uint64_t *s_cand, u
 __global__ void __launch_bounds__(kTopkThreads)
 block_topk_kernel(const float *__restrict__ scores, const int32_t *__restrict__ seq_lens,
                   const int32_t *__restrict__ q_seq, const int32_t *__restrict__ q_pos, int B,
-                  int max_blocks, int32_t *__restrict__ sel, int32_t *dev_err, int staged, int fixed_seq) {
+                  int max_blocks, int32_t *__restrict__ sel, int32_t *dev_err, int staged, int fixed_seq,
+                  const uint32_t *__restrict__ cand_mask, int mask_words) {
     extern __shared__ uint32_t s_keys[];
     __shared__ uint64_t s_surv[kSurvivorCap];
     __shared__ uint64_t s_cand[kTopkWarps * kRemote];
@@ -127,6 +136,7 @@ block_topk_kernel(const float *__restrict__ scores, const int32_t *__restrict__ 
     __shared__ uint32_t s_wmax[kTopkWarps];
     __shared__ uint32_t s_thr;
     __shared__ int s_n;
+    __shared__ int s_allowed;
 
     const int i = blockIdx.x;
     const int tid = threadIdx.x;
@@ -144,34 +154,64 @@ block_topk_kernel(const float *__restrict__ scores, const int32_t *__restrict__ 
     }
     const int nb = r.nb;
     const int nc = nb - kLocal > 0 ? nb - kLocal : 0;
-    if (nc <= kRemote) {
+    const uint32_t *mask = cand_mask ? cand_mask + (size_t)r.b * mask_words : nullptr;
+    if (nc <= kRemote && !mask) {
         // every causal block fits in the 16 slots
         if (tid < kSel) out[tid] = tid < nb ? tid : -1;
         return;
     }
     const float *row = scores + (size_t)i * max_blocks;
-    KeySource key{nullptr, row};
-    if (tid == 0) s_n = 0;
+    KeySource key{nullptr, row, mask};
+    if (tid == 0) {
+        s_n = 0;
+        s_allowed = 0;
+    }
+    __syncthreads();
 
     // ---- 1. stage keys, 2. per-thread then per-warp maximum
     uint32_t tmax = 0;
+    int allowed = 0;
     if (staged) {
 #pragma unroll 8
         for (int j = tid; j < nc; j += kTopkThreads) {
-            const uint32_t k = order_key(__ldcg(row + j));
+            const uint32_t k = key.raw(j);
             s_keys[j] = k;
             tmax = k > tmax ? k : tmax;
+            allowed += k != 0u;
         }
         key.smem = s_keys;
     } else {
         for (int j = tid; j < nc; j += kTopkThreads) {
             const uint32_t k = key(j);
             tmax = k > tmax ? k : tmax;
+            allowed += k != 0u;
         }
     }
     const uint32_t wmax = __reduce_max_sync(0xffffffffu, tmax);
     if (lane == 0) s_wmax[warp] = wmax;
+    if (mask) {
+        const int wa = __reduce_add_sync(0xffffffffu, allowed);
+        if (lane == 0) atomicAdd(&s_allowed, wa);
+    }
     __syncthreads();
+
+    if (mask && s_allowed <= kRemote) {
+        // no more allowed candidates than remote slots: take them all, in id order
+        if (warp == 0) {
+            int pos = 0;
+            for (int base = 0; base < nc; base += 32) {
+                const int j = base + lane;
+                const bool take = j < nc && key(j) != 0u;
+                const unsigned m = __ballot_sync(0xffffffffu, take);
+                if (take) out[pos + __popc(m & ((1u << lane) - 1u))] = j;
+                pos += __popc(m);
+            }
+            const int n_loc = nb < kLocal ? nb : kLocal;
+            if (lane < n_loc) out[pos + lane] = nb - n_loc + lane;
+            if (lane >= pos + n_loc && lane < kSel) out[lane] = -1;
+        }
+        return;
+    }
 
     // ---- threshold = the kRemote-th largest warp maximum (with multiplicity)
     if (warp == 0) {
@@ -235,7 +275,8 @@ block_topk_kernel(const float *__restrict__ scores, const int32_t *__restrict__ 
 
 cudaError_t launch_block_topk(const LaunchCtx &c, const float *scores, const int32_t *seq_lens,
                               const int32_t *q_seq, const int32_t *q_pos, int n_q, int B,
-                              int max_blocks, int32_t *sel, int32_t *dev_err, int fixed_seq) {
+                              int max_blocks, int32_t *sel, int32_t *dev_err, int fixed_seq,
+                              const uint32_t *cand_mask, int mask_words) {
     const int staged = max_blocks <= kTopkSmemKeys;
     const size_t smem = staged ? (size_t)max_blocks * sizeof(uint32_t) : 0;
     if (smem > 16 * 1024) {
@@ -255,7 +296,7 @@ cudaError_t launch_block_topk(const LaunchCtx &c, const float *scores, const int
     cfg.attrs = attr;
     cfg.numAttrs = c.pdl ? 1 : 0;
     return cudaLaunchKernelEx(&cfg, block_topk_kernel, scores, seq_lens, q_seq, q_pos, B, max_blocks,
-                              sel, dev_err, staged, fixed_seq);
+                              sel, dev_err, staged, fixed_seq, cand_mask, mask_words);
 }
 
 }  // namespace uocr

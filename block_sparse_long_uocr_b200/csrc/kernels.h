@@ -25,7 +25,8 @@ cudaError_t launch_index_scan(const LaunchCtx &c, const void *idx_q, const void 
 
 cudaError_t launch_block_topk(const LaunchCtx &c, const float *scores, const int32_t *seq_lens,
                               const int32_t *q_seq, const int32_t *q_pos, int n_q, int B,
-                              int max_blocks, int32_t *sel, int32_t *dev_err, int fixed_seq = -1);
+                              int max_blocks, int32_t *sel, int32_t *dev_err, int fixed_seq = -1,
+                              const uint32_t *cand_mask = nullptr, int mask_words = 0);
 
 cudaError_t launch_sparse_attn(const LaunchCtx &c, const void *q, const void *k, const void *v,
                                const int32_t *bt, const int32_t *seq_lens, const int32_t *q_seq,
@@ -68,5 +69,12 @@ cudaError_t launch_rope_append(const LaunchCtx &c, void *q, void *idx_q, const v
                                const int32_t *q_seq, const int32_t *q_pos, const int32_t *bt,
                                const int32_t *seq_lens, int n, int B, int H, int max_blocks, int num_pages,
                                void *k_cache, void *v_cache, void *idx_k_cache, int32_t *dev_err);
+
+// Block-summary scoring (one summary vector per page) and the mean-key summary builder.
+cudaError_t launch_summary_scan(const LaunchCtx &c, const void *idx_q, const void *summary, const int32_t *bt,
+                                const int32_t *seq_lens, const int32_t *q_seq, const int32_t *q_pos, int n_q, int B,
+                                int max_blocks, int num_pages, float *scores, int32_t *dev_err);
+cudaError_t launch_block_mean(const LaunchCtx &c, const void *idx_k, const int32_t *pages, int n_pages,
+                              int num_pages, void *summary, int32_t *dev_err);
 
 }  // namespace uocr

@@ -237,6 +237,58 @@ uocr_status_t uocr_rope_append(void *q, void *idx_q, const void *k_new, const vo
                                int32_t *dev_err, uocr_stream_t stream);
 
 /*
+ * Block-summary scoring ([lqnn 显存账本]: "learnable summary vectors" per KV
+ * block; [leheaven 二] Token Sieve: score each block by its brief
+ * representation, then read the chosen blocks' tokens).  For every causal block
+ * j < nb_i of query i:  scores[i][j] = idx_q[i] . summary_cache[block_table[b][j]]
+ * with summary_cache bf16 [P][128] (one vector per page, supplied by the caller
+ * or built by uocr_block_summary_mean).  32x fewer bytes than the max-over-tokens
+ * scan.  Same arguments, layouts and errors as uocr_index_score otherwise.
+ */
+uocr_status_t uocr_summary_score(const void *idx_q, const void *summary_cache,
+                                 const int32_t *block_table, const int32_t *seq_lens,
+                                 const int32_t *q_seq, const int32_t *q_pos,
+                                 int n_q, int B, int max_blocks, int num_pages,
+                                 float *scores, int32_t *dev_err, uocr_stream_t stream);
+
+/*
+ * summary_cache[page] = bf16(mean of the page's 32 indexer keys) for the
+ * n_pages pages listed in `pages` (NULL: pages 0 .. n_pages-1).  The mean is the
+ * summary that needs no trained weights.  summary_cache bf16 [num_pages][128].
+ */
+uocr_status_t uocr_block_summary_mean(const void *idx_k_cache, const int32_t *pages, int n_pages,
+                                      int num_pages, void *summary_cache, int32_t *dev_err,
+                                      uocr_stream_t stream);
+
+/*
+ * uocr_sparse_decode with block-summary scoring: uocr_summary_score ->
+ * uocr_block_topk -> uocr_sparse_attn, same arguments except summary_cache
+ * [P][128] in place of the indexer key cache.
+ */
+uocr_status_t uocr_sparse_decode_summary(const void *q, const void *k_cache, const void *v_cache,
+                                         const void *idx_q, const void *summary_cache,
+                                         const int32_t *block_table, const int32_t *seq_lens,
+                                         int B, int H, int max_blocks, int num_pages,
+                                         void *out, int32_t *sel_out,
+                                         void *workspace, size_t workspace_bytes,
+                                         int32_t *dev_err, uocr_stream_t stream);
+
+/*
+ * Block selection under a page-aware candidate constraint ([rkmt 五]
+ * image_bucket_constraint: candidates restricted to the current page's image
+ * blocks + the local window + a global fallback).  As uocr_block_topk, but a
+ * remote candidate j of a query of sequence b may be picked only if bit
+ * (cand_mask[b * mask_words + j / 32] >> (j % 32)) & 1 is set; the local window
+ * is kept regardless.  With at most 12 allowed candidates all of them are
+ * taken; sel is ascending and -1 padded.  mask_words >= ceil(max_blocks / 32).
+ */
+uocr_status_t uocr_block_topk_masked(const float *scores, const int32_t *seq_lens,
+                                     const int32_t *q_seq, const int32_t *q_pos,
+                                     const uint32_t *cand_mask, int mask_words,
+                                     int n_q, int B, int max_blocks, int32_t *sel,
+                                     int32_t *dev_err, uocr_stream_t stream);
+
+/*
  * Comparator decode attention (baselines the pages quote the sparse step
  * against: full attention and R-SWA; release report, leheavengame.com, section
  * 一: 7.0x and 5.6x; R-SWA: Unlimited OCR v1 article, chenxutan.com/d/4261.html,
