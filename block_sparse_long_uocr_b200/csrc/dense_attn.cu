@@ -20,6 +20,7 @@
 
 #include "common.cuh"
 #include "kernels.h"
+#include "scan_core.cuh"
 
 namespace uocr {
 
@@ -58,7 +59,6 @@ dense_attn_chunk_kernel(const uint4 *__restrict__ q, const uint4 *__restrict__ k
 
     float qf[8];
     bf16x8_to_f32(__ldg(q + ((size_t)i * H + h) * (kD / 8) + (lane & 15)), qf);
-    const int tok = 2 * (lane & 15) + (lane >> 4);
     float m_w = -INFINITY, l_w = 0.f;
     float acc[8];
 #pragma unroll
@@ -72,40 +72,8 @@ dense_attn_chunk_kernel(const uint4 *__restrict__ q, const uint4 *__restrict__ k
             if (lane == 0) flag_error(dev_err, UOCR_DEVERR_PAGE);
             continue;
         }
-        const size_t tile = ((size_t)page * H + h) * (kPageElems / 8) + lane;
-        uint4 kv[16];
-#pragma unroll
-        for (int t = 0; t < 16; ++t) kv[t] = ld_stream(kc + tile + t * 32);
-        float z[16];
-#pragma unroll
-        for (int t = 0; t < 16; ++t) {
-            float kf[8];
-            bf16x8_to_f32(kv[t], kf);
-            float a = qf[0] * kf[0];
-#pragma unroll
-            for (int c = 1; c < 8; ++c) a = fmaf(qf[c], kf[c], a);
-            z[t] = a;
-        }
-#pragma unroll
-        for (int t = 0; t < 16; ++t) kv[t] = ld_stream(vc + tile + t * 32);
-        float zt = half_warp_transpose_sum16(z, lane) * scale_log2;
-        if (j * kBlock + tok > r.p) zt = -INFINITY;
-        const float mb = warp_max(zt);                  // finite: token 32j <= p
-        const float m_new = fmaxf(m_w, mb);
-        const float corr = exp2f(m_w - m_new);          // 0 on the first block (m_w = -inf)
-        const float pt = exp2f(zt - m_new);
-        l_w = l_w * corr + warp_sum(pt);
-#pragma unroll
-        for (int c = 0; c < 8; ++c) acc[c] *= corr;
-#pragma unroll
-        for (int t = 0; t < 16; ++t) {
-            const float w = __shfl_sync(0xffffffffu, pt, (lane & 16) | t);
-            float vf[8];
-            bf16x8_to_f32(kv[t], vf);
-#pragma unroll
-            for (int c = 0; c < 8; ++c) acc[c] = fmaf(w, vf[c], acc[c]);
-        }
-        m_w = m_new;
+        attend_block_online(qf, kc, vc, ((size_t)page * H + h) * (kPageElems / 8) + lane, j, r.p, scale_log2,
+                            lane, m_w, l_w, acc);
     }
 #pragma unroll
     for (int c = 0; c < 8; ++c) acc[c] += __shfl_xor_sync(0xffffffffu, acc[c], 16);

@@ -15,11 +15,13 @@
 //   * loads bypass L1 allocation; 16 warps per SM keep ~128 KiB in flight.
 // The grid is flat over (query, chunk of pages); chunks past a query's causal
 // blocks exit at once, so ragged batches need no host-side work list.
+
 #include <cuda_bf16.h>
 #include <math.h>
 
 #include "common.cuh"
 #include "kernels.h"
+#include "scan_core.cuh"
 
 namespace uocr {
 
@@ -47,40 +49,9 @@ index_scan_kernel(const uint4 *__restrict__ idx_q, const uint4 *__restrict__ idx
     float qf[8];
     bf16x8_to_f32(__ldg(idx_q + (size_t)i * (kDIdx / 8) + (lane & 15)), qf);
 
-    const int32_t *bt_row = bt + (size_t)r.b * max_blocks;
-    float *srow = scores + (size_t)i * max_blocks;
-    const int tok = 2 * (lane & 15) + (lane >> 4);
-
-    for (int k = 0; k < pages_per_warp; ++k) {
-        const int j = j0 + warp + k * kScanWarps;
-        if (j >= r.nb) break;
-        const int page = __ldg(bt_row + j);
-        if ((unsigned)page >= (unsigned)num_pages) {
-            if (lane == 0) {
-                flag_error(dev_err, UOCR_DEVERR_PAGE);
-                srow[j] = -INFINITY;
-            }
-            continue;
-        }
-        const uint4 *src = idx_k + (size_t)page * (kBlock * kDIdx / 8) + lane;
-        uint4 v[16];
-#pragma unroll
-        for (int s = 0; s < 16; ++s) v[s] = ld_stream(src + s * 32);
-        float acc[16];
-#pragma unroll
-        for (int s = 0; s < 16; ++s) {
-            float kf[8];
-            bf16x8_to_f32(v[s], kf);
-            float a = qf[0] * kf[0];
-#pragma unroll
-            for (int e = 1; e < 8; ++e) a = fmaf(qf[e], kf[e], a);
-            acc[s] = a;
-        }
-        float dot = half_warp_transpose_sum16(acc, lane);
-        if (j * kBlock + tok > r.p) dot = -INFINITY;
-        const float m = warp_max(dot);
-        if (lane == 0) srow[j] = m;
-    }
+    const int j_end = min(r.nb, j0 + kScanWarps * pages_per_warp);
+    scan_pages(qf, idx_k, bt + (size_t)r.b * max_blocks, r.p, j0 + warp, kScanWarps, j_end, num_pages,
+               scores + (size_t)i * max_blocks, dev_err, lane);
     pdl_launch_dependents();
 }
 
@@ -114,3 +85,4 @@ cudaError_t launch_index_scan(const LaunchCtx &c, const void *idx_q, const void 
 }
 
 }  // namespace uocr
+

@@ -1,0 +1,273 @@
+// topk_core.cuh -- the per-query block selection of the walk-through
+// (news.rkmt.cn/news/25027, section 五 step 3): 4 local blocks + the 12
+// highest-scoring remote blocks (score desc, then lower id), optionally limited
+// to the candidates of a page-aware bitmap.  Shared by block_topk_kernel (one
+// CTA of 512 threads per query) and the fused decode kernel (256 threads).
+//
+// Every candidate's ranking key is the 64-bit composite
+// (order-preserving fp32 key << 32 | ~id): distinct, larger for a higher score
+// and, among equal scores, for the lower id.
+//   1. The candidates' scores are read once from L2 into shared memory as
+//      order-preserving keys (masked-out candidates get key 0).
+//   2. Threshold: the 12th largest of 16 group maxima (groups of T/16
+//      threads).  Those 12 maxima are 12 distinct candidates at or above it, so
+//      every member of the top 12 is at or above it too.
+//   3. Survivors (keys >= threshold; typically a few dozen) are appended to a
+//      shared list and ranked by counting; ranks 0..11 are the answer.
+//   4. One warp writes the 12 ids in ascending order plus the 4 local blocks.
+// If the survivors overflow their list (heavily tied scores) the CTA falls
+// back to an exact two-level extraction (12 rounds of a warp-wide max per warp,
+// then 12 rounds over the warps' survivors).
+#pragma once
+
+#include "common.cuh"
+
+namespace uocr {
+
+constexpr int kSurvivorCap = 2048;          // survivor list capacity (16 KiB)
+constexpr int kTopkGroups = 16;             // threshold from 16 group maxima (>= kRemote)
+
+// Larger key <=> larger float; -0 and +0 map to the same key (they compare equal).
+__device__ __forceinline__ uint32_t order_key(float f) {
+    const uint32_t u = (f == 0.0f) ? 0u : __float_as_uint(f);
+    return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+}
+
+__device__ __forceinline__ uint64_t composite(uint32_t key, int j) {
+    return ((uint64_t)key << 32) | (uint32_t)(~(uint32_t)j);
+}
+
+__device__ __forceinline__ uint64_t warp_max_u64(uint64_t v) {
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+        const uint64_t w = __shfl_xor_sync(0xffffffffu, v, o);
+        v = w > v ? w : v;
+    }
+    return v;
+}
+
+// Keys of one query's candidates: staged in shared memory, or read from the scores row.
+// A candidate that the optional candidate mask excludes gets key 0, below every real key
+// (order_key never returns 0 for a non-NaN score).
+struct KeySource {
+    const uint32_t *smem;
+    const float *row;
+    const uint32_t *mask;   // this sequence's candidate bitmap, or NULL
+    __device__ __forceinline__ uint32_t raw(int j) const {
+        if (mask && !((__ldg(mask + (j >> 5)) >> (j & 31)) & 1u)) return 0u;
+        return order_key(__ldcg(row + j));
+    }
+    __device__ __forceinline__ uint32_t operator()(int j) const { return smem ? smem[j] : raw(j); }
+};
+
+// Largest composite strictly below `cap` among candidates j = first, first + stride, ... < n
+// (0 when there is none; a real composite is never 0 because ~j != 0 for j < 2^31 - 1).
+__device__ __forceinline__ uint64_t best_below(const KeySource &key, int first, int stride, int n,
+                                               uint64_t cap) {
+    uint64_t best = 0;
+    for (int j = first; j < n; j += stride) {
+        const uint64_t c = composite(key(j), j);
+        if (c < cap && c > best) best = c;
+    }
+    return best;
+}
+
+// Exact fallback: the top kRemote composites of candidates [0, nc) into out_c[0..11].
+// Called by every thread of a CTA of T threads.
+template <int T>
+__device__ void topk_two_level(const KeySource &key, int nc, uint64_t *s_cand, uint64_t *out_c) {
+    constexpr int kW = T / 32;
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    uint64_t cap = ~0ull;
+    uint64_t mine = best_below(key, tid, T, nc, cap);
+#pragma unroll 1
+    for (int k = 0; k < kRemote; ++k) {
+        const uint64_t w = warp_max_u64(mine);
+        if (lane == 0) s_cand[warp * kRemote + k] = w;   // 0 when the warp ran out of candidates
+        if (mine == w && w != 0) {
+            cap = mine;
+            mine = best_below(key, tid, T, nc, cap);
+        }
+    }
+    __syncthreads();
+    if (warp == 0) {
+        constexpr int kPer = kW * kRemote / 32;   // survivors per lane
+        static_assert(kW * kRemote % 32 == 0, "warps x 12 survivors must fill whole lanes");
+        uint64_t c[kPer];
+#pragma unroll
+        for (int e = 0; e < kPer; ++e) c[e] = s_cand[lane * kPer + e];
+#pragma unroll 1
+        for (int k = 0; k < kRemote; ++k) {
+            uint64_t best = 0;
+            int at = -1;
+#pragma unroll
+            for (int e = 0; e < kPer; ++e)
+                if (c[e] > best) {
+                    best = c[e];
+                    at = e;
+                }
+            const uint64_t w = warp_max_u64(best);
+            if (best == w && at >= 0) {
+#pragma unroll
+                for (int e = 0; e < kPer; ++e)
+                    if (e == at) c[e] = 0;
+            }
+            if (lane == 0) out_c[k] = w;
+        }
+    }
+    __syncthreads();
+}
+
+
+template <int T>
+struct TopkShared {
+    uint64_t surv[kSurvivorCap];
+    uint64_t cand[(T / 32) * kRemote];
+    uint64_t top[kRemote];
+    uint32_t gmax[kTopkGroups];
+    uint32_t thr;
+    int n;
+    int allowed;
+};
+
+// Selection of one query with nb causal blocks from its score row; every thread of a CTA of
+// T threads calls it (the CTA-wide barriers inside must be reached by all of them).
+// s_keys: shared staging for at least nb - 4 keys, or NULL to read the row from L2 each pass.
+// out: the query's 16 selection slots.
+template <int T>
+__device__ void topk_select(const float *row, int nb, const uint32_t *mask, uint32_t *s_keys,
+                            TopkShared<T> &sm, int32_t *out) {
+    constexpr int kW = T / 32;
+    constexpr int kGroup = T / kTopkGroups;     // threads per group: 16 or 32
+    static_assert(kGroup == 16 || kGroup == 32, "16 groups of a half-warp or a warp");
+    const int tid = threadIdx.x;
+    const int lane = tid & 31, warp = tid >> 5;
+    const int nc = nb - kLocal > 0 ? nb - kLocal : 0;
+    if (nc <= kRemote && !mask) {
+        // every causal block fits in the 16 slots
+        if (tid < kSel) out[tid] = tid < nb ? tid : -1;
+        return;
+    }
+    KeySource key{nullptr, row, mask};
+    if (tid == 0) {
+        sm.n = 0;
+        sm.allowed = 0;
+    }
+    __syncthreads();
+
+    // ---- 1. stage keys, 2. per-thread then per-group maximum
+    uint32_t tmax = 0;
+    int allowed = 0;
+    if (s_keys) {
+#pragma unroll 8
+        for (int j = tid; j < nc; j += T) {
+            const uint32_t k = key.raw(j);
+            s_keys[j] = k;
+            tmax = k > tmax ? k : tmax;
+            allowed += k != 0u;
+        }
+        key.smem = s_keys;
+    } else {
+        for (int j = tid; j < nc; j += T) {
+            const uint32_t k = key(j);
+            tmax = k > tmax ? k : tmax;
+            allowed += k != 0u;
+        }
+    }
+    uint32_t gm = tmax;
+    if (kGroup == 32) {
+        gm = __reduce_max_sync(0xffffffffu, gm);
+    } else {
+#pragma unroll
+        for (int o = 8; o > 0; o >>= 1) {
+            const uint32_t other = __shfl_xor_sync(0xffffffffu, gm, o);
+            gm = other > gm ? other : gm;
+        }
+    }
+    if (tid % kGroup == 0) sm.gmax[tid / kGroup] = gm;
+    if (mask) {
+        const int wa = __reduce_add_sync(0xffffffffu, allowed);
+        if (lane == 0) atomicAdd(&sm.allowed, wa);
+    }
+    __syncthreads();
+
+    if (mask && sm.allowed <= kRemote) {
+        // no more allowed candidates than remote slots: take them all, in id order
+        if (warp == 0) {
+            int pos = 0;
+            for (int base = 0; base < nc; base += 32) {
+                const int j = base + lane;
+                const bool take = j < nc && key(j) != 0u;
+                const unsigned m = __ballot_sync(0xffffffffu, take);
+                if (take) out[pos + __popc(m & ((1u << lane) - 1u))] = j;
+                pos += __popc(m);
+            }
+            const int n_loc = nb < kLocal ? nb : kLocal;
+            if (lane < n_loc) out[pos + lane] = nb - n_loc + lane;
+            if (lane >= pos + n_loc && lane < kSel) out[lane] = -1;
+        }
+        return;
+    }
+
+    // ---- threshold = the kRemote-th largest group maximum (with multiplicity)
+    if (warp == 0) {
+        const uint32_t v = lane < kTopkGroups ? sm.gmax[lane] : 0u;
+        int gt = 0, ge = 0;
+#pragma unroll
+        for (int w = 0; w < kTopkGroups; ++w) {
+            const uint32_t o = sm.gmax[w];
+            gt += o > v;
+            ge += o >= v;
+        }
+        const bool is_thr = lane < kTopkGroups && gt <= kRemote - 1 && kRemote - 1 < ge;
+        const unsigned who = __ballot_sync(0xffffffffu, is_thr);
+        if (lane == __ffs(who) - 1) sm.thr = v;
+    }
+    __syncthreads();
+    const uint32_t thr = sm.thr;
+
+    // ---- 3. survivors: every candidate at or above the threshold
+    for (int j0 = 0; j0 < nc; j0 += T) {
+        const int j = j0 + tid;
+        const uint32_t k = j < nc ? key(j) : 0u;
+        const bool keep = j < nc && k >= thr;
+        const unsigned m = __ballot_sync(0xffffffffu, keep);
+        if (m) {
+            const int leader = __ffs(m) - 1;
+            int base = 0;
+            if (lane == leader) base = atomicAdd(&sm.n, __popc(m));
+            base = __shfl_sync(0xffffffffu, base, leader);
+            const int slot = base + __popc(m & ((1u << lane) - 1u));
+            if (keep && slot < kSurvivorCap) sm.surv[slot] = composite(k, j);
+        }
+    }
+    __syncthreads();
+    const int n = sm.n;
+    if (n <= kSurvivorCap) {
+        for (int a = tid; a < n; a += T) {
+            const uint64_t c = sm.surv[a];
+            int rank = 0;
+            for (int b = 0; b < n; ++b) rank += sm.surv[b] > c;
+            if (rank < kRemote) sm.top[rank] = c;
+        }
+        __syncthreads();
+    } else {
+        topk_two_level<T>(key, nc, sm.cand, sm.top);
+    }
+
+    // ---- 4. the 12 remote ids ascending, then the 4 local blocks
+    if (warp == 0) {
+        const int id = lane < kRemote ? (int)~(uint32_t)(sm.top[lane] & 0xffffffffu) : 0x7fffffff;
+        int rank = 0;
+#pragma unroll
+        for (int k = 0; k < kRemote; ++k) {
+            const int other = __shfl_sync(0xffffffffu, id, k);
+            rank += other < id;
+        }
+        if (lane < kRemote) out[rank] = id;
+        if (lane < kLocal) out[kRemote + lane] = nb - kLocal + lane;
+    }
+    (void)kW;
+}
+
+}  // namespace uocr

@@ -64,7 +64,10 @@ def test_static_decode_matches_the_workspace_entry_on_two_calls_in_a_row(uocr, c
 
 def test_static_decode_refuses_shapes_beyond_its_scratch(uocr, cuda_device):
     B, H = 64, 10
-    mb = 32769                                      # one block more than 8 MiB of scratch holds at B=64
+    mb = 1
+    while uocr.workspace_bytes(B, H, mb + 1) <= uocr.STATIC_SCRATCH_BYTES:   # the largest shape that fits
+        mb += 1
+    mb += 1                                         # one block more than the scratch holds
     assert uocr.workspace_bytes(B, H, mb) > uocr.STATIC_SCRATCH_BYTES >= uocr.workspace_bytes(B, H, mb - 1)
     q = torch.zeros((B, H, 128), dtype=torch.bfloat16, device=cuda_device)
     kv = torch.zeros((1, H, 32, 128), dtype=torch.bfloat16, device=cuda_device)
