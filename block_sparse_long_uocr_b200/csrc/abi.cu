@@ -225,7 +225,8 @@ uocr_status_t uocr_sparse_prefill(const void *q, const void *k_cache, const void
                                         num_pages, scores, dev_err);
     if (e != cudaSuccess) return cuda_status(e);
     c.pdl = true;
-    e = uocr::launch_block_topk(c, scores, seq_lens, nullptr, q_pos, n_q, B, max_blocks, sel_out, dev_err, seq);
+    e = uocr::launch_block_topk(c, scores, seq_lens, nullptr, q_pos, n_q, B, max_blocks, sel_out, dev_err, seq,
+                                nullptr, 0, (int32_t *)(attn_ws + aw.counts_off));
     if (e != cudaSuccess) return cuda_status(e);
     const float scale = 1.0f / sqrtf((float)UOCR_HEAD_DIM);
     e = uocr::launch_prefill_attn(c, q, k_cache, v_cache, bt_row, q_pos, sel_out, n_q, H, max_blocks, num_pages,

@@ -26,7 +26,8 @@ cudaError_t launch_index_scan(const LaunchCtx &c, const void *idx_q, const void 
 cudaError_t launch_block_topk(const LaunchCtx &c, const float *scores, const int32_t *seq_lens,
                               const int32_t *q_seq, const int32_t *q_pos, int n_q, int B,
                               int max_blocks, int32_t *sel, int32_t *dev_err, int fixed_seq = -1,
-                              const uint32_t *cand_mask = nullptr, int mask_words = 0);
+                              const uint32_t *cand_mask = nullptr, int mask_words = 0,
+                              int32_t *counts = nullptr);
 
 cudaError_t launch_sparse_attn(const LaunchCtx &c, const void *q, const void *k, const void *v,
                                const int32_t *bt, const int32_t *seq_lens, const int32_t *q_seq,
@@ -40,13 +41,15 @@ cudaError_t launch_prefill_index_gemm(const LaunchCtx &c, const void *idx_q, con
                                       const int32_t *bt_row, const int32_t *seq_len_ptr, const int32_t *q_pos,
                                       int n_q, int max_blocks, int num_pages, float *scores, int32_t *dev_err);
 
-// Block-centric prefill attention (selection inverted per block, one CTA per (block, head),
-// per-slot partials merged per (query, head)).  Workspace regions, 256-byte aligned.
+// Block-centric prefill attention (selection inverted per block, tensor-core items of 16
+// entries per (block, head), per-slot partials merged per (query, head)).  Workspace regions,
+// 256-byte aligned.
 struct PrefillAttnWs {
-    size_t counts_off, offsets_off, cursor_off, list_off, ml_off, acc_off;
+    size_t counts_off, offsets_off, cursor_off, n_items_off, items_off, list_off, ml_off, acc_off;
 };
 size_t prefill_attn_workspace(int n_q, int H, int max_blocks, PrefillAttnWs *w);
-// `ws` must start with max_blocks zeroed int32 counts (the caller clears them).
+// `ws` must start with the per-block selection counts of `sel` (max_blocks int32), as
+// launch_block_topk writes them when given `counts` zeroed.
 cudaError_t launch_prefill_attn(const LaunchCtx &c, const void *q, const void *k, const void *v,
                                 const int32_t *bt_row, const int32_t *q_pos, const int32_t *sel, int n_q, int H,
                                 int max_blocks, int num_pages, float scale, void *out, void *ws,

@@ -8,17 +8,31 @@
 // a 2048-query chunk, and ~130 times for the local-window blocks that 32
 // consecutive queries share.  Instead:
 //   1. invert the selection: per logical block, the list of (query, slot)
-//      entries that selected it (count with atomics, one-CTA exclusive scan,
-//      fill);
-//   2. one CTA per (block, head) copies the block's K and V tiles (2 x 8 KiB)
-//      into shared memory with 1-D bulk copies (TMA) and runs every entry of
-//      its list against them, one warp per entry, writing the entry's partial
-//      softmax state (m, l, acc[128]) to the workspace.  Blocks are visited
-//      from the last one down, so the heavily shared local-window blocks start
-//      first;
-//   3. one CTA per (query, head) merges its 16 partials (flash-decoding) and
+//      entries that selected it (the top-k kernel counts them, a one-CTA
+//      exclusive scan places the lists and cuts them into items of 16 entries,
+//      a fill kernel writes them);
+//   2. one warp per (item, head) computes the item's 16 x 32 score tile
+//      S = Q K^T and, after a register-resident fp32 softmax per row, the
+//      16 x 128 tile P V on the tensor cores (mma.sync m16n8k16, bf16 in, fp32
+//      accumulate), writing each entry's partial softmax state (m, l, acc[128]);
+//   3. one warp per (query, head) merges the 16 partials (flash-decoding) and
 //      writes the bf16 output.
-// Each (block, head) tile is read from memory once per chunk.
+// Each (block, head) tile is read from memory once per chunk (an item after the
+// first of the same tile finds it in L2).
+//
+// Tensor-core layout of step 2.  The contraction index of S = Q K^T is the head
+// dimension, and any permutation of it applied to both operands leaves S
+// unchanged; this kernel assigns lane (r, t) = (lane / 4, lane % 4) the dims
+// 32u + 8t .. 32u + 8t + 7 for the k-steps 2u and 2u + 1, so that every A (query)
+// and B (key) fragment is one 16-byte load of a row: no shared memory and no
+// shuffles for S.  P V needs V transposed: the warp copies its V tile into shared
+// memory with cp.async, 16-byte chunk c of token x at chunk position c ^ (x & 7),
+// and ldmatrix.trans reads it without bank conflicts.  P is rounded to bf16 for
+// the tensor cores and the row sum l is taken over the rounded weights, so the
+// output is an exact convex combination of the values.  A (block, head) item
+// holds 16 entries -- a remote block is chosen by ~12 queries of a chunk on
+// average -- which is below the 64-row minimum tile of tcgen05; the work is
+// bound by the HBM reads of the tiles and the partials, not by tensor math.
 #include <cuda_bf16.h>
 #include <math.h>
 
@@ -30,55 +44,95 @@ namespace uocr {
 namespace {
 constexpr int kInvThreads = 256;
 constexpr int kScanThreads = 1024;
-constexpr int kBAWarps = 4;
-}  // namespace
+constexpr int kMmaWarps = 4;
+constexpr int kItemRows = 16;
+constexpr int kMergeWarps = 8;
 
-__global__ void __launch_bounds__(kInvThreads)
-prefill_count_kernel(const int32_t *__restrict__ sel, int n_entries, int max_blocks, int32_t *counts) {
-    pdl_wait();
-    const int e = blockIdx.x * kInvThreads + threadIdx.x;
-    if (e < n_entries) {
-        const int j = sel[e];
-        if (j >= 0 && j < max_blocks) atomicAdd(counts + j, 1);
-    }
+__device__ __forceinline__ void cp_async16(uint32_t dst, const void *src) {
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst), "l"(src) : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+__device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_group 0;" ::: "memory"); }
+
+__device__ __forceinline__ void ldsm_x4_trans(uint32_t (&d)[4], uint32_t addr) {
+    asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0, %1, %2, %3}, [%4];"
+                 : "=r"(d[0]), "=r"(d[1]), "=r"(d[2]), "=r"(d[3])
+                 : "r"(addr)
+                 : "memory");
 }
 
-// One CTA: offsets = exclusive prefix sum of counts; cursor = offsets.
+// d += A (16 x 16, row) * B (16 x 8, col); bf16 operands, fp32 accumulators.
+__device__ __forceinline__ void mma_bf16(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
+                                         uint32_t b0, uint32_t b1) {
+    asm volatile(
+        "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, {%8, %9}, "
+        "{%0, %1, %2, %3};"
+        : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+        : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+
+// bf16 pair (lo in the low half) and the sum of the two rounded values.
+__device__ __forceinline__ uint32_t pack_bf16(float lo, float hi, float &sum) {
+    const __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
+    sum += __low2float(v) + __high2float(v);
+    return *reinterpret_cast<const uint32_t *>(&v);
+}
+}  // namespace
+
+// One CTA: offsets = exclusive prefix sum of counts, cursor = offsets, and the work items:
+// block j with n_j entries gives items (j, 0) .. (j, ceil(n_j / 16) - 1), in block order.
 __global__ void __launch_bounds__(kScanThreads)
 prefill_scan_kernel(const int32_t *__restrict__ counts, int max_blocks, int32_t *__restrict__ offsets,
-                    int32_t *__restrict__ cursor) {
-    __shared__ int warp_tot[kScanThreads / 32];
+                    int32_t *__restrict__ cursor, int2 *__restrict__ items, int32_t *__restrict__ n_items) {
+    __shared__ int s_tot[2][kScanThreads / 32];
     pdl_wait();
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int per = (max_blocks + kScanThreads - 1) / kScanThreads;
-    const int lo = tid * per, hi = min(max_blocks, lo + per);
-    int mine = 0;
-    for (int j = lo; j < hi; ++j) mine += counts[j];
-    int incl = mine;
+    const int lo = min(max_blocks, tid * per), hi = min(max_blocks, lo + per);
+    int mine_c = 0, mine_g = 0;
+    for (int j = lo; j < hi; ++j) {
+        const int c = counts[j];
+        mine_c += c;
+        mine_g += (c + kItemRows - 1) / kItemRows;
+    }
+    int inc_c = mine_c, inc_g = mine_g;
 #pragma unroll
     for (int o = 1; o < 32; o <<= 1) {
-        const int n = __shfl_up_sync(0xffffffffu, incl, o);
-        if (lane >= o) incl += n;
+        const int nc = __shfl_up_sync(0xffffffffu, inc_c, o);
+        const int ng = __shfl_up_sync(0xffffffffu, inc_g, o);
+        if (lane >= o) {
+            inc_c += nc;
+            inc_g += ng;
+        }
     }
-    if (lane == 31) warp_tot[warp] = incl;
+    if (lane == 31) {
+        s_tot[0][warp] = inc_c;
+        s_tot[1][warp] = inc_g;
+    }
     __syncthreads();
-    if (warp == 0) {
-        const int w = warp_tot[lane];
+    if (warp < 2) {
+        const int w = s_tot[warp][lane];
         int wi = w;
 #pragma unroll
         for (int o = 1; o < 32; o <<= 1) {
             const int n = __shfl_up_sync(0xffffffffu, wi, o);
             if (lane >= o) wi += n;
         }
-        warp_tot[lane] = wi - w;
+        s_tot[warp][lane] = wi - w;
     }
     __syncthreads();
-    int run = warp_tot[warp] + incl - mine;
+    int run_c = s_tot[0][warp] + inc_c - mine_c;
+    int run_g = s_tot[1][warp] + inc_g - mine_g;
     for (int j = lo; j < hi; ++j) {
-        offsets[j] = run;
-        cursor[j] = run;
-        run += counts[j];
+        const int c = counts[j];
+        offsets[j] = run_c;
+        cursor[j] = run_c;
+        const int g = (c + kItemRows - 1) / kItemRows;
+        for (int k = 0; k < g; ++k) items[run_g + k] = make_int2(j, k);
+        run_c += c;
+        run_g += g;
     }
+    if (tid == kScanThreads - 1) *n_items = run_g;
 }
 
 __global__ void __launch_bounds__(kInvThreads)
@@ -92,129 +146,200 @@ prefill_fill_kernel(const int32_t *__restrict__ sel, int n_entries, int max_bloc
     }
 }
 
-__global__ void __launch_bounds__(kBAWarps * 32)
-prefill_block_attn_kernel(const uint4 *__restrict__ q, const uint4 *__restrict__ kc, const uint4 *__restrict__ vc,
-                          const int32_t *__restrict__ bt_row, const int32_t *__restrict__ q_pos,
-                          const int32_t *__restrict__ counts, const int32_t *__restrict__ offsets,
-                          const int32_t *__restrict__ list, int H, int max_blocks, int num_pages, float scale_log2,
-                          float *__restrict__ part_acc, float *__restrict__ part_ml, int32_t *dev_err) {
-    __shared__ __align__(128) uint4 s_k[kPageElems / 8];
-    __shared__ __align__(128) uint4 s_v[kPageElems / 8];
-    __shared__ __align__(8) uint64_t s_bar;
-
-    const int j = max_blocks - 1 - (int)(blockIdx.x / H);
-    const int h = (int)(blockIdx.x % H);
-    const int warp = threadIdx.x >> 5;
-    const int lane = threadIdx.x & 31;
+// Persistent: warp w takes work units w, w + (warps in the grid), ...; unit = (item, head),
+// heads innermost so that the items of one block run side by side.
+__global__ void __launch_bounds__(kMmaWarps * 32)
+prefill_block_mma_kernel(const uint4 *__restrict__ q, const uint4 *__restrict__ kc, const uint4 *__restrict__ vc,
+                         const int32_t *__restrict__ bt_row, const int32_t *__restrict__ q_pos,
+                         const int32_t *__restrict__ counts, const int32_t *__restrict__ offsets,
+                         const int32_t *__restrict__ list, const int2 *__restrict__ items,
+                         const int32_t *__restrict__ n_items, int H, int num_pages, float scale_log2,
+                         float *__restrict__ part_acc, float *__restrict__ part_ml, int32_t *dev_err) {
+    __shared__ __align__(128) uint4 s_v[kMmaWarps][kPageElems / 8];
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int r = lane >> 2, t = lane & 3;
+    const uint32_t sv = smem_addr(s_v[warp]);
 
     pdl_wait();
-    const int n = counts[j];
-    if (n == 0) return;
-    const int off = offsets[j];
-    const int page = __ldg(bt_row + j);
-    bool have = (unsigned)page < (unsigned)num_pages;
-    if (!have && threadIdx.x == 0) flag_error(dev_err, UOCR_DEVERR_PAGE);
+    const int n_work = __ldg(n_items) * H;
+    for (int w = blockIdx.x * kMmaWarps + warp; w < n_work; w += gridDim.x * kMmaWarps) {
+        const int item = w / H, h = w - item * H;
+        const int2 it = __ldg(items + item);
+        const int j = it.x, g = it.y;
+        const int rows = min(kItemRows, __ldg(counts + j) - g * kItemRows);
+        const int e0 = __ldg(offsets + j) + g * kItemRows;
+        // rows r and r + 8 of the item (rows past its end repeat its last entry and store nothing)
+        const int ent_a = __ldg(list + e0 + min(r, rows - 1));
+        const int ent_b = __ldg(list + e0 + min(r + 8, rows - 1));
+        const int ia = ent_a >> 4, ib = ent_b >> 4;
+        const int page = __ldg(bt_row + j);
 
-    if (have) {
-        if (threadIdx.x == 0) {
+        float o[16][4];
+#pragma unroll
+        for (int n = 0; n < 16; ++n) o[n][0] = o[n][1] = o[n][2] = o[n][3] = 0.f;
+        float ma = -INFINITY, mb = -INFINITY, la = 0.f, lb = 0.f;
+        if ((unsigned)page < (unsigned)num_pages) {
             const size_t tile = ((size_t)page * H + h) * (kPageElems / 8);
-            mbar_init(&s_bar, 1);
-            fence_mbar_init();
-            mbar_arrive_expect_tx(&s_bar, 2 * kPageElems * 2);
-            bulk_copy_g2s(s_k, kc + tile, kPageElems * 2, &s_bar);
-            bulk_copy_g2s(s_v, vc + tile, kPageElems * 2, &s_bar);
-        }
-        __syncthreads();
-        if (!mbar_wait_timed(&s_bar, 0, 2000000000ull, nullptr)) {
-            if (threadIdx.x == 0) flag_error(dev_err, UOCR_DEVERR_TIMEOUT);
-            mbar_wait_timed(&s_bar, 0, 2000000000ull, nullptr);
-            have = false;
-        }
-    }
+            __syncwarp();   // the previous unit's ldmatrix reads of this warp's V buffer are done
+#pragma unroll
+            for (int k = 0; k < 16; ++k) {
+                const int x = k * 32 + lane, tok = x >> 4, c = x & 15;
+                cp_async16(sv + (uint32_t)((tok * 16 + (c ^ (tok & 7))) * 16), vc + tile + x);
+            }
+            cp_async_commit();
 
-    const int tok = 2 * (lane & 15) + (lane >> 4);
-    for (int e = warp; e < n; e += kBAWarps) {
-        const int entry = __ldg(list + off + e);
-        const int i = entry >> 4;
-        const size_t slot = ((size_t)i * H + h) * kSel + (entry & 15);
-        float m_w = -INFINITY, l_w = 0.f;
-        float acc[8];
+            uint4 qa[4], qb[4], kf[4][4];
+            const uint4 *qpa = q + ((size_t)ia * H + h) * (kD / 8) + t;
+            const uint4 *qpb = q + ((size_t)ib * H + h) * (kD / 8) + t;
 #pragma unroll
-        for (int c = 0; c < 8; ++c) acc[c] = 0.f;
-        if (have) {
-            const int p = __ldg(q_pos + i);
-            float qf[8];
-            bf16x8_to_f32(__ldg(q + ((size_t)i * H + h) * (kD / 8) + (lane & 15)), qf);
-            float z[16];
-#pragma unroll
-            for (int t = 0; t < 16; ++t) {
-                float kf[8];
-                bf16x8_to_f32(s_k[t * 32 + lane], kf);
-                float a = qf[0] * kf[0];
-#pragma unroll
-                for (int c = 1; c < 8; ++c) a = fmaf(qf[c], kf[c], a);
-                z[t] = a;
-            }
-            float zt = half_warp_transpose_sum16(z, lane) * scale_log2;
-            if (j * kBlock + tok > p) zt = -INFINITY;
-            m_w = warp_max(zt);                   // finite: a selected block has token 32j <= p
-            const float pt = exp2f(zt - m_w);
-            l_w = warp_sum(pt);
-#pragma unroll
-            for (int t = 0; t < 16; ++t) {
-                const float w = __shfl_sync(0xffffffffu, pt, (lane & 16) | t);
-                float vf[8];
-                bf16x8_to_f32(s_v[t * 32 + lane], vf);
-#pragma unroll
-                for (int c = 0; c < 8; ++c) acc[c] = fmaf(w, vf[c], acc[c]);
+            for (int u = 0; u < 4; ++u) {
+                qa[u] = __ldg(qpa + 4 * u);
+                qb[u] = __ldg(qpb + 4 * u);
             }
 #pragma unroll
-            for (int c = 0; c < 8; ++c) acc[c] += __shfl_xor_sync(0xffffffffu, acc[c], 16);
+            for (int nt = 0; nt < 4; ++nt)
+#pragma unroll
+                for (int u = 0; u < 4; ++u) kf[nt][u] = __ldg(kc + tile + (8 * nt + r) * (kD / 8) + 4 * u + t);
+
+            // S = Q K^T: rows r, r + 8; columns (tokens) 8 nt + 2t, 8 nt + 2t + 1
+            float s[4][4];
+#pragma unroll
+            for (int nt = 0; nt < 4; ++nt) s[nt][0] = s[nt][1] = s[nt][2] = s[nt][3] = 0.f;
+#pragma unroll
+            for (int u = 0; u < 4; ++u)
+#pragma unroll
+                for (int hf = 0; hf < 2; ++hf) {
+                    const uint32_t a0 = hf ? qa[u].z : qa[u].x, a1 = hf ? qb[u].z : qb[u].x;
+                    const uint32_t a2 = hf ? qa[u].w : qa[u].y, a3 = hf ? qb[u].w : qb[u].y;
+#pragma unroll
+                    for (int nt = 0; nt < 4; ++nt)
+                        mma_bf16(s[nt], a0, a1, a2, a3, hf ? kf[nt][u].z : kf[nt][u].x,
+                                 hf ? kf[nt][u].w : kf[nt][u].y);
+                }
+
+            // causal mask t <= p, scale, row maxima over the quad
+            const int pa = __ldg(q_pos + ia), pb = __ldg(q_pos + ib);
+            const int t0 = j * kBlock + 2 * t;
+#pragma unroll
+            for (int nt = 0; nt < 4; ++nt)
+#pragma unroll
+                for (int e = 0; e < 2; ++e) {
+                    const int tok = t0 + 8 * nt + e;
+                    s[nt][e] = tok <= pa ? s[nt][e] * scale_log2 : -INFINITY;
+                    s[nt][2 + e] = tok <= pb ? s[nt][2 + e] * scale_log2 : -INFINITY;
+                    ma = fmaxf(ma, s[nt][e]);
+                    mb = fmaxf(mb, s[nt][2 + e]);
+                }
+#pragma unroll
+            for (int x = 1; x < 4; x <<= 1) {
+                ma = fmaxf(ma, __shfl_xor_sync(0xffffffffu, ma, x));
+                mb = fmaxf(mb, __shfl_xor_sync(0xffffffffu, mb, x));
+            }
+            // finite: a selected block holds a token at or before the query
+            uint32_t pf[4][2];
+#pragma unroll
+            for (int nt = 0; nt < 4; ++nt) {
+                pf[nt][0] = pack_bf16(exp2f(s[nt][0] - ma), exp2f(s[nt][1] - ma), la);
+                pf[nt][1] = pack_bf16(exp2f(s[nt][2] - mb), exp2f(s[nt][3] - mb), lb);
+            }
+#pragma unroll
+            for (int x = 1; x < 4; x <<= 1) {
+                la += __shfl_xor_sync(0xffffffffu, la, x);
+                lb += __shfl_xor_sync(0xffffffffu, lb, x);
+            }
+
+            // O = P V: k-steps of 16 tokens, n-tiles of 8 dims, V^T fragments by ldmatrix.trans
+            cp_async_wait_all();
+            __syncwarp();
+#pragma unroll
+            for (int kk = 0; kk < 2; ++kk) {
+                const int tok = 16 * kk + 8 * ((lane >> 3) & 1) + (lane & 7);
+#pragma unroll
+                for (int np = 0; np < 8; ++np) {
+                    const int c = 2 * np + (lane >> 4);
+                    uint32_t b[4];
+                    ldsm_x4_trans(b, sv + (uint32_t)((tok * 16 + (c ^ (tok & 7))) * 16));
+                    mma_bf16(o[2 * np], pf[2 * kk][0], pf[2 * kk][1], pf[2 * kk + 1][0], pf[2 * kk + 1][1], b[0],
+                             b[1]);
+                    mma_bf16(o[2 * np + 1], pf[2 * kk][0], pf[2 * kk][1], pf[2 * kk + 1][0], pf[2 * kk + 1][1],
+                             b[2], b[3]);
+                }
+            }
+        } else if (lane == 0) {
+            flag_error(dev_err, UOCR_DEVERR_PAGE);   // the entries get an empty partial
         }
-        if (lane < 16) {
-            float4 *dst = reinterpret_cast<float4 *>(part_acc + slot * kD + lane * 8);
-            dst[0] = make_float4(acc[0], acc[1], acc[2], acc[3]);
-            dst[1] = make_float4(acc[4], acc[5], acc[6], acc[7]);
+
+        if (r < rows) {
+            const size_t slot = ((size_t)ia * H + h) * kSel + (ent_a & 15);
+            float *dst = part_acc + slot * kD + 2 * t;
+#pragma unroll
+            for (int n = 0; n < 16; ++n) *reinterpret_cast<float2 *>(dst + 8 * n) = make_float2(o[n][0], o[n][1]);
+            if (t == 0) *reinterpret_cast<float2 *>(part_ml + slot * 2) = make_float2(ma, la);
         }
-        if (lane == 0) {
-            part_ml[slot * 2] = m_w;
-            part_ml[slot * 2 + 1] = l_w;
+        if (r + 8 < rows) {
+            const size_t slot = ((size_t)ib * H + h) * kSel + (ent_b & 15);
+            float *dst = part_acc + slot * kD + 2 * t;
+#pragma unroll
+            for (int n = 0; n < 16; ++n) *reinterpret_cast<float2 *>(dst + 8 * n) = make_float2(o[n][2], o[n][3]);
+            if (t == 0) *reinterpret_cast<float2 *>(part_ml + slot * 2) = make_float2(mb, lb);
         }
     }
 }
 
-// One CTA per (query, head); thread d owns output dim d.
-__global__ void __launch_bounds__(kD)
+// One warp per (query, head): lanes 0..15 hold the 16 slots' (m, l), every lane 4 output dims.
+__global__ void __launch_bounds__(kMergeWarps * 32)
 prefill_merge_kernel(const int32_t *__restrict__ sel, const float *__restrict__ part_acc,
-                     const float *__restrict__ part_ml, int H, __nv_bfloat16 *__restrict__ out) {
-    const int ih = blockIdx.x;
-    const int i = ih / H;
-    const int d = threadIdx.x;
+                     const float *__restrict__ part_ml, int n_q, int H, __nv_bfloat16 *__restrict__ out) {
+    const int lane = threadIdx.x & 31;
+    const long long ih = (long long)blockIdx.x * kMergeWarps + (threadIdx.x >> 5);
     pdl_wait();
-    float M = -INFINITY;
-    int valid = 0;
+    if (ih >= (long long)n_q * H) return;
+    const long long i = ih / H;
+    const int s = lane & 15;
+    const size_t base = (size_t)ih * kSel;
+    const bool valid = __ldg(sel + i * kSel + s) >= 0;
+    const float m = valid ? __ldcs(part_ml + (base + s) * 2) : -INFINITY;
+    const float l = valid ? __ldcs(part_ml + (base + s) * 2 + 1) : 0.f;
+    const unsigned vmask = __ballot_sync(0xffffffffu, valid);
+    float4 v[kSel];
+#pragma unroll
+    for (int k = 0; k < kSel; ++k)
+        v[k] = (vmask >> k & 1u) ? __ldcs(reinterpret_cast<const float4 *>(part_acc + (base + k) * kD) + lane)
+                                 : make_float4(0.f, 0.f, 0.f, 0.f);
+    float M = m;
+#pragma unroll
+    for (int x = 8; x > 0; x >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, x));
+    const float f = M == -INFINITY ? 0.f : exp2f(m - M);
+    float L = l * f;
+#pragma unroll
+    for (int x = 8; x > 0; x >>= 1) L += __shfl_xor_sync(0xffffffffu, L, x);
+    float4 A = make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll
     for (int k = 0; k < kSel; ++k) {
-        if (__ldg(sel + (size_t)i * kSel + k) >= 0) {
-            valid |= 1 << k;
-            M = fmaxf(M, part_ml[((size_t)ih * kSel + k) * 2]);
-        }
+        const float fk = __shfl_sync(0xffffffffu, f, k);
+        A.x = fmaf(fk, v[k].x, A.x);
+        A.y = fmaf(fk, v[k].y, A.y);
+        A.z = fmaf(fk, v[k].z, A.z);
+        A.w = fmaf(fk, v[k].w, A.w);
     }
-    float L = 0.f, A = 0.f;
-    if (M != -INFINITY) {
-#pragma unroll
-        for (int k = 0; k < kSel; ++k) {
-            if (!(valid >> k & 1)) continue;
-            const size_t slot = (size_t)ih * kSel + k;
-            const float f = exp2f(part_ml[slot * 2] - M);
-            L = fmaf(part_ml[slot * 2 + 1], f, L);
-            A = fmaf(part_acc[slot * kD + d], f, A);
-        }
-    }
-    out[(size_t)ih * kD + d] = __float2bfloat16_rn(L > 0.f ? A / L : 0.f);
+    const float inv = L > 0.f ? 1.f / L : 0.f;
+    __nv_bfloat162 lo = __floats2bfloat162_rn(A.x * inv, A.y * inv);
+    __nv_bfloat162 hi = __floats2bfloat162_rn(A.z * inv, A.w * inv);
+    uint2 pk;
+    pk.x = *reinterpret_cast<uint32_t *>(&lo);
+    pk.y = *reinterpret_cast<uint32_t *>(&hi);
+    reinterpret_cast<uint2 *>(out + (size_t)ih * kD)[lane] = pk;
 }
 
 // ------------------------------------------------------------------ host side
+namespace {
+// Items of 16 entries: at most one partly filled item per block that was selected at all.
+size_t item_bound(int n_q, int max_blocks) {
+    const size_t n_entries = (size_t)n_q * kSel;
+    return n_entries / kItemRows + (n_entries < (size_t)max_blocks ? n_entries : (size_t)max_blocks) + 1;
+}
+}  // namespace
+
 size_t prefill_attn_workspace(int n_q, int H, int max_blocks, PrefillAttnWs *w) {
     auto up = [](size_t x) { return (x + 255) / 256 * 256; };
     size_t off = 0;
@@ -225,6 +350,10 @@ size_t prefill_attn_workspace(int n_q, int H, int max_blocks, PrefillAttnWs *w) 
     off += up((size_t)max_blocks * 4);
     l.cursor_off = off;
     off += up((size_t)max_blocks * 4);
+    l.n_items_off = off;
+    off += up(4);
+    l.items_off = off;
+    off += up(item_bound(n_q, max_blocks) * sizeof(int2));
     l.list_off = off;
     off += up((size_t)n_q * kSel * 4);
     l.ml_off = off;
@@ -242,9 +371,11 @@ cudaError_t launch_prefill_attn(const LaunchCtx &c, const void *q, const void *k
     PrefillAttnWs w;
     prefill_attn_workspace(n_q, H, max_blocks, &w);
     char *base = (char *)ws;
-    int32_t *counts = (int32_t *)(base + w.counts_off);
+    const int32_t *counts = (const int32_t *)(base + w.counts_off);
     int32_t *offsets = (int32_t *)(base + w.offsets_off);
     int32_t *cursor = (int32_t *)(base + w.cursor_off);
+    int32_t *n_items = (int32_t *)(base + w.n_items_off);
+    int2 *items = (int2 *)(base + w.items_off);
     int32_t *list = (int32_t *)(base + w.list_off);
     float *ml = (float *)(base + w.ml_off);
     float *acc = (float *)(base + w.acc_off);
@@ -258,29 +389,30 @@ cudaError_t launch_prefill_attn(const LaunchCtx &c, const void *q, const void *k
     cfg.attrs = attr;
     cfg.numAttrs = 1;   // every kernel here follows another kernel of the same call
 
-    cfg.gridDim = dim3((unsigned)((n_entries + kInvThreads - 1) / kInvThreads));
-    cfg.blockDim = dim3(kInvThreads);
-    cudaError_t e = cudaLaunchKernelEx(&cfg, prefill_count_kernel, sel, n_entries, max_blocks, counts);
-    if (e != cudaSuccess) return e;
     cfg.gridDim = dim3(1);
     cfg.blockDim = dim3(kScanThreads);
-    e = cudaLaunchKernelEx(&cfg, prefill_scan_kernel, (const int32_t *)counts, max_blocks, offsets, cursor);
+    cudaError_t e = cudaLaunchKernelEx(&cfg, prefill_scan_kernel, counts, max_blocks, offsets, cursor, items, n_items);
     if (e != cudaSuccess) return e;
     cfg.gridDim = dim3((unsigned)((n_entries + kInvThreads - 1) / kInvThreads));
     cfg.blockDim = dim3(kInvThreads);
     e = cudaLaunchKernelEx(&cfg, prefill_fill_kernel, sel, n_entries, max_blocks, cursor, list);
     if (e != cudaSuccess) return e;
-    const long long ctas = (long long)max_blocks * H;
-    if (ctas > 0x7fffffffLL) return cudaErrorInvalidConfiguration;
-    cfg.gridDim = dim3((unsigned)ctas);
-    cfg.blockDim = dim3(kBAWarps * 32);
-    e = cudaLaunchKernelEx(&cfg, prefill_block_attn_kernel, (const uint4 *)q, (const uint4 *)k, (const uint4 *)v,
-                           bt_row, q_pos, (const int32_t *)counts, (const int32_t *)offsets, (const int32_t *)list,
-                           H, max_blocks, num_pages, scale * kLog2e, acc, ml, dev_err);
+
+    int per_sm = 0;
+    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, prefill_block_mma_kernel, kMmaWarps * 32, 0);
     if (e != cudaSuccess) return e;
-    cfg.gridDim = dim3((unsigned)(n_q * H));
-    cfg.blockDim = dim3(kD);
-    return cudaLaunchKernelEx(&cfg, prefill_merge_kernel, sel, (const float *)acc, (const float *)ml, H,
+    cfg.gridDim = dim3((unsigned)(c.num_sms * (per_sm > 0 ? per_sm : 1)));
+    cfg.blockDim = dim3(kMmaWarps * 32);
+    e = cudaLaunchKernelEx(&cfg, prefill_block_mma_kernel, (const uint4 *)q, (const uint4 *)k, (const uint4 *)v,
+                           bt_row, q_pos, counts, (const int32_t *)offsets, (const int32_t *)list,
+                           (const int2 *)items, (const int32_t *)n_items, H, num_pages, scale * kLog2e, acc, ml,
+                           dev_err);
+    if (e != cudaSuccess) return e;
+    const long long merge_ctas = ((long long)n_q * H + kMergeWarps - 1) / kMergeWarps;
+    if (merge_ctas > 0x7fffffffLL) return cudaErrorInvalidConfiguration;
+    cfg.gridDim = dim3((unsigned)merge_ctas);
+    cfg.blockDim = dim3(kMergeWarps * 32);
+    return cudaLaunchKernelEx(&cfg, prefill_merge_kernel, sel, (const float *)acc, (const float *)ml, n_q, H,
                               (__nv_bfloat16 *)out);
 }
 

@@ -1,8 +1,9 @@
 // topk_core.cuh -- the per-query block selection of the walk-through
 // (news.rkmt.cn/news/25027, section 五 step 3): 4 local blocks + the 12
 // highest-scoring remote blocks (score desc, then lower id), optionally limited
-// to the candidates of a page-aware bitmap.  Shared by block_topk_kernel (one
-// CTA of 512 threads per query) and the fused decode kernel (256 threads).
+// to the candidates of a page-aware bitmap.  topk_select runs one query on a
+// CTA (few long rows: decode); topk_warp_select runs one query on a warp (many
+// rows: a prefill chunk), with the same steps at warp scope.
 //
 // Every candidate's ranking key is the 64-bit composite
 // (order-preserving fp32 key << 32 | ~id): distinct, larger for a higher score
@@ -268,6 +269,179 @@ __device__ void topk_select(const float *row, int nb, const uint32_t *mask, uint
         if (lane < kLocal) out[kRemote + lane] = nb - kLocal + lane;
     }
     (void)kW;
+}
+
+// ------------------------------------------------------------ one warp per query
+constexpr int kWarpSurvivorCap = 256;       // per-warp survivor list (2 KiB)
+
+struct TopkWarpShared {
+    uint64_t surv[kWarpSurvivorCap];
+    uint64_t top[kRemote];
+};
+
+// The 12 remote ids of `top` ascending into out[0..11], the local blocks into out[12..15].
+__device__ __forceinline__ void topk_warp_emit(const uint64_t *top, int nb, int lane, int32_t *out) {
+    const int id = lane < kRemote ? (int)~(uint32_t)(top[lane] & 0xffffffffu) : 0x7fffffff;
+    int rank = 0;
+#pragma unroll
+    for (int k = 0; k < kRemote; ++k) rank += __shfl_sync(0xffffffffu, id, k) < id;
+    if (lane < kRemote) out[rank] = id;
+    if (lane < kLocal) out[kRemote + lane] = nb - kLocal + lane;
+}
+
+// Keys of the 4 candidates j .. j + 3 (j % 4 == 0, all < nc) from one aligned 16-byte load;
+// the 4 share one word of the candidate mask.
+__device__ __forceinline__ void keys4(const float *row, const uint32_t *mask, int j, uint32_t (&k)[4]) {
+    const float4 v = __ldcg(reinterpret_cast<const float4 *>(row + j));
+    const uint32_t mw = mask ? __ldg(mask + (j >> 5)) >> (j & 31) : 0xfu;
+    k[0] = (mw & 1u) ? order_key(v.x) : 0u;
+    k[1] = (mw & 2u) ? order_key(v.y) : 0u;
+    k[2] = (mw & 4u) ? order_key(v.z) : 0u;
+    k[3] = (mw & 8u) ? order_key(v.w) : 0u;
+}
+
+constexpr int kRegQuads = 16;   // rows of up to 32 x 4 x 16 = 2048 candidates keep their keys in registers
+
+// Selection of one query with nb causal blocks by one warp.  Lane l holds the candidates
+// 4l .. 4l + 3, 4l + 128 .., read as aligned float4.  A row of at most 2048 candidates whose
+// start is 16-byte aligned is read once into registers (16 loads in flight per lane); other
+// rows are read twice from L2 (maxima, then survivors), in float4 where aligned.  Threshold
+// = the 12th largest of the 32 lane maxima; the survivors at or above it are ranked by
+// counting; more than kWarpSurvivorCap survivors (heavily tied scores) take the exact
+// fallback of 12 rounds of a warp-wide maximum.
+__device__ void topk_warp_select(const float *row, int nb, const uint32_t *mask, TopkWarpShared &sm,
+                                 int32_t *out) {
+    const int lane = threadIdx.x & 31;
+    const unsigned below = (1u << lane) - 1u;
+    const int nc = nb - kLocal > 0 ? nb - kLocal : 0;
+    if (nc <= kRemote && !mask) {
+        if (lane < kSel) out[lane] = lane < nb ? lane : -1;
+        return;
+    }
+    const KeySource key{nullptr, row, mask};
+    const bool aligned = (reinterpret_cast<uintptr_t>(row) & 15) == 0;
+    const bool in_regs = aligned && nc <= 128 * kRegQuads;
+    const int n_vec = aligned ? (nc & ~3) : 0;
+
+    uint32_t kr[kRegQuads][4];
+    uint32_t tmax = 0;
+    int allowed = 0;
+    if (in_regs) {
+#pragma unroll
+        for (int q = 0; q < kRegQuads; ++q) {
+            const int j = 128 * q + 4 * lane;
+            if (j + 3 < nc) {
+                keys4(row, mask, j, kr[q]);
+            } else {
+#pragma unroll
+                for (int e = 0; e < 4; ++e) kr[q][e] = j + e < nc ? key(j + e) : 0u;
+            }
+        }
+#pragma unroll
+        for (int q = 0; q < kRegQuads; ++q)
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                tmax = kr[q][e] > tmax ? kr[q][e] : tmax;
+                allowed += kr[q][e] != 0u;
+            }
+    } else {
+#pragma unroll 4
+        for (int j = 4 * lane; j < n_vec; j += 128) {
+            uint32_t k[4];
+            keys4(row, mask, j, k);
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                tmax = k[e] > tmax ? k[e] : tmax;
+                allowed += k[e] != 0u;
+            }
+        }
+        for (int j = n_vec + lane; j < nc; j += 32) {
+            const uint32_t k = key(j);
+            tmax = k > tmax ? k : tmax;
+            allowed += k != 0u;
+        }
+    }
+    if (mask && __reduce_add_sync(0xffffffffu, allowed) <= kRemote) {
+        // no more allowed candidates than remote slots: take them all, in id order
+        int pos = 0;
+        for (int base = 0; base < nc; base += 32) {
+            const int j = base + lane;
+            const bool take = j < nc && key(j) != 0u;
+            const unsigned m = __ballot_sync(0xffffffffu, take);
+            if (take) out[pos + __popc(m & below)] = j;
+            pos += __popc(m);
+        }
+        const int n_loc = nb < kLocal ? nb : kLocal;
+        if (lane < n_loc) out[pos + lane] = nb - n_loc + lane;
+        if (lane >= pos + n_loc && lane < kSel) out[lane] = -1;
+        return;
+    }
+
+    // the 12th largest lane maximum, with multiplicity
+    int gt = 0, ge = 0;
+#pragma unroll
+    for (int w = 0; w < 32; ++w) {
+        const uint32_t o = __shfl_sync(0xffffffffu, tmax, w);
+        gt += o > tmax;
+        ge += o >= tmax;
+    }
+    const unsigned who = __ballot_sync(0xffffffffu, gt <= kRemote - 1 && kRemote - 1 < ge);
+    const uint32_t thr = __shfl_sync(0xffffffffu, tmax, __ffs(who) - 1);
+
+    int n = 0;   // warp-uniform survivor count
+    auto append = [&](bool keep, uint32_t k, int j) {
+        const unsigned m = __ballot_sync(0xffffffffu, keep);
+        const int slot = n + __popc(m & below);
+        if (keep && slot < kWarpSurvivorCap) sm.surv[slot] = composite(k, j);
+        n += __popc(m);
+    };
+    // every lane runs the same number of iterations (the ballots need the whole warp)
+    if (in_regs) {
+#pragma unroll
+        for (int q = 0; q < kRegQuads; ++q)
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                const int j = 128 * q + 4 * lane + e;
+                append(j < nc && kr[q][e] >= thr, kr[q][e], j);
+            }
+    } else {
+#pragma unroll 4
+        for (int j0 = 0; j0 < n_vec; j0 += 128) {
+            const int j = j0 + 4 * lane;
+            uint32_t k[4] = {0u, 0u, 0u, 0u};
+            if (j < n_vec) keys4(row, mask, j, k);
+#pragma unroll
+            for (int e = 0; e < 4; ++e) append(j < n_vec && k[e] >= thr, k[e], j + e);
+        }
+        for (int j0 = n_vec; j0 < nc; j0 += 32) {
+            const int j = j0 + lane;
+            const uint32_t k = j < nc ? key(j) : 0u;
+            append(j < nc && k >= thr, k, j);
+        }
+    }
+    __syncwarp();
+    if (n <= kWarpSurvivorCap) {
+        for (int a = lane; a < n; a += 32) {
+            const uint64_t c = sm.surv[a];
+            int rank = 0;
+            for (int b = 0; b < n; ++b) rank += sm.surv[b] > c;
+            if (rank < kRemote) sm.top[rank] = c;
+        }
+    } else {
+        uint64_t cap = ~0ull;
+        uint64_t mine = best_below(key, lane, 32, nc, cap);
+#pragma unroll 1
+        for (int k = 0; k < kRemote; ++k) {
+            const uint64_t w = warp_max_u64(mine);
+            if (lane == 0) sm.top[k] = w;
+            if (mine == w && w != 0) {
+                cap = mine;
+                mine = best_below(key, lane, 32, nc, cap);
+            }
+        }
+    }
+    __syncwarp();
+    topk_warp_emit(sm.top, nb, lane, out);
 }
 
 }  // namespace uocr

@@ -67,6 +67,28 @@ def test_block_topk_is_exact_on_given_scores(uocr, cuda_device, kind):
         assert sel[b].cpu().tolist() == want.tolist(), f"row {b} (nb={nb})"
 
 
+@pytest.mark.parametrize("kind,mb", [("ties", 1024), ("normal", 1023), ("neg", 1024), ("ties", 1021)])
+def test_block_topk_many_rows_is_exact(uocr, cuda_device, kind, mb):
+    """Enough rows for the warp-per-row selection; odd row lengths give rows that start off a
+    16-byte boundary (scalar reads), 'ties' overflows the survivor list (exact fallback)."""
+    g = torch.Generator().manual_seed({"ties": 11, "normal": 12, "neg": 13}[kind] + mb)
+    n = 600
+    edge = [1, 128, 129, 512, 513, 544, 545, 1000, 32 * mb]
+    lens = edge + torch.randint(1, 32 * mb + 1, (n - len(edge),), generator=g).tolist()
+    if kind == "ties":
+        s = torch.randint(-4, 5, (n, mb), generator=g).float()
+    elif kind == "normal":
+        s = torch.randn(n, mb, generator=g)
+    else:
+        s = -torch.rand(n, mb, generator=g) - 1.0
+    seq_lens = torch.tensor(lens, dtype=torch.int32)
+    sel = uocr.block_topk(s.to(cuda_device), seq_lens.to(cuda_device)).cpu()
+    for b, L in enumerate(lens):
+        nb = (L - 1) // 32 + 1
+        want, _ = oracle.select(s[b].double().numpy(), nb)
+        assert sel[b].tolist() == want.tolist(), f"row {b} (nb={nb})"
+
+
 @pytest.mark.parametrize("heads", [1, 3, 10])
 def test_sparse_attn_matches_oracle(uocr, cuda_device, heads):
     lens = [1, 40, 128, 129, 600, 32 * 64, 32 * 100 + 5]

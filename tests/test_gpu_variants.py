@@ -100,6 +100,22 @@ def test_masked_topk_is_exact(uocr, cuda_device, density, kind):
         assert sel[b].cpu().tolist() == want.tolist(), (b, nb)
 
 
+@pytest.mark.parametrize("density,kind", [(0.5, "normal"), (0.01, "ties"), (1.0, "ties")])
+def test_masked_topk_many_rows_is_exact(uocr, cuda_device, density, kind):
+    """The warp-per-row selection (many rows) under a candidate mask."""
+    g = torch.Generator().manual_seed(int(density * 100) + 7)
+    n, mb = 600, 1024
+    lens = [1, 100, 128, 129, 545, 32 * mb] + torch.randint(1, 32 * mb + 1, (n - 6,), generator=g).tolist()
+    s = torch.randint(-4, 5, (n, mb), generator=g).float() if kind == "ties" else torch.randn(n, mb, generator=g)
+    mask = _random_mask(n, mb, density, seed=n)
+    sel = uocr.block_topk_masked(s.to(cuda_device), torch.tensor(lens, dtype=torch.int32, device=cuda_device),
+                                 torch.from_numpy(mask.view(np.int32)).to(cuda_device)).cpu()
+    for b, L in enumerate(lens):
+        nb = (L - 1) // 32 + 1
+        want, _ = oracle.select_masked(s[b].double().numpy(), nb, mask[b])
+        assert sel[b].tolist() == want.tolist(), (b, nb)
+
+
 def test_masked_selection_end_to_end(uocr, cuda_device):
     lens = [32 * 300, 32 * 64 + 5, 32 * 900]
     case = workloads.make_case(lens, shuffle=True, seed=12, device=cuda_device)
