@@ -531,7 +531,8 @@ def run_prefill(args):
                           "bytes_per_step": step_bytes, "flops_per_step": idx_flops + attn_flops},
         "breakdown_us": {"prefill_index_gemm": round(1e3 * gemm_ms, 2), "block_topk": round(1e3 * topk_ms, 2),
                          "sparse_attn": round(1e3 * attn_ms, 2), "prefill_call_graph": round(1e3 * call_ms, 2)},
-        "gpu_launches": args.steps * 3,
+        # per call: scoring GEMM, selection, scan, fill, block attention, merge
+        "gpu_launches": args.steps * 6,
         "clocks": clk.summary(),
     }
     if world > 1:

@@ -45,7 +45,7 @@ cudaError_t launch_prefill_index_gemm(const LaunchCtx &c, const void *idx_q, con
 // entries per (block, head), per-slot partials merged per (query, head)).  Workspace regions,
 // 256-byte aligned.
 struct PrefillAttnWs {
-    size_t counts_off, offsets_off, cursor_off, n_items_off, items_off, list_off, ml_off, acc_off;
+    size_t counts_off, cursor_off, n_items_off, items_off, list_off, ml_off, o_off;
 };
 size_t prefill_attn_workspace(int n_q, int H, int max_blocks, PrefillAttnWs *w);
 // `ws` must start with the per-block selection counts of `sel` (max_blocks int32), as

@@ -14,9 +14,15 @@
 //   2. one warp per (item, head) computes the item's 16 x 32 score tile
 //      S = Q K^T and, after a register-resident fp32 softmax per row, the
 //      16 x 128 tile P V on the tensor cores (mma.sync m16n8k16, bf16 in, fp32
-//      accumulate), writing each entry's partial softmax state (m, l, acc[128]);
-//   3. one warp per (query, head) merges the 16 partials (flash-decoding) and
-//      writes the bf16 output.
+//      accumulate), writing each entry's partial state: the row maximum m and
+//      the weight sum l in fp32, and the normalised output o = acc / l in bf16
+//      (the split-KV partial layout of FlashInfer's merge: the partial output
+//      in the output dtype, the softmax statistics in fp32; o is a convex
+//      combination of the values, so its rounding adds at most 2^-9 max|v| to
+//      the result, the size of the output's own bf16 rounding, and halves the
+//      partials' traffic);
+//   3. one warp per (query, head) merges the 16 partials, weight l 2^(m - M)
+//      each, and writes the bf16 output.
 // Each (block, head) tile is read from memory once per chunk (an item after the
 // first of the same tile finds it in L2).
 //
@@ -44,7 +50,7 @@ namespace uocr {
 namespace {
 constexpr int kInvThreads = 256;
 constexpr int kScanThreads = 1024;
-constexpr int kMmaWarps = 4;
+constexpr int kMmaWarps = 2;
 constexpr int kItemRows = 16;
 constexpr int kMergeWarps = 8;
 
@@ -53,6 +59,7 @@ __device__ __forceinline__ void cp_async16(uint32_t dst, const void *src) {
 }
 __device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
 __device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_group 0;" ::: "memory"); }
+__device__ __forceinline__ void cp_async_wait_1() { asm volatile("cp.async.wait_group 1;" ::: "memory"); }
 
 __device__ __forceinline__ void ldsm_x4_trans(uint32_t (&d)[4], uint32_t addr) {
     asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0, %1, %2, %3}, [%4];"
@@ -79,11 +86,13 @@ __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi, float &sum) {
 }
 }  // namespace
 
-// One CTA: offsets = exclusive prefix sum of counts, cursor = offsets, and the work items:
-// block j with n_j entries gives items (j, 0) .. (j, ceil(n_j / 16) - 1), in block order.
+// One CTA: cursor = exclusive prefix sum of counts (each block's first list position), and the
+// work items:
+// block j with n_j entries gives items (j, 0) .. (j, ceil(n_j / 16) - 1), in block order, each
+// recorded as {j, page of j, first entry, entries (<= 16)} so that a warp needs one load.
 __global__ void __launch_bounds__(kScanThreads)
-prefill_scan_kernel(const int32_t *__restrict__ counts, int max_blocks, int32_t *__restrict__ offsets,
-                    int32_t *__restrict__ cursor, int2 *__restrict__ items, int32_t *__restrict__ n_items) {
+prefill_scan_kernel(const int32_t *__restrict__ counts, const int32_t *__restrict__ bt_row, int max_blocks,
+                    int32_t *__restrict__ cursor, int4 *__restrict__ items, int32_t *__restrict__ n_items) {
     __shared__ int s_tot[2][kScanThreads / 32];
     pdl_wait();
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
@@ -125,170 +134,241 @@ prefill_scan_kernel(const int32_t *__restrict__ counts, int max_blocks, int32_t 
     int run_g = s_tot[1][warp] + inc_g - mine_g;
     for (int j = lo; j < hi; ++j) {
         const int c = counts[j];
-        offsets[j] = run_c;
         cursor[j] = run_c;
         const int g = (c + kItemRows - 1) / kItemRows;
-        for (int k = 0; k < g; ++k) items[run_g + k] = make_int2(j, k);
+        const int page = g ? __ldg(bt_row + j) : 0;
+        for (int k = 0; k < g; ++k)
+            items[run_g + k] = make_int4(j, page, run_c + k * kItemRows, min(kItemRows, c - k * kItemRows));
         run_c += c;
         run_g += g;
     }
     if (tid == kScanThreads - 1) *n_items = run_g;
 }
 
+// list[...] = {entry = query * 16 + slot, position of the query}, grouped by block.
 __global__ void __launch_bounds__(kInvThreads)
-prefill_fill_kernel(const int32_t *__restrict__ sel, int n_entries, int max_blocks, int32_t *cursor,
-                    int32_t *__restrict__ list) {
+prefill_fill_kernel(const int32_t *__restrict__ sel, const int32_t *__restrict__ q_pos, int n_entries,
+                    int max_blocks, int32_t *cursor, int2 *__restrict__ list) {
     pdl_wait();
     const int e = blockIdx.x * kInvThreads + threadIdx.x;
     if (e < n_entries) {
         const int j = sel[e];
-        if (j >= 0 && j < max_blocks) list[atomicAdd(cursor + j, 1)] = e;
+        if (j >= 0 && j < max_blocks) list[atomicAdd(cursor + j, 1)] = make_int2(e, __ldg(q_pos + e / kSel));
     }
 }
 
-// Persistent: warp w takes work units w, w + (warps in the grid), ...; unit = (item, head),
-// heads innermost so that the items of one block run side by side.
+// One unit of work: (item, head) and the item's record and entries.
+struct Unit {
+    int w;          // unit index, or -1 past the end
+    int j, page, rows, h;
+    int2 ea, eb;    // entries {query * 16 + slot, position} of rows r and r + 8
+};
+
+__device__ __forceinline__ Unit load_unit(int w, int n_work, int H, const int4 *items, const int2 *list, int r) {
+    Unit u;
+    u.w = w < n_work ? w : -1;
+    if (u.w < 0) {
+        u.j = u.page = u.h = 0;
+        u.rows = 1;
+        u.ea = u.eb = make_int2(0, 0);
+        return u;
+    }
+    const int4 rec = __ldg(items + w / H);
+    u.j = rec.x;
+    u.page = rec.y;
+    u.rows = rec.w;
+    u.h = w % H;
+    // rows past the item's end repeat its last entry and store nothing
+    u.ea = __ldg(list + rec.z + min(r, rec.w - 1));
+    u.eb = __ldg(list + rec.z + min(r + 8, rec.w - 1));
+    return u;
+}
+
+// Per-warp staging: 16-byte chunk c of row x of K and Q at chunk c ^ ((x & 1) << 2) (the
+// fragment reads touch two rows per 8-lane phase), of V at c ^ (x & 7) (ldmatrix.trans reads
+// eight consecutive rows of one chunk).
+struct WarpStage {
+    uint4 k[kBlock * kD / 8];
+    uint4 v[kBlock * kD / 8];
+    uint4 q[kItemRows * kD / 8];
+};
+
+// Persistent: warp w takes units w, w + (warps in the grid), ...; unit = (item, head), heads
+// innermost so that the items of one block run side by side.  Each warp pipelines its units:
+// the next unit's Q and K copies start once this unit's scores are computed, its V copy once
+// this unit's P V is done, so every copy overlaps the math of the unit before it
+// (cp.async groups, waited for with wait_group 1).
 __global__ void __launch_bounds__(kMmaWarps * 32)
 prefill_block_mma_kernel(const uint4 *__restrict__ q, const uint4 *__restrict__ kc, const uint4 *__restrict__ vc,
-                         const int32_t *__restrict__ bt_row, const int32_t *__restrict__ q_pos,
-                         const int32_t *__restrict__ counts, const int32_t *__restrict__ offsets,
-                         const int32_t *__restrict__ list, const int2 *__restrict__ items,
+                         const int2 *__restrict__ list, const int4 *__restrict__ items,
                          const int32_t *__restrict__ n_items, int H, int num_pages, float scale_log2,
-                         float *__restrict__ part_acc, float *__restrict__ part_ml, int32_t *dev_err) {
-    __shared__ __align__(128) uint4 s_v[kMmaWarps][kPageElems / 8];
+                         __nv_bfloat16 *__restrict__ part_o, float *__restrict__ part_ml, int32_t *dev_err) {
+    __shared__ __align__(128) WarpStage stage[kMmaWarps];
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int r = lane >> 2, t = lane & 3;
-    const uint32_t sv = smem_addr(s_v[warp]);
+    const uint32_t sk = smem_addr(stage[warp].k), sv = smem_addr(stage[warp].v), sq = smem_addr(stage[warp].q);
+    const uint4 *k_s = stage[warp].k, *q_s = stage[warp].q;
 
     pdl_wait();
     const int n_work = __ldg(n_items) * H;
-    for (int w = blockIdx.x * kMmaWarps + warp; w < n_work; w += gridDim.x * kMmaWarps) {
-        const int item = w / H, h = w - item * H;
-        const int2 it = __ldg(items + item);
-        const int j = it.x, g = it.y;
-        const int rows = min(kItemRows, __ldg(counts + j) - g * kItemRows);
-        const int e0 = __ldg(offsets + j) + g * kItemRows;
-        // rows r and r + 8 of the item (rows past its end repeat its last entry and store nothing)
-        const int ent_a = __ldg(list + e0 + min(r, rows - 1));
-        const int ent_b = __ldg(list + e0 + min(r + 8, rows - 1));
-        const int ia = ent_a >> 4, ib = ent_b >> 4;
-        const int page = __ldg(bt_row + j);
+    const int stride = gridDim.x * kMmaWarps;
 
-        float o[16][4];
+    auto page_ok = [&](const Unit &u) { return (unsigned)u.page < (unsigned)num_pages; };
+    // Q rows (16) and the K tile of unit u; then its V tile
+    auto issue_qk = [&](const Unit &u) {
+        if (u.w >= 0) {
 #pragma unroll
-        for (int n = 0; n < 16; ++n) o[n][0] = o[n][1] = o[n][2] = o[n][3] = 0.f;
-        float ma = -INFINITY, mb = -INFINITY, la = 0.f, lb = 0.f;
-        if ((unsigned)page < (unsigned)num_pages) {
-            const size_t tile = ((size_t)page * H + h) * (kPageElems / 8);
-            __syncwarp();   // the previous unit's ldmatrix reads of this warp's V buffer are done
+            for (int k = 0; k < 8; ++k) {
+                const int x = k * 32 + lane, row = x >> 4, c = x & 15;
+                const int src = (row & 7) * 4;
+                const int ea = __shfl_sync(0xffffffffu, u.ea.x, src), eb = __shfl_sync(0xffffffffu, u.eb.x, src);
+                const int ent = row < 8 ? ea : eb;
+                cp_async16(sq + (uint32_t)((row * 16 + (c ^ ((row & 1) << 2))) * 16),
+                           q + ((size_t)(ent >> 4) * H + u.h) * (kD / 8) + c);
+            }
+            if (page_ok(u)) {
+                const uint4 *src = kc + ((size_t)u.page * H + u.h) * (kPageElems / 8);
+#pragma unroll
+                for (int k = 0; k < 16; ++k) {
+                    const int x = k * 32 + lane, tok = x >> 4, c = x & 15;
+                    cp_async16(sk + (uint32_t)((tok * 16 + (c ^ ((tok & 1) << 2))) * 16), src + x);
+                }
+            }
+        }
+        cp_async_commit();
+    };
+    auto issue_v = [&](const Unit &u) {
+        if (u.w >= 0 && page_ok(u)) {
+            const uint4 *src = vc + ((size_t)u.page * H + u.h) * (kPageElems / 8);
 #pragma unroll
             for (int k = 0; k < 16; ++k) {
                 const int x = k * 32 + lane, tok = x >> 4, c = x & 15;
-                cp_async16(sv + (uint32_t)((tok * 16 + (c ^ (tok & 7))) * 16), vc + tile + x);
+                cp_async16(sv + (uint32_t)((tok * 16 + (c ^ (tok & 7))) * 16), src + x);
             }
-            cp_async_commit();
+        }
+        cp_async_commit();
+    };
 
-            uint4 qa[4], qb[4], kf[4][4];
-            const uint4 *qpa = q + ((size_t)ia * H + h) * (kD / 8) + t;
-            const uint4 *qpb = q + ((size_t)ib * H + h) * (kD / 8) + t;
-#pragma unroll
-            for (int u = 0; u < 4; ++u) {
-                qa[u] = __ldg(qpa + 4 * u);
-                qb[u] = __ldg(qpb + 4 * u);
-            }
-#pragma unroll
-            for (int nt = 0; nt < 4; ++nt)
-#pragma unroll
-                for (int u = 0; u < 4; ++u) kf[nt][u] = __ldg(kc + tile + (8 * nt + r) * (kD / 8) + 4 * u + t);
+    Unit cur = load_unit(blockIdx.x * kMmaWarps + warp, n_work, H, items, list, r);
+    if (cur.w < 0) return;
+    issue_qk(cur);
+    issue_v(cur);
+    Unit nxt = load_unit(cur.w + stride, n_work, H, items, list, r);
 
-            // S = Q K^T: rows r, r + 8; columns (tokens) 8 nt + 2t, 8 nt + 2t + 1
-            float s[4][4];
+    while (cur.w >= 0) {
+        // ---- S = Q K^T (rows r, r + 8; tokens 8 nt + 2t, 8 nt + 2t + 1) from this unit's Q, K
+        cp_async_wait_1();
+        __syncwarp();
+        float s[4][4];
 #pragma unroll
-            for (int nt = 0; nt < 4; ++nt) s[nt][0] = s[nt][1] = s[nt][2] = s[nt][3] = 0.f;
+        for (int nt = 0; nt < 4; ++nt) s[nt][0] = s[nt][1] = s[nt][2] = s[nt][3] = 0.f;
+        const int sw = (r & 1) << 2;
 #pragma unroll
-            for (int u = 0; u < 4; ++u)
+        for (int u = 0; u < 4; ++u) {
+            const uint4 qa = q_s[r * 16 + ((4 * u + t) ^ sw)];
+            const uint4 qb = q_s[(r + 8) * 16 + ((4 * u + t) ^ sw)];
+            uint4 kf[4];
 #pragma unroll
-                for (int hf = 0; hf < 2; ++hf) {
-                    const uint32_t a0 = hf ? qa[u].z : qa[u].x, a1 = hf ? qb[u].z : qb[u].x;
-                    const uint32_t a2 = hf ? qa[u].w : qa[u].y, a3 = hf ? qb[u].w : qb[u].y;
-#pragma unroll
-                    for (int nt = 0; nt < 4; ++nt)
-                        mma_bf16(s[nt], a0, a1, a2, a3, hf ? kf[nt][u].z : kf[nt][u].x,
-                                 hf ? kf[nt][u].w : kf[nt][u].y);
-                }
-
-            // causal mask t <= p, scale, row maxima over the quad
-            const int pa = __ldg(q_pos + ia), pb = __ldg(q_pos + ib);
-            const int t0 = j * kBlock + 2 * t;
-#pragma unroll
-            for (int nt = 0; nt < 4; ++nt)
-#pragma unroll
-                for (int e = 0; e < 2; ++e) {
-                    const int tok = t0 + 8 * nt + e;
-                    s[nt][e] = tok <= pa ? s[nt][e] * scale_log2 : -INFINITY;
-                    s[nt][2 + e] = tok <= pb ? s[nt][2 + e] * scale_log2 : -INFINITY;
-                    ma = fmaxf(ma, s[nt][e]);
-                    mb = fmaxf(mb, s[nt][2 + e]);
-                }
-#pragma unroll
-            for (int x = 1; x < 4; x <<= 1) {
-                ma = fmaxf(ma, __shfl_xor_sync(0xffffffffu, ma, x));
-                mb = fmaxf(mb, __shfl_xor_sync(0xffffffffu, mb, x));
-            }
-            // finite: a selected block holds a token at or before the query
-            uint32_t pf[4][2];
+            for (int nt = 0; nt < 4; ++nt) kf[nt] = k_s[(8 * nt + r) * 16 + ((4 * u + t) ^ sw)];
 #pragma unroll
             for (int nt = 0; nt < 4; ++nt) {
-                pf[nt][0] = pack_bf16(exp2f(s[nt][0] - ma), exp2f(s[nt][1] - ma), la);
-                pf[nt][1] = pack_bf16(exp2f(s[nt][2] - mb), exp2f(s[nt][3] - mb), lb);
+                mma_bf16(s[nt], qa.x, qb.x, qa.y, qb.y, kf[nt].x, kf[nt].y);
+                mma_bf16(s[nt], qa.z, qb.z, qa.w, qb.w, kf[nt].z, kf[nt].w);
             }
-#pragma unroll
-            for (int x = 1; x < 4; x <<= 1) {
-                la += __shfl_xor_sync(0xffffffffu, la, x);
-                lb += __shfl_xor_sync(0xffffffffu, lb, x);
-            }
+        }
+        __syncwarp();       // Q and K read: the next unit's copies may land
+        issue_qk(nxt);
 
-            // O = P V: k-steps of 16 tokens, n-tiles of 8 dims, V^T fragments by ldmatrix.trans
-            cp_async_wait_all();
-            __syncwarp();
+        // ---- causal mask t <= p, scale, row maxima and sums over the quad
+        const int pa = cur.ea.y, pb = cur.eb.y;
+        const int t0 = cur.j * kBlock + 2 * t;
+        float ma = -INFINITY, mb = -INFINITY, la = 0.f, lb = 0.f;
 #pragma unroll
-            for (int kk = 0; kk < 2; ++kk) {
-                const int tok = 16 * kk + 8 * ((lane >> 3) & 1) + (lane & 7);
+        for (int nt = 0; nt < 4; ++nt)
 #pragma unroll
-                for (int np = 0; np < 8; ++np) {
-                    const int c = 2 * np + (lane >> 4);
-                    uint32_t b[4];
-                    ldsm_x4_trans(b, sv + (uint32_t)((tok * 16 + (c ^ (tok & 7))) * 16));
-                    mma_bf16(o[2 * np], pf[2 * kk][0], pf[2 * kk][1], pf[2 * kk + 1][0], pf[2 * kk + 1][1], b[0],
-                             b[1]);
-                    mma_bf16(o[2 * np + 1], pf[2 * kk][0], pf[2 * kk][1], pf[2 * kk + 1][0], pf[2 * kk + 1][1],
-                             b[2], b[3]);
-                }
+            for (int e = 0; e < 2; ++e) {
+                const int tok = t0 + 8 * nt + e;
+                s[nt][e] = tok <= pa ? s[nt][e] * scale_log2 : -INFINITY;
+                s[nt][2 + e] = tok <= pb ? s[nt][2 + e] * scale_log2 : -INFINITY;
+                ma = fmaxf(ma, s[nt][e]);
+                mb = fmaxf(mb, s[nt][2 + e]);
             }
-        } else if (lane == 0) {
-            flag_error(dev_err, UOCR_DEVERR_PAGE);   // the entries get an empty partial
+#pragma unroll
+        for (int x = 1; x < 4; x <<= 1) {
+            ma = fmaxf(ma, __shfl_xor_sync(0xffffffffu, ma, x));
+            mb = fmaxf(mb, __shfl_xor_sync(0xffffffffu, mb, x));
+        }
+        // finite: a selected block holds a token at or before the query
+        uint32_t pf[4][2];
+#pragma unroll
+        for (int nt = 0; nt < 4; ++nt) {
+            pf[nt][0] = pack_bf16(exp2f(s[nt][0] - ma), exp2f(s[nt][1] - ma), la);
+            pf[nt][1] = pack_bf16(exp2f(s[nt][2] - mb), exp2f(s[nt][3] - mb), lb);
+        }
+#pragma unroll
+        for (int x = 1; x < 4; x <<= 1) {
+            la += __shfl_xor_sync(0xffffffffu, la, x);
+            lb += __shfl_xor_sync(0xffffffffu, lb, x);
         }
 
-        if (r < rows) {
-            const size_t slot = ((size_t)ia * H + h) * kSel + (ent_a & 15);
-            float *dst = part_acc + slot * kD + 2 * t;
+        // ---- O = P V: k-steps of 16 tokens, n-tiles of 8 dims, V^T fragments by ldmatrix.trans
+        cp_async_wait_1();
+        __syncwarp();
+        float o[16][4];
 #pragma unroll
-            for (int n = 0; n < 16; ++n) *reinterpret_cast<float2 *>(dst + 8 * n) = make_float2(o[n][0], o[n][1]);
+        for (int n = 0; n < 16; ++n) o[n][0] = o[n][1] = o[n][2] = o[n][3] = 0.f;
+#pragma unroll
+        for (int kk = 0; kk < 2; ++kk) {
+            const int tok = 16 * kk + 8 * ((lane >> 3) & 1) + (lane & 7);
+#pragma unroll
+            for (int np = 0; np < 8; ++np) {
+                const int c = 2 * np + (lane >> 4);
+                uint32_t b[4];
+                ldsm_x4_trans(b, sv + (uint32_t)((tok * 16 + (c ^ (tok & 7))) * 16));
+                mma_bf16(o[2 * np], pf[2 * kk][0], pf[2 * kk][1], pf[2 * kk + 1][0], pf[2 * kk + 1][1], b[0], b[1]);
+                mma_bf16(o[2 * np + 1], pf[2 * kk][0], pf[2 * kk][1], pf[2 * kk + 1][0], pf[2 * kk + 1][1], b[2],
+                         b[3]);
+            }
+        }
+        __syncwarp();       // V read: the next unit's V may land
+        issue_v(nxt);
+
+        if (!page_ok(cur)) {
+            // no tile was copied: the entries get an empty partial
+            if (lane == 0) flag_error(dev_err, UOCR_DEVERR_PAGE);
+            ma = mb = -INFINITY;
+            la = lb = 0.f;
+#pragma unroll
+            for (int n = 0; n < 16; ++n) o[n][0] = o[n][1] = o[n][2] = o[n][3] = 0.f;
+        }
+        const int ia = cur.ea.x >> 4, ib = cur.eb.x >> 4;
+        if (r < cur.rows) {
+            const size_t slot = ((size_t)ia * H + cur.h) * kSel + (cur.ea.x & 15);
+            const float inv = la > 0.f ? 1.f / la : 0.f;
+            uint32_t *dst = reinterpret_cast<uint32_t *>(part_o + slot * kD) + t;
+            float unused = 0.f;
+#pragma unroll
+            for (int n = 0; n < 16; ++n) dst[4 * n] = pack_bf16(o[n][0] * inv, o[n][1] * inv, unused);
             if (t == 0) *reinterpret_cast<float2 *>(part_ml + slot * 2) = make_float2(ma, la);
         }
-        if (r + 8 < rows) {
-            const size_t slot = ((size_t)ib * H + h) * kSel + (ent_b & 15);
-            float *dst = part_acc + slot * kD + 2 * t;
+        if (r + 8 < cur.rows) {
+            const size_t slot = ((size_t)ib * H + cur.h) * kSel + (cur.eb.x & 15);
+            const float inv = lb > 0.f ? 1.f / lb : 0.f;
+            uint32_t *dst = reinterpret_cast<uint32_t *>(part_o + slot * kD) + t;
+            float unused = 0.f;
 #pragma unroll
-            for (int n = 0; n < 16; ++n) *reinterpret_cast<float2 *>(dst + 8 * n) = make_float2(o[n][2], o[n][3]);
+            for (int n = 0; n < 16; ++n) dst[4 * n] = pack_bf16(o[n][2] * inv, o[n][3] * inv, unused);
             if (t == 0) *reinterpret_cast<float2 *>(part_ml + slot * 2) = make_float2(mb, lb);
         }
+        cur = nxt;
+        if (cur.w >= 0) nxt = load_unit(cur.w + stride, n_work, H, items, list, r);
     }
+    cp_async_wait_all();
 }
 
 // One warp per (query, head): lanes 0..15 hold the 16 slots' (m, l), every lane 4 output dims.
 __global__ void __launch_bounds__(kMergeWarps * 32)
-prefill_merge_kernel(const int32_t *__restrict__ sel, const float *__restrict__ part_acc,
+prefill_merge_kernel(const int32_t *__restrict__ sel, const __nv_bfloat16 *__restrict__ part_o,
                      const float *__restrict__ part_ml, int n_q, int H, __nv_bfloat16 *__restrict__ out) {
     const int lane = threadIdx.x & 31;
     const long long ih = (long long)blockIdx.x * kMergeWarps + (threadIdx.x >> 5);
@@ -301,33 +381,32 @@ prefill_merge_kernel(const int32_t *__restrict__ sel, const float *__restrict__ 
     const float m = valid ? __ldcs(part_ml + (base + s) * 2) : -INFINITY;
     const float l = valid ? __ldcs(part_ml + (base + s) * 2 + 1) : 0.f;
     const unsigned vmask = __ballot_sync(0xffffffffu, valid);
-    float4 v[kSel];
+    uint2 v[kSel];
 #pragma unroll
     for (int k = 0; k < kSel; ++k)
-        v[k] = (vmask >> k & 1u) ? __ldcs(reinterpret_cast<const float4 *>(part_acc + (base + k) * kD) + lane)
-                                 : make_float4(0.f, 0.f, 0.f, 0.f);
+        v[k] = (vmask >> k & 1u) ? __ldcs(reinterpret_cast<const uint2 *>(part_o + (base + k) * kD) + lane)
+                                 : make_uint2(0u, 0u);
     float M = m;
 #pragma unroll
     for (int x = 8; x > 0; x >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, x));
-    const float f = M == -INFINITY ? 0.f : exp2f(m - M);
-    float L = l * f;
+    const float w = M == -INFINITY ? 0.f : l * exp2f(m - M);
+    float W = w;
 #pragma unroll
-    for (int x = 8; x > 0; x >>= 1) L += __shfl_xor_sync(0xffffffffu, L, x);
-    float4 A = make_float4(0.f, 0.f, 0.f, 0.f);
+    for (int x = 8; x > 0; x >>= 1) W += __shfl_xor_sync(0xffffffffu, W, x);
+    float A[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
     for (int k = 0; k < kSel; ++k) {
-        const float fk = __shfl_sync(0xffffffffu, f, k);
-        A.x = fmaf(fk, v[k].x, A.x);
-        A.y = fmaf(fk, v[k].y, A.y);
-        A.z = fmaf(fk, v[k].z, A.z);
-        A.w = fmaf(fk, v[k].w, A.w);
+        const float wk = __shfl_sync(0xffffffffu, w, k);
+        A[0] = fmaf(wk, __uint_as_float(v[k].x << 16), A[0]);
+        A[1] = fmaf(wk, __uint_as_float(v[k].x & 0xffff0000u), A[1]);
+        A[2] = fmaf(wk, __uint_as_float(v[k].y << 16), A[2]);
+        A[3] = fmaf(wk, __uint_as_float(v[k].y & 0xffff0000u), A[3]);
     }
-    const float inv = L > 0.f ? 1.f / L : 0.f;
-    __nv_bfloat162 lo = __floats2bfloat162_rn(A.x * inv, A.y * inv);
-    __nv_bfloat162 hi = __floats2bfloat162_rn(A.z * inv, A.w * inv);
+    const float inv = W > 0.f ? 1.f / W : 0.f;
+    float unused = 0.f;
     uint2 pk;
-    pk.x = *reinterpret_cast<uint32_t *>(&lo);
-    pk.y = *reinterpret_cast<uint32_t *>(&hi);
+    pk.x = pack_bf16(A[0] * inv, A[1] * inv, unused);
+    pk.y = pack_bf16(A[2] * inv, A[3] * inv, unused);
     reinterpret_cast<uint2 *>(out + (size_t)ih * kD)[lane] = pk;
 }
 
@@ -346,20 +425,18 @@ size_t prefill_attn_workspace(int n_q, int H, int max_blocks, PrefillAttnWs *w) 
     PrefillAttnWs l{};
     l.counts_off = off;
     off += up((size_t)max_blocks * 4);
-    l.offsets_off = off;
-    off += up((size_t)max_blocks * 4);
     l.cursor_off = off;
     off += up((size_t)max_blocks * 4);
     l.n_items_off = off;
     off += up(4);
     l.items_off = off;
-    off += up(item_bound(n_q, max_blocks) * sizeof(int2));
+    off += up(item_bound(n_q, max_blocks) * sizeof(int4));
     l.list_off = off;
-    off += up((size_t)n_q * kSel * 4);
+    off += up((size_t)n_q * kSel * sizeof(int2));
     l.ml_off = off;
     off += up((size_t)n_q * H * kSel * 2 * 4);
-    l.acc_off = off;
-    off += up((size_t)n_q * H * kSel * kD * 4);
+    l.o_off = off;
+    off += up((size_t)n_q * H * kSel * kD * 2);
     if (w) *w = l;
     return off;
 }
@@ -372,13 +449,12 @@ cudaError_t launch_prefill_attn(const LaunchCtx &c, const void *q, const void *k
     prefill_attn_workspace(n_q, H, max_blocks, &w);
     char *base = (char *)ws;
     const int32_t *counts = (const int32_t *)(base + w.counts_off);
-    int32_t *offsets = (int32_t *)(base + w.offsets_off);
     int32_t *cursor = (int32_t *)(base + w.cursor_off);
     int32_t *n_items = (int32_t *)(base + w.n_items_off);
-    int2 *items = (int2 *)(base + w.items_off);
-    int32_t *list = (int32_t *)(base + w.list_off);
+    int4 *items = (int4 *)(base + w.items_off);
+    int2 *list = (int2 *)(base + w.list_off);
     float *ml = (float *)(base + w.ml_off);
-    float *acc = (float *)(base + w.acc_off);
+    __nv_bfloat16 *part_o = (__nv_bfloat16 *)(base + w.o_off);
     const int n_entries = n_q * kSel;
 
     cudaLaunchAttribute attr[1];
@@ -391,11 +467,11 @@ cudaError_t launch_prefill_attn(const LaunchCtx &c, const void *q, const void *k
 
     cfg.gridDim = dim3(1);
     cfg.blockDim = dim3(kScanThreads);
-    cudaError_t e = cudaLaunchKernelEx(&cfg, prefill_scan_kernel, counts, max_blocks, offsets, cursor, items, n_items);
+    cudaError_t e = cudaLaunchKernelEx(&cfg, prefill_scan_kernel, counts, bt_row, max_blocks, cursor, items, n_items);
     if (e != cudaSuccess) return e;
     cfg.gridDim = dim3((unsigned)((n_entries + kInvThreads - 1) / kInvThreads));
     cfg.blockDim = dim3(kInvThreads);
-    e = cudaLaunchKernelEx(&cfg, prefill_fill_kernel, sel, n_entries, max_blocks, cursor, list);
+    e = cudaLaunchKernelEx(&cfg, prefill_fill_kernel, sel, q_pos, n_entries, max_blocks, cursor, list);
     if (e != cudaSuccess) return e;
 
     int per_sm = 0;
@@ -404,16 +480,15 @@ cudaError_t launch_prefill_attn(const LaunchCtx &c, const void *q, const void *k
     cfg.gridDim = dim3((unsigned)(c.num_sms * (per_sm > 0 ? per_sm : 1)));
     cfg.blockDim = dim3(kMmaWarps * 32);
     e = cudaLaunchKernelEx(&cfg, prefill_block_mma_kernel, (const uint4 *)q, (const uint4 *)k, (const uint4 *)v,
-                           bt_row, q_pos, counts, (const int32_t *)offsets, (const int32_t *)list,
-                           (const int2 *)items, (const int32_t *)n_items, H, num_pages, scale * kLog2e, acc, ml,
-                           dev_err);
+                           (const int2 *)list, (const int4 *)items, (const int32_t *)n_items, H, num_pages,
+                           scale * kLog2e, part_o, ml, dev_err);
     if (e != cudaSuccess) return e;
     const long long merge_ctas = ((long long)n_q * H + kMergeWarps - 1) / kMergeWarps;
     if (merge_ctas > 0x7fffffffLL) return cudaErrorInvalidConfiguration;
     cfg.gridDim = dim3((unsigned)merge_ctas);
     cfg.blockDim = dim3(kMergeWarps * 32);
-    return cudaLaunchKernelEx(&cfg, prefill_merge_kernel, sel, (const float *)acc, (const float *)ml, n_q, H,
-                              (__nv_bfloat16 *)out);
+    return cudaLaunchKernelEx(&cfg, prefill_merge_kernel, sel, (const __nv_bfloat16 *)part_o, (const float *)ml, n_q,
+                              H, (__nv_bfloat16 *)out);
 }
 
 }  // namespace uocr

@@ -210,6 +210,7 @@ def test_prefill_workspace_is_a_pure_function_of_shapes(pkg):
     assert pw(0, 10, 64) == 0 and pw(4, 0, 64) == 0 and pw(4, 10, 0) == 0
     a = pw(2048, 10, 2048)
     assert a == pw(2048, 10, 2048) and a % 256 == 0
-    # scores, then the inverted index (3 x max_blocks + 16 n_q ints) and 16 partial states per (query, head)
-    assert a >= ws(2048, 10, 2048) + 2048 * 10 * 16 * 130 * 4 + 2048 * 16 * 4 + 3 * 2048 * 4
+    # scores, then the inverted index (2 x max_blocks ints, 16 n_q (entry, position) pairs, the item
+    # records) and 16 partial states per (query, head): 128 bf16 outputs + fp32 (m, l)
+    assert a >= ws(2048, 10, 2048) + 2048 * 10 * 16 * (128 * 2 + 8) + 2048 * 16 * 8 + 2 * 2048 * 4
     assert pw(2048, 1, 2048) < a and pw(4096, 10, 2048) > a

@@ -12,7 +12,7 @@ import torch
 
 import oracle
 import workloads
-from parity_util import check_queries
+from parity_util import OUT_MAX_ATOL, OUT_MEAN_ATOL, check_queries, oracle_attend
 
 pytestmark = pytest.mark.gpu
 
@@ -95,6 +95,32 @@ def test_prefill_flags_bad_positions_and_pages(uocr, cuda_device):
     torch.cuda.synchronize()
     assert int(err.item()) & uocr.DEVERR_PAGE
     assert torch.isneginf(sc[:, 7]).all() and torch.isfinite(sc[:, 6]).all()
+
+
+def test_sparse_prefill_bad_page_gives_an_empty_block(uocr, cuda_device):
+    """A selected block whose page id is out of range is flagged and contributes nothing: every
+    output equals exact attention over the query's other selected blocks."""
+    total = 32 * 80
+    case = _prefill_case(total, 100, seed=21, device=cuda_device)
+    j_bad = (total - 1) // 32 - 2                       # in the local window of most queries
+    bt = case.block_table.clone()
+    bt[0, j_bad] = case.num_pages + 5
+    err = torch.zeros(1, dtype=torch.int32, device=cuda_device)
+    out, sel = uocr.sparse_prefill(case.q, case.k_pool, case.v_pool, case.idx_q, case.idx_k_pool, bt,
+                                   case.seq_lens, 0, case.q_pos, dev_err=err)
+    torch.cuda.synchronize()
+    assert int(err.item()) & uocr.DEVERR_PAGE
+    assert torch.isfinite(out.float()).all()
+    got, sel = out.float().cpu().numpy(), sel.cpu().numpy()
+    hit = 0
+    for i in range(case.n_q):
+        s = sel[i].copy()
+        hit += int((s == j_bad).any())
+        s[s == j_bad] = -1
+        ref = oracle_attend(case, i, s)
+        d = np.abs(got[i] - ref)
+        assert d.max() <= OUT_MAX_ATOL and d.mean() <= OUT_MEAN_ATOL, f"query {i}"
+    assert hit > 50
 
 
 @pytest.mark.slow
