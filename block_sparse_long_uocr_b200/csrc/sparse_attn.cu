@@ -227,6 +227,9 @@ sparse_attn_kernel(const uint4 *__restrict__ q, const uint4 *__restrict__ kc, co
         out[(size_t)ih * kD + d] = __float2bfloat16_rn(Lt > 0.f ? At / Lt : 0.f);
     }
     cluster_sync();                              // keep every CTA's shared memory alive until read
+    // Warps whose blocks were known in advance never wait on the selection kernel; one thread
+    // waits here so that this grid completes after it (its selection output included).
+    if (blockIdx.x == 0 && threadIdx.x == 0) pdl_wait();
 }
 
 cudaError_t launch_sparse_attn(const LaunchCtx &c, const void *q, const void *k, const void *v,
