@@ -44,15 +44,20 @@ FALLBACK_HBM_GBS = 6650.0
 # dram__bytes_write.sum), per launch of the default workload, and the hash of the
 # kernel source it was taken on.  Reported as null once the source has changed.
 NCU_TRAFFIC = {
-    # ncu --set full on long_decode batch 4 (1 layer), one launch: 134,301,184 B read +
-    # 3,638,272 B written (the write-back of the bench's L2 flush), scaled x4 to 16 queries.
-    "long_decode": {"bytes": 4 * (134301184 + 3638272), "src": "f7c4636027d893b4"},
+    # ncu --set full on long_decode batch 4 (1 layer), one launch: 134,299,392 B read +
+    # 4,135,168 B written (the write-back of the bench's L2 flush), scaled x4 to 16 queries.
+    "long_decode": {"bytes": 4 * (134299392 + 4135168), "src": "db17d3ef40c51c90"},
 }
 
 
-def kernel_source_hash(name: str) -> str:
-    path = os.path.join(ROOT, "block_sparse_long_uocr_b200", "csrc", name)
-    return hashlib.sha256(open(path, "rb").read()).hexdigest()[:16]
+SCAN_SOURCES = ("index_scan.cu", "scan_core.cuh", "common.cuh")
+
+
+def kernel_source_hash(*names: str) -> str:
+    h = hashlib.sha256()
+    for name in names:
+        h.update(open(os.path.join(ROOT, "block_sparse_long_uocr_b200", "csrc", name), "rb").read())
+    return h.hexdigest()[:16]
 
 
 def measured_peaks():
@@ -363,7 +368,7 @@ def run_uocr(args):
     scan_gbs = scan_bytes_call / (scan_ms / 1e3) / 1e9
     step_gbs = bytes_call * n_layers / (ms_per_step / 1e3) / 1e9
     tr = NCU_TRAFFIC.get(args.workload) if (args.workload != "long_decode" or B == 16) else None
-    traffic = tr["bytes"] if tr and tr.get("src") == kernel_source_hash("index_scan.cu") else None
+    traffic = tr["bytes"] if tr and tr.get("src") == kernel_source_hash(*SCAN_SOURCES) else None
 
     # ---- end to end through the public API: pinned host inputs in, results out, every step
     e2e = run_e2e(args, uocr, case, ws, outs, sels, stream, world, dev)
