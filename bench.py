@@ -46,11 +46,11 @@ FALLBACK_HBM_GBS = 6650.0
 NCU_TRAFFIC = {
     # ncu --set full on long_decode batch 4 (1 layer), one launch: 134,299,392 B read +
     # 4,135,168 B written (the write-back of the bench's L2 flush), scaled x4 to 16 queries.
-    "long_decode": {"bytes": 4 * (134299392 + 4135168), "src": "db17d3ef40c51c90"},
+    "long_decode": {"bytes": 4 * (134299392 + 4135168), "src": "838030ba57b367b4"},
 }
 
 
-SCAN_SOURCES = ("index_scan.cu", "scan_core.cuh", "common.cuh")
+SCAN_SOURCES = ("index_scan.cu", "scan_core.cuh")   # the scan kernel and its page loop
 
 
 def kernel_source_hash(*names: str) -> str:

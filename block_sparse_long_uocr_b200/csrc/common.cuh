@@ -172,19 +172,30 @@ __device__ __forceinline__ uint64_t global_timer_ns() {
     return t;
 }
 
+// As mbar_try_wait, but the thread may be suspended for up to `hint_ns` while the phase is
+// incomplete instead of returning at once (no spinning on the issue slots).
+__device__ __forceinline__ bool mbar_try_wait_sleep(uint64_t *bar, uint32_t parity, uint32_t hint_ns) {
+    uint32_t ok;
+    asm volatile(
+        "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n selp.u32 %0, 1, 0, p;\n}"
+        : "=r"(ok)
+        : "r"(smem_addr(bar)), "r"(parity), "r"(hint_ns)
+        : "memory");
+    return ok != 0;
+}
+
 // Wait on phase `parity` of `bar` for at most `timeout_ns` of wall time, giving up early
-// when *abort becomes non-zero.  Returns true when the phase completed.
+// when *abort becomes non-zero.  Returns true when the phase completed.  Each probe may
+// suspend the thread for up to 20 us, so the wait does not spin.
 __device__ __forceinline__ bool mbar_wait_timed(uint64_t *bar, uint32_t parity, uint64_t timeout_ns,
                                                 const volatile int *abort) {
     if (mbar_try_wait(bar, parity)) return true;
     const uint64_t t0 = global_timer_ns();
     for (uint32_t it = 1;; ++it) {
-        if (mbar_try_wait(bar, parity)) return true;
-        if ((it & 63u) == 0) {
-            if (abort && *abort) return false;
-            if (global_timer_ns() - t0 > timeout_ns) return false;
-            if (it > (1u << 30)) return false;   // in case the timer does not advance
-        }
+        if (mbar_try_wait_sleep(bar, parity, 20000u)) return true;
+        if (abort && *abort) return false;
+        if (global_timer_ns() - t0 > timeout_ns) return false;
+        if (it > (1u << 28)) return false;   // in case the timer does not advance
     }
 }
 

@@ -7,19 +7,22 @@
 // maximum of the walk-through (news.rkmt.cn/news/25027, section 五 step 2):
 //   scores[i][j] = max_{t in block j, t <= p_i} S[i][t].
 //
-// Kernel (persistent, one CTA per SM, 320 threads, warp-specialised):
-//   warp 8  TMA producer: per work unit the 128-query A tile (two 64-dim halves,
-//           128-byte swizzle) into a 2-deep ring, and per 256-token N tile the
-//           8 pages' indexer keys (16 boxes of 32 tokens x 64 dims, gathered
-//           through the block table) into a 2-stage ring;
-//   warp 9  MMA issuer: allocates 512 TMEM columns (two 128 x 256 fp32
-//           accumulators) and issues 8 tcgen05.mma (M=128, N=256, K=16) per tile;
-//   warps 0-7 epilogue: tcgen05.ld of the accumulator (warp w owns rows
-//           32(w%4) .. +31 = its TMEM lane quarter, and blocks 4(w/4) .. +3 of
-//           the tile), max over each 32-column block (the causal mask only on
-//           tiles that reach past the row's position), fp32 scores to global
+// Kernel (persistent, one CTA per SM, 320 threads, warp-specialised).  A CTA
+// tile is two 128-query subtiles that share every key tile they load, which
+// halves the key traffic from L2 per FLOP against one subtile per CTA:
+//   warp 8  TMA producer: per work unit the two 128-query A subtiles (two
+//           64-dim halves each, 128-byte swizzle) into a 2-deep ring, and per
+//           128-token N tile the 4 pages' indexer keys (8 boxes of 32 tokens x 64
+//           dims, gathered through the block table) into a 3-stage ring;
+//   warp 9  MMA issuer: allocates 512 TMEM columns (two buffers x two subtiles
+//           of 128 x 128 fp32) and issues 8 tcgen05.mma (M=128, N=128, K=16) per
+//           subtile and tile;
+//   warps 0-7 epilogue: tcgen05.ld of the accumulators (warp w owns rows
+//           32(w%4) .. +31 = its TMEM lane quarter, of subtile w/4, and the
+//           tile's 4 blocks), max over each 32-column block (the causal mask only
+//           on blocks that reach past the row's position), fp32 scores to global
 //           memory, four at a time.
-// Work unit = (128-query tile, chunk of 4 N tiles); units whose tokens all lie
+// Work unit = (256-query tile, chunk of 4 N tiles); units whose tokens all lie
 // past the tile's last query are skipped.  Every mbarrier wait is bounded in
 // wall time: on timeout the CTA reports UOCR_DEVERR_TIMEOUT, every role stops
 // issuing, waits (bounded) for what it issued, and the TMEM is freed.
@@ -35,24 +38,25 @@ namespace uocr {
 
 namespace {
 
-constexpr int kBM = 128;                  // queries per tile (TMEM lanes)
-constexpr int kBN = 256;                  // tokens per N tile (8 pages)
+constexpr int kBM = 128;                  // queries per subtile (TMEM lanes)
+constexpr int kMT = 2;                    // subtiles per CTA tile (they share each key tile)
+constexpr int kBN = 128;                  // tokens per N tile (4 pages)
 constexpr int kPagesPerTile = kBN / kBlock;
 constexpr int kTilesPerUnit = 4;
-constexpr int kStagesB = 2;
+constexpr int kStagesB = 3;
 constexpr int kStagesA = 2;
-constexpr int kHalfBytesA = kBM * 128;    // one 64-dim half of an A tile: 16 KiB
-constexpr int kHalfBytesB = kBN * 128;    // one 64-dim half of a B tile: 32 KiB
+constexpr int kHalfBytesA = kBM * 128;    // one 64-dim half of an A subtile: 16 KiB
+constexpr int kHalfBytesB = kBN * 128;    // one 64-dim half of a B tile: 16 KiB
 constexpr int kBoxBytesB = kBlock * 128;  // one page x 64 dims: 4 KiB
-constexpr int kEpiWarps = 8;             // two warps per TMEM lane quarter, 4 blocks of a tile each
+constexpr int kEpiWarps = 8;             // one warp per (TMEM lane quarter, subtile)
 constexpr int kProducerWarp = 8;
 constexpr int kMmaWarp = 9;
 constexpr int kThreads = 320;
 constexpr uint64_t kTimeoutNs = 2000000000ull;   // 2 s: far above any legitimate wait
 
 struct __align__(1024) Smem {
-    uint8_t a[kStagesA][2][kHalfBytesA];      // 64 KiB
-    uint8_t b[kStagesB][2][kHalfBytesB];      // 128 KiB
+    uint8_t a[kStagesA][kMT][2][kHalfBytesA];   // 128 KiB
+    uint8_t b[kStagesB][2][kHalfBytesB];        // 96 KiB
     uint64_t a_full[kStagesA], a_empty[kStagesA];
     uint64_t b_full[kStagesB], b_empty[kStagesB];
     uint64_t acc_full[2], acc_empty[2];
@@ -63,6 +67,7 @@ struct __align__(1024) Smem {
 
 struct UnitInfo {
     int m0;       // first query of the tile
+    int nsub;     // subtiles holding queries (1 or 2)
     int t0;       // first N tile
     int ntiles;   // tiles to compute (0: skip)
     int nb_max;   // causal blocks of the tile's last valid query
@@ -75,16 +80,24 @@ __device__ __forceinline__ int row_pos(const int32_t *q_pos, int row, int n_q, i
     return p < seq_len ? p : -1;
 }
 
-// Same answer in every role: the unit's tile range, from the queries' positions.
-__device__ __forceinline__ UnitInfo unit_info(int u, int n_chunks, const int32_t *q_pos, int n_q, int seq_len,
-                                              int lane) {
-    UnitInfo w;
-    w.m0 = (u / n_chunks) * kBM;
-    w.t0 = (u % n_chunks) * kTilesPerUnit;
+// Same answer in every role: the unit's tile range, from the queries' positions.  Split in
+// two so that a role can issue the next unit's position loads (lane_pmax) before working on
+// the current unit, and reduce them (unit_info) when it gets there.
+__device__ __forceinline__ int lane_pmax(int u, int n_units, int n_chunks, const int32_t *q_pos, int n_q,
+                                         int seq_len, int lane) {
+    if (u >= n_units) return -1;
+    const int m0 = (u / n_chunks) * (kBM * kMT);
     int pmax = -1;
 #pragma unroll
-    for (int k = 0; k < kBM / 32; ++k) pmax = max(pmax, row_pos(q_pos, w.m0 + k * 32 + lane, n_q, seq_len));
-    pmax = __reduce_max_sync(0xffffffffu, pmax);
+    for (int k = 0; k < kBM * kMT / 32; ++k) pmax = max(pmax, row_pos(q_pos, m0 + k * 32 + lane, n_q, seq_len));
+    return pmax;
+}
+__device__ __forceinline__ UnitInfo unit_info(int u, int n_chunks, int n_q, int pmax_lane) {
+    UnitInfo w;
+    w.m0 = (u / n_chunks) * (kBM * kMT);
+    w.nsub = min(kMT, (n_q - w.m0 + kBM - 1) / kBM);
+    w.t0 = (u % n_chunks) * kTilesPerUnit;
+    const int pmax = __reduce_max_sync(0xffffffffu, pmax_lane);
     w.nb_max = pmax < 0 ? 0 : pmax / kBlock + 1;
     const int tiles_needed = (w.nb_max + kPagesPerTile - 1) / kPagesPerTile;
     w.ntiles = max(0, min(kTilesPerUnit, tiles_needed - w.t0));
@@ -157,35 +170,41 @@ prefill_index_gemm_kernel(const __grid_constant__ CUtensorMap map_q, const __gri
     if (warp == kProducerWarp) {
         // ------------------------------------------------------------ TMA producer
         int it = 0, uc = 0;
-        int b_fills[kStagesB] = {0, 0};
-        int a_fills[kStagesA] = {0, 0};
+        int b_fills[kStagesB] = {};
+        int a_fills[kStagesA] = {};
         bool stop = false;
+        int pm_next = lane_pmax(blockIdx.x, n_units, n_chunks, q_pos, n_q, seq_len_ok, lane);
         for (int u = blockIdx.x; u < n_units && !stop; u += gridDim.x) {
-            const UnitInfo w = unit_info(u, n_chunks, q_pos, n_q, seq_len_ok, lane);
+            const UnitInfo w = unit_info(u, n_chunks, n_q, pm_next);
+            pm_next = lane_pmax(u + gridDim.x, n_units, n_chunks, q_pos, n_q, seq_len_ok, lane);
             if (w.ntiles == 0) continue;
+            // the unit's page ids at once: lane l < 4 * ntiles holds block t0 * 4 + l
+            int upage = -1;
+            if (lane < w.ntiles * kPagesPerTile) {
+                const int j = w.t0 * kPagesPerTile + lane;
+                if (j < w.nb_max) {
+                    upage = __ldg(bt_row + j);
+                    if ((unsigned)upage >= (unsigned)num_pages) {
+                        flag_error(dev_err, UOCR_DEVERR_PAGE);
+                        upage = -1;
+                    }
+                }
+            }
             const int sa = uc % kStagesA;
             if (!warp_wait(&s.a_empty[sa], ((uc / kStagesA) & 1) ^ 1, s, dev_err, lane)) break;
             if (lane == 0) {
-                mbar_arrive_expect_tx(&s.a_full[sa], 2u * a_box_rows * 128u);
-                tc::tma_load_2d(s.a[sa][0], &map_q, 0, w.m0, &s.a_full[sa]);
-                tc::tma_load_2d(s.a[sa][1], &map_q, 64, w.m0, &s.a_full[sa]);
+                mbar_arrive_expect_tx(&s.a_full[sa], (uint32_t)w.nsub * 2u * a_box_rows * 128u);
+                for (int m = 0; m < w.nsub; ++m) {
+                    tc::tma_load_2d(s.a[sa][m][0], &map_q, 0, w.m0 + m * kBM, &s.a_full[sa]);
+                    tc::tma_load_2d(s.a[sa][m][1], &map_q, 64, w.m0 + m * kBM, &s.a_full[sa]);
+                }
             }
             ++a_fills[sa];
             ++uc;
             for (int t = 0; t < w.ntiles; ++t, ++it) {
                 const int st = it % kStagesB;
-                const int tile = w.t0 + t;
-                int page = -1;   // lanes 0..7 look up the tile's pages
-                if (lane < kPagesPerTile) {
-                    const int j = tile * kPagesPerTile + lane;
-                    if (j < w.nb_max) {
-                        page = __ldg(bt_row + j);
-                        if ((unsigned)page >= (unsigned)num_pages) {
-                            flag_error(dev_err, UOCR_DEVERR_PAGE);
-                            page = -1;
-                        }
-                    }
-                }
+                int page = __shfl_sync(0xffffffffu, upage, t * kPagesPerTile + (lane & (kPagesPerTile - 1)));
+                if (lane >= kPagesPerTile) page = -1;   // lanes 0..3 issue the tile's pages
                 const unsigned valid = __ballot_sync(0xffffffffu, page >= 0);
                 if (!warp_wait(&s.b_empty[st], ((it / kStagesB) & 1) ^ 1, s, dev_err, lane)) {
                     stop = true;
@@ -214,15 +233,18 @@ prefill_index_gemm_kernel(const __grid_constant__ CUtensorMap map_q, const __gri
     } else if (warp == kMmaWarp) {
         // ------------------------------------------------------------ MMA issuer
         constexpr uint32_t idesc = tc::idesc_bf16_f32(kBM, kBN);
+        static_assert(kTilesPerUnit * kPagesPerTile <= 32, "a unit's page ids fit in one warp");
+        static_assert(2 * kMT * kBN == 512, "two accumulator buffers of kMT subtiles fill the 512 TMEM columns");
         int it = 0, uc = 0;
         bool issued = false, stop = false;
+        int pm_next = lane_pmax(blockIdx.x, n_units, n_chunks, q_pos, n_q, seq_len_ok, lane);
         for (int u = blockIdx.x; u < n_units && !stop; u += gridDim.x) {
-            const UnitInfo w = unit_info(u, n_chunks, q_pos, n_q, seq_len_ok, lane);
+            const UnitInfo w = unit_info(u, n_chunks, n_q, pm_next);
+            pm_next = lane_pmax(u + gridDim.x, n_units, n_chunks, q_pos, n_q, seq_len_ok, lane);
             if (w.ntiles == 0) continue;
             const int sa = uc % kStagesA;
             if (!warp_wait(&s.a_full[sa], (uc / kStagesA) & 1, s, dev_err, lane)) break;
             ++uc;
-            const uint32_t a0 = smem_addr(s.a[sa][0]), a1 = smem_addr(s.a[sa][1]);
             for (int t = 0; t < w.ntiles; ++t, ++it) {
                 const int st = it % kStagesB;
                 const int acc = it & 1;
@@ -233,13 +255,21 @@ prefill_index_gemm_kernel(const __grid_constant__ CUtensorMap map_q, const __gri
                 }
                 if (lane == 0) {
                     tc::fence_after_sync();
-                    const uint32_t b0 = smem_addr(s.b[st][0]), b1 = smem_addr(s.b[st][1]);
+                    // k-step k reads 16 bf16 = 32 bytes further into the 128-byte swizzle row:
+                    // 2 more in the descriptor's start-address field (16-byte units; the stage
+                    // addresses stay far below the field's 256 KiB range)
+                    const uint64_t bd0 = tc::smem_desc_k_sw128(smem_addr(s.b[st][0]));
+                    const uint64_t bd1 = tc::smem_desc_k_sw128(smem_addr(s.b[st][1]));
+                    for (int m = 0; m < w.nsub; ++m) {
+                        const uint64_t ad0 = tc::smem_desc_k_sw128(smem_addr(s.a[sa][m][0]));
+                        const uint64_t ad1 = tc::smem_desc_k_sw128(smem_addr(s.a[sa][m][1]));
+                        const uint32_t d = tmem + (uint32_t)((acc * kMT + m) * kBN);
 #pragma unroll
-                    for (int k = 0; k < 8; ++k) {
-                        const uint32_t koff = (k & 3) * 32;   // 16 bf16 = 32 bytes inside the swizzle atom
-                        const uint64_t ad = tc::smem_desc_k_sw128((k < 4 ? a0 : a1) + koff);
-                        const uint64_t bd = tc::smem_desc_k_sw128((k < 4 ? b0 : b1) + koff);
-                        tc::mma_bf16(tmem + acc * kBN, ad, bd, idesc, k > 0 ? 1u : 0u);
+                        for (int k = 0; k < 8; ++k) {
+                            const uint64_t koff = (uint64_t)((k & 3) * 2);
+                            tc::mma_bf16(d, (k < 4 ? ad0 : ad1) + koff, (k < 4 ? bd0 : bd1) + koff, idesc,
+                                         k > 0 ? 1u : 0u);
+                        }
                     }
                     tc::commit(&s.b_empty[st]);
                     tc::commit(&s.acc_full[acc]);
@@ -259,15 +289,17 @@ prefill_index_gemm_kernel(const __grid_constant__ CUtensorMap map_q, const __gri
         __syncwarp();
     } else {
         // ------------------------------------------------------------ epilogue, warps 0..7
-        const int quarter = warp & 3;            // TMEM lane quarter = rows 32q .. 32q+31
-        const int half = warp >> 2;              // blocks 4*half .. 4*half+3 of each tile
+        const int quarter = warp & 3;            // TMEM lane quarter = rows 32q .. 32q+31 of a subtile
+        const int sub = warp >> 2;               // subtile
         int it = 0;
         bool stop = false;
+        int pm_next = lane_pmax(blockIdx.x, n_units, n_chunks, q_pos, n_q, seq_len_ok, lane);
         for (int u = blockIdx.x; u < n_units && !stop; u += gridDim.x) {
-            const UnitInfo w = unit_info(u, n_chunks, q_pos, n_q, seq_len_ok, lane);
+            const UnitInfo w = unit_info(u, n_chunks, n_q, pm_next);
+            pm_next = lane_pmax(u + gridDim.x, n_units, n_chunks, q_pos, n_q, seq_len_ok, lane);
             if (w.ntiles == 0) continue;
-            const int row = w.m0 + quarter * 32 + lane;
-            if (row < n_q && half == 0) {
+            const int row = w.m0 + sub * kBM + quarter * 32 + lane;
+            if (row < n_q) {
                 const int p_raw = __ldg(q_pos + row);
                 if (p_raw >= seq_len && w.t0 == 0) flag_error(dev_err, UOCR_DEVERR_POS);
             }
@@ -282,13 +314,16 @@ prefill_index_gemm_kernel(const __grid_constant__ CUtensorMap map_q, const __gri
                 }
                 tc::fence_after_sync();
                 const int tile = w.t0 + t;
-                const int j0 = tile * kPagesPerTile + half * 4;          // first block of this warp
+                const int j0 = tile * kPagesPerTile;                     // first block of the tile
                 const bool interior = (j0 + 4) * kBlock - 1 <= p;        // no masking needed
                 float best[4];
                 const uint32_t tbase =
-                    tmem + ((uint32_t)(quarter * 32) << 16) + (uint32_t)(acc * kBN + half * 4 * kBlock);
+                    tmem + ((uint32_t)(quarter * 32) << 16) + (uint32_t)((acc * kMT + sub) * kBN);
+                // a subtile past the last query holds no accumulator: read nothing, write nothing
+                const bool have = sub < w.nsub;
 #pragma unroll
                 for (int k = 0; k < 4; k += 2) {
+                    if (!have) break;
                     float v0[32], v1[32];
                     tc::tmem_ld_32x32b_x32(tbase + k * 32, v0);
                     tc::tmem_ld_32x32b_x32(tbase + (k + 1) * 32, v1);
@@ -321,6 +356,7 @@ prefill_index_gemm_kernel(const __grid_constant__ CUtensorMap map_q, const __gri
                 if (lane == 0)
                     asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_addr(&s.acc_empty[acc]))
                                  : "memory");
+                if (!have) continue;
                 // a block whose page is not in the pool scores -inf; blocks past the row's
                 // causal range are not written
                 int pg[4];
@@ -388,7 +424,7 @@ cudaError_t launch_prefill_index_gemm(const LaunchCtx &c, const void *idx_q, con
     CUtensorMap map_q, map_k;
     if (!make_map(&map_q, idx_q, (uint64_t)n_q, (uint32_t)a_box_rows)) return cudaErrorInvalidValue;
     if (!make_map(&map_k, idx_k, (uint64_t)num_pages * kBlock, kBlock)) return cudaErrorInvalidValue;
-    const int m_tiles = (n_q + kBM - 1) / kBM;
+    const int m_tiles = (n_q + kBM * kMT - 1) / (kBM * kMT);
     const int n_tiles = (max_blocks + kPagesPerTile - 1) / kPagesPerTile;
     const int n_chunks = (n_tiles + kTilesPerUnit - 1) / kTilesPerUnit;
     const long long units = (long long)m_tiles * n_chunks;
