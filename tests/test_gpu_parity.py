@@ -240,6 +240,17 @@ def test_decode_ragged_paged_workload_sampled(uocr, cuda_device):
 
 
 @pytest.mark.slow
+def test_decode_maximum_lengths_sampled(uocr, cuda_device):
+    """A 1.6M-token row (50,000 blocks: past the selection's shared-memory staging of 49,152
+    candidates, so it reads its scores from L2), a 1M-token row (32,768 blocks, staged), and a
+    short row sharing the same block table width."""
+    lens = [32 * 50000, 32 * 32768 - 5, 700]
+    case = workloads.make_case(lens, shuffle=True, max_blocks=50000, seed=17, device=cuda_device)
+    out, sel, sc = run_decode(uocr, case)
+    check_queries(case, [0, 1, 2], out, sel, sc)
+
+
+@pytest.mark.slow
 def test_chunked_prefill_workload_sampled_step_entries(uocr, cuda_device):
     case = workloads.chunked_prefill(device=cuda_device)
     sc = uocr.index_score(case.idx_q, case.idx_k_pool, case.block_table, case.seq_lens, case.q_seq, case.q_pos)
