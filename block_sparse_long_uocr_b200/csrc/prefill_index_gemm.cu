@@ -7,13 +7,15 @@
 // maximum of the walk-through (news.rkmt.cn/news/25027, section 五 step 2):
 //   scores[i][j] = max_{t in block j, t <= p_i} S[i][t].
 //
-// Kernel (persistent, one CTA per SM, 320 threads, warp-specialised).  A CTA
+// Kernel (persistent, one CTA per SM, 352 threads, warp-specialised).  A CTA
 // tile is two 128-query subtiles that share every key tile they load, which
 // halves the key traffic from L2 per FLOP against one subtile per CTA:
-//   warp 8  TMA producer: per work unit the two 128-query A subtiles (two
-//           64-dim halves each, 128-byte swizzle) into a 2-deep ring, and per
-//           128-token N tile the 4 pages' indexer keys (8 boxes of 32 tokens x 64
-//           dims, gathered through the block table) into a 3-stage ring;
+//   warp 8  TMA producer of queries: per work unit the two 128-query A subtiles
+//           (two 64-dim halves each, 128-byte swizzle) into a 2-deep ring;
+//   warp 10 TMA producer of keys: per 128-token N tile the 4 pages' indexer
+//           keys (8 boxes of 32 tokens x 64 dims, gathered through the block
+//           table) into a 3-stage ring.  The two producers run ahead of the MMAs
+//           independently, each as far as its ring allows;
 //   warp 9  MMA issuer: allocates 512 TMEM columns (two buffers x two subtiles
 //           of 128 x 128 fp32) and issues 8 tcgen05.mma (M=128, N=128, K=16) per
 //           subtile and tile;
@@ -49,9 +51,10 @@ constexpr int kHalfBytesA = kBM * 128;    // one 64-dim half of an A subtile: 16
 constexpr int kHalfBytesB = kBN * 128;    // one 64-dim half of a B tile: 16 KiB
 constexpr int kBoxBytesB = kBlock * 128;  // one page x 64 dims: 4 KiB
 constexpr int kEpiWarps = 8;             // one warp per (TMEM lane quarter, subtile)
-constexpr int kProducerWarp = 8;
+constexpr int kProducerWarp = 8;          // query (A) tiles
 constexpr int kMmaWarp = 9;
-constexpr int kThreads = 320;
+constexpr int kProducerBWarp = 10;        // key (B) tiles
+constexpr int kThreads = 352;
 constexpr uint64_t kTimeoutNs = 2000000000ull;   // 2 s: far above any legitimate wait
 
 struct __align__(1024) Smem {
@@ -168,10 +171,35 @@ prefill_index_gemm_kernel(const __grid_constant__ CUtensorMap map_q, const __gri
     const int seq_len_ok = min(seq_len, max_blocks * kBlock);
 
     if (warp == kProducerWarp) {
-        // ------------------------------------------------------------ TMA producer
-        int it = 0, uc = 0;
-        int b_fills[kStagesB] = {};
+        // ------------------------------------------------------------ TMA producer: query tiles
+        int uc = 0;
         int a_fills[kStagesA] = {};
+        int pm_next = lane_pmax(blockIdx.x, n_units, n_chunks, q_pos, n_q, seq_len_ok, lane);
+        for (int u = blockIdx.x; u < n_units; u += gridDim.x) {
+            const UnitInfo w = unit_info(u, n_chunks, n_q, pm_next);
+            pm_next = lane_pmax(u + gridDim.x, n_units, n_chunks, q_pos, n_q, seq_len_ok, lane);
+            if (w.ntiles == 0) continue;
+            const int sa = uc % kStagesA;
+            if (!warp_wait(&s.a_empty[sa], ((uc / kStagesA) & 1) ^ 1, s, dev_err, lane)) break;
+            if (lane == 0) {
+                mbar_arrive_expect_tx(&s.a_full[sa], (uint32_t)w.nsub * 2u * a_box_rows * 128u);
+                for (int m = 0; m < w.nsub; ++m) {
+                    tc::tma_load_2d(s.a[sa][m][0], &map_q, 0, w.m0 + m * kBM, &s.a_full[sa]);
+                    tc::tma_load_2d(s.a[sa][m][1], &map_q, 64, w.m0 + m * kBM, &s.a_full[sa]);
+                }
+            }
+            ++a_fills[sa];
+            ++uc;
+            if (aborted(s)) break;
+        }
+        // drain: every buffer this warp filled must have landed before the CTA exits
+        if (lane == 0)
+            for (int k = 0; k < kStagesA; ++k)
+                if (a_fills[k] > 0) mbar_wait_timed(&s.a_full[k], (a_fills[k] - 1) & 1, kTimeoutNs, nullptr);
+    } else if (warp == kProducerBWarp) {
+        // ------------------------------------------------------------ TMA producer: key tiles
+        int it = 0;
+        int b_fills[kStagesB] = {};
         bool stop = false;
         int pm_next = lane_pmax(blockIdx.x, n_units, n_chunks, q_pos, n_q, seq_len_ok, lane);
         for (int u = blockIdx.x; u < n_units && !stop; u += gridDim.x) {
@@ -190,17 +218,6 @@ prefill_index_gemm_kernel(const __grid_constant__ CUtensorMap map_q, const __gri
                     }
                 }
             }
-            const int sa = uc % kStagesA;
-            if (!warp_wait(&s.a_empty[sa], ((uc / kStagesA) & 1) ^ 1, s, dev_err, lane)) break;
-            if (lane == 0) {
-                mbar_arrive_expect_tx(&s.a_full[sa], (uint32_t)w.nsub * 2u * a_box_rows * 128u);
-                for (int m = 0; m < w.nsub; ++m) {
-                    tc::tma_load_2d(s.a[sa][m][0], &map_q, 0, w.m0 + m * kBM, &s.a_full[sa]);
-                    tc::tma_load_2d(s.a[sa][m][1], &map_q, 64, w.m0 + m * kBM, &s.a_full[sa]);
-                }
-            }
-            ++a_fills[sa];
-            ++uc;
             for (int t = 0; t < w.ntiles; ++t, ++it) {
                 const int st = it % kStagesB;
                 int page = __shfl_sync(0xffffffffu, upage, t * kPagesPerTile + (lane & (kPagesPerTile - 1)));
@@ -223,13 +240,9 @@ prefill_index_gemm_kernel(const __grid_constant__ CUtensorMap map_q, const __gri
                 }
             }
         }
-        // drain: every buffer this warp filled must have landed before the CTA exits
-        if (lane == 0) {
+        if (lane == 0)
             for (int k = 0; k < kStagesB; ++k)
                 if (b_fills[k] > 0) mbar_wait_timed(&s.b_full[k], (b_fills[k] - 1) & 1, kTimeoutNs, nullptr);
-            for (int k = 0; k < kStagesA; ++k)
-                if (a_fills[k] > 0) mbar_wait_timed(&s.a_full[k], (a_fills[k] - 1) & 1, kTimeoutNs, nullptr);
-        }
     } else if (warp == kMmaWarp) {
         // ------------------------------------------------------------ MMA issuer
         constexpr uint32_t idesc = tc::idesc_bf16_f32(kBM, kBN);
@@ -293,19 +306,35 @@ prefill_index_gemm_kernel(const __grid_constant__ CUtensorMap map_q, const __gri
         const int sub = warp >> 2;               // subtile
         int it = 0;
         bool stop = false;
+        // this thread's row position in unit u (raw, -1 past the queries), fetched a unit ahead
+        auto next_row_p = [&](int u) {
+            if (u >= n_units) return -1;
+            const int r = (u / n_chunks) * (kBM * kMT) + sub * kBM + quarter * 32 + lane;
+            return r < n_q ? __ldg(q_pos + r) : -1;
+        };
+        int p_next = next_row_p(blockIdx.x);
         int pm_next = lane_pmax(blockIdx.x, n_units, n_chunks, q_pos, n_q, seq_len_ok, lane);
         for (int u = blockIdx.x; u < n_units && !stop; u += gridDim.x) {
             const UnitInfo w = unit_info(u, n_chunks, n_q, pm_next);
             pm_next = lane_pmax(u + gridDim.x, n_units, n_chunks, q_pos, n_q, seq_len_ok, lane);
-            if (w.ntiles == 0) continue;
-            const int row = w.m0 + sub * kBM + quarter * 32 + lane;
-            if (row < n_q) {
-                const int p_raw = __ldg(q_pos + row);
-                if (p_raw >= seq_len && w.t0 == 0) flag_error(dev_err, UOCR_DEVERR_POS);
+            if (w.ntiles == 0) {
+                p_next = next_row_p(u + gridDim.x);
+                continue;
             }
-            const int p = row_pos(q_pos, row, n_q, seq_len_ok);
+            const int row = w.m0 + sub * kBM + quarter * 32 + lane;
+            const int p_raw = p_next;
+            p_next = next_row_p(u + gridDim.x);
+            if (row < n_q && p_raw >= seq_len && w.t0 == 0) flag_error(dev_err, UOCR_DEVERR_POS);
+            const int p = (row < n_q && p_raw < seq_len_ok) ? p_raw : -1;
             const int nb_row = p < 0 ? 0 : p / kBlock + 1;
             float *srow = scores + (size_t)(row < n_q ? row : 0) * max_blocks;
+            // which of the unit's blocks have a page in the pool (bit 4t + k), read once per unit
+            // and gathered after the first tile's math, so no tile waits on a block-table load
+            bool in_pool = false;
+            if (lane < w.ntiles * kPagesPerTile) {
+                const int j = w.t0 * kPagesPerTile + lane;
+                if (j < w.nb_max) in_pool = (unsigned)__ldg(bt_row + j) < (unsigned)num_pages;
+            }
             for (int t = 0; t < w.ntiles; ++t, ++it) {
                 const int acc = it & 1;
                 if (!warp_wait(&s.acc_full[acc], (it >> 1) & 1, s, dev_err, lane)) {
@@ -321,34 +350,30 @@ prefill_index_gemm_kernel(const __grid_constant__ CUtensorMap map_q, const __gri
                     tmem + ((uint32_t)(quarter * 32) << 16) + (uint32_t)((acc * kMT + sub) * kBN);
                 // a subtile past the last query holds no accumulator: read nothing, write nothing
                 const bool have = sub < w.nsub;
+                if (have) {
+                    // the tile's 4 blocks in one TMEM round trip (4 x 32 columns in flight)
+                    float v[4][32];
 #pragma unroll
-                for (int k = 0; k < 4; k += 2) {
-                    if (!have) break;
-                    float v0[32], v1[32];
-                    tc::tmem_ld_32x32b_x32(tbase + k * 32, v0);
-                    tc::tmem_ld_32x32b_x32(tbase + (k + 1) * 32, v1);
+                    for (int k = 0; k < 4; ++k) tc::tmem_ld_32x32b_x32(tbase + k * 32, v[k]);
                     tc::tmem_ld_wait();
                     if (interior) {
 #pragma unroll
-                        for (int c = 16; c > 0; c >>= 1) {
+                        for (int k = 0; k < 4; ++k) {
 #pragma unroll
-                            for (int x = 0; x < c; ++x) {
-                                v0[x] = fmaxf(v0[x], v0[x + c]);
-                                v1[x] = fmaxf(v1[x], v1[x + c]);
-                            }
+                            for (int c = 16; c > 0; c >>= 1)
+#pragma unroll
+                                for (int x = 0; x < c; ++x) v[k][x] = fmaxf(v[k][x], v[k][x + c]);
+                            best[k] = v[k][0];
                         }
-                        best[k] = v0[0];
-                        best[k + 1] = v1[0];
                     } else {
-                        const int t0 = (j0 + k) * kBlock, t1 = t0 + kBlock;
-                        float m0 = -INFINITY, m1 = -INFINITY;
 #pragma unroll
-                        for (int c = 0; c < 32; ++c) {
-                            m0 = (t0 + c <= p) ? fmaxf(m0, v0[c]) : m0;
-                            m1 = (t1 + c <= p) ? fmaxf(m1, v1[c]) : m1;
+                        for (int k = 0; k < 4; ++k) {
+                            const int t0 = (j0 + k) * kBlock;
+                            float m = -INFINITY;
+#pragma unroll
+                            for (int c = 0; c < 32; ++c) m = (t0 + c <= p) ? fmaxf(m, v[k][c]) : m;
+                            best[k] = m;
                         }
-                        best[k] = m0;
-                        best[k + 1] = m1;
                     }
                 }
                 tc::fence_before_sync();
@@ -359,12 +384,10 @@ prefill_index_gemm_kernel(const __grid_constant__ CUtensorMap map_q, const __gri
                 if (!have) continue;
                 // a block whose page is not in the pool scores -inf; blocks past the row's
                 // causal range are not written
-                int pg[4];
-#pragma unroll
-                for (int k = 0; k < 4; ++k) pg[k] = (j0 + k < nb_row) ? __ldg(bt_row + j0 + k) : -1;
+                const unsigned pool_mask = __ballot_sync(0xffffffffu, in_pool);
 #pragma unroll
                 for (int k = 0; k < 4; ++k)
-                    if ((unsigned)pg[k] >= (unsigned)num_pages) best[k] = -INFINITY;
+                    if (!((pool_mask >> (t * kPagesPerTile + k)) & 1u)) best[k] = -INFINITY;
                 if (j0 + 4 <= nb_row && (reinterpret_cast<uintptr_t>(srow + j0) & 15u) == 0) {
                     *reinterpret_cast<float4 *>(srow + j0) = make_float4(best[0], best[1], best[2], best[3]);
                 } else {
