@@ -76,30 +76,32 @@ struct UnitInfo {
     int nb_max;   // causal blocks of the tile's last valid query
 };
 
-// Position of query `row`, or -1 when it has no visible token or is invalid.
-__device__ __forceinline__ int row_pos(const int32_t *q_pos, int row, int n_q, int seq_len) {
-    if (row >= n_q) return -1;
-    const int p = __ldg(q_pos + row);
-    return p < seq_len ? p : -1;
-}
-
 // Same answer in every role: the unit's tile range, from the queries' positions.  Split in
-// two so that a role can issue the next unit's position loads (lane_pmax) before working on
-// the current unit, and reduce them (unit_info) when it gets there.
-__device__ __forceinline__ int lane_pmax(int u, int n_units, int n_chunks, const int32_t *q_pos, int n_q,
-                                         int seq_len, int lane) {
-    if (u >= n_units) return -1;
+// two so that a role issues the next unit's position loads (pos_prefetch: predicated loads into
+// registers, nothing consumes them yet) before working on the current unit, and reduces them
+// (unit_info) when it gets there: no role waits on L2 at a unit boundary.
+struct PosPrefetch {
+    int raw[kBM * kMT / 32];   // position of row m0 + 32k + lane, -1 past the queries
+};
+__device__ __forceinline__ PosPrefetch pos_prefetch(int u, int n_units, int n_chunks, const int32_t *q_pos,
+                                                    int n_q, int lane) {
+    PosPrefetch f;
     const int m0 = (u / n_chunks) * (kBM * kMT);
-    int pmax = -1;
 #pragma unroll
-    for (int k = 0; k < kBM * kMT / 32; ++k) pmax = max(pmax, row_pos(q_pos, m0 + k * 32 + lane, n_q, seq_len));
-    return pmax;
+    for (int k = 0; k < kBM * kMT / 32; ++k) {
+        const int row = m0 + k * 32 + lane;
+        f.raw[k] = (u < n_units && row < n_q) ? __ldg(q_pos + row) : -1;
+    }
+    return f;
 }
-__device__ __forceinline__ UnitInfo unit_info(int u, int n_chunks, int n_q, int pmax_lane) {
+__device__ __forceinline__ UnitInfo unit_info(int u, int n_chunks, int n_q, int seq_len, const PosPrefetch &f) {
     UnitInfo w;
     w.m0 = (u / n_chunks) * (kBM * kMT);
     w.nsub = min(kMT, (n_q - w.m0 + kBM - 1) / kBM);
     w.t0 = (u % n_chunks) * kTilesPerUnit;
+    int pmax_lane = -1;
+#pragma unroll
+    for (int k = 0; k < kBM * kMT / 32; ++k) pmax_lane = max(pmax_lane, f.raw[k] < seq_len ? f.raw[k] : -1);
     const int pmax = __reduce_max_sync(0xffffffffu, pmax_lane);
     w.nb_max = pmax < 0 ? 0 : pmax / kBlock + 1;
     const int tiles_needed = (w.nb_max + kPagesPerTile - 1) / kPagesPerTile;
@@ -174,10 +176,10 @@ prefill_index_gemm_kernel(const __grid_constant__ CUtensorMap map_q, const __gri
         // ------------------------------------------------------------ TMA producer: query tiles
         int uc = 0;
         int a_fills[kStagesA] = {};
-        int pm_next = lane_pmax(blockIdx.x, n_units, n_chunks, q_pos, n_q, seq_len_ok, lane);
+        PosPrefetch pf = pos_prefetch(blockIdx.x, n_units, n_chunks, q_pos, n_q, lane);
         for (int u = blockIdx.x; u < n_units; u += gridDim.x) {
-            const UnitInfo w = unit_info(u, n_chunks, n_q, pm_next);
-            pm_next = lane_pmax(u + gridDim.x, n_units, n_chunks, q_pos, n_q, seq_len_ok, lane);
+            const UnitInfo w = unit_info(u, n_chunks, n_q, seq_len_ok, pf);
+            pf = pos_prefetch(u + gridDim.x, n_units, n_chunks, q_pos, n_q, lane);
             if (w.ntiles == 0) continue;
             const int sa = uc % kStagesA;
             if (!warp_wait(&s.a_empty[sa], ((uc / kStagesA) & 1) ^ 1, s, dev_err, lane)) break;
@@ -201,10 +203,10 @@ prefill_index_gemm_kernel(const __grid_constant__ CUtensorMap map_q, const __gri
         int it = 0;
         int b_fills[kStagesB] = {};
         bool stop = false;
-        int pm_next = lane_pmax(blockIdx.x, n_units, n_chunks, q_pos, n_q, seq_len_ok, lane);
+        PosPrefetch pf = pos_prefetch(blockIdx.x, n_units, n_chunks, q_pos, n_q, lane);
         for (int u = blockIdx.x; u < n_units && !stop; u += gridDim.x) {
-            const UnitInfo w = unit_info(u, n_chunks, n_q, pm_next);
-            pm_next = lane_pmax(u + gridDim.x, n_units, n_chunks, q_pos, n_q, seq_len_ok, lane);
+            const UnitInfo w = unit_info(u, n_chunks, n_q, seq_len_ok, pf);
+            pf = pos_prefetch(u + gridDim.x, n_units, n_chunks, q_pos, n_q, lane);
             if (w.ntiles == 0) continue;
             // the unit's page ids at once: lane l < 4 * ntiles holds block t0 * 4 + l
             int upage = -1;
@@ -250,10 +252,10 @@ prefill_index_gemm_kernel(const __grid_constant__ CUtensorMap map_q, const __gri
         static_assert(2 * kMT * kBN == 512, "two accumulator buffers of kMT subtiles fill the 512 TMEM columns");
         int it = 0, uc = 0;
         bool issued = false, stop = false;
-        int pm_next = lane_pmax(blockIdx.x, n_units, n_chunks, q_pos, n_q, seq_len_ok, lane);
+        PosPrefetch pf = pos_prefetch(blockIdx.x, n_units, n_chunks, q_pos, n_q, lane);
         for (int u = blockIdx.x; u < n_units && !stop; u += gridDim.x) {
-            const UnitInfo w = unit_info(u, n_chunks, n_q, pm_next);
-            pm_next = lane_pmax(u + gridDim.x, n_units, n_chunks, q_pos, n_q, seq_len_ok, lane);
+            const UnitInfo w = unit_info(u, n_chunks, n_q, seq_len_ok, pf);
+            pf = pos_prefetch(u + gridDim.x, n_units, n_chunks, q_pos, n_q, lane);
             if (w.ntiles == 0) continue;
             const int sa = uc % kStagesA;
             if (!warp_wait(&s.a_full[sa], (uc / kStagesA) & 1, s, dev_err, lane)) break;
@@ -313,10 +315,10 @@ prefill_index_gemm_kernel(const __grid_constant__ CUtensorMap map_q, const __gri
             return r < n_q ? __ldg(q_pos + r) : -1;
         };
         int p_next = next_row_p(blockIdx.x);
-        int pm_next = lane_pmax(blockIdx.x, n_units, n_chunks, q_pos, n_q, seq_len_ok, lane);
+        PosPrefetch pf = pos_prefetch(blockIdx.x, n_units, n_chunks, q_pos, n_q, lane);
         for (int u = blockIdx.x; u < n_units && !stop; u += gridDim.x) {
-            const UnitInfo w = unit_info(u, n_chunks, n_q, pm_next);
-            pm_next = lane_pmax(u + gridDim.x, n_units, n_chunks, q_pos, n_q, seq_len_ok, lane);
+            const UnitInfo w = unit_info(u, n_chunks, n_q, seq_len_ok, pf);
+            pf = pos_prefetch(u + gridDim.x, n_units, n_chunks, q_pos, n_q, lane);
             if (w.ntiles == 0) {
                 p_next = next_row_p(u + gridDim.x);
                 continue;
@@ -330,11 +332,8 @@ prefill_index_gemm_kernel(const __grid_constant__ CUtensorMap map_q, const __gri
             float *srow = scores + (size_t)(row < n_q ? row : 0) * max_blocks;
             // which of the unit's blocks have a page in the pool (bit 4t + k), read once per unit
             // and gathered after the first tile's math, so no tile waits on a block-table load
-            bool in_pool = false;
-            if (lane < w.ntiles * kPagesPerTile) {
-                const int j = w.t0 * kPagesPerTile + lane;
-                if (j < w.nb_max) in_pool = (unsigned)__ldg(bt_row + j) < (unsigned)num_pages;
-            }
+            const int jp = w.t0 * kPagesPerTile + lane;
+            const int pool_page = (lane < w.ntiles * kPagesPerTile && jp < w.nb_max) ? __ldg(bt_row + jp) : -1;
             for (int t = 0; t < w.ntiles; ++t, ++it) {
                 const int acc = it & 1;
                 if (!warp_wait(&s.acc_full[acc], (it >> 1) & 1, s, dev_err, lane)) {
@@ -384,7 +383,7 @@ prefill_index_gemm_kernel(const __grid_constant__ CUtensorMap map_q, const __gri
                 if (!have) continue;
                 // a block whose page is not in the pool scores -inf; blocks past the row's
                 // causal range are not written
-                const unsigned pool_mask = __ballot_sync(0xffffffffu, in_pool);
+                const unsigned pool_mask = __ballot_sync(0xffffffffu, (unsigned)pool_page < (unsigned)num_pages);
 #pragma unroll
                 for (int k = 0; k < 4; ++k)
                     if (!((pool_mask >> (t * kPagesPerTile + k)) & 1u)) best[k] = -INFINITY;
