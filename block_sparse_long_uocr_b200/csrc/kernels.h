@@ -15,9 +15,6 @@ struct LaunchCtx {
     bool pdl;   // launch with programmatic stream serialization
 };
 
-// CTAs (split-K partitions, one thread-block cluster) per (query, head) in the attention.
-int attn_splits(int n_q, int H);
-
 cudaError_t launch_index_scan(const LaunchCtx &c, const void *idx_q, const void *idx_k,
                               const int32_t *bt, const int32_t *seq_lens, const int32_t *q_seq,
                               const int32_t *q_pos, int n_q, int B, int max_blocks, int num_pages,

@@ -6,7 +6,8 @@
 // lane l holds token 2s + l/16, dims 8*(l%16) .. +8), does 8 fp32 FMAs per load
 // against the lane's 8 query dims, reduces with the 15-shuffle transposed
 // half-warp sum (each lane ends with one token's dot product) and a 5-shuffle
-// warp max.  Shared by index_scan_kernel and the fused decode kernel.
+// warp max.  attend_block_online is the per-block online-softmax step of the
+// comparator decode attention (dense_attn.cu).
 #pragma once
 
 #include "common.cuh"

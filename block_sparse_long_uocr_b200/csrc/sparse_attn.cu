@@ -34,7 +34,6 @@ namespace uocr {
 constexpr int kAttnWarps = 4;                     // blocks per CTA (one per warp)
 constexpr int kAttnCluster = kSel / kAttnWarps;   // CTAs per (query, head)
 
-int attn_splits(int, int) { return kAttnCluster; }
 
 __device__ __forceinline__ uint32_t cluster_ctarank() {
     uint32_t r;

@@ -191,15 +191,22 @@ uocr_status_t uocr_prefill_index_score(const void *idx_q, const void *idx_k_cach
 
 /*
  * The whole chunked-prefill step for n_q queries of sequence `seq` at
- * positions q_pos (their K/V and indexer keys already cached):
- * uocr_prefill_index_score -> uocr_block_topk -> uocr_sparse_attn with
- * scale = 1/sqrt(128), launched back to back on `stream`.  Each query selects
- * its own 4 local + 12 remote blocks over its causal prefix.  out [n_q][H][128]
- * bf16, sel_out [n_q][16].  The attention is block-centric: the selection is
- * inverted per block and every selected (block, head) K/V tile is read once
- * for all the queries that chose it, with per-slot partial softmax states
- * merged per query.  Workspace: uocr_prefill_workspace_bytes(n_q, H, max_blocks)
- * bytes (the block scores first, then the inverted index and the partials).
+ * positions q_pos (their K/V and indexer keys already cached), launched back
+ * to back on `stream`: block scores on the tensor cores (as
+ * uocr_prefill_index_score), the selection (as uocr_block_topk: each query
+ * keeps its own 4 local + 12 remote blocks over its causal prefix), and exact
+ * attention over the selected blocks with scale = 1/sqrt(128) (the result of
+ * uocr_sparse_attn).  out [n_q][H][128] bf16, sel_out [n_q][16] int32.
+ * The attention is block-centric: the selection is inverted per block, every
+ * selected (block, head) K/V tile is read once for all the queries that chose
+ * it, and each (query, slot, head) partial -- the row maximum and weight sum in
+ * fp32, the normalised partial output in bf16 -- is merged per (query, head);
+ * the bf16 partial adds at most 2^-9 max|v| to an output, the size of the
+ * output's own bf16 rounding.  Workspace: uocr_prefill_workspace_bytes(n_q, H,
+ * max_blocks) bytes, 256-byte aligned (the block scores first, then the
+ * inverted index and the partials).  Errors as uocr_sparse_decode; a selected
+ * block whose page is outside the pool contributes nothing to the output and
+ * sets UOCR_DEVERR_PAGE.
  */
 /* Workspace bytes uocr_sparse_prefill needs; a pure function of the shapes. */
 size_t uocr_prefill_workspace_bytes(int n_q, int H, int max_blocks);
