@@ -508,6 +508,11 @@ def run_prefill(args):
     attn_ms = graph_time_fn(lambda st: uocr.sparse_attn(case.q, case.k_pool, case.v_pool, case.block_table,
                                                         case.seq_lens, sel, case.q_seq, case.q_pos, out=out,
                                                         stream=st), stream, n_rep, flush_buf)
+    seq_ws = torch.empty(max(uocr.sparse_attn_seq_workspace_bytes(n_q, H, mb), 1), dtype=torch.uint8, device=dev)
+    out_seq = torch.empty_like(out)
+    attn_seq_ms = graph_time_fn(lambda st: uocr.sparse_attn_seq(case.q, case.k_pool, case.v_pool, case.block_table,
+                                                                case.seq_lens, 0, case.q_pos, sel, out=out_seq,
+                                                                workspace=seq_ws, stream=st), stream, n_rep, flush_buf)
     call_ms = graph_time_fn(lambda st: step(st), stream, n_rep, flush_buf)
     pos = case.q_pos.cpu().long()
     idx_flops = float(((pos + 1) * 128 * 2).sum())                 # causal q_idx . k_idx products
@@ -518,6 +523,9 @@ def run_prefill(args):
     hbm_peak = float(peaks.get("hbm_gbs", FALLBACK_HBM_GBS))
     gemm_tflops = idx_flops / (gemm_ms / 1e3) / 1e12
     kv_union = case.num_pages * H * 32 * 128 * 2 * 2               # every page is selected by some query
+    n_sel_blocks = int(torch.unique(sel[sel >= 0]).numel())
+    attn_bytes = n_sel_blocks * H * 32 * 128 * 2 * 2 + 2 * n_q * H * 128 * 2   # selected K/V tiles once, q, out
+    attn_gbs = attn_bytes / (attn_seq_ms / 1e3) / 1e9
     step_bytes = kv_union + case.num_pages * 32 * 128 * 2 + 2 * n_q * mb * 4 + 2 * n_q * H * 128 * 2
     result = {
         "metric": "chunked-prefill queries/s per layer; tensor-core TFLOP/s of the scoring GEMM vs peak",
@@ -534,8 +542,15 @@ def run_prefill(args):
                           "peak": hbm_peak, "unit": "GB/s",
                           "frac": round(step_bytes / (call_ms / 1e3) / 1e9 / hbm_peak, 4),
                           "bytes_per_step": step_bytes, "flops_per_step": idx_flops + attn_flops},
+        "attn_roofline": {"bound": "hbm", "entry": "uocr_sparse_attn_seq: selection check, inversion, "
+                          "tensor-core block kernel, merge (5 kernels)", "achieved": round(attn_gbs, 1),
+                          "peak": hbm_peak, "unit": "GB/s", "frac": round(attn_gbs / hbm_peak, 4),
+                          "bytes_per_launch": attn_bytes, "avg_launch_ms": round(attn_seq_ms, 5),
+                          "selected_blocks": n_sel_blocks},
         "breakdown_us": {"prefill_index_gemm": round(1e3 * gemm_ms, 2), "block_topk": round(1e3 * topk_ms, 2),
-                         "sparse_attn": round(1e3 * attn_ms, 2), "prefill_call_graph": round(1e3 * call_ms, 2)},
+                         "sparse_attn_seq": round(1e3 * attn_seq_ms, 2),
+                         "sparse_attn_query_centric": round(1e3 * attn_ms, 2),
+                         "prefill_call_graph": round(1e3 * call_ms, 2)},
         # per call: scoring GEMM, selection, scan, fill, block attention, merge
         "gpu_launches": args.steps * 6,
         "clocks": clk.summary(),

@@ -93,6 +93,10 @@ def _load() -> ctypes.CDLL:
     lib.uocr_prefill_index_score.restype = I
     lib.uocr_sparse_prefill.argtypes = [P, P, P, P, P, P, P, I, P, I, I, I, I, I, P, P, P, Z, P, P]
     lib.uocr_sparse_prefill.restype = I
+    lib.uocr_sparse_attn_seq_workspace_bytes.argtypes = [I, I, I]
+    lib.uocr_sparse_attn_seq_workspace_bytes.restype = Z
+    lib.uocr_sparse_attn_seq.argtypes = [P, P, P, P, P, I, P, P, I, I, I, I, I, F, P, P, Z, P, P]
+    lib.uocr_sparse_attn_seq.restype = I
     lib.uocr_sparse_decode_static.argtypes = [P, P, P, P, P, P, P, I, I, I, I, P, P, P, P]
     lib.uocr_sparse_decode_static.restype = I
     return lib
@@ -158,6 +162,10 @@ def prefill_workspace_bytes(n_q: int, heads: int, max_blocks: int) -> int:
 def alloc_prefill_workspace(n_q: int, heads: int, max_blocks: int, device) -> torch.Tensor:
     """uint8 workspace for sparse_prefill; its first n_q*max_blocks*4 bytes hold the block scores."""
     return torch.empty(max(prefill_workspace_bytes(n_q, heads, max_blocks), 1), dtype=torch.uint8, device=device)
+
+
+def sparse_attn_seq_workspace_bytes(n_q: int, heads: int, max_blocks: int) -> int:
+    return int(_lib().uocr_sparse_attn_seq_workspace_bytes(int(n_q), int(heads), int(max_blocks)))
 
 
 def alloc_workspace(n_q: int, heads: int, max_blocks: int, device) -> torch.Tensor:
@@ -283,6 +291,30 @@ def sparse_prefill(q, k_cache, v_cache, idx_q, idx_k_cache, block_table, seq_len
         int(seq), _ptr(q_pos), n_q, B, H, mb, k_cache.shape[0], _ptr(out), _ptr(sel), _ptr(workspace),
         workspace.numel(), _ptr(dev_err), _stream(stream)))
     return out, sel
+
+
+def sparse_attn_seq(q, k_cache, v_cache, block_table, seq_lens, seq: int, q_pos, sel, *, scale=None,
+                    out=None, workspace=None, dev_err=None, stream=None) -> torch.Tensor:
+    """Attention of many queries of sequence `seq` over the given selection (block-centric).
+    Returns out [n_q,H,128] bf16."""
+    for t, n, dt, nd in ((q, "q", torch.bfloat16, 3), (k_cache, "k_cache", torch.bfloat16, 4),
+                         (v_cache, "v_cache", torch.bfloat16, 4), (block_table, "block_table", torch.int32, 2),
+                         (seq_lens, "seq_lens", torch.int32, 1), (q_pos, "q_pos", torch.int32, 1),
+                         (sel, "sel", torch.int32, 2)):
+        _dev(t, n, dt, nd)
+    n_q, H = q.shape[0], q.shape[1]
+    B, mb = block_table.shape
+    if out is None:
+        out = torch.empty_like(q)
+    if workspace is None:
+        workspace = torch.empty(max(sparse_attn_seq_workspace_bytes(n_q, H, mb), 1), dtype=torch.uint8,
+                                device=q.device)
+    sc = float(scale) if scale is not None else HEAD_DIM ** -0.5
+    _check("uocr_sparse_attn_seq", _lib().uocr_sparse_attn_seq(
+        _ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(block_table), _ptr(seq_lens), int(seq), _ptr(q_pos), _ptr(sel),
+        n_q, B, H, mb, k_cache.shape[0], sc, _ptr(out), _ptr(workspace), workspace.numel(), _ptr(dev_err),
+        _stream(stream)))
+    return out
 
 
 def summary_score(idx_q, summary_cache, block_table, seq_lens, q_seq=None, q_pos=None, *,

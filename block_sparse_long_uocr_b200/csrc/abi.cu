@@ -234,6 +234,42 @@ uocr_status_t uocr_sparse_prefill(const void *q, const void *k_cache, const void
     return cuda_status(e);
 }
 
+size_t uocr_sparse_attn_seq_workspace_bytes(int n_q, int H, int max_blocks) {
+    if (n_q <= 0 || H <= 0 || max_blocks <= 0) return 0;
+    return uocr::prefill_attn_workspace(n_q, H, max_blocks, nullptr);
+}
+
+uocr_status_t uocr_sparse_attn_seq(const void *q, const void *k_cache, const void *v_cache,
+                                   const int32_t *block_table, const int32_t *seq_lens, int seq,
+                                   const int32_t *q_pos, const int32_t *sel, int n_q, int B, int H,
+                                   int max_blocks, int num_pages, float scale, void *out, void *workspace,
+                                   size_t workspace_bytes, int32_t *dev_err, uocr_stream_t stream) {
+    uocr_status_t st = check_common(n_q, B, max_blocks, num_pages, block_table, seq_lens, nullptr, q_pos, dev_err);
+    if (st != UOCR_OK) return st;
+    if (!bf16_ok(q) || !bf16_ok(k_cache) || !bf16_ok(v_cache) || !bf16_ok(out) || !q_pos) return UOCR_ERR_INVALID_ARG;
+    if (!sel || !aligned(sel, 4)) return UOCR_ERR_INVALID_ARG;
+    if (seq < 0 || seq >= B) return UOCR_ERR_INVALID_ARG;
+    if (H < 1 || H > UOCR_MAX_HEADS) return UOCR_ERR_UNSUPPORTED;
+    if (!isfinite(scale)) return UOCR_ERR_INVALID_ARG;
+    if (n_q == 0) return UOCR_OK;
+    if ((long long)n_q * UOCR_N_SEL > 0x7fffffffLL || (long long)n_q * H > 0x7fffffffLL) return UOCR_ERR_UNSUPPORTED;
+    if (!workspace || !aligned(workspace, kWsAlign) ||
+        workspace_bytes < uocr_sparse_attn_seq_workspace_bytes(n_q, H, max_blocks))
+        return UOCR_ERR_WORKSPACE;
+    uocr::LaunchCtx c;
+    if ((st = make_ctx(stream, false, c)) != UOCR_OK) return st;
+    uocr::PrefillAttnWs aw;
+    uocr::prefill_attn_workspace(n_q, H, max_blocks, &aw);
+    char *ws = (char *)workspace;
+    cudaError_t e = cudaMemsetAsync(ws + aw.counts_off, 0, (size_t)max_blocks * sizeof(int32_t), c.stream);
+    if (e != cudaSuccess) return cuda_status(e);
+    e = uocr::launch_prefill_select_count(c, sel, q_pos, seq_lens + seq, n_q, max_blocks, workspace, dev_err);
+    if (e != cudaSuccess) return cuda_status(e);
+    return cuda_status(uocr::launch_prefill_attn(c, q, k_cache, v_cache, block_table + (size_t)seq * max_blocks,
+                                                 q_pos, (const int32_t *)(ws + aw.sel_off), n_q, H, max_blocks,
+                                                 num_pages, scale, out, workspace, dev_err));
+}
+
 size_t uocr_dense_workspace_bytes(int B, int H, int max_blocks) {
     if (B <= 0 || H <= 0 || max_blocks <= 0) return 0;
     return uocr::dense_attn_workspace(B, H, max_blocks);

@@ -42,11 +42,16 @@ cudaError_t launch_prefill_index_gemm(const LaunchCtx &c, const void *idx_q, con
 // entries per (block, head), per-slot partials merged per (query, head)).  Workspace regions,
 // 256-byte aligned.
 struct PrefillAttnWs {
-    size_t counts_off, cursor_off, n_items_off, items_off, list_off, ml_off, o_off;
+    size_t counts_off, cursor_off, n_items_off, items_off, list_off, sel_off, ml_off, o_off;
 };
 size_t prefill_attn_workspace(int n_q, int H, int max_blocks, PrefillAttnWs *w);
 // `ws` must start with the per-block selection counts of `sel` (max_blocks int32), as
 // launch_block_topk writes them when given `counts` zeroed.
+// For a caller's selection: a validated copy of it into the workspace's sel region and the
+// per-block counts (zeroed by the caller) that launch_prefill_attn expects.
+cudaError_t launch_prefill_select_count(const LaunchCtx &c, const int32_t *sel, const int32_t *q_pos,
+                                       const int32_t *seq_len_ptr, int n_q, int max_blocks, void *ws,
+                                       int32_t *dev_err);
 cudaError_t launch_prefill_attn(const LaunchCtx &c, const void *q, const void *k, const void *v,
                                 const int32_t *bt_row, const int32_t *q_pos, const int32_t *sel, int n_q, int H,
                                 int max_blocks, int num_pages, float scale, void *out, void *ws,

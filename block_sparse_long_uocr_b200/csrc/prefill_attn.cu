@@ -86,6 +86,33 @@ __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi, float &sum) {
 }
 }  // namespace
 
+// A caller's selection for many queries of one sequence (uocr_sparse_attn_seq): sel_ws keeps
+// the slots that name a causal block of a query at a valid position (0 <= j < p / 32 + 1,
+// 0 <= p < seq_len) and -1 elsewhere, flagging UOCR_DEVERR_SEL / UOCR_DEVERR_POS as
+// sparse_attn does; counts[j] += 1 for every kept slot.
+__global__ void __launch_bounds__(kInvThreads)
+prefill_select_count_kernel(const int32_t *__restrict__ sel, const int32_t *__restrict__ q_pos,
+                            const int32_t *__restrict__ seq_len_ptr, int n_entries, int max_blocks,
+                            int32_t *__restrict__ sel_ws, int32_t *counts, int32_t *dev_err) {
+    pdl_wait();
+    const int e = blockIdx.x * kInvThreads + threadIdx.x;
+    if (e >= n_entries) return;
+    const int seq_len = min(__ldg(seq_len_ptr), max_blocks * kBlock);
+    const int p = __ldg(q_pos + e / kSel);
+    int j = __ldg(sel + e);
+    if (p < 0 || p >= seq_len) {
+        if ((e & (kSel - 1)) == 0) flag_error(dev_err, UOCR_DEVERR_POS);
+        j = -1;
+    } else if (j >= p / kBlock + 1) {
+        flag_error(dev_err, UOCR_DEVERR_SEL);
+        j = -1;
+    } else if (j < 0) {
+        j = -1;
+    }
+    sel_ws[e] = j;
+    if (j >= 0) atomicAdd(counts + j, 1);
+}
+
 // One CTA: cursor = exclusive prefix sum of counts (each block's first list position), and the
 // work items:
 // block j with n_j entries gives items (j, 0) .. (j, ceil(n_j / 16) - 1), in block order, each
@@ -433,12 +460,34 @@ size_t prefill_attn_workspace(int n_q, int H, int max_blocks, PrefillAttnWs *w) 
     off += up(item_bound(n_q, max_blocks) * sizeof(int4));
     l.list_off = off;
     off += up((size_t)n_q * kSel * sizeof(int2));
+    l.sel_off = off;
+    off += up((size_t)n_q * kSel * 4);
     l.ml_off = off;
     off += up((size_t)n_q * H * kSel * 2 * 4);
     l.o_off = off;
     off += up((size_t)n_q * H * kSel * kD * 2);
     if (w) *w = l;
     return off;
+}
+
+cudaError_t launch_prefill_select_count(const LaunchCtx &c, const int32_t *sel, const int32_t *q_pos,
+                                       const int32_t *seq_len_ptr, int n_q, int max_blocks, void *ws,
+                                       int32_t *dev_err) {
+    PrefillAttnWs w;
+    prefill_attn_workspace(n_q, 1, max_blocks, &w);   // the regions before the partials do not depend on H
+    char *base = (char *)ws;
+    const int n_entries = n_q * kSel;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cudaLaunchConfig_t cfg = {};
+    cfg.stream = c.stream;
+    cfg.attrs = attr;
+    cfg.numAttrs = c.pdl ? 1 : 0;
+    cfg.gridDim = dim3((unsigned)((n_entries + kInvThreads - 1) / kInvThreads));
+    cfg.blockDim = dim3(kInvThreads);
+    return cudaLaunchKernelEx(&cfg, prefill_select_count_kernel, sel, q_pos, seq_len_ptr, n_entries, max_blocks,
+                              (int32_t *)(base + w.sel_off), (int32_t *)(base + w.counts_off), dev_err);
 }
 
 cudaError_t launch_prefill_attn(const LaunchCtx &c, const void *q, const void *k, const void *v,

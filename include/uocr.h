@@ -190,6 +190,32 @@ uocr_status_t uocr_prefill_index_score(const void *idx_q, const void *idx_k_cach
                                        int32_t *dev_err, uocr_stream_t stream);
 
 /*
+ * Exact attention of n_q queries of one sequence `seq` over the blocks a
+ * caller selected for them: the result of uocr_sparse_attn with q_seq all
+ * `seq`, computed block-centrically for many queries (the attention of
+ * uocr_sparse_prefill).  [rkmt 五 step 4]
+ *   q        [n_q][H][128] bf16 (device)
+ *   q_pos    [n_q] int32 positions, required; sel [n_q][16] int32 block ids
+ *            (-1 = empty slot), in any order
+ *   out      [n_q][H][128] bf16 (device)
+ * A slot naming a block that is not causal for its query (id >= p / 32 + 1)
+ * is ignored and sets UOCR_DEVERR_SEL; a query at a position outside
+ * [0, seq_len) gets a zero output and sets UOCR_DEVERR_POS; a block whose page
+ * is outside the pool contributes nothing and sets UOCR_DEVERR_PAGE.  The
+ * per-slot partial outputs are rounded to bf16 before the merge (at most
+ * 2^-9 max|v| on an output).  Workspace: uocr_sparse_attn_seq_workspace_bytes
+ * bytes, 256-byte aligned, owned by the caller, a pure function of the shapes.
+ */
+size_t uocr_sparse_attn_seq_workspace_bytes(int n_q, int H, int max_blocks);
+
+uocr_status_t uocr_sparse_attn_seq(const void *q, const void *k_cache, const void *v_cache,
+                                   const int32_t *block_table, const int32_t *seq_lens, int seq,
+                                   const int32_t *q_pos, const int32_t *sel, int n_q, int B, int H,
+                                   int max_blocks, int num_pages, float scale, void *out,
+                                   void *workspace, size_t workspace_bytes,
+                                   int32_t *dev_err, uocr_stream_t stream);
+
+/*
  * The whole chunked-prefill step for n_q queries of sequence `seq` at
  * positions q_pos (their K/V and indexer keys already cached), launched back
  * to back on `stream`: block scores on the tensor cores (as

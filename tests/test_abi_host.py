@@ -205,6 +205,32 @@ def test_sparse_prefill_rejects(pkg, over, code):
     assert st == code
 
 
+@no_gpu
+@pytest.mark.parametrize("over,code", [
+    (dict(q_pos=None), 1), (dict(seq=5), 1), (dict(seq=-1), 1), (dict(sel=None), 1), (dict(sel=MIS), 1),
+    (dict(out=MIS), 1), (dict(q=None), 1), (dict(H=0), 2), (dict(H=65), 2), (dict(scale=float("nan")), 1),
+    (dict(ws=None), 3), (dict(wsb=16), 3), (dict(ws=FAKE + 64), 3), (dict(mb=0), 1), (dict(P=0), 1),
+])
+def test_sparse_attn_seq_rejects(pkg, over, code):
+    a = dict(q=FAKE, k=FAKE, v=FAKE, bt=FAKE, sl=FAKE, seq=0, q_pos=FAKE, sel=FAKE, n_q=4, B=4, H=10, mb=64, P=256,
+             scale=0.088, out=FAKE, ws=FAKE, wsb=1 << 30)
+    a.update(over)
+    st = pkg.lib.uocr_sparse_attn_seq(a["q"], a["k"], a["v"], a["bt"], a["sl"], a["seq"], a["q_pos"], a["sel"],
+                                      a["n_q"], a["B"], a["H"], a["mb"], a["P"], a["scale"], a["out"], a["ws"],
+                                      a["wsb"], None, None)
+    assert st == code
+
+
+def test_sparse_attn_seq_workspace_is_a_pure_function_of_shapes(pkg):
+    f = pkg.sparse_attn_seq_workspace_bytes
+    assert f(0, 10, 64) == 0 and f(4, 0, 64) == 0 and f(4, 10, 0) == 0
+    a = f(2048, 10, 2048)
+    assert a == f(2048, 10, 2048) and a % 256 == 0
+    # the inversion (counts, cursor, items, entries, the checked selection) and the partial states
+    assert a >= 2048 * 10 * 16 * (128 * 2 + 8) + 2048 * 16 * (8 + 4) + 2 * 2048 * 4
+    assert f(2048, 1, 2048) < a and f(4096, 10, 2048) > a
+
+
 def test_prefill_workspace_is_a_pure_function_of_shapes(pkg):
     pw, ws = pkg.prefill_workspace_bytes, pkg.workspace_bytes
     assert pw(0, 10, 64) == 0 and pw(4, 0, 64) == 0 and pw(4, 10, 0) == 0

@@ -123,6 +123,61 @@ def test_sparse_prefill_bad_page_gives_an_empty_block(uocr, cuda_device):
     assert hit > 50
 
 
+def _random_selection(case, seed, empty_frac=0.2):
+    """Per query: distinct causal blocks (up to 16) in random slots, some slots empty (-1)."""
+    g = np.random.default_rng(seed)
+    sel = np.full((case.n_q, 16), -1, np.int32)
+    for i in range(case.n_q):
+        nb = int(case.q_pos[i]) // 32 + 1
+        k = min(16, nb)
+        picks = g.choice(nb, size=k, replace=False)
+        keep = g.random(k) >= empty_frac
+        keep[0] = True
+        slots = g.permutation(16)[:k]
+        sel[i, slots[keep]] = picks[keep]
+    return sel
+
+
+def test_sparse_attn_seq_matches_oracle(uocr, cuda_device):
+    """Block-centric attention of a caller's selection (ragged n_q, several 16-entry items per
+    block, empty slots, blocks shared by many queries) against the oracle, query by query."""
+    case = _prefill_case(32 * 90 + 11, 333, (0, 5, 31, 32, 700), seed=31, device=cuda_device)
+    sel = _random_selection(case, 31)
+    sel_d = torch.from_numpy(sel).to(cuda_device)
+    out = uocr.sparse_attn_seq(case.q, case.k_pool, case.v_pool, case.block_table, case.seq_lens, 0, case.q_pos,
+                               sel_d)
+    ref_q = uocr.sparse_attn(case.q, case.k_pool, case.v_pool, case.block_table, case.seq_lens, sel_d,
+                             case.q_seq, case.q_pos)
+    torch.cuda.synchronize()
+    got = out.float().cpu().numpy()
+    for i in range(case.n_q):
+        ref = oracle_attend(case, i, sel[i])
+        d = np.abs(got[i] - ref)
+        assert d.max() <= OUT_MAX_ATOL and d.mean() <= OUT_MEAN_ATOL, f"query {i}"
+    # and the query-centric entry on the same selection agrees to within both roundings
+    assert (out.float() - ref_q.float()).abs().max().item() <= 2e-2
+
+
+def test_sparse_attn_seq_flags_bad_selections(uocr, cuda_device):
+    case = _prefill_case(32 * 40, 64, seed=32, device=cuda_device, heads=3)
+    sel = _random_selection(case, 32, empty_frac=0.0)
+    sel[5, 3] = int(case.q_pos[5]) // 32 + 1           # one block past the query's causal range
+    q_pos = case.q_pos.clone()
+    q_pos[7] = int(case.seq_lens[0])                    # a position at the sequence length: invalid
+    err = torch.zeros(1, dtype=torch.int32, device=cuda_device)
+    out = uocr.sparse_attn_seq(case.q, case.k_pool, case.v_pool, case.block_table, case.seq_lens, 0, q_pos,
+                               torch.from_numpy(sel).to(cuda_device), dev_err=err)
+    torch.cuda.synchronize()
+    assert int(err.item()) & uocr.DEVERR_SEL and int(err.item()) & uocr.DEVERR_POS
+    got = out.float().cpu().numpy()
+    assert np.isfinite(got).all() and (got[7] == 0).all()
+    s5 = sel[5].copy()
+    s5[3] = -1
+    for i, s in ((5, s5), (6, sel[6])):
+        d = np.abs(got[i] - oracle_attend(case, i, s))
+        assert d.max() <= OUT_MAX_ATOL and d.mean() <= OUT_MEAN_ATOL, f"query {i}"
+
+
 @pytest.mark.slow
 def test_chunked_prefill_workload_sampled(uocr, cuda_device):
     case = workloads.chunked_prefill(device=cuda_device)
