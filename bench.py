@@ -44,9 +44,9 @@ FALLBACK_HBM_GBS = 6650.0
 # dram__bytes_write.sum), per launch of the default workload, and the hash of the
 # kernel source it was taken on.  Reported as null once the source has changed.
 NCU_TRAFFIC = {
-    # ncu --set full on long_decode batch 4 (1 layer), one launch: 134,299,392 B read +
-    # 4,135,168 B written (the write-back of the bench's L2 flush), scaled x4 to 16 queries.
-    "long_decode": {"bytes": 4 * (134299392 + 4135168), "src": "838030ba57b367b4"},
+    # ncu --set full on long_decode batch 4 (1 layer), one launch: 134,299,136 B read +
+    # 3,573,248 B written (the write-back of the bench's L2 flush), scaled x4 to 16 queries.
+    "long_decode": {"bytes": 4 * (134299136 + 3573248), "src": "91046180f0834582"},
 }
 
 
@@ -363,9 +363,11 @@ def run_uocr(args):
         del summ
         for o in outs:
             o.zero_()
+    read_cal = read_calibration(dev, stream)
     peaks, peak_kind = measured_peaks()
     peak = float(peaks.get("hbm_gbs", FALLBACK_HBM_GBS))
     scan_gbs = scan_bytes_call / (scan_ms / 1e3) / 1e9
+    read_cal["scan_frac_of_read"] = round(scan_gbs / read_cal["gbs"], 4)
     step_gbs = bytes_call * n_layers / (ms_per_step / 1e3) / 1e9
     tr = NCU_TRAFFIC.get(args.workload) if (args.workload != "long_decode" or B == 16) else None
     traffic = tr["bytes"] if tr and tr.get("src") == kernel_source_hash(*SCAN_SOURCES) else None
@@ -396,6 +398,7 @@ def run_uocr(args):
                          "note": "device time per launch from CUDA-graph replays of each entry point alone; "
                                  "the decode call chains the three with programmatic dependent launch"},
         "comparators": comparators,
+        "hbm_read_calibration": read_cal,
         "e2e": e2e,
         "gpu_launches": args.steps * n_layers * 3,
         "clocks": clocks,
@@ -406,6 +409,26 @@ def run_uocr(args):
         torch.distributed.destroy_process_group()
     if rank == 0:
         print(json.dumps(result), flush=True)
+
+
+def read_calibration(dev, stream, gib: int = 4, reps: int = 5):
+    """Read-only HBM stream for context beside the copy peak: torch.sum over `gib` GiB of bf16
+    (the scan is a pure read stream, which can run above a copy's read + write rate)."""
+    x = torch.ones(gib * (1 << 30) // 2, dtype=torch.bfloat16, device=dev)
+    for _ in range(2):
+        x.sum()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(reps):
+        x.sum()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    ms = e0.elapsed_time(e1) / reps
+    gbs = x.numel() * 2 / (ms / 1e3) / 1e9
+    del x
+    torch.cuda.empty_cache()
+    return {"kind": f"torch.sum over {gib} GiB bf16", "gbs": round(gbs, 1), "ms": round(ms, 4)}
 
 
 def graph_time_fn(fn, stream, n_rep, flush_buf=None):
