@@ -580,7 +580,7 @@ def run_prefill(args):
     }
     result["e2e"] = run_prefill_e2e(args, uocr, case, ws, out, sel, stream, world, dev)
     if rank == 0 and not args.no_cpu_baseline:
-        result["cpu_baseline"] = cpu_baseline(case, args.cpu_budget, max_passes=1)
+        result["cpu_baseline"] = cpu_baseline(case, args.cpu_budget)
     if world > 1:
         torch.distributed.destroy_process_group()
     if rank == 0:
@@ -724,38 +724,66 @@ def _gather_kv(case, layer, queries, sel):
     return kp[pidx].cpu(), vp[pidx].cpu(), np.stack(rows)
 
 
+class OracleInputs:
+    """Host copies of what the oracle reads for `queries` of one layer: their queries, the
+    sequences' indexer pages, and (after a first selection) the selected K/V pages."""
+
+    def __init__(self, case, layer, queries):
+        import oracle
+        self.n = len(queries)
+        self.q, self.qi, self.mini_idx, self.bt, self.qs, self.qp = _gather_for_oracle(case, layer, queries)
+        H = self.q.shape[1]
+        dummy = torch.zeros((1, H, 32, 128), dtype=torch.bfloat16)
+        r = oracle.run(self.q, self.qi, dummy, dummy, self.mini_idx, self.bt, self.qs, self.qp, want_out=False,
+                       want_scores=False)
+        self.sel = r["sel"]
+        self.kp, self.vp, self.bt2 = _gather_kv(case, layer, queries, self.sel)
+        self.dummy = dummy
+
+    def time(self, threads=0):
+        """Seconds of oracle work (scores + selection, then attention over the selection)."""
+        import numpy as np
+        import oracle
+        t0 = time.perf_counter()
+        r = oracle.run(self.q, self.qi, self.dummy, self.dummy, self.mini_idx, self.bt, self.qs, self.qp,
+                       want_out=False, want_scores=False, threads=threads)
+        t1 = time.perf_counter()
+        own_row = np.arange(self.n, dtype=np.int32)     # bt2 has one row per query
+        r2 = oracle.run(self.q, self.qi, self.kp, self.vp, self.mini_idx[:1], self.bt2, own_row, self.qp,
+                        sel_in=r["sel"], threads=threads)
+        t2 = time.perf_counter()
+        return t2 - t0, r["threads"], r2
+
+
 def oracle_time_queries(case, layer, queries, threads=0):
     """Seconds of oracle work (scores + selection, then attention) for `queries` of one layer."""
-    import numpy as np
-    import oracle
-    q, qi, mini_idx, bt, qs, qp = _gather_for_oracle(case, layer, queries)
-    H = q.shape[1]
-    dummy = torch.zeros((1, H, 32, 128), dtype=torch.bfloat16)
-    t0 = time.perf_counter()
-    r = oracle.run(q, qi, dummy, dummy, mini_idx, bt, qs, qp, want_out=False, want_scores=False, threads=threads)
-    t1 = time.perf_counter()
-    kp, vp, bt2 = _gather_kv(case, layer, queries, r["sel"])
-    t2 = time.perf_counter()
-    own_row = np.arange(len(queries), dtype=np.int32)     # bt2 has one row per query
-    r2 = oracle.run(q, qi, kp, vp, mini_idx[:1], bt2, own_row, qp, sel_in=r["sel"], threads=threads)
-    t3 = time.perf_counter()
-    return (t1 - t0) + (t3 - t2), r["threads"], r2
+    return OracleInputs(case, layer, queries).time(threads)
 
 
-def cpu_baseline(case, budget_s: float = 10.0, max_passes: int = 4):
+def cpu_baseline(case, budget_s: float = 10.0, max_layers: int = 2):
     """The oracle as it stands, on this host's cores, on a bounded sample of the same workload:
-    whole layers of queries, cycling over the layers, until about budget_s seconds of oracle time."""
-    n_layers = len(case.layers)
+    whole layers of queries (the inputs of up to `max_layers` layers read back once), timed pass
+    after pass until about budget_s seconds of oracle time."""
+    n_layers = min(len(case.layers), max_layers)
+    inputs = [OracleInputs(case, l, list(range(case.n_q))) for l in range(n_layers)]
     done, secs, threads, calls = 0, 0.0, 1, 0
-    while secs < budget_s and calls < max_passes * n_layers:
-        t, threads, _ = oracle_time_queries(case, calls % n_layers, list(range(case.n_q)))
+    while secs < budget_s and calls < 1000:
+        t, threads, _ = inputs[calls % n_layers].time()
         secs += t
         done += case.n_q
         calls += 1
+    # the same oracle on one thread, on a few queries of the first layer (about 2 s)
+    one, n1 = 0.0, 0
+    while one < 2.0 and n1 < case.n_q:
+        k = min(max(1, n1), case.n_q - n1)
+        t, _, _ = oracle_time_queries(case, 0, list(range(n1, n1 + k)), threads=1)
+        one += t
+        n1 += k
     return {"value": round(done / secs, 2), "unit": UNIT, "cores": threads, "kind": "oracle",
-            "sample": f"{done} queries ({calls} layer calls of {case.n_q} queries) of {case.name}, "
-                      f"fp64, {secs:.1f} s of oracle time (host reads excluded)",
-            "host_cpus": os.cpu_count()}
+            "sample": f"{done} queries ({calls} passes over {n_layers} layer(s) of {case.n_q} queries) of "
+                      f"{case.name}, fp64, {secs:.1f} s of oracle time (host reads excluded)",
+            "host_cpus": os.cpu_count(),
+            "value_1_thread": round(n1 / one, 2), "sample_1_thread": f"{n1} queries, {one:.1f} s"}
 
 
 # --------------------------------------------------------------------------- reference arm
