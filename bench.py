@@ -354,12 +354,30 @@ def run_uocr(args):
                              generator=torch.Generator(device=dev).manual_seed(1))
         masked_topk_ms = graph_time(lambda l, st: uocr.block_topk_masked(scores, case.seq_lens, mask, sel=sels[l],
                                                                          stream=st))
+        # the step before the scan (row f2): page2d rotation of one new token per sequence and its
+        # append to the caches, here into a separate small cache (one page per sequence) so that the
+        # workload's caches stay as they are
+        g = torch.Generator(device=dev).manual_seed(3)
+        rq = torch.randn((B, H, 128), generator=g, device=dev).to(torch.bfloat16)
+        rqi = torch.randn((B, 128), generator=g, device=dev).to(torch.bfloat16)
+        rk, rv = torch.randn_like(rq.float()).to(torch.bfloat16), torch.randn_like(rq.float()).to(torch.bfloat16)
+        rki = torch.randn_like(rqi.float()).to(torch.bfloat16)
+        rpos = case.seq_lens - 1
+        rpage = rpos // 4096
+        rbt = torch.arange(B, dtype=torch.int32, device=dev).view(B, 1)
+        rsl = torch.full((B,), 32, dtype=torch.int32, device=dev)
+        rkc = torch.zeros((B, H, 32, 128), dtype=torch.bfloat16, device=dev)
+        rvc, rkic = torch.zeros_like(rkc), torch.zeros((B, 32, 128), dtype=torch.bfloat16, device=dev)
+        rope_ms = graph_time(lambda l, st: uocr.rope_append(rq, rqi, rk, rv, rki, rpos, rpage, rbt, rsl, rkc, rvc,
+                                                            rkic, stream=st))
+        del rq, rqi, rk, rv, rki, rkc, rvc, rkic
         summary_bytes = B * (256 * mb + KV_BYTES_PER_QUERY)     # one 256-byte summary per causal block
         comparators["variants"] = {
             "summary_decode_us": round(1e3 * summary_ms, 2),
             "summary_decode_gbs": round(summary_bytes / (summary_ms / 1e3) / 1e9, 1),
             "summary_speedup_vs_token_scan": round(decode_ms / summary_ms, 2),
-            "masked_topk_us": round(1e3 * masked_topk_ms, 2), "topk_us": round(1e3 * topk_ms, 2)}
+            "masked_topk_us": round(1e3 * masked_topk_ms, 2), "topk_us": round(1e3 * topk_ms, 2),
+            "rope_append_us": round(1e3 * rope_ms, 2), "rope_append_tokens": B}
         del summ
         for o in outs:
             o.zero_()

@@ -13,7 +13,8 @@
 // 1e5 radians, where an fp32 product alone would be off by ~0.01 rad), reduced
 // to [-pi, pi] and passed to sincosf; then the H query heads and the indexer
 // query are rotated in place, and the H key heads, the indexer key (rotated) and
-// the H value heads (unchanged) are written to the token's cache row.
+// the H value heads (unchanged) are written to the token's cache row, 16 bytes
+// (8 pairs) per thread and step.
 #include <cuda_bf16.h>
 #include <math.h>
 
@@ -67,10 +68,11 @@ rope_append_kernel(__nv_bfloat16 *__restrict__ q, __nv_bfloat16 *__restrict__ id
         }
     }
 
-    // rotation work items: (vector v, pair d) for v in [q heads..., idx_q, k heads..., idx_k]
+    // rotation work items: (vector v, chunk c) for v in [q heads..., idx_q, k heads..., idx_k]; chunk c
+    // holds pairs 8c .. 8c + 7, i.e. dims 8c .. 8c + 7 and 64 + 8c .. 64 + 8c + 7 (two 16-byte loads)
     const int n_vec = 2 * H + 2;
-    for (int w = tid; w < n_vec * kPairs; w += kRopeThreads) {
-        const int v = w / kPairs, d = w % kPairs;
+    for (int w = tid; w < n_vec * (kPairs / 8); w += kRopeThreads) {
+        const int v = w / (kPairs / 8), c = w % (kPairs / 8);
         const __nv_bfloat16 *src;
         __nv_bfloat16 *dst;
         if (v < H) {
@@ -86,12 +88,23 @@ rope_append_kernel(__nv_bfloat16 *__restrict__ q, __nv_bfloat16 *__restrict__ id
             dst = page >= 0 ? idx_k_cache + ((size_t)page * kBlock + row) * kDIdx : nullptr;
         }
         if (!dst) continue;
-        const float x0 = __bfloat162float(src[d]), x1 = __bfloat162float(src[d + kPairs]);
-        const float c = s_cos[d], s = s_sin[d];
-        const float y0 = x0 * c - x1 * s;
-        const float y1 = x1 * c + x0 * s;
-        dst[d] = __float2bfloat16_rn(y0);
-        dst[d + kPairs] = __float2bfloat16_rn(y1);
+        const uint4 lo = reinterpret_cast<const uint4 *>(src)[c];
+        const uint4 hi = reinterpret_cast<const uint4 *>(src + kPairs)[c];
+        const __nv_bfloat162 *l2 = reinterpret_cast<const __nv_bfloat162 *>(&lo);
+        const __nv_bfloat162 *h2 = reinterpret_cast<const __nv_bfloat162 *>(&hi);
+        uint4 olo, ohi;
+        __nv_bfloat162 *ol = reinterpret_cast<__nv_bfloat162 *>(&olo);
+        __nv_bfloat162 *oh = reinterpret_cast<__nv_bfloat162 *>(&ohi);
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+            const float2 x0 = __bfloat1622float2(l2[e]), x1 = __bfloat1622float2(h2[e]);
+            const int d = 8 * c + 2 * e;
+            const float c0 = s_cos[d], s0 = s_sin[d], c1 = s_cos[d + 1], s1 = s_sin[d + 1];
+            ol[e] = __floats2bfloat162_rn(x0.x * c0 - x1.x * s0, x0.y * c1 - x1.y * s1);
+            oh[e] = __floats2bfloat162_rn(x1.x * c0 + x0.x * s0, x1.y * c1 + x0.y * s1);
+        }
+        reinterpret_cast<uint4 *>(dst)[c] = olo;
+        reinterpret_cast<uint4 *>(dst + kPairs)[c] = ohi;
     }
     // values are cached as they are
     if (page >= 0) {
