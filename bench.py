@@ -584,7 +584,7 @@ def run_prefill(args):
                           "frac": round(step_bytes / (call_ms / 1e3) / 1e9 / hbm_peak, 4),
                           "bytes_per_step": step_bytes, "flops_per_step": idx_flops + attn_flops},
         "attn_roofline": {"bound": "hbm", "entry": "uocr_sparse_attn_seq: selection check, inversion, "
-                          "tensor-core block kernel, merge (5 kernels)", "achieved": round(attn_gbs, 1),
+                          "tensor-core block kernel, merge (4 kernels)", "achieved": round(attn_gbs, 1),
                           "peak": hbm_peak, "unit": "GB/s", "frac": round(attn_gbs / hbm_peak, 4),
                           "bytes_per_launch": attn_bytes, "avg_launch_ms": round(attn_seq_ms, 5),
                           "selected_blocks": n_sel_blocks},
@@ -592,8 +592,8 @@ def run_prefill(args):
                          "sparse_attn_seq": round(1e3 * attn_seq_ms, 2),
                          "sparse_attn_query_centric": round(1e3 * attn_ms, 2),
                          "prefill_call_graph": round(1e3 * call_ms, 2)},
-        # per call: scoring GEMM, selection, scan, fill, block attention, merge
-        "gpu_launches": args.steps * 6,
+        # per call: scoring GEMM, selection, inversion, block attention, merge
+        "gpu_launches": args.steps * 5,
         "clocks": clk.summary(),
     }
     result["e2e"] = run_prefill_e2e(args, uocr, case, ws, out, sel, stream, world, dev)

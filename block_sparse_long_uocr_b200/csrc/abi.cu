@@ -218,7 +218,7 @@ uocr_status_t uocr_sparse_prefill(const void *q, const void *k_cache, const void
     char *attn_ws = (char *)workspace + w.total;
     uocr::PrefillAttnWs aw;
     uocr::prefill_attn_workspace(n_q, H, max_blocks, &aw);
-    cudaError_t e = cudaMemsetAsync(attn_ws + aw.counts_off, 0, (size_t)max_blocks * sizeof(int32_t), c.stream);
+    cudaError_t e = cudaMemsetAsync(attn_ws, 0, aw.zero_bytes, c.stream);
     if (e != cudaSuccess) return cuda_status(e);
     const int32_t *bt_row = block_table + (size_t)seq * max_blocks;
     e = uocr::launch_prefill_index_gemm(c, idx_q, idx_k_cache, bt_row, seq_lens + seq, q_pos, n_q, max_blocks,
@@ -261,7 +261,7 @@ uocr_status_t uocr_sparse_attn_seq(const void *q, const void *k_cache, const voi
     uocr::PrefillAttnWs aw;
     uocr::prefill_attn_workspace(n_q, H, max_blocks, &aw);
     char *ws = (char *)workspace;
-    cudaError_t e = cudaMemsetAsync(ws + aw.counts_off, 0, (size_t)max_blocks * sizeof(int32_t), c.stream);
+    cudaError_t e = cudaMemsetAsync(ws, 0, aw.zero_bytes, c.stream);
     if (e != cudaSuccess) return cuda_status(e);
     e = uocr::launch_prefill_select_count(c, sel, q_pos, seq_lens + seq, n_q, max_blocks, workspace, dev_err);
     if (e != cudaSuccess) return cuda_status(e);

@@ -40,9 +40,11 @@ cudaError_t launch_prefill_index_gemm(const LaunchCtx &c, const void *idx_q, con
 
 // Block-centric prefill attention (selection inverted per block, tensor-core items of 16
 // entries per (block, head), per-slot partials merged per (query, head)).  Workspace regions,
-// 256-byte aligned.
+// 256-byte aligned.  The first zero_bytes bytes (the per-block selector counts and list
+// counters) must be zero before the call's first kernel.
 struct PrefillAttnWs {
-    size_t counts_off, cursor_off, n_items_off, items_off, list_off, sel_off, ml_off, o_off;
+    size_t counts_off, fill_off, n_items_off, items_off, list_off, sel_off, ml_off, o_off;
+    size_t zero_bytes;
 };
 size_t prefill_attn_workspace(int n_q, int H, int max_blocks, PrefillAttnWs *w);
 // `ws` must start with the per-block selection counts of `sel` (max_blocks int32), as

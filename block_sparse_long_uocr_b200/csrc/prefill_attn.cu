@@ -8,9 +8,9 @@
 // a 2048-query chunk, and ~130 times for the local-window blocks that 32
 // consecutive queries share.  Instead:
 //   1. invert the selection: per logical block, the list of (query, slot)
-//      entries that selected it (the top-k kernel counts them, a one-CTA
-//      exclusive scan places the lists and cuts them into items of 16 entries,
-//      a fill kernel writes them);
+//      entries that selected it (the top-k kernel counts them; one kernel
+//      places the lists by the prefix sums of the counts, writes them and cuts
+//      them into items of 16 entries);
 //   2. one warp per (item, head) computes the item's 16 x 32 score tile
 //      S = Q K^T and, after a register-resident fp32 softmax per row, the
 //      16 x 128 tile P V on the tensor cores (mma.sync m16n8k16, bf16 in, fp32
@@ -49,7 +49,8 @@ namespace uocr {
 
 namespace {
 constexpr int kInvThreads = 256;
-constexpr int kScanThreads = 1024;
+constexpr int kInvPerThread = 8;
+constexpr int kInvTile = kInvThreads * kInvPerThread;   // blocks per prefix-sum tile of the inversion
 constexpr int kMmaWarps = 2;
 constexpr int kItemRows = 16;
 constexpr int kMergeWarps = 8;
@@ -113,75 +114,94 @@ prefill_select_count_kernel(const int32_t *__restrict__ sel, const int32_t *__re
     if (j >= 0) atomicAdd(counts + j, 1);
 }
 
-// One CTA: cursor = exclusive prefix sum of counts (each block's first list position), and the
-// work items:
-// block j with n_j entries gives items (j, 0) .. (j, ceil(n_j / 16) - 1), in block order, each
-// recorded as {j, page of j, first entry, entries (<= 16)} so that a warp needs one load.
-__global__ void __launch_bounds__(kScanThreads)
-prefill_scan_kernel(const int32_t *__restrict__ counts, const int32_t *__restrict__ bt_row, int max_blocks,
-                    int32_t *__restrict__ cursor, int4 *__restrict__ items, int32_t *__restrict__ n_items) {
-    __shared__ int s_tot[2][kScanThreads / 32];
+// The selection inverted in one grid: CTA b places the entries e in [256 b, 256 b + 256) in the
+// per-block lists, grouped by block ({entry = query * 16 + slot, position of the query}), and
+// writes the work items of the blocks j with j % gridDim.x == b: block j with n_j entries gives
+// items (j, 0) .. (j, ceil(n_j / 16) - 1), in block order, each recorded as {j, page of j, first
+// entry, entries (<= 16)} so that a warp needs one load.  Each CTA computes the exclusive prefix
+// sums of counts (each block's first list position and first item) itself, 2048 blocks at a time
+// (8 KiB of counts from L2 per tile); a block's entries take consecutive list positions from a
+// counter per block (fill, zero before the call).
+__global__ void __launch_bounds__(kInvThreads)
+prefill_invert_kernel(const int32_t *counts, const int32_t *__restrict__ bt_row, const int32_t *sel,
+                      const int32_t *__restrict__ q_pos, int n_entries, int max_blocks, int32_t *fill,
+                      int4 *__restrict__ items, int32_t *__restrict__ n_items, int2 *__restrict__ list) {
+    __shared__ int s_c[kInvTile], s_g[kInvTile];   // exclusive prefixes (entries, items) inside the tile
+    __shared__ int s_wc[kInvThreads / 32], s_wg[kInvThreads / 32];
     pdl_wait();
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-    const int per = (max_blocks + kScanThreads - 1) / kScanThreads;
-    const int lo = min(max_blocks, tid * per), hi = min(max_blocks, lo + per);
-    int mine_c = 0, mine_g = 0;
-    for (int j = lo; j < hi; ++j) {
-        const int c = counts[j];
-        mine_c += c;
-        mine_g += (c + kItemRows - 1) / kItemRows;
+    const int e = blockIdx.x * kInvThreads + tid;
+    // this thread's entry, loaded before the scan so that the load overlaps it
+    int j = -1, p = 0;
+    if (e < n_entries) {
+        j = sel[e];
+        if (j >= max_blocks) j = -1;
+        if (j >= 0) p = __ldg(q_pos + e / kSel);
     }
-    int inc_c = mine_c, inc_g = mine_g;
+    int base_c = 0, base_g = 0;   // entries and items of the blocks before the tile
+    for (int t0 = 0; t0 < max_blocks; t0 += kInvTile) {
+        // thread tid sums blocks t0 + 8 tid .. t0 + 8 tid + 7
+        int c[kInvPerThread], sc = 0, sg = 0;
 #pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-        const int nc = __shfl_up_sync(0xffffffffu, inc_c, o);
-        const int ng = __shfl_up_sync(0xffffffffu, inc_g, o);
-        if (lane >= o) {
-            inc_c += nc;
-            inc_g += ng;
+        for (int k = 0; k < kInvPerThread; ++k) {
+            const int jb = t0 + kInvPerThread * tid + k;
+            c[k] = jb < max_blocks ? counts[jb] : 0;
+            sc += c[k];
+            sg += (c[k] + kItemRows - 1) / kItemRows;
         }
-    }
-    if (lane == 31) {
-        s_tot[0][warp] = inc_c;
-        s_tot[1][warp] = inc_g;
-    }
-    __syncthreads();
-    if (warp < 2) {
-        const int w = s_tot[warp][lane];
-        int wi = w;
+        int ic = sc, ig = sg;
 #pragma unroll
         for (int o = 1; o < 32; o <<= 1) {
-            const int n = __shfl_up_sync(0xffffffffu, wi, o);
-            if (lane >= o) wi += n;
+            const int nc = __shfl_up_sync(0xffffffffu, ic, o);
+            const int ng = __shfl_up_sync(0xffffffffu, ig, o);
+            if (lane >= o) {
+                ic += nc;
+                ig += ng;
+            }
         }
-        s_tot[warp][lane] = wi - w;
+        if (lane == 31) {
+            s_wc[warp] = ic;
+            s_wg[warp] = ig;
+        }
+        __syncthreads();
+        int rc = ic - sc, rg = ig - sg, tot_c = 0, tot_g = 0;
+#pragma unroll
+        for (int w = 0; w < kInvThreads / 32; ++w) {
+            if (w < warp) {
+                rc += s_wc[w];
+                rg += s_wg[w];
+            }
+            tot_c += s_wc[w];
+            tot_g += s_wg[w];
+        }
+#pragma unroll
+        for (int k = 0; k < kInvPerThread; ++k) {
+            s_c[kInvPerThread * tid + k] = rc;
+            s_g[kInvPerThread * tid + k] = rg;
+            rc += c[k];
+            rg += (c[k] + kItemRows - 1) / kItemRows;
+        }
+        __syncthreads();
+        if (j >= t0 && j < t0 + kInvTile)
+            list[base_c + s_c[j - t0] + atomicAdd(fill + j, 1)] = make_int2(e, p);
+        // the items of this CTA's blocks in the tile: local index x with (t0 + x) % gridDim.x == b
+        const int len = min(kInvTile, max_blocks - t0);
+        const int G = (int)gridDim.x;
+        const int first = (int)((blockIdx.x + (unsigned)G - (unsigned)(t0 % G)) % (unsigned)G);
+        for (int x = first + tid * G; x < len; x += kInvThreads * G) {
+            const int cnt = (x + 1 < kInvTile ? s_c[x + 1] : tot_c) - s_c[x];
+            if (cnt == 0) continue;
+            const int jb = t0 + x;
+            const int page = __ldg(bt_row + jb);
+            const int g0 = base_g + s_g[x], c0 = base_c + s_c[x];
+            for (int k = 0; k * kItemRows < cnt; ++k)
+                items[g0 + k] = make_int4(jb, page, c0 + k * kItemRows, min(kItemRows, cnt - k * kItemRows));
+        }
+        base_c += tot_c;
+        base_g += tot_g;
+        __syncthreads();   // the next tile reuses s_c, s_g, s_wc, s_wg
     }
-    __syncthreads();
-    int run_c = s_tot[0][warp] + inc_c - mine_c;
-    int run_g = s_tot[1][warp] + inc_g - mine_g;
-    for (int j = lo; j < hi; ++j) {
-        const int c = counts[j];
-        cursor[j] = run_c;
-        const int g = (c + kItemRows - 1) / kItemRows;
-        const int page = g ? __ldg(bt_row + j) : 0;
-        for (int k = 0; k < g; ++k)
-            items[run_g + k] = make_int4(j, page, run_c + k * kItemRows, min(kItemRows, c - k * kItemRows));
-        run_c += c;
-        run_g += g;
-    }
-    if (tid == kScanThreads - 1) *n_items = run_g;
-}
-
-// list[...] = {entry = query * 16 + slot, position of the query}, grouped by block.
-__global__ void __launch_bounds__(kInvThreads)
-prefill_fill_kernel(const int32_t *__restrict__ sel, const int32_t *__restrict__ q_pos, int n_entries,
-                    int max_blocks, int32_t *cursor, int2 *__restrict__ list) {
-    pdl_wait();
-    const int e = blockIdx.x * kInvThreads + threadIdx.x;
-    if (e < n_entries) {
-        const int j = sel[e];
-        if (j >= 0 && j < max_blocks) list[atomicAdd(cursor + j, 1)] = make_int2(e, __ldg(q_pos + e / kSel));
-    }
+    if (blockIdx.x == 0 && tid == 0) *n_items = base_g;
 }
 
 // One unit of work: (item, head) and the item's record and entries.
@@ -452,8 +472,9 @@ size_t prefill_attn_workspace(int n_q, int H, int max_blocks, PrefillAttnWs *w) 
     PrefillAttnWs l{};
     l.counts_off = off;
     off += up((size_t)max_blocks * 4);
-    l.cursor_off = off;
+    l.fill_off = off;
     off += up((size_t)max_blocks * 4);
+    l.zero_bytes = off;
     l.n_items_off = off;
     off += up(4);
     l.items_off = off;
@@ -498,7 +519,7 @@ cudaError_t launch_prefill_attn(const LaunchCtx &c, const void *q, const void *k
     prefill_attn_workspace(n_q, H, max_blocks, &w);
     char *base = (char *)ws;
     const int32_t *counts = (const int32_t *)(base + w.counts_off);
-    int32_t *cursor = (int32_t *)(base + w.cursor_off);
+    int32_t *fill = (int32_t *)(base + w.fill_off);
     int32_t *n_items = (int32_t *)(base + w.n_items_off);
     int4 *items = (int4 *)(base + w.items_off);
     int2 *list = (int2 *)(base + w.list_off);
@@ -514,13 +535,10 @@ cudaError_t launch_prefill_attn(const LaunchCtx &c, const void *q, const void *k
     cfg.attrs = attr;
     cfg.numAttrs = 1;   // every kernel here follows another kernel of the same call
 
-    cfg.gridDim = dim3(1);
-    cfg.blockDim = dim3(kScanThreads);
-    cudaError_t e = cudaLaunchKernelEx(&cfg, prefill_scan_kernel, counts, bt_row, max_blocks, cursor, items, n_items);
-    if (e != cudaSuccess) return e;
     cfg.gridDim = dim3((unsigned)((n_entries + kInvThreads - 1) / kInvThreads));
     cfg.blockDim = dim3(kInvThreads);
-    e = cudaLaunchKernelEx(&cfg, prefill_fill_kernel, sel, q_pos, n_entries, max_blocks, cursor, list);
+    cudaError_t e = cudaLaunchKernelEx(&cfg, prefill_invert_kernel, counts, bt_row, sel, q_pos, n_entries, max_blocks,
+                                       fill, items, n_items, list);
     if (e != cudaSuccess) return e;
 
     int per_sm = 0;

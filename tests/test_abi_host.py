@@ -226,7 +226,7 @@ def test_sparse_attn_seq_workspace_is_a_pure_function_of_shapes(pkg):
     assert f(0, 10, 64) == 0 and f(4, 0, 64) == 0 and f(4, 10, 0) == 0
     a = f(2048, 10, 2048)
     assert a == f(2048, 10, 2048) and a % 256 == 0
-    # the inversion (counts, cursor, items, entries, the checked selection) and the partial states
+    # the inversion (counts, list counters, items, entries, the checked selection) and the partial states
     assert a >= 2048 * 10 * 16 * (128 * 2 + 8) + 2048 * 16 * (8 + 4) + 2 * 2048 * 4
     assert f(2048, 1, 2048) < a and f(4096, 10, 2048) > a
 
