@@ -7,7 +7,7 @@
 // maximum of the walk-through (news.rkmt.cn/news/25027, section 五 step 2):
 //   scores[i][j] = max_{t in block j, t <= p_i} S[i][t].
 //
-// Kernel (persistent, one CTA per SM, 352 threads, warp-specialised).  A CTA
+// Kernel (persistent, one CTA per SM, 384 threads, warp-specialised).  A CTA
 // tile is two 128-query subtiles that share every key tile they load, which
 // halves the key traffic from L2 per FLOP against one subtile per CTA:
 //   warp 8  TMA producer of queries: per work unit the two 128-query A subtiles
@@ -16,9 +16,11 @@
 //           keys (8 boxes of 32 tokens x 64 dims, gathered through the block
 //           table) into a 3-stage ring.  The two producers run ahead of the MMAs
 //           independently, each as far as its ring allows;
-//   warp 9  MMA issuer: allocates 512 TMEM columns (two buffers x two subtiles
-//           of 128 x 128 fp32) and issues 8 tcgen05.mma (M=128, N=128, K=16) per
-//           subtile and tile;
+//   warps 9, 11  MMA issuers, one per subtile: warp 9 allocates 512 TMEM columns
+//           (two buffers x two subtiles of 128 x 128 fp32); each issues 8
+//           tcgen05.mma (M=128, N=128, K=16) per tile into its subtile's
+//           accumulator, so that one thread's barrier waits and commits overlap
+//           the other's MMAs and the tensor pipe does not drain between tiles;
 //   warps 0-7 epilogue: tcgen05.ld of the accumulators (warp w owns rows
 //           32(w%4) .. +31 = its TMEM lane quarter, of subtile w/4, and the
 //           tile's 4 blocks), max over each 32-column block (the causal mask only
@@ -52,9 +54,10 @@ constexpr int kHalfBytesB = kBN * 128;    // one 64-dim half of a B tile: 16 KiB
 constexpr int kBoxBytesB = kBlock * 128;  // one page x 64 dims: 4 KiB
 constexpr int kEpiWarps = 8;             // one warp per (TMEM lane quarter, subtile)
 constexpr int kProducerWarp = 8;          // query (A) tiles
-constexpr int kMmaWarp = 9;
+constexpr int kMmaWarp = 9;               // MMA issuer of subtile 0; allocates the TMEM
 constexpr int kProducerBWarp = 10;        // key (B) tiles
-constexpr int kThreads = 352;
+constexpr int kMmaWarp1 = 11;             // MMA issuer of subtile 1
+constexpr int kThreads = 384;
 constexpr uint64_t kTimeoutNs = 2000000000ull;   // 2 s: far above any legitimate wait
 
 struct __align__(1024) Smem {
@@ -62,8 +65,8 @@ struct __align__(1024) Smem {
     uint8_t b[kStagesB][2][kHalfBytesB];        // 96 KiB
     uint64_t a_full[kStagesA], a_empty[kStagesA];
     uint64_t b_full[kStagesB], b_empty[kStagesB];
-    uint64_t acc_full[2], acc_empty[2];
-    uint64_t mma_done;
+    uint64_t acc_full[2][kMT], acc_empty[2][kMT];   // per accumulator buffer and subtile
+    uint64_t mma_done[kMT];
     uint32_t tmem_base;
     int abort_flag;
 };
@@ -140,17 +143,18 @@ prefill_index_gemm_kernel(const __grid_constant__ CUtensorMap map_q, const __gri
     if (threadIdx.x == 0) {
         for (int k = 0; k < kStagesA; ++k) {
             mbar_init(&s.a_full[k], 1);
-            mbar_init(&s.a_empty[k], 1);
+            mbar_init(&s.a_empty[k], kMT);
         }
         for (int k = 0; k < kStagesB; ++k) {
             mbar_init(&s.b_full[k], 1);
-            mbar_init(&s.b_empty[k], 1);
+            mbar_init(&s.b_empty[k], kMT);
         }
-        for (int k = 0; k < 2; ++k) {
-            mbar_init(&s.acc_full[k], 1);
-            mbar_init(&s.acc_empty[k], kEpiWarps);
-        }
-        mbar_init(&s.mma_done, 1);
+        for (int k = 0; k < 2; ++k)
+            for (int m = 0; m < kMT; ++m) {
+                mbar_init(&s.acc_full[k][m], 1);
+                mbar_init(&s.acc_empty[k][m], kEpiWarps / kMT);
+            }
+        for (int m = 0; m < kMT; ++m) mbar_init(&s.mma_done[m], 1);
         s.abort_flag = 0;
         fence_mbar_init();
     }
@@ -245,11 +249,15 @@ prefill_index_gemm_kernel(const __grid_constant__ CUtensorMap map_q, const __gri
         if (lane == 0)
             for (int k = 0; k < kStagesB; ++k)
                 if (b_fills[k] > 0) mbar_wait_timed(&s.b_full[k], (b_fills[k] - 1) & 1, kTimeoutNs, nullptr);
-    } else if (warp == kMmaWarp) {
-        // ------------------------------------------------------------ MMA issuer
+    } else if (warp == kMmaWarp || warp == kMmaWarp1) {
+        // ------------------------------------------------------------ MMA issuers, one per subtile
+        // Two issuing threads: while one waits on a barrier or commits, the other's MMAs keep
+        // the tensor pipe busy.  Each stage and accumulator is released by both (count kMT).
+        const int m = warp == kMmaWarp ? 0 : 1;
         constexpr uint32_t idesc = tc::idesc_bf16_f32(kBM, kBN);
         static_assert(kTilesPerUnit * kPagesPerTile <= 32, "a unit's page ids fit in one warp");
         static_assert(2 * kMT * kBN == 512, "two accumulator buffers of kMT subtiles fill the 512 TMEM columns");
+        static_assert(kMT == 2, "one issuing warp per subtile");
         int it = 0, uc = 0;
         bool issued = false, stop = false;
         PosPrefetch pf = pos_prefetch(blockIdx.x, n_units, n_chunks, q_pos, n_q, lane);
@@ -260,22 +268,23 @@ prefill_index_gemm_kernel(const __grid_constant__ CUtensorMap map_q, const __gri
             const int sa = uc % kStagesA;
             if (!warp_wait(&s.a_full[sa], (uc / kStagesA) & 1, s, dev_err, lane)) break;
             ++uc;
+            const bool mine = m < w.nsub;   // this subtile holds queries in the unit
             for (int t = 0; t < w.ntiles; ++t, ++it) {
                 const int st = it % kStagesB;
                 const int acc = it & 1;
                 if (!warp_wait(&s.b_full[st], (it / kStagesB) & 1, s, dev_err, lane) ||
-                    !warp_wait(&s.acc_empty[acc], ((it >> 1) & 1) ^ 1, s, dev_err, lane)) {
+                    !warp_wait(&s.acc_empty[acc][m], ((it >> 1) & 1) ^ 1, s, dev_err, lane)) {
                     stop = true;
                     break;
                 }
                 if (lane == 0) {
-                    tc::fence_after_sync();
-                    // k-step k reads 16 bf16 = 32 bytes further into the 128-byte swizzle row:
-                    // 2 more in the descriptor's start-address field (16-byte units; the stage
-                    // addresses stay far below the field's 256 KiB range)
-                    const uint64_t bd0 = tc::smem_desc_k_sw128(smem_addr(s.b[st][0]));
-                    const uint64_t bd1 = tc::smem_desc_k_sw128(smem_addr(s.b[st][1]));
-                    for (int m = 0; m < w.nsub; ++m) {
+                    if (mine) {
+                        tc::fence_after_sync();
+                        // k-step k reads 16 bf16 = 32 bytes further into the 128-byte swizzle row:
+                        // 2 more in the descriptor's start-address field (16-byte units; the stage
+                        // addresses stay far below the field's 256 KiB range)
+                        const uint64_t bd0 = tc::smem_desc_k_sw128(smem_addr(s.b[st][0]));
+                        const uint64_t bd1 = tc::smem_desc_k_sw128(smem_addr(s.b[st][1]));
                         const uint64_t ad0 = tc::smem_desc_k_sw128(smem_addr(s.a[sa][m][0]));
                         const uint64_t ad1 = tc::smem_desc_k_sw128(smem_addr(s.a[sa][m][1]));
                         const uint32_t d = tmem + (uint32_t)((acc * kMT + m) * kBN);
@@ -285,21 +294,30 @@ prefill_index_gemm_kernel(const __grid_constant__ CUtensorMap map_q, const __gri
                             tc::mma_bf16(d, (k < 4 ? ad0 : ad1) + koff, (k < 4 ? bd0 : bd1) + koff, idesc,
                                          k > 0 ? 1u : 0u);
                         }
+                        tc::commit(&s.b_empty[st]);
+                        tc::commit(&s.acc_full[acc][m]);
+                        issued = true;
+                    } else {
+                        // nothing read or written: release at once
+                        mbar_arrive(&s.b_empty[st]);
+                        mbar_arrive(&s.acc_full[acc][m]);
                     }
-                    tc::commit(&s.b_empty[st]);
-                    tc::commit(&s.acc_full[acc]);
                 }
-                issued = true;
                 __syncwarp();
             }
-            if (lane == 0) tc::commit(&s.a_empty[sa]);   // the A tile is free once its MMAs complete
+            if (lane == 0) {   // the A subtile is free once its MMAs complete
+                if (mine)
+                    tc::commit(&s.a_empty[sa]);
+                else
+                    mbar_arrive(&s.a_empty[sa]);
+            }
             __syncwarp();
             if (aborted(s)) break;
         }
         // drain: every MMA this thread issued has completed before TMEM is freed
         if (lane == 0 && issued) {
-            tc::commit(&s.mma_done);
-            mbar_wait_timed(&s.mma_done, 0, kTimeoutNs, nullptr);
+            tc::commit(&s.mma_done[m]);
+            mbar_wait_timed(&s.mma_done[m], 0, kTimeoutNs, nullptr);
         }
         __syncwarp();
     } else {
@@ -336,7 +354,7 @@ prefill_index_gemm_kernel(const __grid_constant__ CUtensorMap map_q, const __gri
             const int pool_page = (lane < w.ntiles * kPagesPerTile && jp < w.nb_max) ? __ldg(bt_row + jp) : -1;
             for (int t = 0; t < w.ntiles; ++t, ++it) {
                 const int acc = it & 1;
-                if (!warp_wait(&s.acc_full[acc], (it >> 1) & 1, s, dev_err, lane)) {
+                if (!warp_wait(&s.acc_full[acc][sub], (it >> 1) & 1, s, dev_err, lane)) {
                     stop = true;
                     break;
                 }
@@ -378,8 +396,7 @@ prefill_index_gemm_kernel(const __grid_constant__ CUtensorMap map_q, const __gri
                 tc::fence_before_sync();
                 __syncwarp();
                 if (lane == 0)
-                    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_addr(&s.acc_empty[acc]))
-                                 : "memory");
+                    mbar_arrive(&s.acc_empty[acc][sub]);
                 if (!have) continue;
                 // a block whose page is not in the pool scores -inf; blocks past the row's
                 // causal range are not written
