@@ -125,6 +125,24 @@ __device__ __forceinline__ bool warp_wait(uint64_t *bar, uint32_t parity, Smem &
     return __shfl_sync(0xffffffffu, ok, 0) != 0;
 }
 
+// Two barriers at once: both probes are issued before either result is used, so their latencies
+// overlap; only a phase that is not complete yet is waited for.
+__device__ __forceinline__ bool warp_wait2(uint64_t *bar0, uint32_t parity0, uint64_t *bar1, uint32_t parity1, Smem &s,
+                                           int32_t *dev_err, int lane) {
+    int ok = 1;
+    if (lane == 0) {
+        const bool r0 = mbar_try_wait(bar0, parity0);
+        const bool r1 = mbar_try_wait(bar1, parity1);
+        ok = (r0 || mbar_wait_timed(bar0, parity0, kTimeoutNs, &s.abort_flag)) &&
+             (r1 || mbar_wait_timed(bar1, parity1, kTimeoutNs, &s.abort_flag));
+        if (!ok) {
+            if (!*(volatile int *)&s.abort_flag) flag_error(dev_err, UOCR_DEVERR_TIMEOUT);
+            atomicExch(&s.abort_flag, 1);
+        }
+    }
+    return __shfl_sync(0xffffffffu, ok, 0) != 0;
+}
+
 __device__ __forceinline__ bool aborted(Smem &s) { return *(volatile int *)&s.abort_flag != 0; }
 
 }  // namespace
@@ -272,8 +290,8 @@ prefill_index_gemm_kernel(const __grid_constant__ CUtensorMap map_q, const __gri
             for (int t = 0; t < w.ntiles; ++t, ++it) {
                 const int st = it % kStagesB;
                 const int acc = it & 1;
-                if (!warp_wait(&s.b_full[st], (it / kStagesB) & 1, s, dev_err, lane) ||
-                    !warp_wait(&s.acc_empty[acc][m], ((it >> 1) & 1) ^ 1, s, dev_err, lane)) {
+                if (!warp_wait2(&s.b_full[st], (it / kStagesB) & 1, &s.acc_empty[acc][m], ((it >> 1) & 1) ^ 1, s,
+                                dev_err, lane)) {
                     stop = true;
                     break;
                 }
@@ -294,13 +312,11 @@ prefill_index_gemm_kernel(const __grid_constant__ CUtensorMap map_q, const __gri
                             tc::mma_bf16(d, (k < 4 ? ad0 : ad1) + koff, (k < 4 ? bd0 : bd1) + koff, idesc,
                                          k > 0 ? 1u : 0u);
                         }
-                        tc::commit(&s.b_empty[st]);
+                        // the epilogue frees the key stage once it sees the accumulator complete
                         tc::commit(&s.acc_full[acc][m]);
                         issued = true;
                     } else {
-                        // nothing read or written: release at once
-                        mbar_arrive(&s.b_empty[st]);
-                        mbar_arrive(&s.acc_full[acc][m]);
+                        mbar_arrive(&s.acc_full[acc][m]);   // nothing written: at once
                     }
                 }
                 __syncwarp();
@@ -358,6 +374,8 @@ prefill_index_gemm_kernel(const __grid_constant__ CUtensorMap map_q, const __gri
                     stop = true;
                     break;
                 }
+                // this subtile's MMAs of the tile are complete: its reads of the key stage are done
+                if (quarter == 0 && lane == 0) mbar_arrive(&s.b_empty[it % kStagesB]);
                 tc::fence_after_sync();
                 const int tile = w.t0 + t;
                 const int j0 = tile * kPagesPerTile;                     // first block of the tile
