@@ -67,6 +67,7 @@ struct __align__(1024) Smem {
     uint64_t b_full[kStagesB], b_empty[kStagesB];
     uint64_t acc_full[2][kMT], acc_empty[2][kMT];   // per accumulator buffer and subtile
     uint64_t mma_done[kMT];
+    int unit_tiles[kStagesA], unit_nsub[kStagesA];   // the unit of each A stage (0 tiles: no more units)
     uint32_t tmem_base;
     int abort_flag;
 };
@@ -83,6 +84,15 @@ struct UnitInfo {
 // two so that a role issues the next unit's position loads (pos_prefetch: predicated loads into
 // registers, nothing consumes them yet) before working on the current unit, and reduces them
 // (unit_info) when it gets there: no role waits on L2 at a unit boundary.
+// A read-only load issued where it stands in the program: the volatile asm keeps the compiler
+// from sinking a prefetch down to its first use (a unit later), which would put the memory
+// latency back on the unit boundary.
+__device__ __forceinline__ int ld_pinned(const int32_t *p) {
+    int v;
+    asm volatile("ld.global.nc.b32 %0, [%1];" : "=r"(v) : "l"(p));
+    return v;
+}
+
 struct PosPrefetch {
     int raw[kBM * kMT / 32];   // position of row m0 + 32k + lane, -1 past the queries
 };
@@ -93,7 +103,7 @@ __device__ __forceinline__ PosPrefetch pos_prefetch(int u, int n_units, int n_ch
 #pragma unroll
     for (int k = 0; k < kBM * kMT / 32; ++k) {
         const int row = m0 + k * 32 + lane;
-        f.raw[k] = (u < n_units && row < n_q) ? __ldg(q_pos + row) : -1;
+        f.raw[k] = (u < n_units && row < n_q) ? ld_pinned(q_pos + row) : -1;
     }
     return f;
 }
@@ -206,6 +216,9 @@ prefill_index_gemm_kernel(const __grid_constant__ CUtensorMap map_q, const __gri
             const int sa = uc % kStagesA;
             if (!warp_wait(&s.a_empty[sa], ((uc / kStagesA) & 1) ^ 1, s, dev_err, lane)) break;
             if (lane == 0) {
+                // the unit's shape travels with its A stage (visible to whoever sees the phase complete)
+                s.unit_tiles[sa] = w.ntiles;
+                s.unit_nsub[sa] = w.nsub;
                 mbar_arrive_expect_tx(&s.a_full[sa], (uint32_t)w.nsub * 2u * a_box_rows * 128u);
                 for (int m = 0; m < w.nsub; ++m) {
                     tc::tma_load_2d(s.a[sa][m][0], &map_q, 0, w.m0 + m * kBM, &s.a_full[sa]);
@@ -216,31 +229,51 @@ prefill_index_gemm_kernel(const __grid_constant__ CUtensorMap map_q, const __gri
             ++uc;
             if (aborted(s)) break;
         }
-        // drain: every buffer this warp filled must have landed before the CTA exits
+        // drain: every buffer this warp filled must have landed before the CTA exits (before the
+        // end marker below completes one more phase of a stage)
         if (lane == 0)
             for (int k = 0; k < kStagesA; ++k)
                 if (a_fills[k] > 0) mbar_wait_timed(&s.a_full[k], (a_fills[k] - 1) & 1, kTimeoutNs, nullptr);
+        __syncwarp();
+        // end marker for the MMA issuers: a stage that holds no unit
+        if (!aborted(s)) {
+            const int sa = uc % kStagesA;
+            if (warp_wait(&s.a_empty[sa], ((uc / kStagesA) & 1) ^ 1, s, dev_err, lane) && lane == 0) {
+                s.unit_tiles[sa] = 0;
+                mbar_arrive(&s.a_full[sa]);
+            }
+        }
     } else if (warp == kProducerBWarp) {
         // ------------------------------------------------------------ TMA producer: key tiles
         int it = 0;
         int b_fills[kStagesB] = {};
         bool stop = false;
+        // a unit's page ids, read a unit ahead (the block table row is read whole, in bounds, before
+        // the unit's causal range is known): lane l < 4 * kTilesPerUnit holds block t0 * 4 + l
+        auto unit_pages = [&](int u) {
+            int pg = -1;
+            if (u < n_units && lane < kTilesPerUnit * kPagesPerTile) {
+                const int j = (u % n_chunks) * kTilesPerUnit * kPagesPerTile + lane;
+                if (j < max_blocks) pg = ld_pinned(bt_row + j);
+            }
+            return pg;
+        };
         PosPrefetch pf = pos_prefetch(blockIdx.x, n_units, n_chunks, q_pos, n_q, lane);
+        int pages_next = unit_pages(blockIdx.x);
         for (int u = blockIdx.x; u < n_units && !stop; u += gridDim.x) {
             const UnitInfo w = unit_info(u, n_chunks, n_q, seq_len_ok, pf);
             pf = pos_prefetch(u + gridDim.x, n_units, n_chunks, q_pos, n_q, lane);
+            int upage = pages_next;
+            pages_next = unit_pages(u + gridDim.x);
             if (w.ntiles == 0) continue;
-            // the unit's page ids at once: lane l < 4 * ntiles holds block t0 * 4 + l
-            int upage = -1;
-            if (lane < w.ntiles * kPagesPerTile) {
-                const int j = w.t0 * kPagesPerTile + lane;
-                if (j < w.nb_max) {
-                    upage = __ldg(bt_row + j);
-                    if ((unsigned)upage >= (unsigned)num_pages) {
-                        flag_error(dev_err, UOCR_DEVERR_PAGE);
-                        upage = -1;
-                    }
+            // keep the blocks of the unit's tiles inside the causal range; flag pages outside the pool
+            if (lane < w.ntiles * kPagesPerTile && w.t0 * kPagesPerTile + lane < w.nb_max) {
+                if ((unsigned)upage >= (unsigned)num_pages) {
+                    flag_error(dev_err, UOCR_DEVERR_PAGE);
+                    upage = -1;
                 }
+            } else {
+                upage = -1;
             }
             for (int t = 0; t < w.ntiles; ++t, ++it) {
                 const int st = it % kStagesB;
@@ -276,18 +309,18 @@ prefill_index_gemm_kernel(const __grid_constant__ CUtensorMap map_q, const __gri
         static_assert(kTilesPerUnit * kPagesPerTile <= 32, "a unit's page ids fit in one warp");
         static_assert(2 * kMT * kBN == 512, "two accumulator buffers of kMT subtiles fill the 512 TMEM columns");
         static_assert(kMT == 2, "one issuing warp per subtile");
+        // the units come from the query producer with their A stages: no unit logic here
         int it = 0, uc = 0;
         bool issued = false, stop = false;
-        PosPrefetch pf = pos_prefetch(blockIdx.x, n_units, n_chunks, q_pos, n_q, lane);
-        for (int u = blockIdx.x; u < n_units && !stop; u += gridDim.x) {
-            const UnitInfo w = unit_info(u, n_chunks, n_q, seq_len_ok, pf);
-            pf = pos_prefetch(u + gridDim.x, n_units, n_chunks, q_pos, n_q, lane);
-            if (w.ntiles == 0) continue;
+        while (!stop) {
             const int sa = uc % kStagesA;
             if (!warp_wait(&s.a_full[sa], (uc / kStagesA) & 1, s, dev_err, lane)) break;
+            const int ntiles = *(volatile int *)&s.unit_tiles[sa];
+            const int nsub = *(volatile int *)&s.unit_nsub[sa];
+            if (ntiles == 0) break;   // end marker
             ++uc;
-            const bool mine = m < w.nsub;   // this subtile holds queries in the unit
-            for (int t = 0; t < w.ntiles; ++t, ++it) {
+            const bool mine = m < nsub;   // this subtile holds queries in the unit
+            for (int t = 0; t < ntiles; ++t, ++it) {
                 const int st = it % kStagesB;
                 const int acc = it & 1;
                 if (!warp_wait2(&s.b_full[st], (it / kStagesB) & 1, &s.acc_empty[acc][m], ((it >> 1) & 1) ^ 1, s,
@@ -346,7 +379,7 @@ prefill_index_gemm_kernel(const __grid_constant__ CUtensorMap map_q, const __gri
         auto next_row_p = [&](int u) {
             if (u >= n_units) return -1;
             const int r = (u / n_chunks) * (kBM * kMT) + sub * kBM + quarter * 32 + lane;
-            return r < n_q ? __ldg(q_pos + r) : -1;
+            return r < n_q ? ld_pinned(q_pos + r) : -1;
         };
         int p_next = next_row_p(blockIdx.x);
         PosPrefetch pf = pos_prefetch(blockIdx.x, n_units, n_chunks, q_pos, n_q, lane);
