@@ -44,12 +44,13 @@ block_topk_kernel(const float *__restrict__ scores, const int32_t *__restrict__ 
     const int tid = threadIdx.x;
     int32_t *out = sel + (size_t)i * kSel;
 
+    // the query's metadata are inputs of the call, not outputs of the preceding kernel
+    QueryRef r;
+    const bool ok = resolve_query(i, seq_lens, q_seq, q_pos, B, max_blocks, dev_err, tid == 0, r, fixed_seq);
     pdl_wait();
     // the attention kernel of a decode call may start its prologue while this runs
     pdl_launch_dependents();
-
-    QueryRef r;
-    if (!resolve_query(i, seq_lens, q_seq, q_pos, B, max_blocks, dev_err, tid == 0, r, fixed_seq)) {
+    if (!ok) {
         if (tid < kSel) out[tid] = -1;
         return;
     }

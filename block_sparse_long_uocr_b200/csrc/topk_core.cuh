@@ -55,8 +55,10 @@ struct KeySource {
     const float *row;
     const uint32_t *mask;   // this sequence's candidate bitmap, or NULL
     __device__ __forceinline__ uint32_t raw(int j) const {
-        if (mask && !((__ldg(mask + (j >> 5)) >> (j & 31)) & 1u)) return 0u;
-        return order_key(__ldcg(row + j));
+        // both loads are issued before either is used
+        const float f = __ldcg(row + j);
+        const bool ok = !mask || ((__ldg(mask + (j >> 5)) >> (j & 31)) & 1u);
+        return ok ? order_key(f) : 0u;
     }
     __device__ __forceinline__ uint32_t operator()(int j) const { return smem ? smem[j] : raw(j); }
 };
@@ -120,6 +122,8 @@ __device__ void topk_two_level(const KeySource &key, int nc, uint64_t *s_cand, u
 }
 
 
+constexpr int kTopkRegKeys = 8;            // rows of at most 8 T candidates keep their keys in registers
+
 template <int T>
 struct TopkShared {
     uint64_t surv[kSurvivorCap];
@@ -157,9 +161,25 @@ __device__ void topk_select(const float *row, int nb, const uint32_t *mask, uint
     __syncthreads();
 
     // ---- 1. stage keys, 2. per-thread then per-group maximum
+    // Rows of at most kTopkRegKeys * T candidates: thread tid holds candidates tid + u T in
+    // registers, all loads issued before any is used; longer rows are staged in shared memory
+    // (or re-read from L2 when they do not fit there).
+    const bool in_regs = nc <= kTopkRegKeys * T;
+    uint32_t kr[kTopkRegKeys];
     uint32_t tmax = 0;
     int allowed = 0;
-    if (s_keys) {
+    if (in_regs) {
+#pragma unroll
+        for (int u = 0; u < kTopkRegKeys; ++u) {
+            const int j = tid + u * T;
+            kr[u] = j < nc ? key.raw(j) : 0u;
+        }
+#pragma unroll
+        for (int u = 0; u < kTopkRegKeys; ++u) {
+            tmax = kr[u] > tmax ? kr[u] : tmax;
+            allowed += kr[u] != 0u;
+        }
+    } else if (s_keys) {
 #pragma unroll 8
         for (int j = tid; j < nc; j += T) {
             const uint32_t k = key.raw(j);
@@ -228,6 +248,24 @@ __device__ void topk_select(const float *row, int nb, const uint32_t *mask, uint
     const uint32_t thr = sm.thr;
 
     // ---- 3. survivors: every candidate at or above the threshold
+    auto append = [&](uint32_t k, int j, bool keep) {
+        const unsigned m = __ballot_sync(0xffffffffu, keep);
+        if (m) {
+            const int leader = __ffs(m) - 1;
+            int base = 0;
+            if (lane == leader) base = atomicAdd(&sm.n, __popc(m));
+            base = __shfl_sync(0xffffffffu, base, leader);
+            const int slot = base + __popc(m & ((1u << lane) - 1u));
+            if (keep && slot < kSurvivorCap) sm.surv[slot] = composite(k, j);
+        }
+    };
+    if (in_regs) {
+#pragma unroll
+        for (int u = 0; u < kTopkRegKeys; ++u) {
+            const int j = tid + u * T;
+            append(kr[u], j, j < nc && kr[u] >= thr);   // the staged path's test
+        }
+    } else {
     for (int j0 = 0; j0 < nc; j0 += T) {
         const int j = j0 + tid;
         const uint32_t k = j < nc ? key(j) : 0u;
@@ -241,6 +279,7 @@ __device__ void topk_select(const float *row, int nb, const uint32_t *mask, uint
             const int slot = base + __popc(m & ((1u << lane) - 1u));
             if (keep && slot < kSurvivorCap) sm.surv[slot] = composite(k, j);
         }
+    }
     }
     __syncthreads();
     const int n = sm.n;
