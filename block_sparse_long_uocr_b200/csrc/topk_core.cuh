@@ -161,21 +161,31 @@ __device__ void topk_select(const float *row, int nb, const uint32_t *mask, uint
     __syncthreads();
 
     // ---- 1. stage keys, 2. per-thread then per-group maximum
-    // Rows of at most kTopkRegKeys * T candidates: thread tid holds candidates tid + u T in
-    // registers, all loads issued before any is used; longer rows are staged in shared memory
-    // (or re-read from L2 when they do not fit there).
+    // Rows of at most kTopkRegKeys * T candidates: thread tid holds the candidates
+    // kTopkRegKeys tid .. + kTopkRegKeys - 1 in registers (two 16-byte loads on an aligned row,
+    // else scalar loads, all issued before any is used; one word of the candidate mask); longer
+    // rows are staged in shared memory (or re-read from L2 when they do not fit there).
+    static_assert(kTopkRegKeys == 8, "a thread's candidates are two float4 and one byte of a mask word");
     const bool in_regs = nc <= kTopkRegKeys * T;
+    const int jr = kTopkRegKeys * tid;   // first candidate of this thread on the register path
     uint32_t kr[kTopkRegKeys];
     uint32_t tmax = 0;
     int allowed = 0;
     if (in_regs) {
+        float f[kTopkRegKeys];
+        if ((reinterpret_cast<uintptr_t>(row) & 15) == 0 && jr + kTopkRegKeys <= nc) {
+            const float4 a = __ldcg(reinterpret_cast<const float4 *>(row + jr));
+            const float4 b = __ldcg(reinterpret_cast<const float4 *>(row + jr) + 1);
+            f[0] = a.x; f[1] = a.y; f[2] = a.z; f[3] = a.w;
+            f[4] = b.x; f[5] = b.y; f[6] = b.z; f[7] = b.w;
+        } else {
 #pragma unroll
-        for (int u = 0; u < kTopkRegKeys; ++u) {
-            const int j = tid + u * T;
-            kr[u] = j < nc ? key.raw(j) : 0u;
+            for (int u = 0; u < kTopkRegKeys; ++u) f[u] = jr + u < nc ? __ldcg(row + jr + u) : 0.f;
         }
+        const uint32_t mbits = mask ? (jr < nc ? __ldg(mask + (jr >> 5)) >> (jr & 31) : 0u) : 0xffu;
 #pragma unroll
         for (int u = 0; u < kTopkRegKeys; ++u) {
+            kr[u] = (jr + u < nc && ((mbits >> u) & 1u)) ? order_key(f[u]) : 0u;
             tmax = kr[u] > tmax ? kr[u] : tmax;
             allowed += kr[u] != 0u;
         }
@@ -260,10 +270,30 @@ __device__ void topk_select(const float *row, int nb, const uint32_t *mask, uint
         }
     };
     if (in_regs) {
+        // this thread's survivors (the staged path's test), placed by one warp prefix sum and
+        // one shared atomic per warp
+        unsigned keep = 0;
 #pragma unroll
-        for (int u = 0; u < kTopkRegKeys; ++u) {
-            const int j = tid + u * T;
-            append(kr[u], j, j < nc && kr[u] >= thr);   // the staged path's test
+        for (int u = 0; u < kTopkRegKeys; ++u)
+            if (jr + u < nc && kr[u] >= thr) keep |= 1u << u;
+        const int cnt = __popc(keep);
+        int incl = cnt;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const int v = __shfl_up_sync(0xffffffffu, incl, o);
+            if (lane >= o) incl += v;
+        }
+        const int wtot = __shfl_sync(0xffffffffu, incl, 31);
+        int base = 0;
+        if (wtot > 0) {
+            if (lane == 31) base = atomicAdd(&sm.n, wtot);
+            base = __shfl_sync(0xffffffffu, base, 31) + incl - cnt;
+#pragma unroll
+            for (int u = 0; u < kTopkRegKeys; ++u)
+                if ((keep >> u) & 1u) {
+                    if (base < kSurvivorCap) sm.surv[base] = composite(kr[u], jr + u);
+                    ++base;
+                }
         }
     } else {
     for (int j0 = 0; j0 < nc; j0 += T) {
@@ -283,7 +313,16 @@ __device__ void topk_select(const float *row, int nb, const uint32_t *mask, uint
     }
     __syncthreads();
     const int n = sm.n;
-    if (n <= kSurvivorCap) {
+    if (n <= 32) {
+        // one survivor per lane of warp 0, ranked by counting over shuffles
+        if (warp == 0) {
+            const uint64_t c = lane < n ? sm.surv[lane] : 0ull;
+            int rank = 0;
+            for (int b = 0; b < n; ++b) rank += __shfl_sync(0xffffffffu, c, b) > c;
+            if (lane < n && rank < kRemote) sm.top[rank] = c;
+        }
+        __syncthreads();
+    } else if (n <= kSurvivorCap) {
         for (int a = tid; a < n; a += T) {
             const uint64_t c = sm.surv[a];
             int rank = 0;
