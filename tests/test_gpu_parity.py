@@ -46,15 +46,21 @@ def test_index_score_matches_oracle_on_ragged_tails(uocr, cuda_device):
         assert torch.isneginf(sc[b, nb:]).all()
 
 
-@pytest.mark.parametrize("kind", ["ties", "normal", "neg"])
-def test_block_topk_is_exact_on_given_scores(uocr, cuda_device, kind):
-    g = torch.Generator().manual_seed({"ties": 1, "normal": 2, "neg": 3}[kind])
+@pytest.mark.parametrize("mb", [4096, 4093, 1021])
+@pytest.mark.parametrize("kind", ["ties", "normal", "neg", "binary"])
+def test_block_topk_is_exact_on_given_scores(uocr, cuda_device, kind, mb):
+    """Few rows: one CTA per row.  Rows of up to 8 x 512 candidates are held in registers (odd
+    row lengths start off a 16-byte boundary: scalar reads); 'normal' leaves a few dozen
+    survivors (ranked by one warp), 'ties' hundreds (ranked by the CTA), 'binary' more than the
+    survivor list holds (exact fallback)."""
+    g = torch.Generator().manual_seed({"ties": 1, "normal": 2, "neg": 3, "binary": 4}[kind] + mb)
     lens = [1, 128, 129, 512, 513, 544, 545, 1000, 32 * 1024, 32 * 4096, 77777]
-    mb = 4096
     if kind == "ties":
         s = torch.randint(-4, 5, (len(lens), mb), generator=g).float()
     elif kind == "normal":
         s = torch.randn(len(lens), mb, generator=g)
+    elif kind == "binary":
+        s = (torch.rand(len(lens), mb, generator=g) < 0.6).float()
     else:
         s = -torch.rand(len(lens), mb, generator=g) - 1.0
     lens = [min(L, mb * 32) for L in lens]
