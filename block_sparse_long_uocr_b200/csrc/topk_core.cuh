@@ -405,15 +405,36 @@ __device__ void topk_warp_select(const float *row, int nb, const uint32_t *mask,
     uint32_t tmax = 0;
     int allowed = 0;
     if (in_regs) {
+        // every load is issued before any is used: the whole quads first, then the mask words
+        // (one branch: the mask pointer is the same for the warp), then the one partial quad
+        float4 v[kRegQuads];
 #pragma unroll
         for (int q = 0; q < kRegQuads; ++q) {
             const int j = 128 * q + 4 * lane;
-            if (j + 3 < nc) {
-                keys4(row, mask, j, kr[q]);
-            } else {
+            v[q] = j + 3 < nc ? __ldcg(reinterpret_cast<const float4 *>(row + j)) : make_float4(0.f, 0.f, 0.f, 0.f);
+        }
+        uint32_t mw[kRegQuads];
+        if (mask) {
 #pragma unroll
-                for (int e = 0; e < 4; ++e) kr[q][e] = j + e < nc ? key(j + e) : 0u;
+            for (int q = 0; q < kRegQuads; ++q) {
+                const int j = 128 * q + 4 * lane;
+                mw[q] = j < nc ? __ldg(mask + (j >> 5)) >> (j & 31) : 0u;
             }
+        } else {
+#pragma unroll
+            for (int q = 0; q < kRegQuads; ++q) mw[q] = 0xfu;
+        }
+#pragma unroll
+        for (int q = 0; q < kRegQuads; ++q) {
+            const int j = 128 * q + 4 * lane;
+            if (j < nc && j + 3 >= nc) {   // the quad that holds the row's end: scalar reads
+                v[q].x = __ldcg(row + j);
+                v[q].y = j + 1 < nc ? __ldcg(row + j + 1) : 0.f;
+                v[q].z = j + 2 < nc ? __ldcg(row + j + 2) : 0.f;
+            }
+            const float f[4] = {v[q].x, v[q].y, v[q].z, v[q].w};
+#pragma unroll
+            for (int e = 0; e < 4; ++e) kr[q][e] = (j + e < nc && ((mw[q] >> e) & 1u)) ? order_key(f[e]) : 0u;
         }
 #pragma unroll
         for (int q = 0; q < kRegQuads; ++q)
