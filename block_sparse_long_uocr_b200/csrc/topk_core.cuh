@@ -161,13 +161,18 @@ __device__ void topk_select(const float *row, int nb, const uint32_t *mask, uint
     __syncthreads();
 
     // ---- 1. stage keys, 2. per-thread then per-group maximum
-    // Rows of at most kTopkRegKeys * T candidates: thread tid holds the candidates
-    // kTopkRegKeys tid .. + kTopkRegKeys - 1 in registers (two 16-byte loads on an aligned row,
-    // else scalar loads, all issued before any is used; one word of the candidate mask); longer
-    // rows are staged in shared memory (or re-read from L2 when they do not fit there).
+    // Rows of at most kTopkRegKeys * T candidates: a thread holds one chunk of kTopkRegKeys
+    // consecutive candidates in registers (two 16-byte loads on an aligned row, else scalar
+    // loads, all issued before any is used; one byte of a word of the candidate mask).  Chunk k
+    // goes to thread (k % 16) * kGroup + k / 16, so that consecutive chunks fall in different
+    // groups and every group holds candidates whenever the row has 16 chunks: a short row packed
+    // into the first groups would leave the other group maxima at 0, the threshold at 0 and
+    // every candidate a survivor.  Longer rows are staged in shared memory (or re-read from L2
+    // when they do not fit there).
     static_assert(kTopkRegKeys == 8, "a thread's candidates are two float4 and one byte of a mask word");
     const bool in_regs = nc <= kTopkRegKeys * T;
-    const int jr = kTopkRegKeys * tid;   // first candidate of this thread on the register path
+    // first candidate of this thread's chunk on the register path
+    const int jr = kTopkRegKeys * ((tid % kGroup) * kTopkGroups + tid / kGroup);
     uint32_t kr[kTopkRegKeys];
     uint32_t tmax = 0;
     int allowed = 0;
