@@ -33,7 +33,8 @@ __device__ __forceinline__ void count_selected(const int32_t *out, int slot, int
     if (v >= 0) atomicAdd(counts + v, 1);
 }
 
-__global__ void __launch_bounds__(kTopkThreads)
+// (512, 1): without the block count ptxas fits 4 CTAs per SM in 32 registers and spills
+__global__ void __launch_bounds__(kTopkThreads, 1)
 block_topk_kernel(const float *__restrict__ scores, const int32_t *__restrict__ seq_lens,
                   const int32_t *__restrict__ q_seq, const int32_t *__restrict__ q_pos, int B,
                   int max_blocks, int32_t *__restrict__ sel, int32_t *dev_err, int staged, int fixed_seq,
