@@ -35,6 +35,7 @@ def _prefill_case(total, n_new, extra_pos=(), seed=0, shuffle=True, device="cpu"
     (4096 + 17, 300, (0, 1, 4000)),                # 3 M tiles (ragged), 17 N tiles (ragged)
     (2048, 128, ()),                               # exactly one M tile
     (2048, 129, ()),                               # one query over
+    (32768 + 5, 1100, ()),                         # 325 work units: 3 on some CTAs (the A ring wraps)
 ])
 def test_prefill_scores_match_oracle(uocr, cuda_device, total, n_new, extra):
     case = _prefill_case(total, n_new, extra, seed=total + n_new, device=cuda_device, heads=1)
