@@ -6,11 +6,11 @@
 // uses a hard top-k.  Ranking: score descending, then lower block id.
 //
 // Few rows (decode): one CTA of 512 threads per query runs topk_select
-// (topk_core.cuh): scores staged in shared memory, a threshold from 16 warp
-// maxima, survivors ranked by counting, an exact two-level fallback for heavily
-// tied rows, and an optional page-aware candidate bitmap (section 五
-// image_bucket_constraint).  Rows longer than the shared-memory budget are read
-// from L2 instead of staged.  Many rows (a prefill chunk): one warp per query
+// (topk_core.cuh): keys in registers (rows of up to 4096 candidates) or staged
+// in shared memory, a threshold from 16 warp maxima, survivors ranked by
+// counting, an exact two-level fallback for heavily tied rows, and an optional
+// page-aware candidate bitmap (section 五 image_bucket_constraint).  Rows longer
+// than the shared-memory budget are read from L2 instead of staged.  Many rows (a prefill chunk): one warp per query
 // runs topk_warp_select, the same steps at warp scope, so that every row is in
 // flight at once.  Either kernel can also count, per block, the queries that
 // selected it (the first step of the block-centric prefill attention).

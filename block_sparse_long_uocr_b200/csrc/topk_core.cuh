@@ -8,8 +8,9 @@
 // Every candidate's ranking key is the 64-bit composite
 // (order-preserving fp32 key << 32 | ~id): distinct, larger for a higher score
 // and, among equal scores, for the lower id.
-//   1. The candidates' scores are read once from L2 into shared memory as
-//      order-preserving keys (masked-out candidates get key 0).
+//   1. The candidates' scores are read once from L2 as order-preserving keys
+//      (masked-out candidates get key 0): into registers for rows of up to
+//      8 T candidates, else into shared memory.
 //   2. Threshold: the 12th largest of 16 group maxima (groups of T/16
 //      threads).  Those 12 maxima are 12 distinct candidates at or above it, so
 //      every member of the top 12 is at or above it too.
