@@ -15,14 +15,14 @@
 //      S = Q K^T and, after a register-resident fp32 softmax per row, the
 //      16 x 128 tile P V on the tensor cores (mma.sync m16n8k16, bf16 in, fp32
 //      accumulate), writing each entry's partial state: the row maximum m and
-//      the weight sum l in fp32, and the normalised output o = acc / l in bf16
-//      (the split-KV partial layout of FlashInfer's merge: the partial output
-//      in the output dtype, the softmax statistics in fp32; o is a convex
-//      combination of the values, so its rounding adds at most 2^-9 max|v| to
-//      the result, the size of the output's own bf16 rounding, and halves the
+//      the weight sum l in fp32, and the unnormalised output acc = sum_t
+//      2^(z_t - m) v_t in bf16 (the partial output in the output dtype, the
+//      softmax statistics in fp32; |acc| <= l max|v|, so its rounding adds at
+//      most 2^-9 max|v| to the result after the merge divides by the summed
+//      weights, the size of the output's own bf16 rounding, and halves the
 //      partials' traffic);
-//   3. one warp per (query, head) merges the 16 partials, weight l 2^(m - M)
-//      each, and writes the bf16 output.
+//   3. one warp per (query, head) merges the 16 partials: out = sum_k
+//      2^(m_k - M) acc_k / sum_k 2^(m_k - M) l_k, written in bf16.
 // Each (block, head) tile is read from memory once per chunk (an item after the
 // first of the same tile finds it in L2).
 //
@@ -330,16 +330,30 @@ prefill_block_mma_kernel(const uint4 *__restrict__ q, const uint4 *__restrict__ 
         const int pa = cur.ea.y, pb = cur.eb.y;
         const int t0 = cur.j * kBlock + 2 * t;
         float ma = -INFINITY, mb = -INFINITY, la = 0.f, lb = 0.f;
+        // a block wholly at or before every row's position (every remote block) needs no mask
+        const bool visible = cur.j * kBlock + kBlock - 1 <= __reduce_min_sync(0xffffffffu, min(pa, pb));
+        if (visible) {
 #pragma unroll
-        for (int nt = 0; nt < 4; ++nt)
+            for (int nt = 0; nt < 4; ++nt)
 #pragma unroll
-            for (int e = 0; e < 2; ++e) {
-                const int tok = t0 + 8 * nt + e;
-                s[nt][e] = tok <= pa ? s[nt][e] * scale_log2 : -INFINITY;
-                s[nt][2 + e] = tok <= pb ? s[nt][2 + e] * scale_log2 : -INFINITY;
-                ma = fmaxf(ma, s[nt][e]);
-                mb = fmaxf(mb, s[nt][2 + e]);
-            }
+                for (int e = 0; e < 2; ++e) {
+                    s[nt][e] *= scale_log2;
+                    s[nt][2 + e] *= scale_log2;
+                    ma = fmaxf(ma, s[nt][e]);
+                    mb = fmaxf(mb, s[nt][2 + e]);
+                }
+        } else {
+#pragma unroll
+            for (int nt = 0; nt < 4; ++nt)
+#pragma unroll
+                for (int e = 0; e < 2; ++e) {
+                    const int tok = t0 + 8 * nt + e;
+                    s[nt][e] = tok <= pa ? s[nt][e] * scale_log2 : -INFINITY;
+                    s[nt][2 + e] = tok <= pb ? s[nt][2 + e] * scale_log2 : -INFINITY;
+                    ma = fmaxf(ma, s[nt][e]);
+                    mb = fmaxf(mb, s[nt][2 + e]);
+                }
+        }
 #pragma unroll
         for (int x = 1; x < 4; x <<= 1) {
             ma = fmaxf(ma, __shfl_xor_sync(0xffffffffu, ma, x));
@@ -389,22 +403,22 @@ prefill_block_mma_kernel(const uint4 *__restrict__ q, const uint4 *__restrict__ 
             for (int n = 0; n < 16; ++n) o[n][0] = o[n][1] = o[n][2] = o[n][3] = 0.f;
         }
         const int ia = cur.ea.x >> 4, ib = cur.eb.x >> 4;
+        // the partial is stored unnormalised (sum of weight x value); the merge divides by the sum
+        // of the weights
         if (r < cur.rows) {
             const size_t slot = ((size_t)ia * H + cur.h) * kSel + (cur.ea.x & 15);
-            const float inv = la > 0.f ? 1.f / la : 0.f;
             uint32_t *dst = reinterpret_cast<uint32_t *>(part_o + slot * kD) + t;
             float unused = 0.f;
 #pragma unroll
-            for (int n = 0; n < 16; ++n) dst[4 * n] = pack_bf16(o[n][0] * inv, o[n][1] * inv, unused);
+            for (int n = 0; n < 16; ++n) dst[4 * n] = pack_bf16(o[n][0], o[n][1], unused);
             if (t == 0) *reinterpret_cast<float2 *>(part_ml + slot * 2) = make_float2(ma, la);
         }
         if (r + 8 < cur.rows) {
             const size_t slot = ((size_t)ib * H + cur.h) * kSel + (cur.eb.x & 15);
-            const float inv = lb > 0.f ? 1.f / lb : 0.f;
             uint32_t *dst = reinterpret_cast<uint32_t *>(part_o + slot * kD) + t;
             float unused = 0.f;
 #pragma unroll
-            for (int n = 0; n < 16; ++n) dst[4 * n] = pack_bf16(o[n][2] * inv, o[n][3] * inv, unused);
+            for (int n = 0; n < 16; ++n) dst[4 * n] = pack_bf16(o[n][2], o[n][3], unused);
             if (t == 0) *reinterpret_cast<float2 *>(part_ml + slot * 2) = make_float2(mb, lb);
         }
         cur = nxt;
@@ -436,8 +450,9 @@ prefill_merge_kernel(const int32_t *__restrict__ sel, const __nv_bfloat16 *__res
     float M = m;
 #pragma unroll
     for (int x = 8; x > 0; x >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, x));
-    const float w = M == -INFINITY ? 0.f : l * exp2f(m - M);
-    float W = w;
+    // partial k holds sum_t 2^(z_t - m_k) v_t and l_k = sum_t 2^(z_t - m_k): rescale both to M
+    const float w = M == -INFINITY ? 0.f : exp2f(m - M);
+    float W = l * w;
 #pragma unroll
     for (int x = 8; x > 0; x >>= 1) W += __shfl_xor_sync(0xffffffffu, W, x);
     float A[4] = {0.f, 0.f, 0.f, 0.f};
