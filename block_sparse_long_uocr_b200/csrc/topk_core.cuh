@@ -29,10 +29,12 @@ namespace uocr {
 constexpr int kSurvivorCap = 2048;          // survivor list capacity (16 KiB)
 constexpr int kTopkGroups = 16;             // threshold from 16 group maxima (>= kRemote)
 
-// Larger key <=> larger float; -0 and +0 map to the same key (they compare equal).
+// Larger key <=> larger float; -0 and +0 map to the same key (they compare equal): adding +0
+// turns -0 into +0 (round to nearest), then negative floats have all bits flipped and
+// non-negative ones the sign bit set.
 __device__ __forceinline__ uint32_t order_key(float f) {
-    const uint32_t u = (f == 0.0f) ? 0u : __float_as_uint(f);
-    return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+    const uint32_t u = __float_as_uint(f + 0.0f);
+    return u ^ ((uint32_t)((int32_t)u >> 31) | 0x80000000u);
 }
 
 __device__ __forceinline__ uint64_t composite(uint32_t key, int j) {
