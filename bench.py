@@ -605,41 +605,116 @@ def run_prefill(args):
         print(json.dumps(result), flush=True)
 
 
-def run_prefill_e2e(args, uocr, case, ws, out, sel, stream, world, dev):
-    """Same metric through sparse_prefill, end to end: every step copies the chunk's queries,
-    indexer queries and positions from pinned host memory in one transfer, runs the call, and
-    copies the output and the selection back in one transfer, inside the timed region.  The
-    caches stay resident (the sequence's state; the chunk's own keys are already appended)."""
-    inputs = [case.q, case.idx_q, case.q_pos]
-    h_in, h_views = _packed(inputs, "cpu", pin=True)
-    for hv, t in zip(h_views, inputs):
+def _serial_e2e(args, inputs, results, run_step, stream, dev):
+    """Time `steps` end-to-end steps on one stream: copy every input from pinned host memory (one
+    transfer), run `run_step`, copy every result back to pinned host memory (one transfer), step
+    after step.  Returns device ms."""
+    h_in, h_in_views = _packed(inputs, "cpu", pin=True)
+    for hv, t in zip(h_in_views, inputs):
         hv.copy_(t.cpu())
-    d_in, (d_q, d_qi, d_pos) = _packed(inputs, dev)
-    results = [out, sel]
-    d_out, (o_view, s_view) = _packed(results, dev)
+    d_in, d_in_views = _packed(inputs, dev)
+    d_out, d_out_views = _packed(results, dev)
     h_out, _ = _packed(results, "cpu", pin=True)
 
     def step():
         d_in.copy_(h_in, non_blocking=True)
-        uocr.sparse_prefill(d_q, case.k_pool, case.v_pool, d_qi, case.idx_k_pool, case.block_table, case.seq_lens,
-                            0, d_pos, out=o_view, sel=s_view, workspace=ws, stream=stream)
+        run_step(d_in_views, d_out_views)
         h_out.copy_(d_out, non_blocking=True)
+
+    for _ in range(max(1, args.warmup)):
+        step()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(max(1, args.steps)):
+        step()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    return e0.elapsed_time(e1)
+
+
+def _e2e(args, inputs, results, run_step, stream, dev, units_per_step, world):
+    """Both ways of running end-to-end steps, each with every step's copies inside the timed
+    region: serial (one stream) and pipelined (copies of neighbouring steps overlap the compute).
+    Pipelining hides the copies of long steps; a step of a few microseconds is bound by the host
+    issuing three streams' work, where the serial loop is faster.  The faster mode is the reported
+    value; the other is kept beside it."""
+    steps = max(1, args.steps)
+    res = {}
+    for mode, fn in (("serial", _serial_e2e), ("pipelined", _pipelined_e2e)):
+        ms = udist.max_over_ranks(fn(args, inputs, results, run_step, stream, dev), dev)
+        res[mode] = {"value": round(world * units_per_step * steps / (ms / 1e3), 1), "ms_per_step": round(ms / steps, 4)}
+    best = max(res, key=lambda m: res[m]["value"])
+    other = "serial" if best == "pipelined" else "pipelined"
+    return {"value": res[best]["value"], "unit": UNIT,
+            "h2d_bytes_per_step": sum(t.numel() * t.element_size() for t in inputs),
+            "d2h_bytes_per_step": sum(t.numel() * t.element_size() for t in results),
+            "ms_per_step": res[best]["ms_per_step"], "copies_per_step": 2, "mode": best, other: res[other]}
+
+
+def _pipelined_e2e(args, inputs, results, run_step, stream, dev):
+    """Time `steps` end-to-end steps: step k copies every input from pinned host memory (one
+    transfer), runs `run_step` on the device copy and copies every result back to pinned host
+    memory (one transfer).  Device inputs and results are double-buffered and the two copies run
+    on their own streams, so step k + 1's inputs travel while step k computes and step k's results
+    travel while step k + 1 computes, as in a serving loop; every copy of every step is inside the
+    timed region (from the first input copy to the last result copy).  Returns device ms."""
+    h_in, h_in_views = _packed(inputs, "cpu", pin=True)
+    for hv, t in zip(h_in_views, inputs):
+        hv.copy_(t.cpu())
+    d_in = [_packed(inputs, dev) for _ in range(2)]
+    d_out = [_packed(results, dev) for _ in range(2)]
+    h_out = [_packed(results, "cpu", pin=True)[0] for _ in range(2)]
+    h2d, d2h = torch.cuda.Stream(dev), torch.cuda.Stream(dev)
+    ev = {name: [torch.cuda.Event() for _ in range(2)] for name in ("in", "comp", "out")}
+    k = [0]
+
+    def step():
+        b, reuse = k[0] % 2, k[0] >= 2
+        with torch.cuda.stream(h2d):
+            if reuse:
+                h2d.wait_event(ev["comp"][b])          # step k - 2 has read this input buffer
+            d_in[b][0].copy_(h_in, non_blocking=True)
+            ev["in"][b].record(h2d)
+        stream.wait_event(ev["in"][b])
+        if reuse:
+            stream.wait_event(ev["out"][b])            # step k - 2's results have left this buffer
+        run_step(d_in[b][1], d_out[b][1])
+        ev["comp"][b].record(stream)
+        with torch.cuda.stream(d2h):
+            d2h.wait_event(ev["comp"][b])
+            h_out[b].copy_(d_out[b][0], non_blocking=True)
+            ev["out"][b].record(d2h)
+        k[0] += 1
 
     for _ in range(max(1, args.warmup)):
         step()
     torch.cuda.synchronize()
     steps = max(1, args.steps)
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    e0.record(stream)
+    e0.record(h2d)
     for _ in range(steps):
         step()
-    e1.record(stream)
+    e1.record(d2h)
     torch.cuda.synchronize()
-    ms = udist.max_over_ranks(e0.elapsed_time(e1), dev)
-    return {"value": round(world * case.n_q * steps / (ms / 1e3), 1), "unit": UNIT,
-            "h2d_bytes_per_step": sum(t.numel() * t.element_size() for t in inputs),
-            "d2h_bytes_per_step": sum(t.numel() * t.element_size() for t in results),
-            "ms_per_step": round(ms / steps, 4), "copies_per_step": 2}
+    return e0.elapsed_time(e1)
+
+
+def run_prefill_e2e(args, uocr, case, ws, out, sel, stream, world, dev):
+    """Same metric through sparse_prefill, end to end: every step copies the chunk's queries,
+    indexer queries and positions from pinned host memory in one transfer, runs the call, and
+    copies the output and the selection back in one transfer, inside the timed region (serial or
+    pipelined across steps, see _e2e).  The caches stay resident (the sequence's state; the
+    chunk's own keys are already appended)."""
+    inputs = [case.q, case.idx_q, case.q_pos]
+    results = [out, sel]
+
+    def run_step(din, dout):
+        d_q, d_qi, d_pos = din
+        uocr.sparse_prefill(d_q, case.k_pool, case.v_pool, d_qi, case.idx_k_pool, case.block_table, case.seq_lens,
+                            0, d_pos, out=dout[0], sel=dout[1], workspace=ws, stream=stream)
+
+    return _e2e(args, inputs, results, run_step, stream, dev, case.n_q, world)
 
 
 def _packed(tensors, device, pin=False):
@@ -659,44 +734,21 @@ def run_e2e(args, uocr, case, ws, outs, sels, stream, world, dev):
     """Same metric through sparse_decode, end to end: every step copies its inputs (the block table,
     the lengths and every layer's query and indexer query) from pinned host memory in one transfer,
     runs the 12 layer calls, and copies every layer's output and selection back in one transfer,
-    all inside the timed region.  The KV / indexer caches stay resident (the decode state)."""
+    all inside the timed region (serial or pipelined across steps, see _e2e).  The KV / indexer
+    caches stay resident (the decode state)."""
     n_layers = len(case.layers)
     inputs = [case.block_table, case.seq_lens] + [case.q_layers[l][0] for l in range(n_layers)] + \
              [case.q_layers[l][1] for l in range(n_layers)]
-    h_in, h_views = _packed(inputs, "cpu", pin=True)
-    for hv, t in zip(h_views, inputs):
-        hv.copy_(t.cpu())
-    d_in, d_views = _packed(inputs, dev)
-    d_bt, d_sl = d_views[0], d_views[1]
-    d_q, d_qi = d_views[2: 2 + n_layers], d_views[2 + n_layers:]
     results = list(outs) + list(sels)
-    d_out, d_out_views = _packed(results, dev)
-    h_out, _ = _packed(results, "cpu", pin=True)
-    o_views, s_views = d_out_views[:n_layers], d_out_views[n_layers:]
 
-    def step():
-        d_in.copy_(h_in, non_blocking=True)
+    def run_step(din, dout):
+        d_bt, d_sl = din[0], din[1]
         for l in range(n_layers):
             kp, vp, ikp = case.layers[l]
-            uocr.sparse_decode(d_q[l], kp, vp, d_qi[l], ikp, d_bt, d_sl, out=o_views[l], sel=s_views[l],
-                               workspace=ws, stream=stream)
-        h_out.copy_(d_out, non_blocking=True)
+            uocr.sparse_decode(din[2 + l], kp, vp, din[2 + n_layers + l], ikp, d_bt, d_sl, out=dout[l],
+                               sel=dout[n_layers + l], workspace=ws, stream=stream)
 
-    for _ in range(max(1, args.warmup)):
-        step()
-    torch.cuda.synchronize()
-    steps = max(1, args.steps)
-    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    e0.record(stream)
-    for _ in range(steps):
-        step()
-    e1.record(stream)
-    torch.cuda.synchronize()
-    ms = udist.max_over_ranks(e0.elapsed_time(e1), dev)
-    value = world * case.n_q * n_layers * steps / (ms / 1e3)
-    return {"value": round(value, 1), "unit": UNIT, "h2d_bytes_per_step": sum(t.numel() * t.element_size() for t in inputs),
-            "d2h_bytes_per_step": sum(t.numel() * t.element_size() for t in results),
-            "ms_per_step": round(ms / steps, 4), "copies_per_step": 2}
+    return _e2e(args, inputs, results, run_step, stream, dev, case.n_q * n_layers, world)
 
 
 # --------------------------------------------------------------------------- oracle timing
