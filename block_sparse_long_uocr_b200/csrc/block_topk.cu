@@ -24,7 +24,7 @@ namespace uocr {
 
 constexpr int kTopkThreads = 512;
 constexpr int kTopkSmemKeys = 48 * 1024;    // stage rows up to 48K candidates (192 KiB of keys)
-constexpr int kTopkWarpRows = 8;            // queries (warps) per CTA of the warp-per-row kernel
+constexpr int kTopkWarpRows = 14;           // queries (warps) per CTA of the warp-per-row kernel: 2048 rows fill 147 SMs evenly
 constexpr int kWarpRowsFrom = 512;          // use the warp-per-row kernel from this many queries
 
 // counts[v] += 1 for every selected block v of one query's 16 slots (lanes 0..15 of the caller).
