@@ -226,7 +226,7 @@ uocr_status_t uocr_sparse_attn_seq(const void *q, const void *k_cache, const voi
  * The attention is block-centric: the selection is inverted per block, every
  * selected (block, head) K/V tile is read once for all the queries that chose
  * it, and each (query, slot, head) partial -- the row maximum and weight sum in
- * fp32, the normalised partial output in bf16 -- is merged per (query, head);
+ * fp32, the unnormalised partial output in bf16 -- is merged per (query, head);
  * the bf16 partial adds at most 2^-9 max|v| to an output, the size of the
  * output's own bf16 rounding.  Workspace: uocr_prefill_workspace_bytes(n_q, H,
  * max_blocks) bytes, 256-byte aligned (the block scores first, then the
