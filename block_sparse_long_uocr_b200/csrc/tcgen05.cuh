@@ -1,6 +1,6 @@
 // tcgen05.cuh -- thin inline-PTX wrappers for the sm_100a tensor-core path:
 // TMEM allocation, tcgen05.mma (kind::f16, one CTA), commit to an mbarrier,
-// TMEM loads, and 2-D TMA tile loads (no cluster multicast).
+// TMEM loads, and plain 2-D TMA tile loads into this CTA's shared memory.
 #pragma once
 
 #include <cuda.h>
@@ -87,7 +87,7 @@ __device__ __forceinline__ void tmem_ld_32x32b_x32(uint32_t taddr, float (&v)[32
 }
 __device__ __forceinline__ void tmem_ld_wait() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
 
-// ---- 2-D TMA tile load into shared memory, completing bytes on `bar` (no multicast).
+// ---- 2-D TMA tile load into this CTA's shared memory, completing bytes on `bar`.
 // x (innermost coordinate) must be a multiple of 16 bytes / element size.
 __device__ __forceinline__ void tma_load_2d(void *dst, const CUtensorMap *map, int x, int y, uint64_t *bar) {
     asm volatile(
