@@ -51,6 +51,8 @@ namespace {
 constexpr int kInvThreads = 256;
 constexpr int kInvPerThread = 8;
 constexpr int kInvTile = kInvThreads * kInvPerThread;   // blocks per prefix-sum tile of the inversion
+constexpr int kInvEntries = 4;   // selection entries per thread of the inversion (each CTA recomputes
+                                 // the prefix sums, so fewer CTAs re-read fewer counts)
 constexpr int kMmaWarps = 2;
 constexpr int kItemRows = 16;
 constexpr int kMergeWarps = 8;
@@ -114,7 +116,7 @@ prefill_select_count_kernel(const int32_t *__restrict__ sel, const int32_t *__re
     if (j >= 0) atomicAdd(counts + j, 1);
 }
 
-// The selection inverted in one grid: CTA b places the entries e in [256 b, 256 b + 256) in the
+// The selection inverted in one grid: CTA b places the entries e in [1024 b, 1024 b + 1024) in the
 // per-block lists, grouped by block ({entry = query * 16 + slot, position of the query}), and
 // writes the work items of the blocks j with j % gridDim.x == b: block j with n_j entries gives
 // items (j, 0) .. (j, ceil(n_j / 16) - 1), in block order, each recorded as {j, page of j, first
@@ -130,13 +132,19 @@ prefill_invert_kernel(const int32_t *counts, const int32_t *__restrict__ bt_row,
     __shared__ int s_wc[kInvThreads / 32], s_wg[kInvThreads / 32];
     pdl_wait();
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-    const int e = blockIdx.x * kInvThreads + tid;
-    // this thread's entry, loaded before the scan so that the load overlaps it
-    int j = -1, p = 0;
-    if (e < n_entries) {
-        j = sel[e];
-        if (j >= max_blocks) j = -1;
-        if (j >= 0) p = __ldg(q_pos + e / kSel);
+    // this thread's entries (kInvEntries, kInvThreads apart), loaded before the scan so that the
+    // loads overlap it
+    int ej[kInvEntries], ep[kInvEntries];
+#pragma unroll
+    for (int k = 0; k < kInvEntries; ++k) {
+        const int e = (blockIdx.x * kInvEntries + k) * kInvThreads + tid;
+        ej[k] = -1;
+        ep[k] = 0;
+        if (e < n_entries) {
+            ej[k] = sel[e];
+            if (ej[k] >= max_blocks) ej[k] = -1;
+            if (ej[k] >= 0) ep[k] = __ldg(q_pos + e / kSel);
+        }
     }
     int base_c = 0, base_g = 0;   // entries and items of the blocks before the tile
     for (int t0 = 0; t0 < max_blocks; t0 += kInvTile) {
@@ -182,8 +190,13 @@ prefill_invert_kernel(const int32_t *counts, const int32_t *__restrict__ bt_row,
             rg += (c[k] + kItemRows - 1) / kItemRows;
         }
         __syncthreads();
-        if (j >= t0 && j < t0 + kInvTile)
-            list[base_c + s_c[j - t0] + atomicAdd(fill + j, 1)] = make_int2(e, p);
+#pragma unroll
+        for (int k = 0; k < kInvEntries; ++k) {
+            const int j = ej[k];
+            if (j >= t0 && j < t0 + kInvTile)
+                list[base_c + s_c[j - t0] + atomicAdd(fill + j, 1)] =
+                    make_int2((blockIdx.x * kInvEntries + k) * kInvThreads + tid, ep[k]);
+        }
         // the items of this CTA's blocks in the tile: local index x with (t0 + x) % gridDim.x == b
         const int len = min(kInvTile, max_blocks - t0);
         const int G = (int)gridDim.x;
@@ -550,7 +563,7 @@ cudaError_t launch_prefill_attn(const LaunchCtx &c, const void *q, const void *k
     cfg.attrs = attr;
     cfg.numAttrs = 1;   // every kernel here follows another kernel of the same call
 
-    cfg.gridDim = dim3((unsigned)((n_entries + kInvThreads - 1) / kInvThreads));
+    cfg.gridDim = dim3((unsigned)((n_entries + kInvThreads * kInvEntries - 1) / (kInvThreads * kInvEntries)));
     cfg.blockDim = dim3(kInvThreads);
     cudaError_t e = cudaLaunchKernelEx(&cfg, prefill_invert_kernel, counts, bt_row, sel, q_pos, n_entries, max_blocks,
                                        fill, items, n_items, list);
