@@ -186,7 +186,7 @@ uocr_status_t uocr_prefill_index_score(const void *idx_q, const void *idx_k_cach
     if ((st = make_ctx(stream, false, c)) != UOCR_OK) return st;
     return cuda_status(uocr::launch_prefill_index_gemm(c, idx_q, idx_k_cache, block_table + (size_t)seq * max_blocks,
                                                        seq_lens + seq, q_pos, n_q, max_blocks, num_pages, scores,
-                                                       dev_err));
+                                                       nullptr, dev_err));
 }
 
 size_t uocr_prefill_workspace_bytes(int n_q, int H, int max_blocks) {
@@ -222,7 +222,7 @@ uocr_status_t uocr_sparse_prefill(const void *q, const void *k_cache, const void
     if (e != cudaSuccess) return cuda_status(e);
     const int32_t *bt_row = block_table + (size_t)seq * max_blocks;
     e = uocr::launch_prefill_index_gemm(c, idx_q, idx_k_cache, bt_row, seq_lens + seq, q_pos, n_q, max_blocks,
-                                        num_pages, scores, dev_err);
+                                        num_pages, scores, (int32_t *)(attn_ws + aw.sched_off), dev_err);
     if (e != cudaSuccess) return cuda_status(e);
     c.pdl = true;
     e = uocr::launch_block_topk(c, scores, seq_lens, nullptr, q_pos, n_q, B, max_blocks, sel_out, dev_err, seq,

@@ -33,17 +33,19 @@ cudaError_t launch_sparse_attn(const LaunchCtx &c, const void *q, const void *k,
                                bool implicit_local, int fixed_seq, bool head_major, int32_t *dev_err);
 
 // tcgen05 block scoring of n_q queries of one sequence (block table row bt_row,
-// length *seq_len_ptr) into scores [n_q][max_blocks].
+// length *seq_len_ptr) into scores [n_q][max_blocks].  sched: a zeroed int32 work-unit counter
+// for this launch alone (CTAs take units as they go), or NULL for a round-robin split.
 cudaError_t launch_prefill_index_gemm(const LaunchCtx &c, const void *idx_q, const void *idx_k,
                                       const int32_t *bt_row, const int32_t *seq_len_ptr, const int32_t *q_pos,
-                                      int n_q, int max_blocks, int num_pages, float *scores, int32_t *dev_err);
+                                      int n_q, int max_blocks, int num_pages, float *scores, int32_t *sched,
+                                      int32_t *dev_err);
 
 // Block-centric prefill attention (selection inverted per block, tensor-core items of 16
 // entries per (block, head), per-slot partials merged per (query, head)).  Workspace regions,
 // 256-byte aligned.  The first zero_bytes bytes (the per-block selector counts and list
 // counters) must be zero before the call's first kernel.
 struct PrefillAttnWs {
-    size_t counts_off, fill_off, n_items_off, items_off, list_off, sel_off, ml_off, o_off;
+    size_t counts_off, fill_off, sched_off, n_items_off, items_off, list_off, sel_off, ml_off, o_off;
     size_t zero_bytes;
 };
 size_t prefill_attn_workspace(int n_q, int H, int max_blocks, PrefillAttnWs *w);

@@ -502,6 +502,8 @@ size_t prefill_attn_workspace(int n_q, int H, int max_blocks, PrefillAttnWs *w) 
     off += up((size_t)max_blocks * 4);
     l.fill_off = off;
     off += up((size_t)max_blocks * 4);
+    l.sched_off = off;   // the scoring GEMM's work-unit counter
+    off += up(4);
     l.zero_bytes = off;
     l.n_items_off = off;
     off += up(4);

@@ -27,7 +27,9 @@
 //           on blocks that reach past the row's position), fp32 scores to global
 //           memory, four at a time.
 // Work unit = (256-query tile, chunk of 4 N tiles); units whose tokens all lie
-// past the tile's last query are skipped.  Every mbarrier wait is bounded in
+// past the tile's last query are skipped.  The query producer picks the CTA's
+// units (from a per-launch queue when one is given, else round-robin) and
+// publishes each with its A stage -- shape, page ids -- for every other role.  Every mbarrier wait is bounded in
 // wall time: on timeout the CTA reports UOCR_DEVERR_TIMEOUT, every role stops
 // issuing, waits (bounded) for what it issued, and the TMEM is freed.
 #include <cuda.h>
@@ -67,7 +69,13 @@ struct __align__(1024) Smem {
     uint64_t b_full[kStagesB], b_empty[kStagesB];
     uint64_t acc_full[2][kMT], acc_empty[2][kMT];   // per accumulator buffer and subtile
     uint64_t mma_done[kMT];
-    int unit_tiles[kStagesA], unit_nsub[kStagesA];   // the unit of each A stage (0 tiles: no more units)
+    // The work unit of each A stage, written by the query producer before it arrives on desc_full
+    // and read by every other role (0 tiles: no more units); the stage is rewritten only after the
+    // two MMA issuers, the key producer and the 8 epilogue warps have released it (a_empty).
+    uint64_t desc_full[kStagesA];
+    int unit_u[kStagesA], unit_tiles[kStagesA], unit_nsub[kStagesA];
+    int unit_pages[kStagesA][kTilesPerUnit * kPagesPerTile];   // -1: not loaded (outside the pool or
+                                                               // past the unit's causal range)
     uint32_t tmem_base;
     int abort_flag;
 };
@@ -162,7 +170,7 @@ prefill_index_gemm_kernel(const __grid_constant__ CUtensorMap map_q, const __gri
                           const int32_t *__restrict__ bt_row, const int32_t *__restrict__ seq_len_ptr,
                           const int32_t *__restrict__ q_pos, int n_q, int a_box_rows, int num_pages,
                           int max_blocks, int n_chunks, int n_units, float *__restrict__ scores,
-                          int32_t *dev_err) {
+                          int32_t *sched, int32_t *dev_err) {
     extern __shared__ uint8_t smem_raw[];
     Smem &s = *reinterpret_cast<Smem *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     const int warp = threadIdx.x >> 5;
@@ -171,7 +179,8 @@ prefill_index_gemm_kernel(const __grid_constant__ CUtensorMap map_q, const __gri
     if (threadIdx.x == 0) {
         for (int k = 0; k < kStagesA; ++k) {
             mbar_init(&s.a_full[k], 1);
-            mbar_init(&s.a_empty[k], kMT);
+            mbar_init(&s.a_empty[k], kMT + 1 + kEpiWarps);
+            mbar_init(&s.desc_full[k], 1);
         }
         for (int k = 0; k < kStagesB; ++k) {
             mbar_init(&s.b_full[k], 1);
@@ -206,19 +215,61 @@ prefill_index_gemm_kernel(const __grid_constant__ CUtensorMap map_q, const __gri
 
     if (warp == kProducerWarp) {
         // ------------------------------------------------------------ TMA producer: query tiles
+        // It picks the CTA's work units -- from the launch's queue when `sched` is given (a CTA that
+        // runs faster takes more units), else round-robin -- one unit ahead, so that the next
+        // unit's positions and page ids are in flight while the current one is published.
         int uc = 0;
         int a_fills[kStagesA] = {};
-        PosPrefetch pf = pos_prefetch(blockIdx.x, n_units, n_chunks, q_pos, n_q, lane);
-        for (int u = blockIdx.x; u < n_units; u += gridDim.x) {
+        auto pick = [&](int prev) {
+            if (!sched) return prev < 0 ? (int)blockIdx.x : prev + (int)gridDim.x;
+            int v = 0;
+            if (lane == 0) v = atomicAdd(sched, 1);
+            return __shfl_sync(0xffffffffu, v, 0);
+        };
+        // a unit's page ids (the block table row is read in bounds before the unit's causal range
+        // is known): lane l < 4 * kTilesPerUnit holds block t0 * 4 + l
+        auto unit_pages = [&](int u) {
+            int pg = -1;
+            if (u < n_units && lane < kTilesPerUnit * kPagesPerTile) {
+                const int j = (u % n_chunks) * kTilesPerUnit * kPagesPerTile + lane;
+                if (j < max_blocks) pg = ld_pinned(bt_row + j);
+            }
+            return pg;
+        };
+        int u = pick(-1);
+        PosPrefetch pf = pos_prefetch(u, n_units, n_chunks, q_pos, n_q, lane);
+        int pages_pf = unit_pages(u);
+        int u_next = u < n_units ? pick(u) : n_units;
+        while (u < n_units) {
             const UnitInfo w = unit_info(u, n_chunks, n_q, seq_len_ok, pf);
-            pf = pos_prefetch(u + gridDim.x, n_units, n_chunks, q_pos, n_q, lane);
+            int upage = pages_pf;
+            const int u_cur = u;
+            pf = pos_prefetch(u_next, n_units, n_chunks, q_pos, n_q, lane);
+            pages_pf = unit_pages(u_next);
+            u = u_next;
+            u_next = u < n_units ? pick(u) : n_units;
             if (w.ntiles == 0) continue;
+            // keep the blocks of the unit's tiles inside the causal range; flag pages outside the pool
+            if (lane < w.ntiles * kPagesPerTile && w.t0 * kPagesPerTile + lane < w.nb_max) {
+                if ((unsigned)upage >= (unsigned)num_pages) {
+                    flag_error(dev_err, UOCR_DEVERR_PAGE);
+                    upage = -1;
+                }
+            } else {
+                upage = -1;
+            }
             const int sa = uc % kStagesA;
             if (!warp_wait(&s.a_empty[sa], ((uc / kStagesA) & 1) ^ 1, s, dev_err, lane)) break;
+            if (lane < kTilesPerUnit * kPagesPerTile) s.unit_pages[sa][lane] = upage;
             if (lane == 0) {
-                // the unit's shape travels with its A stage (visible to whoever sees the phase complete)
+                s.unit_u[sa] = u_cur;
                 s.unit_tiles[sa] = w.ntiles;
                 s.unit_nsub[sa] = w.nsub;
+            }
+            __syncwarp();
+            if (lane == 0) {
+                // the descriptor is visible to whoever sees either phase complete
+                mbar_arrive(&s.desc_full[sa]);
                 mbar_arrive_expect_tx(&s.a_full[sa], (uint32_t)w.nsub * 2u * a_box_rows * 128u);
                 for (int m = 0; m < w.nsub; ++m) {
                     tc::tma_load_2d(s.a[sa][m][0], &map_q, 0, w.m0 + m * kBM, &s.a_full[sa]);
@@ -235,47 +286,31 @@ prefill_index_gemm_kernel(const __grid_constant__ CUtensorMap map_q, const __gri
             for (int k = 0; k < kStagesA; ++k)
                 if (a_fills[k] > 0) mbar_wait_timed(&s.a_full[k], (a_fills[k] - 1) & 1, kTimeoutNs, nullptr);
         __syncwarp();
-        // end marker for the MMA issuers: a stage that holds no unit
+        // end marker for every other role: a stage that holds no unit
         if (!aborted(s)) {
             const int sa = uc % kStagesA;
             if (warp_wait(&s.a_empty[sa], ((uc / kStagesA) & 1) ^ 1, s, dev_err, lane) && lane == 0) {
                 s.unit_tiles[sa] = 0;
+                mbar_arrive(&s.desc_full[sa]);
                 mbar_arrive(&s.a_full[sa]);
             }
         }
     } else if (warp == kProducerBWarp) {
         // ------------------------------------------------------------ TMA producer: key tiles
-        int it = 0;
+        int it = 0, uc = 0;
         int b_fills[kStagesB] = {};
         bool stop = false;
-        // a unit's page ids, read a unit ahead (the block table row is read whole, in bounds, before
-        // the unit's causal range is known): lane l < 4 * kTilesPerUnit holds block t0 * 4 + l
-        auto unit_pages = [&](int u) {
-            int pg = -1;
-            if (u < n_units && lane < kTilesPerUnit * kPagesPerTile) {
-                const int j = (u % n_chunks) * kTilesPerUnit * kPagesPerTile + lane;
-                if (j < max_blocks) pg = ld_pinned(bt_row + j);
-            }
-            return pg;
-        };
-        PosPrefetch pf = pos_prefetch(blockIdx.x, n_units, n_chunks, q_pos, n_q, lane);
-        int pages_next = unit_pages(blockIdx.x);
-        for (int u = blockIdx.x; u < n_units && !stop; u += gridDim.x) {
-            const UnitInfo w = unit_info(u, n_chunks, n_q, seq_len_ok, pf);
-            pf = pos_prefetch(u + gridDim.x, n_units, n_chunks, q_pos, n_q, lane);
-            int upage = pages_next;
-            pages_next = unit_pages(u + gridDim.x);
-            if (w.ntiles == 0) continue;
-            // keep the blocks of the unit's tiles inside the causal range; flag pages outside the pool
-            if (lane < w.ntiles * kPagesPerTile && w.t0 * kPagesPerTile + lane < w.nb_max) {
-                if ((unsigned)upage >= (unsigned)num_pages) {
-                    flag_error(dev_err, UOCR_DEVERR_PAGE);
-                    upage = -1;
-                }
-            } else {
-                upage = -1;
-            }
-            for (int t = 0; t < w.ntiles; ++t, ++it) {
+        while (!stop) {
+            const int sa = uc % kStagesA;
+            if (!warp_wait(&s.desc_full[sa], (uc / kStagesA) & 1, s, dev_err, lane)) break;
+            const int ntiles = *(volatile int *)&s.unit_tiles[sa];
+            if (ntiles == 0) break;   // end marker
+            // lane l < 4 * kTilesPerUnit: block t0 * 4 + l
+            const int upage = lane < kTilesPerUnit * kPagesPerTile ? *(volatile int *)&s.unit_pages[sa][lane] : -1;
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&s.a_empty[sa]);   // descriptor read
+            ++uc;
+            for (int t = 0; t < ntiles; ++t, ++it) {
                 const int st = it % kStagesB;
                 int page = __shfl_sync(0xffffffffu, upage, t * kPagesPerTile + (lane & (kPagesPerTile - 1)));
                 if (lane >= kPagesPerTile) page = -1;   // lanes 0..3 issue the tile's pages
@@ -373,35 +408,30 @@ prefill_index_gemm_kernel(const __grid_constant__ CUtensorMap map_q, const __gri
         // ------------------------------------------------------------ epilogue, warps 0..7
         const int quarter = warp & 3;            // TMEM lane quarter = rows 32q .. 32q+31 of a subtile
         const int sub = warp >> 2;               // subtile
-        int it = 0;
+        int it = 0, uc = 0;
         bool stop = false;
-        // this thread's row position in unit u (raw, -1 past the queries), fetched a unit ahead
-        auto next_row_p = [&](int u) {
-            if (u >= n_units) return -1;
-            const int r = (u / n_chunks) * (kBM * kMT) + sub * kBM + quarter * 32 + lane;
-            return r < n_q ? ld_pinned(q_pos + r) : -1;
-        };
-        int p_next = next_row_p(blockIdx.x);
-        PosPrefetch pf = pos_prefetch(blockIdx.x, n_units, n_chunks, q_pos, n_q, lane);
-        for (int u = blockIdx.x; u < n_units && !stop; u += gridDim.x) {
-            const UnitInfo w = unit_info(u, n_chunks, n_q, seq_len_ok, pf);
-            pf = pos_prefetch(u + gridDim.x, n_units, n_chunks, q_pos, n_q, lane);
-            if (w.ntiles == 0) {
-                p_next = next_row_p(u + gridDim.x);
-                continue;
-            }
-            const int row = w.m0 + sub * kBM + quarter * 32 + lane;
-            const int p_raw = p_next;
-            p_next = next_row_p(u + gridDim.x);
-            if (row < n_q && p_raw >= seq_len && w.t0 == 0) flag_error(dev_err, UOCR_DEVERR_POS);
+        while (!stop) {
+            const int sa = uc % kStagesA;
+            if (!warp_wait(&s.desc_full[sa], (uc / kStagesA) & 1, s, dev_err, lane)) break;
+            const int ntiles = *(volatile int *)&s.unit_tiles[sa];
+            if (ntiles == 0) break;   // end marker
+            const int u = *(volatile int *)&s.unit_u[sa];
+            const int nsub = *(volatile int *)&s.unit_nsub[sa];
+            // which of the unit's blocks have a page in the pool and in the causal range (bit 4t + k)
+            const unsigned pool_mask = __ballot_sync(
+                0xffffffffu, lane < kTilesPerUnit * kPagesPerTile && *(volatile int *)&s.unit_pages[sa][lane] >= 0);
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&s.a_empty[sa]);   // descriptor read
+            ++uc;
+            const int m0 = (u / n_chunks) * (kBM * kMT), t0u = (u % n_chunks) * kTilesPerUnit;
+            const int row = m0 + sub * kBM + quarter * 32 + lane;
+            // the row's position: its load overlaps the wait for the unit's first accumulator
+            const int p_raw = row < n_q ? __ldg(q_pos + row) : -1;
+            if (row < n_q && p_raw >= seq_len && t0u == 0) flag_error(dev_err, UOCR_DEVERR_POS);
             const int p = (row < n_q && p_raw < seq_len_ok) ? p_raw : -1;
             const int nb_row = p < 0 ? 0 : p / kBlock + 1;
             float *srow = scores + (size_t)(row < n_q ? row : 0) * max_blocks;
-            // which of the unit's blocks have a page in the pool (bit 4t + k), read once per unit
-            // and gathered after the first tile's math, so no tile waits on a block-table load
-            const int jp = w.t0 * kPagesPerTile + lane;
-            const int pool_page = (lane < w.ntiles * kPagesPerTile && jp < w.nb_max) ? __ldg(bt_row + jp) : -1;
-            for (int t = 0; t < w.ntiles; ++t, ++it) {
+            for (int t = 0; t < ntiles; ++t, ++it) {
                 const int acc = it & 1;
                 if (!warp_wait(&s.acc_full[acc][sub], (it >> 1) & 1, s, dev_err, lane)) {
                     stop = true;
@@ -410,14 +440,14 @@ prefill_index_gemm_kernel(const __grid_constant__ CUtensorMap map_q, const __gri
                 // this subtile's MMAs of the tile are complete: its reads of the key stage are done
                 if (quarter == 0 && lane == 0) mbar_arrive(&s.b_empty[it % kStagesB]);
                 tc::fence_after_sync();
-                const int tile = w.t0 + t;
+                const int tile = t0u + t;
                 const int j0 = tile * kPagesPerTile;                     // first block of the tile
                 const bool interior = (j0 + 4) * kBlock - 1 <= p;        // no masking needed
                 float best[4];
                 const uint32_t tbase =
                     tmem + ((uint32_t)(quarter * 32) << 16) + (uint32_t)((acc * kMT + sub) * kBN);
                 // a subtile past the last query holds no accumulator: read nothing, write nothing
-                const bool have = sub < w.nsub;
+                const bool have = sub < nsub;
                 if (have) {
                     // the tile's 4 blocks in one TMEM round trip (4 x 32 columns in flight)
                     float v[4][32];
@@ -451,7 +481,6 @@ prefill_index_gemm_kernel(const __grid_constant__ CUtensorMap map_q, const __gri
                 if (!have) continue;
                 // a block whose page is not in the pool scores -inf; blocks past the row's
                 // causal range are not written
-                const unsigned pool_mask = __ballot_sync(0xffffffffu, (unsigned)pool_page < (unsigned)num_pages);
 #pragma unroll
                 for (int k = 0; k < 4; ++k)
                     if (!((pool_mask >> (t * kPagesPerTile + k)) & 1u)) best[k] = -INFINITY;
@@ -509,7 +538,8 @@ size_t prefill_index_gemm_smem() { return sizeof(Smem) + 1024; }
 
 cudaError_t launch_prefill_index_gemm(const LaunchCtx &c, const void *idx_q, const void *idx_k,
                                       const int32_t *bt_row, const int32_t *seq_len_ptr, const int32_t *q_pos,
-                                      int n_q, int max_blocks, int num_pages, float *scores, int32_t *dev_err) {
+                                      int n_q, int max_blocks, int num_pages, float *scores, int32_t *sched,
+                                      int32_t *dev_err) {
     const int a_box_rows = n_q < kBM ? n_q : kBM;
     CUtensorMap map_q, map_k;
     if (!make_map(&map_q, idx_q, (uint64_t)n_q, (uint32_t)a_box_rows)) return cudaErrorInvalidValue;
@@ -535,7 +565,7 @@ cudaError_t launch_prefill_index_gemm(const LaunchCtx &c, const void *idx_q, con
     cfg.attrs = attr;
     cfg.numAttrs = c.pdl ? 1 : 0;
     return cudaLaunchKernelEx(&cfg, prefill_index_gemm_kernel, map_q, map_k, bt_row, seq_len_ptr, q_pos, n_q,
-                              a_box_rows, num_pages, max_blocks, n_chunks, (int)units, scores, dev_err);
+                              a_box_rows, num_pages, max_blocks, n_chunks, (int)units, scores, sched, dev_err);
 }
 
 }  // namespace uocr
