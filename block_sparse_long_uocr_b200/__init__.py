@@ -15,6 +15,8 @@ Entry points (same names as the C ABI, without the ``uocr_`` prefix):
 * :func:`sparse_decode` -- the three fused into one decode call;
 * :func:`prefill_index_score` -- the block scores of a prefill chunk on the tcgen05 tensor cores;
 * :func:`sparse_prefill` -- tensor-core scoring, selection and attention for a prefill chunk;
+* :func:`sparse_attn_seq` -- the block-centric attention of many queries of one sequence over a
+  caller's selection (the attention stage of :func:`sparse_prefill`);
 * :func:`summary_score`, :func:`block_summary_mean`, :func:`sparse_decode_summary` -- block-summary
   scoring (one vector per block) and the decode step built on it;
 * :func:`block_topk_masked` -- selection under a page-aware candidate bitmap;
