@@ -12,8 +12,8 @@
 // builds the simplest untrained one, the mean of the page's 32 indexer keys.
 //
 // Scan layout: a half-warp per page (16 lanes x 16 bytes = one summary), 8 fp32
-// FMAs per lane and a 4-shuffle reduction; the grid is flat over (query, chunk
-// of pages) like the token scan.
+// FMAs per lane and a 4-shuffle reduction, 8 pages per half-warp in flight; the
+// grid is flat over (query, chunk of pages) like the token scan.
 #include <cuda_bf16.h>
 #include <math.h>
 
@@ -24,6 +24,7 @@ namespace uocr {
 
 namespace {
 constexpr int kSumWarps = 8;
+constexpr int kSumBatch = 8;   // pages per half-warp whose loads are in flight together
 }  // namespace
 
 __global__ void __launch_bounds__(kSumWarps * 32)
@@ -45,22 +46,40 @@ summary_scan_kernel(const uint4 *__restrict__ idx_q, const uint4 *__restrict__ s
     const int32_t *bt_row = bt + (size_t)r.b * max_blocks;
     float *srow = scores + (size_t)i * max_blocks;
     const int jend = min(r.nb, j0 + pages_per_cta);
-    for (int j = j0 + warp * 2 + half; j < jend; j += kSumWarps * 2) {
-        const int page = __ldg(bt_row + j);
-        float a = 0.f;
-        const bool ok = (unsigned)page < (unsigned)num_pages;
-        if (ok) {
+    // A half-warp's pages are jw + half, + 16, ..., kSumBatch at a time: all block-table loads
+    // issued, then all summary loads, then the math, so that the two dependent round trips are
+    // paid once per batch instead of once per page.  The loop bound is the warp's (the same for
+    // both half-warps).
+    for (int jw = j0 + warp * 2; jw < jend; jw += kSumBatch * kSumWarps * 2) {
+        const int jb = jw + half;
+        int page[kSumBatch];
+#pragma unroll
+        for (int k = 0; k < kSumBatch; ++k) {
+            const int j = jb + k * kSumWarps * 2;
+            page[k] = j < jend ? __ldg(bt_row + j) : -1;
+        }
+        uint4 v[kSumBatch];
+#pragma unroll
+        for (int k = 0; k < kSumBatch; ++k)
+            v[k] = (unsigned)page[k] < (unsigned)num_pages ? ld_stream(summary + (size_t)page[k] * (kDIdx / 8) + hl)
+                                                          : make_uint4(0u, 0u, 0u, 0u);
+#pragma unroll
+        for (int k = 0; k < kSumBatch; ++k) {
+            const int j = jb + k * kSumWarps * 2;
             float kf[8];
-            bf16x8_to_f32(ld_stream(summary + (size_t)page * (kDIdx / 8) + hl), kf);
-            a = qf[0] * kf[0];
+            bf16x8_to_f32(v[k], kf);
+            float a = qf[0] * kf[0];
 #pragma unroll
             for (int c = 1; c < 8; ++c) a = fmaf(qf[c], kf[c], a);
-        }
+            // both half-warps run the same iterations (j past jend only idles), so the whole warp
+            // takes part in every shuffle
 #pragma unroll
-        for (int o = 8; o > 0; o >>= 1) a += __shfl_xor_sync(__activemask(), a, o);
-        if (hl == 0) {
-            if (!ok) flag_error(dev_err, UOCR_DEVERR_PAGE);
-            srow[j] = ok ? a : -INFINITY;
+            for (int o = 8; o > 0; o >>= 1) a += __shfl_xor_sync(0xffffffffu, a, o);
+            if (hl == 0 && j < jend) {
+                const bool ok = (unsigned)page[k] < (unsigned)num_pages;
+                if (!ok) flag_error(dev_err, UOCR_DEVERR_PAGE);
+                srow[j] = ok ? a : -INFINITY;
+            }
         }
     }
     pdl_launch_dependents();
