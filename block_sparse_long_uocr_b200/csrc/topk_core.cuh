@@ -197,21 +197,24 @@ __device__ void topk_select(const float *row, int nb, const uint32_t *mask, uint
             tmax = kr[u] > tmax ? kr[u] : tmax;
             allowed += kr[u] != 0u;
         }
-    } else if (s_keys) {
-#pragma unroll 8
-        for (int j = tid; j < nc; j += T) {
-            const uint32_t k = key.raw(j);
-            s_keys[j] = k;
-            tmax = k > tmax ? k : tmax;
-            allowed += k != 0u;
-        }
-        key.smem = s_keys;
     } else {
-        for (int j = tid; j < nc; j += T) {
-            const uint32_t k = key(j);
-            tmax = k > tmax ? k : tmax;
-            allowed += k != 0u;
+        // batches of kTopkRegKeys loads per thread, all issued before any is used
+        for (int jb = 0; jb < nc; jb += kTopkRegKeys * T) {
+            uint32_t kk[kTopkRegKeys];
+#pragma unroll
+            for (int u = 0; u < kTopkRegKeys; ++u) {
+                const int j = jb + u * T + tid;
+                kk[u] = j < nc ? key.raw(j) : 0u;
+            }
+#pragma unroll
+            for (int u = 0; u < kTopkRegKeys; ++u) {
+                const int j = jb + u * T + tid;
+                if (j < nc && s_keys) s_keys[j] = kk[u];
+                tmax = kk[u] > tmax ? kk[u] : tmax;
+                allowed += kk[u] != 0u;
+            }
         }
+        if (s_keys) key.smem = s_keys;
     }
     uint32_t gm = tmax;
     if (kGroup == 32) {
