@@ -12,7 +12,7 @@
 //   * 8 fp32 FMAs per load against the lane's 8 query dims (kept in registers);
 //   * a 15-shuffle transposed reduction leaves each lane with one full token
 //     dot product, then a 5-shuffle warp max gives the block score;
-//   * loads bypass L1 allocation; 16 warps per SM keep ~128 KiB in flight.
+//   * loads bypass L1 allocation; 32 warps per SM (4 CTAs of 8) keep the HBM busy.
 // The grid is flat over (query, chunk of pages); chunks past a query's causal
 // blocks exit at once, so ragged batches need no host-side work list.
 
@@ -27,7 +27,8 @@ namespace uocr {
 
 constexpr int kScanWarps = 8;
 
-__global__ void __launch_bounds__(kScanWarps * 32, 2)
+// (256, 4): 64 registers, 4 CTAs x 8 warps per SM (2 CTAs at 96 registers and 5 at 48 are slower)
+__global__ void __launch_bounds__(kScanWarps * 32, 4)
 index_scan_kernel(const uint4 *__restrict__ idx_q, const uint4 *__restrict__ idx_k,
                   const int32_t *__restrict__ bt, const int32_t *__restrict__ seq_lens,
                   const int32_t *__restrict__ q_seq, const int32_t *__restrict__ q_pos, int B,
@@ -59,9 +60,9 @@ cudaError_t launch_index_scan(const LaunchCtx &c, const void *idx_q, const void 
                               const int32_t *bt, const int32_t *seq_lens, const int32_t *q_seq,
                               const int32_t *q_pos, int n_q, int B, int max_blocks, int num_pages,
                               float *scores, int32_t *dev_err) {
-    // Pages per warp: enough CTAs for ~8 waves of 2 CTAs per SM, at most 8 pages per warp.
+    // Pages per warp: enough CTAs for ~16 waves of 4 CTAs per SM, at most 8 pages per warp.
     const long long total_pages = (long long)n_q * max_blocks;
-    const long long target_ctas = 16LL * c.num_sms * 2;
+    const long long target_ctas = 16LL * c.num_sms * 4;
     long long ppw = total_pages / (target_ctas * kScanWarps);
     if (ppw < 1) ppw = 1;
     if (ppw > 8) ppw = 8;
