@@ -60,6 +60,33 @@ constexpr int kMergeWarps = 8;
 __device__ __forceinline__ void cp_async16(uint32_t dst, const void *src) {
     asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst), "l"(src) : "memory");
 }
+// L2 eviction policies (PTX createpolicy): the K/V tiles stream through L2 once per chunk and go
+// first; the partials, which the merge kernel of the same call reads back, stay.
+__device__ __forceinline__ uint64_t l2_evict_first() {
+    uint64_t p;
+    asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(p));
+    return p;
+}
+__device__ __forceinline__ uint64_t l2_evict_last() {
+    uint64_t p;
+    asm volatile("createpolicy.fractional.L2::evict_last.b64 %0, 1.0;" : "=l"(p));
+    return p;
+}
+__device__ __forceinline__ void cp_async16_pol(uint32_t dst, const void *src, uint64_t pol) {
+    asm volatile("cp.async.cg.shared.global.L2::cache_hint [%0], [%1], 16, %2;" ::"r"(dst), "l"(src), "l"(pol)
+                 : "memory");
+}
+__device__ __forceinline__ void st_u32_pol(uint32_t *p, uint32_t v, uint64_t pol) {
+    asm volatile("st.global.L2::cache_hint.b32 [%0], %1, %2;" ::"l"(p), "r"(v), "l"(pol) : "memory");
+}
+__device__ __forceinline__ void st_f2_pol(float *p, float a, float b, uint64_t pol) {
+    asm volatile("st.global.L2::cache_hint.v2.f32 [%0], {%1, %2}, %3;" ::"l"(p), "f"(a), "f"(b), "l"(pol)
+                 : "memory");
+}
+// Drops a 128-byte line from L2 without writing it back (its contents become undefined).
+__device__ __forceinline__ void l2_discard_line(const void *p) {
+    asm volatile("discard.global.L2 [%0], 128;" ::"l"(p) : "memory");
+}
 __device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
 __device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_group 0;" ::: "memory"); }
 __device__ __forceinline__ void cp_async_wait_1() { asm volatile("cp.async.wait_group 1;" ::: "memory"); }
@@ -269,6 +296,7 @@ prefill_block_mma_kernel(const uint4 *__restrict__ q, const uint4 *__restrict__ 
     const uint32_t sk = smem_addr(stage[warp].k), sv = smem_addr(stage[warp].v), sq = smem_addr(stage[warp].q);
     const uint4 *k_s = stage[warp].k, *q_s = stage[warp].q;
 
+    const uint64_t pol_kv = l2_evict_first(), pol_part = l2_evict_last();
     pdl_wait();
     const int n_work = __ldg(n_items) * H;
     const int stride = gridDim.x * kMmaWarps;
@@ -291,7 +319,7 @@ prefill_block_mma_kernel(const uint4 *__restrict__ q, const uint4 *__restrict__ 
 #pragma unroll
                 for (int k = 0; k < 16; ++k) {
                     const int x = k * 32 + lane, tok = x >> 4, c = x & 15;
-                    cp_async16(sk + (uint32_t)((tok * 16 + (c ^ ((tok & 1) << 2))) * 16), src + x);
+                    cp_async16_pol(sk + (uint32_t)((tok * 16 + (c ^ ((tok & 1) << 2))) * 16), src + x, pol_kv);
                 }
             }
         }
@@ -303,7 +331,7 @@ prefill_block_mma_kernel(const uint4 *__restrict__ q, const uint4 *__restrict__ 
 #pragma unroll
             for (int k = 0; k < 16; ++k) {
                 const int x = k * 32 + lane, tok = x >> 4, c = x & 15;
-                cp_async16(sv + (uint32_t)((tok * 16 + (c ^ (tok & 7))) * 16), src + x);
+                cp_async16_pol(sv + (uint32_t)((tok * 16 + (c ^ (tok & 7))) * 16), src + x, pol_kv);
             }
         }
         cp_async_commit();
@@ -423,16 +451,16 @@ prefill_block_mma_kernel(const uint4 *__restrict__ q, const uint4 *__restrict__ 
             uint32_t *dst = reinterpret_cast<uint32_t *>(part_o + slot * kD) + t;
             float unused = 0.f;
 #pragma unroll
-            for (int n = 0; n < 16; ++n) dst[4 * n] = pack_bf16(o[n][0], o[n][1], unused);
-            if (t == 0) *reinterpret_cast<float2 *>(part_ml + slot * 2) = make_float2(ma, la);
+            for (int n = 0; n < 16; ++n) st_u32_pol(dst + 4 * n, pack_bf16(o[n][0], o[n][1], unused), pol_part);
+            if (t == 0) st_f2_pol(part_ml + slot * 2, ma, la, pol_part);
         }
         if (r + 8 < cur.rows) {
             const size_t slot = ((size_t)ib * H + cur.h) * kSel + (cur.eb.x & 15);
             uint32_t *dst = reinterpret_cast<uint32_t *>(part_o + slot * kD) + t;
             float unused = 0.f;
 #pragma unroll
-            for (int n = 0; n < 16; ++n) dst[4 * n] = pack_bf16(o[n][2], o[n][3], unused);
-            if (t == 0) *reinterpret_cast<float2 *>(part_ml + slot * 2) = make_float2(mb, lb);
+            for (int n = 0; n < 16; ++n) st_u32_pol(dst + 4 * n, pack_bf16(o[n][2], o[n][3], unused), pol_part);
+            if (t == 0) st_f2_pol(part_ml + slot * 2, mb, lb, pol_part);
         }
         cur = nxt;
         if (cur.w >= 0) nxt = load_unit(cur.w + stride, n_work, H, items, list, r);
@@ -477,6 +505,13 @@ prefill_merge_kernel(const int32_t *__restrict__ sel, const __nv_bfloat16 *__res
         A[2] = fmaf(wk, __uint_as_float(v[k].y << 16), A[2]);
         A[3] = fmaf(wk, __uint_as_float(v[k].y & 0xffff0000u), A[3]);
     }
+    // Every lane has its loads' values: drop this (query, head)'s partial lines from L2 (its 16
+    // x 256 bytes of outputs are 32 lines, one per lane, and its 16 (m, l) pairs one line), so
+    // that they are never written back.  The block kernel writes every slot the merge reads
+    // within the same call, before the merge starts.
+    __syncwarp();
+    l2_discard_line(part_o + base * kD + 64 * lane);
+    if (lane == 0) l2_discard_line(part_ml + base * 2);
     const float inv = W > 0.f ? 1.f / W : 0.f;
     float unused = 0.f;
     uint2 pk;
