@@ -219,7 +219,7 @@ def run_uocr(args):
     stream = torch.cuda.current_stream()
     l2 = torch.cuda.get_device_properties(dev).L2_cache_size
     flush = bytes_call * n_layers < 4 * l2
-    flush_buf = torch.empty(2 * l2 if flush else 1, dtype=torch.uint8, device=dev)
+    flush_l2 = L2Flush(l2, dev) if flush else None
 
     def step(st=None):
         for l in range(n_layers):
@@ -235,7 +235,7 @@ def run_uocr(args):
     clk = ClockSampler(physical_gpu(local_rank)).start()
     for _ in range(args.warmup):
         if flush:
-            flush_buf.zero_()
+            flush_l2()
         step()
     step_graph = capture_step(step, stream) if flush else None
     torch.cuda.synchronize()
@@ -247,7 +247,7 @@ def run_uocr(args):
         # L2 flushed between steps; each step (one graph replay) timed on its own
         times = []
         for _ in range(args.steps):
-            flush_buf.zero_()
+            flush_l2()
             e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
             e0.record(stream)
             step_graph.replay()
@@ -289,14 +289,14 @@ def run_uocr(args):
         with torch.cuda.graph(g, stream=side):
             for r in range(n_rep):
                 if flush:
-                    flush_buf.zero_()
+                    flush_l2()
                 fn(r % n_layers, side)
         flush_g = None
         if flush:
             flush_g = torch.cuda.CUDAGraph()
             with torch.cuda.graph(flush_g, stream=side):
                 for r in range(n_rep):
-                    flush_buf.zero_()
+                    flush_l2()
         g.replay()
         torch.cuda.synchronize()
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
@@ -402,7 +402,7 @@ def run_uocr(args):
         "config": {"workload": case.name, "batch_per_gpu": B, "context": int(case.seq_lens.max().item()),
                    "layers": n_layers, "heads": H, "head_dim": 128, "block": 32, "local_blocks": 4,
                    "remote_blocks": 12, "max_blocks": mb,
-                   "l2": "flushed between steps" if flush else "inputs larger than L2 (no flush)",
+                   "l2": L2_FLUSH_NOTE if flush else "inputs larger than L2 (no flush)",
                    "launch": "one CUDA-graph replay per step" if flush else "stream launches queued ahead",
                    "parallelism": f"dp{world} (independent sequence shards)"},
         "roofline": {"bound": "hbm", "kernel": "index_scan_kernel", "achieved": round(scan_gbs, 1),
@@ -451,6 +451,25 @@ def read_calibration(dev, stream, gib: int = 4, reps: int = 5):
     return {"kind": f"torch.sum over {gib} GiB bf16", "gbs": round(gbs, 1), "ms": round(ms, 4)}
 
 
+L2_FLUSH_NOTE = "flushed between steps (2 x L2 written, then 2 x L2 of another buffer read)"
+
+
+class L2Flush:
+    """Evicts a step's data from L2 between timed steps: writes a buffer of twice the L2 size, then
+    reads another of the same size.  The write is the flush; the read pass then evicts the flush's
+    own dirty lines (written back here, outside the timed region), so that the next step starts with
+    none of its inputs in L2 and no foreign write-back in its DRAM traffic."""
+
+    def __init__(self, l2_bytes, dev):
+        self.w = torch.empty(2 * l2_bytes, dtype=torch.uint8, device=dev)
+        self.r = torch.zeros(2 * l2_bytes // 4, dtype=torch.float32, device=dev)
+        self.acc = torch.zeros((), dtype=torch.float32, device=dev)
+
+    def __call__(self):
+        self.w.zero_()
+        torch.sum(self.r, dim=0, out=self.acc)
+
+
 def capture_step(fn, stream):
     """One call of fn(stream) captured in a CUDA graph (after one eager call on a side stream, so
     that lazily created resources exist).  The timed loops of the L2-flushed workloads replay it,
@@ -467,9 +486,9 @@ def capture_step(fn, stream):
     return g
 
 
-def graph_time_fn(fn, stream, n_rep, flush_buf=None):
+def graph_time_fn(fn, stream, n_rep, flush_l2=None):
     """Device ms per call of fn(stream) from n_rep calls captured in one CUDA graph
-    (minus the captured L2 flushes between them, when flush_buf is given)."""
+    (minus the captured L2 flushes between them, when an L2Flush is given)."""
     side = torch.cuda.Stream()
     side.wait_stream(stream)
     with torch.cuda.stream(side):
@@ -478,15 +497,15 @@ def graph_time_fn(fn, stream, n_rep, flush_buf=None):
     g = torch.cuda.CUDAGraph()
     with torch.cuda.graph(g, stream=side):
         for _ in range(n_rep):
-            if flush_buf is not None:
-                flush_buf.zero_()
+            if flush_l2 is not None:
+                flush_l2()
             fn(side)
     fg = None
-    if flush_buf is not None:
+    if flush_l2 is not None:
         fg = torch.cuda.CUDAGraph()
         with torch.cuda.graph(fg, stream=side):
             for _ in range(n_rep):
-                flush_buf.zero_()
+                flush_l2()
     g.replay()
     torch.cuda.synchronize()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
@@ -524,7 +543,7 @@ def run_prefill(args):
     scores = ws[: n_q * mb * 4].view(torch.float32).view(n_q, mb)
     stream = torch.cuda.current_stream()
     l2 = torch.cuda.get_device_properties(dev).L2_cache_size
-    flush_buf = torch.empty(2 * l2, dtype=torch.uint8, device=dev)
+    flush_l2 = L2Flush(l2, dev)
 
     def step(st=None):
         uocr.sparse_prefill(case.q, case.k_pool, case.v_pool, case.idx_q, case.idx_k_pool, case.block_table,
@@ -536,7 +555,7 @@ def run_prefill(args):
 
     clk = ClockSampler(physical_gpu(local_rank)).start()
     for _ in range(args.warmup):
-        flush_buf.zero_()
+        flush_l2()
         step()
     step_graph = capture_step(step, stream)
     torch.cuda.synchronize()
@@ -545,7 +564,7 @@ def run_prefill(args):
     clk.mark_start()
     times = []
     for _ in range(args.steps):
-        flush_buf.zero_()
+        flush_l2()
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         e0.record(stream)
         step_graph.replay()
@@ -563,18 +582,18 @@ def run_prefill(args):
     n_rep = 10
     gemm_ms = graph_time_fn(lambda st: uocr.prefill_index_score(case.idx_q, case.idx_k_pool, case.block_table,
                                                                 case.seq_lens, 0, case.q_pos, scores=scores,
-                                                                stream=st), stream, n_rep, flush_buf)
+                                                                stream=st), stream, n_rep, flush_l2)
     topk_ms = graph_time_fn(lambda st: uocr.block_topk(scores, case.seq_lens, case.q_seq, case.q_pos, sel=sel,
-                                                       stream=st), stream, n_rep, flush_buf)
+                                                       stream=st), stream, n_rep, flush_l2)
     attn_ms = graph_time_fn(lambda st: uocr.sparse_attn(case.q, case.k_pool, case.v_pool, case.block_table,
                                                         case.seq_lens, sel, case.q_seq, case.q_pos, out=out,
-                                                        stream=st), stream, n_rep, flush_buf)
+                                                        stream=st), stream, n_rep, flush_l2)
     seq_ws = torch.empty(max(uocr.sparse_attn_seq_workspace_bytes(n_q, H, mb), 1), dtype=torch.uint8, device=dev)
     out_seq = torch.empty_like(out)
     attn_seq_ms = graph_time_fn(lambda st: uocr.sparse_attn_seq(case.q, case.k_pool, case.v_pool, case.block_table,
                                                                 case.seq_lens, 0, case.q_pos, sel, out=out_seq,
-                                                                workspace=seq_ws, stream=st), stream, n_rep, flush_buf)
-    call_ms = graph_time_fn(lambda st: step(st), stream, n_rep, flush_buf)
+                                                                workspace=seq_ws, stream=st), stream, n_rep, flush_l2)
+    call_ms = graph_time_fn(lambda st: step(st), stream, n_rep, flush_l2)
     pos = case.q_pos.cpu().long()
     idx_flops = float(((pos + 1) * 128 * 2).sum())                 # causal q_idx . k_idx products
     attn_flops = float(n_q * H * 16 * 32 * 128 * 4)                 # QK and PV over 512 tokens
@@ -594,7 +613,7 @@ def run_prefill(args):
         "warmup": args.warmup, "ms_per_step": round(ms_per_step, 4), "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
         "config": {"workload": case.name, "queries": n_q, "context": int(case.seq_lens[0]), "heads": H,
-                   "max_blocks": mb, "l2": "flushed between steps", "launch": "one CUDA-graph replay per step",
+                   "max_blocks": mb, "l2": L2_FLUSH_NOTE, "launch": "one CUDA-graph replay per step",
                    "parallelism": f"dp{world}"},
         "roofline": {"bound": "tensor", "kernel": "prefill_index_gemm_kernel", "achieved": round(gemm_tflops, 1),
                      "peak": tc_peak, "unit": "TFLOP/s", "frac": round(gemm_tflops / tc_peak, 4), "traffic": None,
