@@ -167,14 +167,21 @@ prefill_invert_kernel(const int32_t *counts, const int32_t *__restrict__ bt_row,
         const int e = (blockIdx.x * kInvEntries + k) * kInvThreads + tid;
         ej[k] = -1;
         ep[k] = 0;
-        if (e < n_entries) {
+        if (e < n_entries) {   // both loads in flight together
             ej[k] = sel[e];
+            ep[k] = __ldg(q_pos + e / kSel);
             if (ej[k] >= max_blocks) ej[k] = -1;
-            if (ej[k] >= 0) ep[k] = __ldg(q_pos + e / kSel);
         }
     }
     int base_c = 0, base_g = 0;   // entries and items of the blocks before the tile
+    const int G = (int)gridDim.x;
     for (int t0 = 0; t0 < max_blocks; t0 += kInvTile) {
+        // the first block of the tile whose items this thread records (local index x with
+        // (t0 + x) % G == blockIdx.x), and its page, loaded ahead of the prefix sums
+        const int len = min(kInvTile, max_blocks - t0);
+        const int first = (int)((blockIdx.x + (unsigned)G - (unsigned)(t0 % G)) % (unsigned)G);
+        const int x0 = first + tid * G;
+        const int page0 = x0 < len ? __ldg(bt_row + t0 + x0) : 0;
         // thread tid sums blocks t0 + 8 tid .. t0 + 8 tid + 7
         int c[kInvPerThread], sc = 0, sg = 0;
 #pragma unroll
@@ -224,15 +231,12 @@ prefill_invert_kernel(const int32_t *counts, const int32_t *__restrict__ bt_row,
                 list[base_c + s_c[j - t0] + atomicAdd(fill + j, 1)] =
                     make_int2((blockIdx.x * kInvEntries + k) * kInvThreads + tid, ep[k]);
         }
-        // the items of this CTA's blocks in the tile: local index x with (t0 + x) % gridDim.x == b
-        const int len = min(kInvTile, max_blocks - t0);
-        const int G = (int)gridDim.x;
-        const int first = (int)((blockIdx.x + (unsigned)G - (unsigned)(t0 % G)) % (unsigned)G);
-        for (int x = first + tid * G; x < len; x += kInvThreads * G) {
+        // the items of this CTA's blocks in the tile
+        for (int x = x0; x < len; x += kInvThreads * G) {
             const int cnt = (x + 1 < kInvTile ? s_c[x + 1] : tot_c) - s_c[x];
             if (cnt == 0) continue;
             const int jb = t0 + x;
-            const int page = __ldg(bt_row + jb);
+            const int page = x == x0 ? page0 : __ldg(bt_row + jb);
             const int g0 = base_g + s_g[x], c0 = base_c + s_c[x];
             for (int k = 0; k * kItemRows < cnt; ++k)
                 items[g0 + k] = make_int4(jb, page, c0 + k * kItemRows, min(kItemRows, cnt - k * kItemRows));
