@@ -159,6 +159,32 @@ def test_sparse_attn_seq_matches_oracle(uocr, cuda_device):
     assert (out.float() - ref_q.float()).abs().max().item() <= 2e-2
 
 
+def test_sparse_attn_seq_reuses_one_workspace(uocr, cuda_device):
+    """Consecutive calls on one workspace, each checked against the oracle on its own selection.
+    The merge drops the partials it has read from L2, leaving their memory undefined; a call
+    writes every slot it uses before its merge reads it, so a slot that was empty in one call and
+    selected in the next (and the reverse) must not carry anything over."""
+    case = _prefill_case(32 * 70 + 7, 200, (0, 31, 64), seed=41, device=cuda_device)
+    mb = int(case.block_table.shape[1])
+    ws = torch.empty(uocr.sparse_attn_seq_workspace_bytes(case.n_q, 10, mb), dtype=torch.uint8,
+                     device=cuda_device)
+    first = _random_selection(case, 41, empty_frac=0.5)
+    second = _random_selection(case, 42, empty_frac=0.0)
+    third = second.copy()
+    third[:, 1::2] = -1                                 # slots full in the second call, empty now
+    none = (third < 0).all(axis=1)
+    third[none] = second[none]                          # a query keeps at least one block
+    for sel in (first, second, third, first):
+        out = uocr.sparse_attn_seq(case.q, case.k_pool, case.v_pool, case.block_table, case.seq_lens, 0,
+                                   case.q_pos, torch.from_numpy(sel).to(cuda_device), workspace=ws)
+        torch.cuda.synchronize()
+        got = out.float().cpu().numpy()
+        for i in range(case.n_q):
+            ref = oracle_attend(case, i, sel[i])
+            d = np.abs(got[i] - ref)
+            assert d.max() <= OUT_MAX_ATOL and d.mean() <= OUT_MEAN_ATOL, f"query {i}"
+
+
 def test_sparse_attn_seq_flags_bad_selections(uocr, cuda_device):
     case = _prefill_case(32 * 40, 64, seed=32, device=cuda_device, heads=3)
     sel = _random_selection(case, 32, empty_frac=0.0)
