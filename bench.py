@@ -47,10 +47,15 @@ NCU_TRAFFIC = {
     # ncu --set full on long_decode batch 4 (1 layer), one launch: 134,299,392 B read +
     # 3,379,200 B written (the write-back of the bench's L2 flush), scaled x4 to 16 queries.
     "long_decode": {"bytes": 4 * (134299392 + 3379200), "src": "aea494e8d3b8c4ea"},
+    # launch list of chunked_prefill with dram__bytes_read.sum / dram__bytes_write.sum and
+    # --cache-control none, averaged over the scoring GEMM's 16 launches: 17,253,056 B read (the
+    # indexer keys and queries) + 198,288 B written (the scores stay in L2 for the selection).
+    "chunked_prefill": {"bytes": 17253056 + 198288, "src": "a8fa49b30f1463f8"},
 }
 
 
 SCAN_SOURCES = ("index_scan.cu", "scan_core.cuh")   # the scan kernel and its page loop
+GEMM_SOURCES = ("prefill_index_gemm.cu", "tcgen05.cuh")   # the scoring GEMM and its tcgen05 helpers
 
 
 def kernel_source_hash(*names: str) -> str:
@@ -602,6 +607,8 @@ def run_prefill(args):
     tc_sust = float(peaks.get("bf16_tflops_sustained", 1400.0))
     hbm_peak = float(peaks.get("hbm_gbs", FALLBACK_HBM_GBS))
     gemm_tflops = idx_flops / (gemm_ms / 1e3) / 1e12
+    tr = NCU_TRAFFIC.get("chunked_prefill")
+    gemm_traffic = tr["bytes"] if tr and tr.get("src") == kernel_source_hash(*GEMM_SOURCES) else None
     kv_union = case.num_pages * H * 32 * 128 * 2 * 2               # every page is selected by some query
     n_sel_blocks = int(torch.unique(sel[sel >= 0]).numel())
     attn_bytes = n_sel_blocks * H * 32 * 128 * 2 * 2 + 2 * n_q * H * 128 * 2   # selected K/V tiles once, q, out
@@ -616,7 +623,7 @@ def run_prefill(args):
                    "max_blocks": mb, "l2": L2_FLUSH_NOTE, "launch": "one CUDA-graph replay per step",
                    "parallelism": f"dp{world}"},
         "roofline": {"bound": "tensor", "kernel": "prefill_index_gemm_kernel", "achieved": round(gemm_tflops, 1),
-                     "peak": tc_peak, "unit": "TFLOP/s", "frac": round(gemm_tflops / tc_peak, 4), "traffic": None,
+                     "peak": tc_peak, "unit": "TFLOP/s", "frac": round(gemm_tflops / tc_peak, 4), "traffic": gemm_traffic,
                      "peak_kind": f"{peak_kind} bf16 burst", "frac_of_sustained": round(gemm_tflops / tc_sust, 4),
                      "flops_per_launch": idx_flops, "avg_launch_ms": round(gemm_ms, 5)},
         "step_roofline": {"bound": "hbm", "achieved": round(step_bytes / (call_ms / 1e3) / 1e9, 1),
