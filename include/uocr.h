@@ -205,6 +205,8 @@ uocr_status_t uocr_prefill_index_score(const void *idx_q, const void *idx_k_cach
  * per-slot partial outputs are rounded to bf16 before the merge (at most
  * 2^-9 max|v| on an output).  Workspace: uocr_sparse_attn_seq_workspace_bytes
  * bytes, 256-byte aligned, owned by the caller, a pure function of the shapes.
+ * After the call its partial region holds undefined bytes: the merge drops the
+ * partials' L2 lines once it has read them, without writing them back.
  */
 size_t uocr_sparse_attn_seq_workspace_bytes(int n_q, int H, int max_blocks);
 
@@ -230,7 +232,9 @@ uocr_status_t uocr_sparse_attn_seq(const void *q, const void *k_cache, const voi
  * the bf16 partial adds at most 2^-9 max|v| to an output, the size of the
  * output's own bf16 rounding.  Workspace: uocr_prefill_workspace_bytes(n_q, H,
  * max_blocks) bytes, 256-byte aligned (the block scores first, then the
- * inverted index and the partials).  Errors as uocr_sparse_decode; a selected
+ * inverted index and the partials; after the call the block scores are
+ * readable and the partial region holds undefined bytes, dropped from L2 by
+ * the merge without being written back).  Errors as uocr_sparse_decode; a selected
  * block whose page is outside the pool contributes nothing to the output and
  * sets UOCR_DEVERR_PAGE.
  */
