@@ -23,8 +23,9 @@
 //      partials' traffic);
 //   3. one warp per (query, head) merges the 16 partials: out = sum_k
 //      2^(m_k - M) acc_k / sum_k 2^(m_k - M) l_k, written in bf16.
-// Each (block, head) tile is read from memory once per chunk (an item after the
-// first of the same tile finds it in L2).
+// Each (block, head) tile is read from memory about once per chunk (an item after
+// the first of the same tile runs beside it and finds it in L2; the DRAM reads come
+// to ~6 % above the selected tiles, queries and item records).
 //
 // Tensor-core layout of step 2.  The contraction index of S = Q K^T is the head
 // dimension, and any permutation of it applied to both operands leaves S
