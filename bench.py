@@ -12,6 +12,12 @@ Metric: decode queries/s per layer (= 16 * 12 / step time) and achieved HBM
 bandwidth on the algorithmic bytes (256 B of indexer key per causal token +
 512 tokens x 10 heads x 128 dims x 2 B x (K and V) per query).
 
+The default run (long_decode on one GPU) also measures the other workloads, each on its own
+after the headline's caches are freed, into a ``configs`` record: tiny, batched and ragged
+paged decode (queries/s, HBM fractions of the call and of the scan kernel) and the chunked
+prefill (queries/s, the scoring GEMM's tensor-core fraction, the attention stage's and the
+whole call's HBM fractions), each with the clocks of its own timed region.
+
 Prints ONE JSON line on rank 0.  Under torchrun each rank runs its own shard
 of sequences (weak scaling, no collective on the data path).
 """
@@ -430,6 +436,22 @@ def run_uocr(args):
     }
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         result["cpu_baseline"] = cpu_baseline(case, budget_s=args.cpu_budget)
+    if world == 1 and args.workload == "long_decode" and not args.no_configs:
+        # the other workloads, each measured on its own after the headline's caches are freed
+        del case, ws, outs, sels, scores, step_graph, flush_l2, step
+        import gc
+        gc.collect()
+        torch.cuda.empty_cache()
+        cfg_steps = max(5, min(args.steps, 50))
+        result["configs"] = {
+            "tiny_decode": decode_config_record("tiny_decode", args, uocr, dev, cfg_steps),
+            "batched_decode": decode_config_record("batched_decode", args, uocr, dev, cfg_steps),
+            "ragged_paged_decode": decode_config_record("ragged_paged_decode", args, uocr, dev, cfg_steps),
+            "chunked_prefill": prefill_config_record(args, uocr, dev, cfg_steps),
+            "note": "each workload measured alone after the headline (its own warm-up, timed calls and clocks); "
+                    "value = queries of one call / device time of one call",
+        }
+        result["gpu_launches"] += sum(v["gpu_launches"] for k, v in result["configs"].items() if k != "note")
     if world > 1:
         torch.distributed.destroy_process_group()
     if rank == 0:
@@ -540,6 +562,16 @@ def run_prefill(args):
         torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
     import block_sparse_long_uocr_b200 as uocr
 
+    result = prefill_measure(args, uocr, dev, rank, local_rank, world, args.steps, extras=True)
+    if world > 1:
+        torch.distributed.destroy_process_group()
+    if rank == 0:
+        print(json.dumps(result), flush=True)
+
+
+def prefill_measure(args, uocr, dev, rank, local_rank, world, steps, extras):
+    """The chunked-prefill measurement: `steps` timed calls (L2 flushed before each), the per-kernel
+    breakdown, the rooflines; with `extras` also the end-to-end leg and the oracle baseline."""
     case = workloads.chunked_prefill(device=dev, seed=udist.shard_seed(args.seed, rank))
     n_q, H, mb = case.n_q, case.q.shape[1], case.max_blocks
     ws = uocr.alloc_prefill_workspace(n_q, H, mb, dev)
@@ -568,7 +600,7 @@ def run_prefill(args):
     torch.cuda.synchronize()
     clk.mark_start()
     times = []
-    for _ in range(args.steps):
+    for _ in range(steps):
         flush_l2()
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         e0.record(stream)
@@ -581,8 +613,8 @@ def run_prefill(args):
     elapsed_ms = sum(a.elapsed_time(b) for a, b in times)
     barrier()
     max_ms = udist.max_over_ranks(elapsed_ms, dev)
-    ms_per_step = max_ms / args.steps
-    value = world * n_q * args.steps / (max_ms / 1e3)
+    ms_per_step = max_ms / steps
+    value = world * n_q * steps / (max_ms / 1e3)
 
     n_rep = 10
     gemm_ms = graph_time_fn(lambda st: uocr.prefill_index_score(case.idx_q, case.idx_k_pool, case.block_table,
@@ -616,7 +648,7 @@ def run_prefill(args):
     step_bytes = kv_union + case.num_pages * 32 * 128 * 2 + 2 * n_q * mb * 4 + 2 * n_q * H * 128 * 2
     result = {
         "metric": "chunked-prefill queries/s per layer; tensor-core TFLOP/s of the scoring GEMM vs peak",
-        "value": round(value, 1), "unit": "queries/s per layer", "n_gpus": world, "steps": args.steps,
+        "value": round(value, 1), "unit": "queries/s per layer", "n_gpus": world, "steps": steps,
         "warmup": args.warmup, "ms_per_step": round(ms_per_step, 4), "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
         "config": {"workload": case.name, "queries": n_q, "context": int(case.seq_lens[0]), "heads": H,
@@ -639,17 +671,102 @@ def run_prefill(args):
                          "sparse_attn_seq": round(1e3 * attn_seq_ms, 2),
                          "sparse_attn_query_centric": round(1e3 * attn_ms, 2),
                          "prefill_call_graph": round(1e3 * call_ms, 2)},
-        # per call: scoring GEMM, selection, inversion, block attention, merge
-        "gpu_launches": args.steps * 5,
+        "gpu_launches": steps * PREFILL_LAUNCHES,
         "clocks": clk.summary(),
     }
-    result["e2e"] = run_prefill_e2e(args, uocr, case, ws, out, sel, stream, world, dev)
-    if rank == 0 and not args.no_cpu_baseline:
-        result["cpu_baseline"] = cpu_baseline(case, args.cpu_budget)
-    if world > 1:
-        torch.distributed.destroy_process_group()
-    if rank == 0:
-        print(json.dumps(result), flush=True)
+    if extras:
+        result["e2e"] = run_prefill_e2e(args, uocr, case, ws, out, sel, stream, world, dev)
+        if rank == 0 and not args.no_cpu_baseline:
+            result["cpu_baseline"] = cpu_baseline(case, args.cpu_budget)
+    return result
+
+
+# kernels of one uocr_sparse_prefill call: scoring GEMM, selection, inversion, block attention, merge
+PREFILL_LAUNCHES = 5
+
+
+def decode_config_record(name, args, uocr, dev, steps):
+    """One decode workload measured on its own for the `configs` record of the default run:
+    `steps` timed decode calls (each replaying one captured call, L2 flushed before it when the
+    call's bytes would otherwise stay in L2), the scan kernel and the whole call from CUDA-graph
+    replays, the HBM fractions on the algorithmic bytes, and the clocks of its timed region."""
+    case = build_workload(name, dev, args.seed)
+    B, H, mb = case.n_q, case.q.shape[1], case.max_blocks
+    bytes_call, scan_bytes = algorithmic_bytes(case)
+    ws = uocr.alloc_workspace(B, H, mb, dev)
+    out = torch.empty_like(case.q)
+    sel = torch.empty((B, 16), dtype=torch.int32, device=dev)
+    scores = torch.empty((B, mb), dtype=torch.float32, device=dev)
+    stream = torch.cuda.current_stream()
+    l2 = torch.cuda.get_device_properties(dev).L2_cache_size
+    flush = bytes_call < 4 * l2
+    flush_l2 = L2Flush(l2, dev) if flush else None
+
+    def call(st=None):
+        uocr.sparse_decode(case.q, case.k_pool, case.v_pool, case.idx_q, case.idx_k_pool, case.block_table,
+                           case.seq_lens, out=out, sel=sel, workspace=ws, stream=st or stream)
+
+    for _ in range(max(3, args.warmup)):
+        if flush:
+            flush_l2()
+        call()
+    g = capture_step(call, stream)
+    torch.cuda.synchronize()
+    clk = ClockSampler(physical_gpu(torch.cuda.current_device())).start()
+    clk.mark_start()
+    times = []
+    for _ in range(steps):
+        if flush:
+            flush_l2()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        g.replay()
+        e1.record(stream)
+        times.append((e0, e1))
+    torch.cuda.synchronize()
+    clk.mark_end()
+    clk.stop()
+    call_ms = sum(a.elapsed_time(b) for a, b in times) / steps
+    n_rep = 20
+    scan_ms = graph_time_fn(lambda st: uocr.index_score(case.idx_q, case.idx_k_pool, case.block_table, case.seq_lens,
+                                                        scores=scores, stream=st), stream, n_rep, flush_l2)
+    peaks, peak_kind = measured_peaks()
+    peak = float(peaks.get("hbm_gbs", FALLBACK_HBM_GBS))
+    gbs = bytes_call / (call_ms / 1e3) / 1e9
+    scan_gbs = scan_bytes / (scan_ms / 1e3) / 1e9
+    tr = NCU_TRAFFIC.get(name)
+    traffic = tr["bytes"] if tr and tr.get("src") == kernel_source_hash(*SCAN_SOURCES) else None
+    rec = {"workload": case.name, "queries_per_call": B,
+           "value": round(B / (call_ms / 1e3), 1), "unit": "queries/s per layer",
+           "ms_per_call": round(call_ms, 5), "steps": steps,
+           "l2": L2_FLUSH_NOTE if flush else "inputs larger than L2 (no flush)",
+           "roofline": {"bound": "hbm", "achieved": round(gbs, 1), "peak": peak, "unit": "GB/s",
+                        "frac": round(gbs / peak, 4), "frac_of_8tbs": round(gbs / NOMINAL_HBM_GBS, 4),
+                        "bytes_per_call": bytes_call, "peak_kind": f"{peak_kind} hbm copy"},
+           "scan": {"kernel": "index_scan_kernel", "achieved": round(scan_gbs, 1), "frac": round(scan_gbs / peak, 4),
+                    "bytes_per_launch": scan_bytes, "avg_launch_ms": round(scan_ms, 5), "traffic": traffic},
+           "gpu_launches": steps * 3, "clocks": clk.summary()}
+    del case, ws, out, sel, scores, g, flush_l2
+    torch.cuda.empty_cache()
+    return rec
+
+
+def prefill_config_record(args, uocr, dev, steps):
+    """The chunked-prefill workload for the `configs` record of the default run."""
+    full = prefill_measure(args, uocr, dev, 0, torch.cuda.current_device(), 1, steps, extras=False)
+    r = full["roofline"]
+    rec = {"workload": full["config"]["workload"], "queries_per_call": full["config"]["queries"],
+           "value": full["value"], "unit": full["unit"], "ms_per_call": full["ms_per_step"], "steps": steps,
+           "l2": full["config"]["l2"],
+           "gemm": {"kernel": r["kernel"], "bound": "tensor", "achieved": r["achieved"], "unit": "TFLOP/s",
+                    "peak": r["peak"], "frac": r["frac"], "frac_of_sustained": r["frac_of_sustained"],
+                    "flops_per_launch": r["flops_per_launch"], "avg_launch_ms": r["avg_launch_ms"],
+                    "traffic": r["traffic"]},
+           "attention_stage": full["attn_roofline"],
+           "roofline": full["step_roofline"],
+           "breakdown_us": full["breakdown_us"], "gpu_launches": full["gpu_launches"], "clocks": full["clocks"]}
+    torch.cuda.empty_cache()
+    return rec
 
 
 def _serial_e2e(args, inputs, results, run_step, stream, dev):
@@ -951,6 +1068,8 @@ def main():
     ap.add_argument("--layers", type=int, default=None, help="long_decode only: layer caches (default 12)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-comparators", action="store_true", help="skip the full-attention / R-SWA timings")
+    ap.add_argument("--no-configs", action="store_true",
+                    help="long_decode only: skip the per-workload records of the other configs")
     ap.add_argument("--cpu-budget", type=float, default=10.0)
     args = ap.parse_args()
     if args.warmup < 3 and args.impl == "uocr":

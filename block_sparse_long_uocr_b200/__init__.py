@@ -144,8 +144,47 @@ def _dev(t: torch.Tensor, name: str, dtype: torch.dtype, ndim: int | None = None
     return t
 
 
-def _opt_i32(t, name):
-    return None if t is None else _dev(t, name, torch.int32, 1)
+def _opt_i32(t, name, n=None):
+    if t is None:
+        return None
+    _dev(t, name, torch.int32, 1)
+    if n is not None:
+        _shape(t, name, (n,))
+    return t
+
+
+def _shape(t: torch.Tensor, name: str, shape) -> torch.Tensor:
+    """Refuse, before any launch, a tensor whose shape differs from what the kernels will index
+    (None in `shape` accepts any extent): a smaller buffer would be written or read past its end
+    on the device."""
+    got = tuple(t.shape)
+    if len(got) != len(shape) or any(e is not None and g != e for g, e in zip(got, shape)):
+        want = "[" + ", ".join("*" if e is None else str(e) for e in shape) + "]"
+        raise ValueError(f"{name} must have shape {want}, got {list(got)}")
+    return t
+
+
+def _check_caches(k_cache, v_cache, H):
+    """K / V caches [P, H, 32, 128] of the same shape."""
+    _shape(k_cache, "k_cache", (None, H, BLOCK, HEAD_DIM))
+    _shape(v_cache, "v_cache", tuple(k_cache.shape))
+
+
+def _check_decode_args(q, k_cache, v_cache, idx_q, idx_k_cache, block_table, seq_lens, out, sel):
+    """One decode query per sequence: every per-sequence tensor has B rows, the caches agree on
+    the head count and the pool size, and the outputs match the queries."""
+    B, H = q.shape[0], q.shape[1]
+    _shape(q, "q", (B, H, HEAD_DIM))
+    _check_caches(k_cache, v_cache, H)
+    _shape(idx_q, "idx_q", (B, IDX_DIM))
+    if idx_k_cache is not None:
+        _shape(idx_k_cache, "idx_k_cache", (k_cache.shape[0], BLOCK, IDX_DIM))
+    _shape(block_table, "block_table", (B, None))
+    _shape(seq_lens, "seq_lens", (B,))
+    if out is not None:
+        _shape(out, "out", (B, H, HEAD_DIM))
+    if sel is not None:
+        _shape(sel, "sel", (B, N_SEL))
 
 
 def _stream(stream) -> ctypes.c_void_p:
@@ -184,12 +223,16 @@ def index_score(idx_q, idx_k_cache, block_table, seq_lens, q_seq=None, q_pos=Non
     _dev(block_table, "block_table", torch.int32, 2)
     _dev(seq_lens, "seq_lens", torch.int32, 1)
     n_q, B, mb = idx_q.shape[0], block_table.shape[0], block_table.shape[1]
+    _shape(idx_q, "idx_q", (n_q, IDX_DIM))
+    _shape(idx_k_cache, "idx_k_cache", (None, BLOCK, IDX_DIM))
+    _shape(seq_lens, "seq_lens", (B,))
     if scores is None:
         scores = torch.full((n_q, mb), float("-inf"), dtype=torch.float32, device=idx_q.device)
     _dev(scores, "scores", torch.float32, 2)
+    _shape(scores, "scores", (n_q, mb))
     _check("uocr_index_score", _lib().uocr_index_score(
-        _ptr(idx_q), _ptr(idx_k_cache), _ptr(block_table), _ptr(seq_lens), _ptr(_opt_i32(q_seq, "q_seq")),
-        _ptr(_opt_i32(q_pos, "q_pos")), n_q, B, mb, idx_k_cache.shape[0], _ptr(scores),
+        _ptr(idx_q), _ptr(idx_k_cache), _ptr(block_table), _ptr(seq_lens), _ptr(_opt_i32(q_seq, "q_seq", n_q)),
+        _ptr(_opt_i32(q_pos, "q_pos", n_q)), n_q, B, mb, idx_k_cache.shape[0], _ptr(scores),
         _ptr(dev_err), _stream(stream)))
     return scores
 
@@ -202,8 +245,9 @@ def block_topk(scores, seq_lens, q_seq=None, q_pos=None, *, sel=None, dev_err=No
     if sel is None:
         sel = torch.empty((n_q, N_SEL), dtype=torch.int32, device=scores.device)
     _dev(sel, "sel", torch.int32, 2)
+    _shape(sel, "sel", (n_q, N_SEL))
     _check("uocr_block_topk", _lib().uocr_block_topk(
-        _ptr(scores), _ptr(seq_lens), _ptr(_opt_i32(q_seq, "q_seq")), _ptr(_opt_i32(q_pos, "q_pos")),
+        _ptr(scores), _ptr(seq_lens), _ptr(_opt_i32(q_seq, "q_seq", n_q)), _ptr(_opt_i32(q_pos, "q_pos", n_q)),
         n_q, seq_lens.shape[0], mb, _ptr(sel), _ptr(dev_err), _stream(stream)))
     return sel
 
@@ -219,12 +263,18 @@ def sparse_attn(q, k_cache, v_cache, block_table, seq_lens, sel, q_seq=None, q_p
     _dev(sel, "sel", torch.int32, 2)
     n_q, H = q.shape[0], q.shape[1]
     B, mb = block_table.shape
+    _shape(q, "q", (n_q, H, HEAD_DIM))
+    _check_caches(k_cache, v_cache, H)
+    _shape(seq_lens, "seq_lens", (B,))
+    _shape(sel, "sel", (n_q, N_SEL))
     if out is None:
         out = torch.empty_like(q)
+    _dev(out, "out", torch.bfloat16, 3)
+    _shape(out, "out", (n_q, H, HEAD_DIM))
     sc = float(scale) if scale is not None else HEAD_DIM ** -0.5
     _check("uocr_sparse_attn", _lib().uocr_sparse_attn(
         _ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(block_table), _ptr(seq_lens),
-        _ptr(_opt_i32(q_seq, "q_seq")), _ptr(_opt_i32(q_pos, "q_pos")), _ptr(sel), n_q, B, H, mb,
+        _ptr(_opt_i32(q_seq, "q_seq", n_q)), _ptr(_opt_i32(q_pos, "q_pos", n_q)), _ptr(sel), n_q, B, H, mb,
         k_cache.shape[0], ctypes.c_float(sc), _ptr(out), _ptr(dev_err), _stream(stream)))
     return out
 
@@ -245,6 +295,9 @@ def sparse_decode(q, k_cache, v_cache, idx_q, idx_k_cache, block_table, seq_lens
         out = torch.empty_like(q)
     if sel is None:
         sel = torch.empty((B, N_SEL), dtype=torch.int32, device=q.device)
+    _dev(out, "out", torch.bfloat16, 3)
+    _dev(sel, "sel", torch.int32, 2)
+    _check_decode_args(q, k_cache, v_cache, idx_q, idx_k_cache, block_table, seq_lens, out, sel)
     if workspace is None:
         workspace = alloc_workspace(B, H, mb, q.device)
     _check("uocr_sparse_decode", _lib().uocr_sparse_decode(
@@ -263,9 +316,14 @@ def prefill_index_score(idx_q, idx_k_cache, block_table, seq_lens, seq: int, q_p
     _dev(seq_lens, "seq_lens", torch.int32, 1)
     _dev(q_pos, "q_pos", torch.int32, 1)
     n_q, B, mb = idx_q.shape[0], block_table.shape[0], block_table.shape[1]
+    _shape(idx_q, "idx_q", (n_q, IDX_DIM))
+    _shape(idx_k_cache, "idx_k_cache", (None, BLOCK, IDX_DIM))
+    _shape(seq_lens, "seq_lens", (B,))
+    _shape(q_pos, "q_pos", (n_q,))
     if scores is None:
         scores = torch.full((n_q, mb), float("-inf"), dtype=torch.float32, device=idx_q.device)
     _dev(scores, "scores", torch.float32, 2)
+    _shape(scores, "scores", (n_q, mb))
     _check("uocr_prefill_index_score", _lib().uocr_prefill_index_score(
         _ptr(idx_q), _ptr(idx_k_cache), _ptr(block_table), _ptr(seq_lens), int(seq), _ptr(q_pos), n_q, B, mb,
         idx_k_cache.shape[0], _ptr(scores), _ptr(dev_err), _stream(stream)))
@@ -286,6 +344,16 @@ def sparse_prefill(q, k_cache, v_cache, idx_q, idx_k_cache, block_table, seq_len
         out = torch.empty_like(q)
     if sel is None:
         sel = torch.empty((n_q, N_SEL), dtype=torch.int32, device=q.device)
+    _dev(out, "out", torch.bfloat16, 3)
+    _dev(sel, "sel", torch.int32, 2)
+    _shape(q, "q", (n_q, H, HEAD_DIM))
+    _check_caches(k_cache, v_cache, H)
+    _shape(idx_q, "idx_q", (n_q, IDX_DIM))
+    _shape(idx_k_cache, "idx_k_cache", (k_cache.shape[0], BLOCK, IDX_DIM))
+    _shape(seq_lens, "seq_lens", (B,))
+    _shape(q_pos, "q_pos", (n_q,))
+    _shape(out, "out", (n_q, H, HEAD_DIM))
+    _shape(sel, "sel", (n_q, N_SEL))
     if workspace is None:
         workspace = alloc_prefill_workspace(n_q, H, mb, q.device)
     _check("uocr_sparse_prefill", _lib().uocr_sparse_prefill(
@@ -308,6 +376,13 @@ def sparse_attn_seq(q, k_cache, v_cache, block_table, seq_lens, seq: int, q_pos,
     B, mb = block_table.shape
     if out is None:
         out = torch.empty_like(q)
+    _dev(out, "out", torch.bfloat16, 3)
+    _shape(q, "q", (n_q, H, HEAD_DIM))
+    _check_caches(k_cache, v_cache, H)
+    _shape(seq_lens, "seq_lens", (B,))
+    _shape(q_pos, "q_pos", (n_q,))
+    _shape(sel, "sel", (n_q, N_SEL))
+    _shape(out, "out", (n_q, H, HEAD_DIM))
     if workspace is None:
         workspace = torch.empty(max(sparse_attn_seq_workspace_bytes(n_q, H, mb), 1), dtype=torch.uint8,
                                 device=q.device)
@@ -327,11 +402,16 @@ def summary_score(idx_q, summary_cache, block_table, seq_lens, q_seq=None, q_pos
     _dev(block_table, "block_table", torch.int32, 2)
     _dev(seq_lens, "seq_lens", torch.int32, 1)
     n_q, B, mb = idx_q.shape[0], block_table.shape[0], block_table.shape[1]
+    _shape(idx_q, "idx_q", (n_q, IDX_DIM))
+    _shape(summary_cache, "summary_cache", (None, IDX_DIM))
+    _shape(seq_lens, "seq_lens", (B,))
     if scores is None:
         scores = torch.full((n_q, mb), float("-inf"), dtype=torch.float32, device=idx_q.device)
+    _dev(scores, "scores", torch.float32, 2)
+    _shape(scores, "scores", (n_q, mb))
     _check("uocr_summary_score", _lib().uocr_summary_score(
-        _ptr(idx_q), _ptr(summary_cache), _ptr(block_table), _ptr(seq_lens), _ptr(_opt_i32(q_seq, "q_seq")),
-        _ptr(_opt_i32(q_pos, "q_pos")), n_q, B, mb, summary_cache.shape[0], _ptr(scores), _ptr(dev_err),
+        _ptr(idx_q), _ptr(summary_cache), _ptr(block_table), _ptr(seq_lens), _ptr(_opt_i32(q_seq, "q_seq", n_q)),
+        _ptr(_opt_i32(q_pos, "q_pos", n_q)), n_q, B, mb, summary_cache.shape[0], _ptr(scores), _ptr(dev_err),
         _stream(stream)))
     return scores
 
@@ -340,9 +420,11 @@ def block_summary_mean(idx_k_cache, summary_cache=None, pages=None, *, dev_err=N
     """bf16 [P, 128]: the mean of each (listed) page's indexer keys."""
     _dev(idx_k_cache, "idx_k_cache", torch.bfloat16, 3)
     P = idx_k_cache.shape[0]
+    _shape(idx_k_cache, "idx_k_cache", (P, BLOCK, IDX_DIM))
     if summary_cache is None:
         summary_cache = torch.zeros((P, IDX_DIM), dtype=torch.bfloat16, device=idx_k_cache.device)
     _dev(summary_cache, "summary_cache", torch.bfloat16, 2)
+    _shape(summary_cache, "summary_cache", (P, IDX_DIM))
     n = P if pages is None else _dev(pages, "pages", torch.int32, 1).shape[0]
     _check("uocr_block_summary_mean", _lib().uocr_block_summary_mean(
         _ptr(idx_k_cache), _ptr(pages), n, P, _ptr(summary_cache), _ptr(dev_err), _stream(stream)))
@@ -363,6 +445,10 @@ def sparse_decode_summary(q, k_cache, v_cache, idx_q, summary_cache, block_table
         out = torch.empty_like(q)
     if sel is None:
         sel = torch.empty((B, N_SEL), dtype=torch.int32, device=q.device)
+    _dev(out, "out", torch.bfloat16, 3)
+    _dev(sel, "sel", torch.int32, 2)
+    _shape(summary_cache, "summary_cache", (k_cache.shape[0], IDX_DIM))
+    _check_decode_args(q, k_cache, v_cache, idx_q, None, block_table, seq_lens, out, sel)
     if workspace is None:
         workspace = alloc_workspace(B, H, mb, q.device)
     _check("uocr_sparse_decode_summary", _lib().uocr_sparse_decode_summary(
@@ -379,10 +465,13 @@ def block_topk_masked(scores, seq_lens, cand_mask, q_seq=None, q_pos=None, *, se
     _dev(seq_lens, "seq_lens", torch.int32, 1)
     _dev(cand_mask, "cand_mask", torch.int32, 2)
     n_q, mb = scores.shape
+    _shape(cand_mask, "cand_mask", (seq_lens.shape[0], None))
     if sel is None:
         sel = torch.empty((n_q, N_SEL), dtype=torch.int32, device=scores.device)
+    _dev(sel, "sel", torch.int32, 2)
+    _shape(sel, "sel", (n_q, N_SEL))
     _check("uocr_block_topk_masked", _lib().uocr_block_topk_masked(
-        _ptr(scores), _ptr(seq_lens), _ptr(_opt_i32(q_seq, "q_seq")), _ptr(_opt_i32(q_pos, "q_pos")),
+        _ptr(scores), _ptr(seq_lens), _ptr(_opt_i32(q_seq, "q_seq", n_q)), _ptr(_opt_i32(q_pos, "q_pos", n_q)),
         _ptr(cand_mask), cand_mask.shape[1], n_q, seq_lens.shape[0], mb, _ptr(sel), _ptr(dev_err), _stream(stream)))
     return sel
 
@@ -400,9 +489,19 @@ def rope_append(q, idx_q, k_new, v_new, idx_k_new, tok_pos, page_pos, block_tabl
         _dev(t, n, dt, nd)
     n, H = q.shape[0], q.shape[1]
     B, mb = block_table.shape
+    _shape(q, "q", (n, H, HEAD_DIM))
+    _shape(idx_q, "idx_q", (n, IDX_DIM))
+    _shape(k_new, "k_new", (n, H, HEAD_DIM))
+    _shape(v_new, "v_new", (n, H, HEAD_DIM))
+    _shape(idx_k_new, "idx_k_new", (n, IDX_DIM))
+    _shape(tok_pos, "tok_pos", (n,))
+    _shape(page_pos, "page_pos", (n,))
+    _shape(seq_lens, "seq_lens", (B,))
+    _check_caches(k_cache, v_cache, H)
+    _shape(idx_k_cache, "idx_k_cache", (k_cache.shape[0], BLOCK, IDX_DIM))
     _check("uocr_rope_append", _lib().uocr_rope_append(
         _ptr(q), _ptr(idx_q), _ptr(k_new), _ptr(v_new), _ptr(idx_k_new), _ptr(tok_pos), _ptr(page_pos),
-        _ptr(_opt_i32(q_seq, "q_seq")), _ptr(_opt_i32(q_pos, "q_pos")), _ptr(block_table), _ptr(seq_lens),
+        _ptr(_opt_i32(q_seq, "q_seq", n)), _ptr(_opt_i32(q_pos, "q_pos", n)), _ptr(block_table), _ptr(seq_lens),
         n, B, H, mb, k_cache.shape[0], _ptr(k_cache), _ptr(v_cache), _ptr(idx_k_cache), _ptr(dev_err),
         _stream(stream)))
     return q, idx_q
@@ -425,6 +524,12 @@ def dense_decode(q, k_cache, v_cache, block_table, seq_lens, *, ref_blocks: int 
     rb = mb if ref_blocks is None else int(ref_blocks)
     if out is None:
         out = torch.empty_like(q)
+    _dev(out, "out", torch.bfloat16, 3)
+    _shape(q, "q", (B, H, HEAD_DIM))
+    _check_caches(k_cache, v_cache, H)
+    _shape(block_table, "block_table", (B, None))
+    _shape(seq_lens, "seq_lens", (B,))
+    _shape(out, "out", (B, H, HEAD_DIM))
     if workspace is None:
         workspace = torch.empty(max(dense_workspace_bytes(B, H, mb), 1), dtype=torch.uint8, device=q.device)
     _check("uocr_dense_decode", _lib().uocr_dense_decode(
@@ -453,6 +558,7 @@ def sparse_decode_static(q, k_cache, v_cache, idx_q, idx_k_cache, block_table, s
                          (seq_lens, "seq_lens", torch.int32, 1), (out, "out", torch.bfloat16, 3),
                          (sel, "sel", torch.int32, 2)):
         _dev(t, n, dt, nd)
+    _check_decode_args(q, k_cache, v_cache, idx_q, idx_k_cache, block_table, seq_lens, out, sel)
     B, H = q.shape[0], q.shape[1]
     _check("uocr_sparse_decode_static", _lib().uocr_sparse_decode_static(
         _ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(idx_q), _ptr(idx_k_cache), _ptr(block_table),

@@ -7,6 +7,8 @@
 #include <math.h>
 #include <stdint.h>
 
+#include <atomic>
+
 #include "common.cuh"
 #include "kernels.h"
 #include "uocr.h"
@@ -32,6 +34,11 @@ inline WsLayout ws_layout(int n_q, int /*H*/, int max_blocks) {
     return w;
 }
 
+// Limit of the first bounded wait of the decode attention and of the scoring GEMM's epilogue
+// (LaunchCtx::first_wait_ns), negative for the library default.  Set only by the test hook
+// uocr_test_first_wait_limit_ns below.
+std::atomic<long long> g_first_wait_ns{-1};
+
 inline uocr_status_t make_ctx(uocr_stream_t stream, bool pdl, uocr::LaunchCtx &c) {
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess) return UOCR_ERR_CUDA;
@@ -41,6 +48,8 @@ inline uocr_status_t make_ctx(uocr_stream_t stream, bool pdl, uocr::LaunchCtx &c
     c.stream = (cudaStream_t)stream;
     c.num_sms = sms;
     c.pdl = pdl;
+    const long long w = g_first_wait_ns.load(std::memory_order_relaxed);
+    c.first_wait_ns = w < 0 ? uocr::kWaitLimitNs : (uint64_t)w;
     return UOCR_OK;
 }
 
@@ -81,6 +90,13 @@ const char *uocr_status_string(uocr_status_t status) {
 }
 
 int uocr_abi_version(void) { return 2; }
+
+// Test hook, not part of the ABI in uocr.h: sets the wall-time limit of the first bounded wait
+// of the decode attention (its V copy) and of the scoring GEMM's epilogue (its first
+// accumulator) for the calls that follow, process-wide; ns = 0 makes those waits give up at
+// once, a negative ns restores the default (2 s).  The drain waits that follow a timeout keep
+// the default limit.  Used by the tests to run the timeout paths without a stuck copy.
+void uocr_test_first_wait_limit_ns(long long ns) { g_first_wait_ns.store(ns, std::memory_order_relaxed); }
 
 size_t uocr_workspace_bytes(int n_q, int H, int max_blocks) {
     if (n_q <= 0 || H <= 0 || max_blocks <= 0) return 0;
@@ -140,12 +156,14 @@ uocr_status_t uocr_sparse_attn(const void *q, const void *k_cache, const void *v
                                                 out, false, -1, false, dev_err));
 }
 
-uocr_status_t uocr_sparse_decode(const void *q, const void *k_cache, const void *v_cache,
-                                 const void *idx_q, const void *idx_k_cache,
-                                 const int32_t *block_table, const int32_t *seq_lens, int B, int H,
-                                 int max_blocks, int num_pages, void *out, int32_t *sel_out,
-                                 void *workspace, size_t workspace_bytes, int32_t *dev_err,
-                                 uocr_stream_t stream) {
+}  // extern "C"
+
+namespace uocr {
+// Every check of uocr_sparse_decode that does not concern the workspace, in its order.
+uocr_status_t check_sparse_decode_args(const void *q, const void *k_cache, const void *v_cache, const void *idx_q,
+                                       const void *idx_k_cache, const int32_t *block_table,
+                                       const int32_t *seq_lens, int B, int H, int max_blocks, int num_pages,
+                                       const void *out, const int32_t *sel_out, const int32_t *dev_err) {
     uocr_status_t st = check_common(B, B, max_blocks, num_pages, block_table, seq_lens, nullptr,
                                     nullptr, dev_err);
     if (st != UOCR_OK) return st;
@@ -154,6 +172,21 @@ uocr_status_t uocr_sparse_decode(const void *q, const void *k_cache, const void 
         return UOCR_ERR_INVALID_ARG;
     if (!sel_out || !aligned(sel_out, 4)) return UOCR_ERR_INVALID_ARG;
     if (H < 1 || H > UOCR_MAX_HEADS) return UOCR_ERR_UNSUPPORTED;
+    return UOCR_OK;
+}
+}  // namespace uocr
+
+extern "C" {
+
+uocr_status_t uocr_sparse_decode(const void *q, const void *k_cache, const void *v_cache,
+                                 const void *idx_q, const void *idx_k_cache,
+                                 const int32_t *block_table, const int32_t *seq_lens, int B, int H,
+                                 int max_blocks, int num_pages, void *out, int32_t *sel_out,
+                                 void *workspace, size_t workspace_bytes, int32_t *dev_err,
+                                 uocr_stream_t stream) {
+    uocr_status_t st = uocr::check_sparse_decode_args(q, k_cache, v_cache, idx_q, idx_k_cache, block_table,
+                                                      seq_lens, B, H, max_blocks, num_pages, out, sel_out, dev_err);
+    if (st != UOCR_OK) return st;
     const WsLayout w = ws_layout(B, H, max_blocks);
     if (!workspace || !aligned(workspace, kWsAlign) || workspace_bytes < w.total) return UOCR_ERR_WORKSPACE;
     uocr::LaunchCtx c;

@@ -16,6 +16,10 @@ constexpr int kD = UOCR_HEAD_DIM;
 constexpr int kDIdx = UOCR_IDX_DIM;
 constexpr int kPageElems = kBlock * kD;   // elements of one (page, head) tile: 4096 bf16 = 8 KiB
 constexpr float kLog2e = 1.4426950408889634f;
+// Wall-time bound of every mbarrier wait in the library: far above any legitimate wait for an
+// asynchronous copy or tensor-core operation (microseconds), short enough that a stuck wait
+// ends the kernel with UOCR_DEVERR_TIMEOUT instead of hanging the device.
+constexpr uint64_t kWaitLimitNs = 2000000000ull;
 
 // Query position and sequence for query i, with the device-side checks the
 // ABI documents.  Returns false (and flags dev_err) when the query is invalid;
@@ -163,14 +167,6 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t *bar, uint32_t parity) {
     return ok != 0;
 }
 
-// Bounded wait on phase `parity` of `bar`: false after `max_tries` unsuccessful probes
-// (each probe may suspend the thread for a hardware-defined interval).
-__device__ __forceinline__ bool mbar_wait_bounded(uint64_t *bar, uint32_t parity, int max_tries) {
-    for (int it = 0; it < max_tries; ++it)
-        if (mbar_try_wait(bar, parity)) return true;
-    return false;
-}
-
 __device__ __forceinline__ uint64_t global_timer_ns() {
     uint64_t t;
     asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
@@ -191,9 +187,11 @@ __device__ __forceinline__ bool mbar_try_wait_sleep(uint64_t *bar, uint32_t pari
 
 // Wait on phase `parity` of `bar` for at most `timeout_ns` of wall time, giving up early
 // when *abort becomes non-zero.  Returns true when the phase completed.  Each probe may
-// suspend the thread for up to 20 us, so the wait does not spin.
+// suspend the thread for up to 20 us, so the wait does not spin.  A zero limit gives up at
+// once without probing (the way the timeout paths are exercised).
 __device__ __forceinline__ bool mbar_wait_timed(uint64_t *bar, uint32_t parity, uint64_t timeout_ns,
                                                 const volatile int *abort) {
+    if (timeout_ns == 0) return false;
     if (mbar_try_wait(bar, parity)) return true;
     const uint64_t t0 = global_timer_ns();
     for (uint32_t it = 1;; ++it) {

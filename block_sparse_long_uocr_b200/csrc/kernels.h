@@ -13,6 +13,10 @@ struct LaunchCtx {
     cudaStream_t stream;
     int num_sms;
     bool pdl;   // launch with programmatic stream serialization
+    // Limit of the first bounded wait of the decode attention (its V copy) and of the scoring
+    // GEMM's epilogue (its first accumulator); kWaitLimitNs except when a test shortens it to
+    // exercise the timeout path.  Every other wait keeps kWaitLimitNs.
+    uint64_t first_wait_ns;
 };
 
 cudaError_t launch_index_scan(const LaunchCtx &c, const void *idx_q, const void *idx_k,
@@ -31,6 +35,13 @@ cudaError_t launch_sparse_attn(const LaunchCtx &c, const void *q, const void *k,
                                const int32_t *q_pos, const int32_t *sel, int n_q, int B, int H,
                                int max_blocks, int num_pages, float scale, void *out,
                                bool implicit_local, int fixed_seq, bool head_major, int32_t *dev_err);
+
+// The argument checks of uocr_sparse_decode other than the workspace's (shared with
+// uocr_sparse_decode_static, which checks its fixed scratch size after them).
+uocr_status_t check_sparse_decode_args(const void *q, const void *k_cache, const void *v_cache, const void *idx_q,
+                                       const void *idx_k_cache, const int32_t *block_table,
+                                       const int32_t *seq_lens, int B, int H, int max_blocks, int num_pages,
+                                       const void *out, const int32_t *sel_out, const int32_t *dev_err);
 
 // tcgen05 block scoring of n_q queries of one sequence (block table row bt_row,
 // length *seq_len_ptr) into scores [n_q][max_blocks].  sched: a zeroed int32 work-unit counter

@@ -60,7 +60,6 @@ constexpr int kMmaWarp = 9;               // MMA issuer of subtile 0; allocates 
 constexpr int kProducerBWarp = 10;        // key (B) tiles
 constexpr int kMmaWarp1 = 11;             // MMA issuer of subtile 1
 constexpr int kThreads = 384;
-constexpr uint64_t kTimeoutNs = 2000000000ull;   // 2 s: far above any legitimate wait
 
 struct __align__(1024) Smem {
     uint8_t a[kStagesA][kMT][2][kHalfBytesA];   // 128 KiB
@@ -131,10 +130,11 @@ __device__ __forceinline__ UnitInfo unit_info(int u, int n_chunks, int n_q, int 
 }
 
 // Lane 0 waits; the verdict is broadcast so the whole warp leaves its loops together.
-__device__ __forceinline__ bool warp_wait(uint64_t *bar, uint32_t parity, Smem &s, int32_t *dev_err, int lane) {
+__device__ __forceinline__ bool warp_wait(uint64_t *bar, uint32_t parity, Smem &s, int32_t *dev_err, int lane,
+                                          uint64_t limit_ns = kWaitLimitNs) {
     int ok = 1;
     if (lane == 0) {
-        ok = mbar_wait_timed(bar, parity, kTimeoutNs, &s.abort_flag);
+        ok = mbar_wait_timed(bar, parity, limit_ns, &s.abort_flag);
         if (!ok) {
             if (!*(volatile int *)&s.abort_flag) flag_error(dev_err, UOCR_DEVERR_TIMEOUT);
             atomicExch(&s.abort_flag, 1);
@@ -151,8 +151,8 @@ __device__ __forceinline__ bool warp_wait2(uint64_t *bar0, uint32_t parity0, uin
     if (lane == 0) {
         const bool r0 = mbar_try_wait(bar0, parity0);
         const bool r1 = mbar_try_wait(bar1, parity1);
-        ok = (r0 || mbar_wait_timed(bar0, parity0, kTimeoutNs, &s.abort_flag)) &&
-             (r1 || mbar_wait_timed(bar1, parity1, kTimeoutNs, &s.abort_flag));
+        ok = (r0 || mbar_wait_timed(bar0, parity0, kWaitLimitNs, &s.abort_flag)) &&
+             (r1 || mbar_wait_timed(bar1, parity1, kWaitLimitNs, &s.abort_flag));
         if (!ok) {
             if (!*(volatile int *)&s.abort_flag) flag_error(dev_err, UOCR_DEVERR_TIMEOUT);
             atomicExch(&s.abort_flag, 1);
@@ -170,7 +170,7 @@ prefill_index_gemm_kernel(const __grid_constant__ CUtensorMap map_q, const __gri
                           const int32_t *__restrict__ bt_row, const int32_t *__restrict__ seq_len_ptr,
                           const int32_t *__restrict__ q_pos, int n_q, int a_box_rows, int num_pages,
                           int max_blocks, int n_chunks, int n_units, float *__restrict__ scores,
-                          int32_t *sched, int32_t *dev_err) {
+                          int32_t *sched, int32_t *dev_err, uint64_t first_wait_ns) {
     extern __shared__ uint8_t smem_raw[];
     Smem &s = *reinterpret_cast<Smem *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     const int warp = threadIdx.x >> 5;
@@ -284,7 +284,7 @@ prefill_index_gemm_kernel(const __grid_constant__ CUtensorMap map_q, const __gri
         // end marker below completes one more phase of a stage)
         if (lane == 0)
             for (int k = 0; k < kStagesA; ++k)
-                if (a_fills[k] > 0) mbar_wait_timed(&s.a_full[k], (a_fills[k] - 1) & 1, kTimeoutNs, nullptr);
+                if (a_fills[k] > 0) mbar_wait_timed(&s.a_full[k], (a_fills[k] - 1) & 1, kWaitLimitNs, nullptr);
         __syncwarp();
         // end marker for every other role: a stage that holds no unit
         if (!aborted(s)) {
@@ -334,7 +334,7 @@ prefill_index_gemm_kernel(const __grid_constant__ CUtensorMap map_q, const __gri
         }
         if (lane == 0)
             for (int k = 0; k < kStagesB; ++k)
-                if (b_fills[k] > 0) mbar_wait_timed(&s.b_full[k], (b_fills[k] - 1) & 1, kTimeoutNs, nullptr);
+                if (b_fills[k] > 0) mbar_wait_timed(&s.b_full[k], (b_fills[k] - 1) & 1, kWaitLimitNs, nullptr);
     } else if (warp == kMmaWarp || warp == kMmaWarp1) {
         // ------------------------------------------------------------ MMA issuers, one per subtile
         // Two issuing threads: while one waits on a barrier or commits, the other's MMAs keep
@@ -401,7 +401,7 @@ prefill_index_gemm_kernel(const __grid_constant__ CUtensorMap map_q, const __gri
         // drain: every MMA this thread issued has completed before TMEM is freed
         if (lane == 0 && issued) {
             tc::commit(&s.mma_done[m]);
-            mbar_wait_timed(&s.mma_done[m], 0, kTimeoutNs, nullptr);
+            mbar_wait_timed(&s.mma_done[m], 0, kWaitLimitNs, nullptr);
         }
         __syncwarp();
     } else {
@@ -433,7 +433,8 @@ prefill_index_gemm_kernel(const __grid_constant__ CUtensorMap map_q, const __gri
             float *srow = scores + (size_t)(row < n_q ? row : 0) * max_blocks;
             for (int t = 0; t < ntiles; ++t, ++it) {
                 const int acc = it & 1;
-                if (!warp_wait(&s.acc_full[acc][sub], (it >> 1) & 1, s, dev_err, lane)) {
+                if (!warp_wait(&s.acc_full[acc][sub], (it >> 1) & 1, s, dev_err, lane,
+                               it == 0 ? first_wait_ns : kWaitLimitNs)) {
                     stop = true;
                     break;
                 }
@@ -565,7 +566,8 @@ cudaError_t launch_prefill_index_gemm(const LaunchCtx &c, const void *idx_q, con
     cfg.attrs = attr;
     cfg.numAttrs = c.pdl ? 1 : 0;
     return cudaLaunchKernelEx(&cfg, prefill_index_gemm_kernel, map_q, map_k, bt_row, seq_len_ptr, q_pos, n_q,
-                              a_box_rows, num_pages, max_blocks, n_chunks, (int)units, scores, sched, dev_err);
+                              a_box_rows, num_pages, max_blocks, n_chunks, (int)units, scores, sched, dev_err,
+                              c.first_wait_ns);
 }
 
 }  // namespace uocr

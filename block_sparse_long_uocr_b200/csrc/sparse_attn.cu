@@ -68,7 +68,7 @@ sparse_attn_kernel(const uint4 *__restrict__ q, const uint4 *__restrict__ kc, co
                    const int32_t *__restrict__ q_seq, const int32_t *__restrict__ q_pos,
                    const int32_t *__restrict__ sel, int B, int H, int max_blocks, int num_pages,
                    float scale_log2, int implicit_local, int fixed_seq, int head_major, int n_q,
-                   __nv_bfloat16 *__restrict__ out, int32_t *dev_err) {
+                   __nv_bfloat16 *__restrict__ out, int32_t *dev_err, uint64_t first_wait_ns) {
     __shared__ float s_m[kAttnWarps], s_l[kAttnWarps];
     __shared__ float s_acc[kAttnWarps][kD];
     __shared__ float s_cta_ml[2];
@@ -150,11 +150,16 @@ sparse_attn_kernel(const uint4 *__restrict__ q, const uint4 *__restrict__ kc, co
         const float pt = exp2f(zt - m_w);
         l_w = warp_sum(pt);
 
-        const bool ready = mbar_wait_bounded(bar, 0, 1 << 20);
+        // every lane waits (bounded in wall time) and observes the copy's completion itself
+        const bool ready = __all_sync(0xffffffffu, mbar_wait_timed(bar, 0, first_wait_ns, nullptr));
         if (!ready) {
-            // the copy did not land in time: report it, let it finish, and drop the block
+            // The copy did not land in time: report it and drop the block.  Before the warp goes
+            // on, a second wait (default limit) lets the copy finish, so that the CTA does not
+            // retire with a bulk copy still writing into its shared memory.  If that wait too runs
+            // out (a copy stuck for seconds: a broken memory system), the kernel ends regardless,
+            // bounded, rather than wait forever.
             if (lane == 0) flag_error(dev_err, UOCR_DEVERR_TIMEOUT);
-            mbar_wait_bounded(bar, 0, 1 << 20);
+            mbar_wait_timed(bar, 0, kWaitLimitNs, nullptr);
             m_w = -INFINITY;
             l_w = 0.f;
         } else {
@@ -255,7 +260,7 @@ cudaError_t launch_sparse_attn(const LaunchCtx &c, const void *q, const void *k,
     return cudaLaunchKernelEx(&cfg, sparse_attn_kernel, (const uint4 *)q, (const uint4 *)k, (const uint4 *)v, bt,
                               seq_lens, q_seq, q_pos, sel, B, H, max_blocks, num_pages, scale * kLog2e,
                               implicit_local ? 1 : 0, fixed_seq, head_major ? 1 : 0, n_q, (__nv_bfloat16 *)out,
-                              dev_err);
+                              dev_err, c.first_wait_ns);
 }
 
 }  // namespace uocr

@@ -5,6 +5,10 @@ device: the sequence's indexer pages (for scores and selection) and the K/V
 pages of the selected blocks (for attention), re-indexed into small host
 pools.  That lets full-size workloads be checked on sampled queries.
 
+``check_all_queries`` does the same for every query of a one-sequence case
+(a prefill chunk) with one host copy of the sequence's pages and the oracle
+run over all queries at once (OpenMP).
+
 Acceptance (per query):
   * block scores: |gpu - oracle| <= SCORE_ATOL on every causal block;
   * selection: identical to the oracle's, unless the oracle flags a near tie
@@ -107,3 +111,43 @@ def check_queries(case, queries, out_gpu, sel_gpu, scores_gpu=None, layer=0, rep
     if report is not None:
         report.extend(stats)
     return stats
+
+
+def check_all_queries(case, out_gpu, sel_gpu, scores_gpu=None, layer=0, threads=0):
+    """check_queries for every query of a case whose queries all belong to one sequence, with the
+    sequence's pages copied to the host once and the oracle run over all queries in one call.
+    Returns (max abs error, mean abs error, near ties) over all queries."""
+    q, idx_q = case.q_layers[layer]
+    kp, vp, ikp = case.layers[layer]
+    seqs = set(case.q_seq.cpu().tolist())
+    assert len(seqs) == 1, "one sequence only"
+    b = seqs.pop()
+    nb_max = int(case.q_pos.max().item()) // 32 + 1
+    pages = case.block_table[b, :nb_max].long()
+    h_idx, h_k, h_v = ikp[pages].cpu(), kp[pages].cpu(), vp[pages].cpu()
+    bt = np.arange(nb_max, dtype=np.int32).reshape(1, nb_max)     # logical block j -> host page j
+    qs = np.zeros(case.n_q, np.int32)
+    qp = case.q_pos.cpu().numpy().astype(np.int32)
+    h_q, h_qi = q.cpu(), idx_q.cpu()
+    r = oracle.run(h_q, h_qi, h_k[:1], h_v[:1], h_idx, bt, qs, qp, want_out=False, threads=threads)
+    sel = sel_gpu.cpu().numpy()
+    sc = scores_gpu.cpu().numpy() if scores_gpu is not None else None
+    ties = 0
+    for i in range(case.n_q):
+        nb = int(qp[i]) // 32 + 1 if qp[i] >= 0 else 0
+        s = r["scores"][i, :nb]
+        if sc is not None and nb:
+            err = np.abs(sc[i, :nb].astype(np.float64) - s).max()
+            assert err <= SCORE_ATOL, f"query {i}: score error {err}"
+        tie = bool(r["near_tie"][i])
+        ties += int(tie)
+        assert accept_selection(s, r["sel"][i], sel[i], tie), \
+            f"query {i}: selection {sel[i].tolist()} vs oracle {r['sel'][i].tolist()} (near tie {tie})"
+    ref = oracle.run(h_q, h_qi, h_k, h_v, h_idx[:1], bt, qs, qp, sel_in=sel, threads=threads)["out"]
+    got = out_gpu.float().cpu().numpy()
+    d = np.abs(got - ref)
+    per_max = d.reshape(case.n_q, -1).max(axis=1)
+    per_mean = d.reshape(case.n_q, -1).mean(axis=1)
+    bad = np.nonzero((per_max > OUT_MAX_ATOL) | (per_mean > OUT_MEAN_ATOL))[0]
+    assert bad.size == 0, f"queries {bad[:10].tolist()}: out max {per_max[bad[:10]].tolist()}"
+    return float(d.max()), float(d.mean()), ties

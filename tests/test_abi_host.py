@@ -161,6 +161,30 @@ def test_sparse_decode_rejects(pkg, over, code):
     assert st == code
 
 
+@no_gpu
+@pytest.mark.parametrize("over,code", [
+    (dict(q=None), 1), (dict(sel=None), 1), (dict(idx_k=MIS), 1), (dict(H=0), 2), (dict(B=0), 1),
+    (dict(mb=1 << 27), 2),                               # too many blocks: UNSUPPORTED, not WORKSPACE
+    (dict(q=None, B=64, mb=1 << 20), 1),                 # a NULL pointer with a shape past the scratch
+    (dict(P=0, B=64, mb=1 << 20), 1),                    # a bad pool size with a shape past the scratch
+    (dict(B=64, mb=1 << 20), 3),                         # valid arguments, scratch too small
+])
+def test_sparse_decode_static_checks_in_the_order_of_sparse_decode(pkg, over, code):
+    """The static entry returns what uocr_sparse_decode would for the same arguments; only a call
+    that passes all of those checks can fail on its fixed scratch size (UOCR_ERR_WORKSPACE)."""
+    a = dict(q=FAKE, k=FAKE, v=FAKE, idx_q=FAKE, idx_k=FAKE, bt=FAKE, sl=FAKE, B=4, H=10, mb=64, P=256,
+             out=FAKE, sel=FAKE)
+    a.update(over)
+    st = pkg.lib.uocr_sparse_decode_static(a["q"], a["k"], a["v"], a["idx_q"], a["idx_k"], a["bt"], a["sl"],
+                                           a["B"], a["H"], a["mb"], a["P"], a["out"], a["sel"], None, None)
+    assert st == code
+    if code != 3:
+        ws = pkg.workspace_bytes(a["B"], a["H"], a["mb"]) if a["B"] > 0 and a["H"] > 0 and a["mb"] > 0 else 0
+        st2 = pkg.lib.uocr_sparse_decode(a["q"], a["k"], a["v"], a["idx_q"], a["idx_k"], a["bt"], a["sl"], a["B"],
+                                         a["H"], a["mb"], a["P"], a["out"], a["sel"], FAKE, max(ws, 256), None, None)
+        assert st2 == code
+
+
 def test_python_binding_refuses_cpu_tensors(pkg):
     x = torch.zeros(2, 128, dtype=torch.bfloat16)
     with pytest.raises(ValueError, match="CUDA"):

@@ -1,8 +1,9 @@
 """Parity of the CUDA path (through the C ABI) with the fp64 oracle.
 
-Small cases are checked on every query and every block score; the full-size
-workloads are checked on sampled queries (the oracle reads back only those
-queries' pages).  Tolerances: scores 1e-3 absolute; outputs 2e-2 max and
+Every case, the full-size workloads included, is checked on every query and
+every block score (the long-decode workload on every query of its first, a
+middle and its last layer; the oracle reads back only each query's pages).
+Tolerances: scores 1e-3 absolute; outputs 2e-2 max and
 2e-3 mean absolute error; selections exact except oracle-flagged near ties.
 """
 import numpy as np
@@ -11,7 +12,7 @@ import torch
 
 import oracle
 import workloads
-from parity_util import check_queries
+from parity_util import check_all_queries, check_queries
 
 pytestmark = pytest.mark.gpu
 
@@ -228,25 +229,85 @@ def test_device_errors_are_flagged_not_trapped(uocr, cuda_device):
     assert torch.isfinite(out.float()).all()
 
 
+def _first_wait_limit(uocr, ns):
+    """Test hook of the library (not in uocr.h): the limit of the first bounded wait of the decode
+    attention and of the scoring GEMM's epilogue; 0 gives up at once, -1 restores the default."""
+    import ctypes
+    fn = uocr.lib.uocr_test_first_wait_limit_ns
+    fn.argtypes = [ctypes.c_longlong]
+    fn.restype = None
+    fn(int(ns))
+
+
+def test_decode_attention_wait_timeout_is_flagged_and_recovers(uocr, cuda_device):
+    """The decode attention's wait for its V copy gives up at once: every block is dropped and
+    UOCR_DEVERR_TIMEOUT is set, the kernel still drains its copies and ends, the outputs are finite
+    (zeros: no block contributes), and the next call with the default limit matches the oracle."""
+    case = workloads.make_case([32 * 300 + 5, 32 * 40, 700], shuffle=True, seed=12, device=cuda_device)
+    err = torch.zeros(1, dtype=torch.int32, device=cuda_device)
+    _first_wait_limit(uocr, 0)
+    try:
+        out, sel = uocr.sparse_decode(case.q, case.k_pool, case.v_pool, case.idx_q, case.idx_k_pool,
+                                      case.block_table, case.seq_lens, dev_err=err)
+        torch.cuda.synchronize()
+    finally:
+        _first_wait_limit(uocr, -1)
+    assert int(err.item()) & uocr.DEVERR_TIMEOUT
+    assert torch.isfinite(out.float()).all() and (out == 0).all()
+    err.zero_()
+    out, sel, sc = run_decode(uocr, case)
+    check_queries(case, range(case.n_q), out, sel, sc)
+
+
+def test_binding_refuses_wrong_output_shapes_before_launching(uocr, cuda_device):
+    """A selection buffer of 12 slots or an output of the wrong shape is refused by the binding
+    with nothing launched (the caller's buffers keep their contents)."""
+    case = workloads.make_case([32 * 64, 32 * 70], seed=13, device=cuda_device)
+    B = case.n_q
+    bad_sel = torch.full((B, 12), -5, dtype=torch.int32, device=cuda_device)
+    out = torch.full_like(case.q, 3.0)
+    sel = torch.full((B, 16), -5, dtype=torch.int32, device=cuda_device)
+    bad_out = torch.full((B, 10, 64), 3.0, dtype=torch.bfloat16, device=cuda_device)
+    for fn in (uocr.sparse_decode, uocr.sparse_decode_static):
+        with pytest.raises(ValueError, match="sel"):
+            fn(case.q, case.k_pool, case.v_pool, case.idx_q, case.idx_k_pool, case.block_table, case.seq_lens,
+               out=out, sel=bad_sel)
+        with pytest.raises(ValueError, match="out"):
+            fn(case.q, case.k_pool, case.v_pool, case.idx_q, case.idx_k_pool, case.block_table, case.seq_lens,
+               out=bad_out, sel=sel)
+        with pytest.raises(ValueError, match="seq_lens"):
+            fn(case.q, case.k_pool, case.v_pool, case.idx_q, case.idx_k_pool, case.block_table,
+               case.seq_lens[:1].contiguous(), out=out, sel=sel)
+    with pytest.raises(ValueError, match="sel"):
+        uocr.sparse_attn(case.q, case.k_pool, case.v_pool, case.block_table, case.seq_lens, bad_sel)
+    torch.cuda.synchronize()
+    assert (bad_sel == -5).all() and (sel == -5).all() and (out == 3.0).all() and (bad_out == 3.0).all()
+
+
 # ----------------------------------------------------------------------------- full-size workloads
 @pytest.mark.slow
-def test_decode_long_context_workload_sampled(uocr, cuda_device):
-    case = workloads.long_decode(device=cuda_device, n_layers=1)
-    out, sel, sc = run_decode(uocr, case)
-    check_queries(case, [0, 5, 15], out, sel, sc)
+def test_decode_long_context_workload_every_query(uocr, cuda_device):
+    """The long-decode workload as the bench runs it (16 sequences x 131072 tokens, 12 layer caches,
+    126 GiB): every query of the first, a middle and the last layer against the oracle."""
+    case = workloads.long_decode(device=cuda_device)
+    for layer in (0, 5, 11):
+        out, sel, sc = run_decode(uocr, case, layer=layer)
+        check_queries(case, range(case.n_q), out, sel, sc, layer=layer)
+    del case
+    torch.cuda.empty_cache()
 
 
 @pytest.mark.slow
-def test_decode_ragged_paged_workload_sampled(uocr, cuda_device):
+def test_decode_ragged_paged_workload_every_query(uocr, cuda_device):
     case = workloads.ragged_paged_decode(device=cuda_device)
     out, sel, sc = run_decode(uocr, case)
-    lens = case.seq_lens.cpu()
-    picks = sorted({int(lens.argmin()), int(lens.argmax()), 0, 13, 31, 63})
-    check_queries(case, picks, out, sel, sc)
+    check_queries(case, range(case.n_q), out, sel, sc)
+    del case
+    torch.cuda.empty_cache()
 
 
 @pytest.mark.slow
-def test_decode_maximum_lengths_sampled(uocr, cuda_device):
+def test_decode_maximum_lengths(uocr, cuda_device):
     """A 1.6M-token row (50,000 blocks: past the selection's shared-memory staging of 49,152
     candidates, so it reads its scores from L2), a 1M-token row (32,768 blocks, staged), and a
     short row sharing the same block table width."""
@@ -257,11 +318,13 @@ def test_decode_maximum_lengths_sampled(uocr, cuda_device):
 
 
 @pytest.mark.slow
-def test_chunked_prefill_workload_sampled_step_entries(uocr, cuda_device):
+def test_chunked_prefill_workload_every_query_step_entries(uocr, cuda_device):
+    """The chunked-prefill workload through the per-step entry points (scan, selection,
+    query-centric attention): every score, selection and output of the 2048 queries."""
     case = workloads.chunked_prefill(device=cuda_device)
     sc = uocr.index_score(case.idx_q, case.idx_k_pool, case.block_table, case.seq_lens, case.q_seq, case.q_pos)
     sel = uocr.block_topk(sc, case.seq_lens, case.q_seq, case.q_pos)
     out = uocr.sparse_attn(case.q, case.k_pool, case.v_pool, case.block_table, case.seq_lens, sel,
                            case.q_seq, case.q_pos)
     torch.cuda.synchronize()
-    check_queries(case, [0, 1, 31, 32, 1000, 2046, 2047], out, sel, sc)
+    check_all_queries(case, out, sel, sc)
