@@ -662,8 +662,8 @@ def prefill_measure(args, uocr, dev, rank, local_rank, world, steps, extras):
                           "peak": hbm_peak, "unit": "GB/s",
                           "frac": round(step_bytes / (call_ms / 1e3) / 1e9 / hbm_peak, 4),
                           "bytes_per_step": step_bytes, "flops_per_step": idx_flops + attn_flops},
-        "attn_roofline": {"bound": "hbm", "entry": "uocr_sparse_attn_seq: selection check, inversion, "
-                          "tensor-core block kernel, merge (4 kernels)", "achieved": round(attn_gbs, 1),
+        "attn_roofline": {"bound": "hbm", "entry": "uocr_sparse_attn_seq: classification, tcgen05 local-window "
+                          "kernel, inversion, block kernel, merge (5 kernels)", "achieved": round(attn_gbs, 1),
                           "peak": hbm_peak, "unit": "GB/s", "frac": round(attn_gbs / hbm_peak, 4),
                           "bytes_per_launch": attn_bytes, "avg_launch_ms": round(attn_seq_ms, 5),
                           "selected_blocks": n_sel_blocks},
@@ -681,8 +681,9 @@ def prefill_measure(args, uocr, dev, rank, local_rank, world, steps, extras):
     return result
 
 
-# kernels of one uocr_sparse_prefill call: scoring GEMM, selection, inversion, block attention, merge
-PREFILL_LAUNCHES = 5
+# kernels of one uocr_sparse_prefill call: scoring GEMM, selection, classification, local-window
+# attention (tcgen05), inversion, block attention, merge
+PREFILL_LAUNCHES = 7
 
 
 def decode_config_record(name, args, uocr, dev, steps):

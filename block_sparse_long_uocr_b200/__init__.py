@@ -65,6 +65,8 @@ def _load() -> ctypes.CDLL:
     lib.uocr_status_string.restype = ctypes.c_char_p
     lib.uocr_abi_version.argtypes = []
     lib.uocr_abi_version.restype = I
+    lib.uocr_last_cuda_error.argtypes = []
+    lib.uocr_last_cuda_error.restype = ctypes.c_char_p
     lib.uocr_workspace_bytes.argtypes = [I, I, I]
     lib.uocr_workspace_bytes.restype = Z
     lib.uocr_index_score.argtypes = [P, P, P, P, P, P, I, I, I, I, P, P, P]
@@ -123,7 +125,10 @@ def __getattr__(name):
 # --------------------------------------------------------------------------- helpers
 def _check(fn: str, st: int):
     if st != 0:
-        raise UocrError(fn, st, _lib().uocr_status_string(st).decode())
+        msg = _lib().uocr_status_string(st).decode()
+        if st == 4:   # UOCR_ERR_CUDA: name the CUDA error behind it
+            msg += f" ({_lib().uocr_last_cuda_error().decode()})"
+        raise UocrError(fn, st, msg)
 
 
 def _ptr(t: torch.Tensor | None):

@@ -34,6 +34,16 @@ inline WsLayout ws_layout(int n_q, int /*H*/, int max_blocks) {
     return w;
 }
 
+// The CUDA error behind this thread's last UOCR_ERR_CUDA (uocr_last_cuda_error).
+thread_local cudaError_t t_last_cuda_error = cudaSuccess;
+
+inline uocr_status_t cuda_status(cudaError_t e) {
+    if (e == cudaSuccess) return UOCR_OK;
+    t_last_cuda_error = e;
+    (void)cudaGetLastError();   // clear the sticky-free launch error so later calls are clean
+    return UOCR_ERR_CUDA;
+}
+
 // Limit of the first bounded wait of the decode attention and of the scoring GEMM's epilogue
 // (LaunchCtx::first_wait_ns), negative for the library default.  Set only by the test hook
 // uocr_test_first_wait_limit_ns below.
@@ -41,22 +51,17 @@ std::atomic<long long> g_first_wait_ns{-1};
 
 inline uocr_status_t make_ctx(uocr_stream_t stream, bool pdl, uocr::LaunchCtx &c) {
     int dev = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess) return UOCR_ERR_CUDA;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return cuda_status(e);
     int sms = 0;
-    if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
-        return UOCR_ERR_CUDA;
+    e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    if (e != cudaSuccess) return cuda_status(e);
     c.stream = (cudaStream_t)stream;
     c.num_sms = sms;
     c.pdl = pdl;
     const long long w = g_first_wait_ns.load(std::memory_order_relaxed);
     c.first_wait_ns = w < 0 ? uocr::kWaitLimitNs : (uint64_t)w;
     return UOCR_OK;
-}
-
-inline uocr_status_t cuda_status(cudaError_t e) {
-    if (e == cudaSuccess) return UOCR_OK;
-    (void)cudaGetLastError();   // clear the sticky-free launch error so later calls are clean
-    return UOCR_ERR_CUDA;
 }
 
 // Common shape checks shared by every compute entry point.
@@ -90,6 +95,10 @@ const char *uocr_status_string(uocr_status_t status) {
 }
 
 int uocr_abi_version(void) { return 2; }
+
+const char *uocr_last_cuda_error(void) {
+    return t_last_cuda_error == cudaSuccess ? "no error" : cudaGetErrorString(t_last_cuda_error);
+}
 
 // Test hook, not part of the ABI in uocr.h: sets the wall-time limit of the first bounded wait
 // of the decode attention (its V copy) and of the scoring GEMM's epilogue (its first
@@ -242,6 +251,7 @@ uocr_status_t uocr_sparse_prefill(const void *q, const void *k_cache, const void
     if (H < 1 || H > UOCR_MAX_HEADS) return UOCR_ERR_UNSUPPORTED;
     if (n_q == 0) return UOCR_OK;
     if ((long long)n_q * UOCR_N_SEL > 0x7fffffffLL || (long long)n_q * H > 0x7fffffffLL) return UOCR_ERR_UNSUPPORTED;
+    if ((long long)num_pages * H > 0x7fffffffLL) return UOCR_ERR_UNSUPPORTED;   // TMA tile coordinates are int32
     const WsLayout w = ws_layout(n_q, H, max_blocks);
     if (!workspace || !aligned(workspace, kWsAlign) || workspace_bytes < uocr_prefill_workspace_bytes(n_q, H, max_blocks))
         return UOCR_ERR_WORKSPACE;
@@ -258,12 +268,11 @@ uocr_status_t uocr_sparse_prefill(const void *q, const void *k_cache, const void
                                         num_pages, scores, (int32_t *)(attn_ws + aw.sched_off), dev_err);
     if (e != cudaSuccess) return cuda_status(e);
     c.pdl = true;
-    e = uocr::launch_block_topk(c, scores, seq_lens, nullptr, q_pos, n_q, B, max_blocks, sel_out, dev_err, seq,
-                                nullptr, 0, (int32_t *)(attn_ws + aw.counts_off));
+    e = uocr::launch_block_topk(c, scores, seq_lens, nullptr, q_pos, n_q, B, max_blocks, sel_out, dev_err, seq);
     if (e != cudaSuccess) return cuda_status(e);
     const float scale = 1.0f / sqrtf((float)UOCR_HEAD_DIM);
-    e = uocr::launch_prefill_attn(c, q, k_cache, v_cache, bt_row, q_pos, sel_out, n_q, H, max_blocks, num_pages,
-                                  scale, out, attn_ws, dev_err);
+    e = uocr::launch_prefill_attn(c, q, k_cache, v_cache, bt_row, seq_lens + seq, q_pos, sel_out, n_q, H, max_blocks,
+                                  num_pages, scale, out, attn_ws, dev_err);
     return cuda_status(e);
 }
 
@@ -286,6 +295,7 @@ uocr_status_t uocr_sparse_attn_seq(const void *q, const void *k_cache, const voi
     if (!isfinite(scale)) return UOCR_ERR_INVALID_ARG;
     if (n_q == 0) return UOCR_OK;
     if ((long long)n_q * UOCR_N_SEL > 0x7fffffffLL || (long long)n_q * H > 0x7fffffffLL) return UOCR_ERR_UNSUPPORTED;
+    if ((long long)num_pages * H > 0x7fffffffLL) return UOCR_ERR_UNSUPPORTED;   // TMA tile coordinates are int32
     if (!workspace || !aligned(workspace, kWsAlign) ||
         workspace_bytes < uocr_sparse_attn_seq_workspace_bytes(n_q, H, max_blocks))
         return UOCR_ERR_WORKSPACE;
@@ -296,11 +306,9 @@ uocr_status_t uocr_sparse_attn_seq(const void *q, const void *k_cache, const voi
     char *ws = (char *)workspace;
     cudaError_t e = cudaMemsetAsync(ws, 0, aw.zero_bytes, c.stream);
     if (e != cudaSuccess) return cuda_status(e);
-    e = uocr::launch_prefill_select_count(c, sel, q_pos, seq_lens + seq, n_q, max_blocks, workspace, dev_err);
-    if (e != cudaSuccess) return cuda_status(e);
     return cuda_status(uocr::launch_prefill_attn(c, q, k_cache, v_cache, block_table + (size_t)seq * max_blocks,
-                                                 q_pos, (const int32_t *)(ws + aw.sel_off), n_q, H, max_blocks,
-                                                 num_pages, scale, out, workspace, dev_err));
+                                                 seq_lens + seq, q_pos, sel, n_q, H, max_blocks, num_pages, scale, out,
+                                                 workspace, dev_err));
 }
 
 size_t uocr_dense_workspace_bytes(int B, int H, int max_blocks) {

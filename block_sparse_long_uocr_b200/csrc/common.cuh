@@ -67,6 +67,14 @@ __device__ __forceinline__ void bf16x8_to_f32(const uint4 &v, float (&f)[8]) {
     }
 }
 
+// A read-only load issued where it stands in the program: the volatile asm keeps the compiler
+// from sinking a load issued ahead of a wait down to its first use after the wait.
+__device__ __forceinline__ int ld_pinned(const int32_t *p) {
+    int v;
+    asm volatile("ld.global.nc.b32 %0, [%1];" : "=r"(v) : "l"(p));
+    return v;
+}
+
 // Streaming 16-byte load that bypasses L1 allocation (each byte is read once).
 __device__ __forceinline__ uint4 ld_stream(const uint4 *p) {
     uint4 v;
@@ -200,6 +208,12 @@ __device__ __forceinline__ bool mbar_wait_timed(uint64_t *bar, uint32_t parity, 
         if (global_timer_ns() - t0 > timeout_ns) return false;
         if (it > (1u << 28)) return false;   // in case the timer does not advance
     }
+}
+
+// A drain wait (the copies or MMAs a warp issued must complete before its CTA ends or frees
+// what they use): bounded like every wait, and a wait that runs out is reported as a timeout.
+__device__ __forceinline__ void mbar_drain(uint64_t *bar, uint32_t parity, int32_t *dev_err) {
+    if (!mbar_wait_timed(bar, parity, kWaitLimitNs, nullptr)) flag_error(dev_err, UOCR_DEVERR_TIMEOUT);
 }
 
 // Programmatic dependent launch: wait for the preceding grid's memory, and

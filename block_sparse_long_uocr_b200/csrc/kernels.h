@@ -1,6 +1,7 @@
 // kernels.h -- internal launchers of libuocr (not part of the public ABI).
 #pragma once
 
+#include <cuda.h>
 #include <cuda_runtime.h>
 #include <stddef.h>
 #include <stdint.h>
@@ -51,26 +52,44 @@ cudaError_t launch_prefill_index_gemm(const LaunchCtx &c, const void *idx_q, con
                                       int n_q, int max_blocks, int num_pages, float *scores, int32_t *sched,
                                       int32_t *dev_err);
 
-// Block-centric prefill attention (selection inverted per block, tensor-core items of 16
-// entries per (block, head), per-slot partials merged per (query, head)).  Workspace regions,
-// 256-byte aligned.  The first zero_bytes bytes (the per-block selector counts and list
-// counters) must be zero before the call's first kernel.
+// cuTensorMapEncodeTiled through the runtime's driver entry point (NULL if unavailable).
+typedef CUresult (*EncodeTiledFn)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *, const cuuint64_t *,
+                                  const cuuint64_t *, const cuuint32_t *, const cuuint32_t *, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+EncodeTiledFn tensor_map_encoder();
+
+// Prefill attention of many queries of one sequence over their selection: the selection is
+// classified per 128-query tile (local-window entries of tiles whose windows fit 8 blocks go to
+// the tensor-core local kernel, the rest to the block kernel), the block kernel's entries are
+// inverted per block and attended in items of 16 entries per (block, head), and a merge kernel
+// combines each row's partial states.  Workspace regions, 256-byte aligned.  The first zero_bytes
+// bytes (per-block entry counts, list counters, the scoring GEMM's unit counter) must be zero
+// before the call's first kernel.
 struct PrefillAttnWs {
-    size_t counts_off, fill_off, sched_off, n_items_off, items_off, list_off, sel_off, ml_off, o_off;
+    size_t counts_off, fill_off, sched_off, n_items_off, items_off, list_off, sel_off, loc_off, tile_off, ml_off,
+        o_off, loc_ml_off, loc_o_off;
     size_t zero_bytes;
 };
 size_t prefill_attn_workspace(int n_q, int H, int max_blocks, PrefillAttnWs *w);
-// `ws` must start with the per-block selection counts of `sel` (max_blocks int32), as
-// launch_block_topk writes them when given `counts` zeroed.
-// For a caller's selection: a validated copy of it into the workspace's sel region and the
-// per-block counts (zeroed by the caller) that launch_prefill_attn expects.
-cudaError_t launch_prefill_select_count(const LaunchCtx &c, const int32_t *sel, const int32_t *q_pos,
-                                       const int32_t *seq_len_ptr, int n_q, int max_blocks, void *ws,
-                                       int32_t *dev_err);
+// sel: the queries' selection ([n_q][16], any order, -1 for an empty slot), validated here.
 cudaError_t launch_prefill_attn(const LaunchCtx &c, const void *q, const void *k, const void *v,
-                                const int32_t *bt_row, const int32_t *q_pos, const int32_t *sel, int n_q, int H,
-                                int max_blocks, int num_pages, float scale, void *out, void *ws,
-                                int32_t *dev_err);
+                                const int32_t *bt_row, const int32_t *seq_len_ptr, const int32_t *q_pos,
+                                const int32_t *sel, int n_q, int H, int max_blocks, int num_pages, float scale,
+                                void *out, void *ws, int32_t *dev_err);
+// The kernels of prefill_local.cu (launched by launch_prefill_attn).
+int prefill_local_tiles(int n_q);
+// TMA map of a K or V cache [P][H][32][128] bf16 as a 3-D tensor (dim, token, page * H + head)
+// read in boxes of 64 dims x 32 tokens with the 128-byte swizzle.
+bool prefill_kv_tensor_map(CUtensorMap *map, const void *cache, int num_pages, int H);
+cudaError_t launch_prefill_classify(const LaunchCtx &c, const int32_t *sel, const int32_t *q_pos,
+                                    const int32_t *seq_len_ptr, int n_q, int max_blocks, int32_t *sel_ws,
+                                    int32_t *counts, int32_t *loc_info, int2 *tile_info, int32_t *dev_err);
+cudaError_t launch_prefill_local(const LaunchCtx &c, const void *q, const void *k, const void *v,
+                                 const int32_t *bt_row, const int32_t *q_pos, const int32_t *loc_info,
+                                 const int2 *tile_info, int n_q, int H, int num_pages, float scale, void *loc_o,
+                                 float2 *loc_ml, int32_t *dev_err);
+cudaError_t launch_prefill_merge(const LaunchCtx &c, const int32_t *sel_ws, const void *part_o, const float *part_ml,
+                                 const void *loc_o, const float2 *loc_ml, int n_q, int H, void *out);
 
 // Comparator decode attention over [0, min(ref_blocks, nb)) U the 4-block local window.
 int dense_chunks(int max_blocks);

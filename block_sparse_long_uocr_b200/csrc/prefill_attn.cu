@@ -1,18 +1,22 @@
-// prefill_attn.cu -- block-centric sparse attention for a prefill chunk.
+// prefill_attn.cu -- block-centric sparse attention for a prefill chunk: the
+// entries that the local-window kernel (prefill_local.cu) does not take.
 //
 // Same arithmetic as sparse_attn.cu (Unlimited-OCR-2 walk-through,
 // news.rkmt.cn/news/25027, section 五 step 4: exact softmax attention of each
-// query over its 16 selected 32-token blocks), organised for many queries of
-// one sequence.  Query-by-query gathering would read every selected (block,
-// head) tile once per query that picked it -- ~16 times per tile on average in
-// a 2048-query chunk, and ~130 times for the local-window blocks that 32
-// consecutive queries share.  Instead:
-//   1. invert the selection: per logical block, the list of (query, slot)
-//      entries that selected it (the top-k kernel counts them; one kernel
-//      places the lists by the prefix sums of the counts, writes them and cuts
-//      them into items of 16 entries);
-//   2. one warp per (item, head) computes the item's 16 x 32 score tile
-//      S = Q K^T and, after a register-resident fp32 softmax per row, the
+// query over its selected 32-token blocks), organised for many queries of one
+// sequence.  Query-by-query gathering would read every selected (block, head)
+// tile once per query that picked it -- ~12 times per remote tile on average in
+// a 2048-query chunk.  Instead:
+//   1. the selection is classified per 128-query tile (prefill_local.cu): the
+//      local-window entries of tiles whose windows fit one 8-block window go
+//      to the tensor-core local kernel, which runs beside the inversion; every
+//      other entry (the 12 remote blocks of a query, and all entries of other
+//      tiles) stays here, counted per block;
+//   2. the inversion: per logical block, the list of (query, slot) entries
+//      that selected it (one kernel places the lists by the prefix sums of the
+//      counts, writes them and cuts them into items of 16 entries);
+//   3. one warp per (item, head) unit computes the item's 16 x 32 score
+//      tile S = Q K^T and, after a register-resident fp32 softmax per row, the
 //      16 x 128 tile P V on the tensor cores (mma.sync m16n8k16, bf16 in, fp32
 //      accumulate), writing each entry's partial state: the row maximum m and
 //      the weight sum l in fp32, and the unnormalised output acc = sum_t
@@ -21,25 +25,26 @@
 //      most 2^-9 max|v| to the result after the merge divides by the summed
 //      weights, the size of the output's own bf16 rounding, and halves the
 //      partials' traffic);
-//   3. one warp per (query, head) merges the 16 partials: out = sum_k
-//      2^(m_k - M) acc_k / sum_k 2^(m_k - M) l_k, written in bf16.
+//   4. the merge kernel (prefill_local.cu) combines each (query, head)'s
+//      partials, its local window's included: out = sum_k 2^(m_k - M) acc_k /
+//      sum_k 2^(m_k - M) l_k.
 // Each (block, head) tile is read from memory about once per chunk (an item after
-// the first of the same tile runs beside it and finds it in L2; the DRAM reads come
-// to ~6 % above the selected tiles, queries and item records).
+// the first of the same tile runs beside it and finds it in L2).
 //
-// Tensor-core layout of step 2.  The contraction index of S = Q K^T is the head
+// Tensor-core layout of step 3.  The contraction index of S = Q K^T is the head
 // dimension, and any permutation of it applied to both operands leaves S
 // unchanged; this kernel assigns lane (r, t) = (lane / 4, lane % 4) the dims
 // 32u + 8t .. 32u + 8t + 7 for the k-steps 2u and 2u + 1, so that every A (query)
-// and B (key) fragment is one 16-byte load of a row: no shared memory and no
-// shuffles for S.  P V needs V transposed: the warp copies its V tile into shared
-// memory with cp.async, 16-byte chunk c of token x at chunk position c ^ (x & 7),
-// and ldmatrix.trans reads it without bank conflicts.  P is rounded to bf16 for
-// the tensor cores and the row sum l is taken over the rounded weights, so the
-// output is an exact convex combination of the values.  A (block, head) item
-// holds 16 entries -- a remote block is chosen by ~12 queries of a chunk on
-// average -- which is below the 64-row minimum tile of tcgen05; the work is
-// bound by the HBM reads of the tiles and the partials, not by tensor math.
+// and B (key) fragment is one 16-byte load of a row: no shuffles for S.  P V
+// needs V transposed: the warp copies its V tile into shared memory with
+// cp.async, 16-byte chunk c of token x at chunk position c ^ (x & 7), and
+// ldmatrix.trans reads it without bank conflicts.  P is rounded to bf16 for the
+// tensor cores and the row sum l is taken over the rounded weights, so the
+// output is an exact convex combination of the values (the normalised weights
+// move by at most ~2^-8 of their size, the output by ~2^-9 times the range of
+// the values).  An item holds at most 16 entries -- a remote block is chosen by
+// ~12 queries of a chunk on average -- below the 64-row minimum tile of
+// tcgen05, so these products stay on the warp-level tensor-core instructions.
 #include <cuda_bf16.h>
 #include <math.h>
 
@@ -54,9 +59,8 @@ constexpr int kInvPerThread = 8;
 constexpr int kInvTile = kInvThreads * kInvPerThread;   // blocks per prefix-sum tile of the inversion
 constexpr int kInvEntries = 4;   // selection entries per thread of the inversion (each CTA recomputes
                                  // the prefix sums, so fewer CTAs re-read fewer counts)
-constexpr int kMmaWarps = 2;
 constexpr int kItemRows = 16;
-constexpr int kMergeWarps = 8;
+constexpr int kMmaWarps = 2;
 
 __device__ __forceinline__ void cp_async16(uint32_t dst, const void *src) {
     asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst), "l"(src) : "memory");
@@ -73,10 +77,6 @@ __device__ __forceinline__ uint64_t l2_evict_last() {
     asm volatile("createpolicy.fractional.L2::evict_last.b64 %0, 1.0;" : "=l"(p));
     return p;
 }
-__device__ __forceinline__ void cp_async16_pol(uint32_t dst, const void *src, uint64_t pol) {
-    asm volatile("cp.async.cg.shared.global.L2::cache_hint [%0], [%1], 16, %2;" ::"r"(dst), "l"(src), "l"(pol)
-                 : "memory");
-}
 __device__ __forceinline__ void st_u32_pol(uint32_t *p, uint32_t v, uint64_t pol) {
     asm volatile("st.global.L2::cache_hint.b32 [%0], %1, %2;" ::"l"(p), "r"(v), "l"(pol) : "memory");
 }
@@ -84,9 +84,9 @@ __device__ __forceinline__ void st_f2_pol(float *p, float a, float b, uint64_t p
     asm volatile("st.global.L2::cache_hint.v2.f32 [%0], {%1, %2}, %3;" ::"l"(p), "f"(a), "f"(b), "l"(pol)
                  : "memory");
 }
-// Drops a 128-byte line from L2 without writing it back (its contents become undefined).
-__device__ __forceinline__ void l2_discard_line(const void *p) {
-    asm volatile("discard.global.L2 [%0], 128;" ::"l"(p) : "memory");
+__device__ __forceinline__ void cp_async16_pol(uint32_t dst, const void *src, uint64_t pol) {
+    asm volatile("cp.async.cg.shared.global.L2::cache_hint [%0], [%1], 16, %2;" ::"r"(dst), "l"(src), "l"(pol)
+                 : "memory");
 }
 __device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
 __device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_group 0;" ::: "memory"); }
@@ -117,33 +117,6 @@ __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi, float &sum) {
 }
 }  // namespace
 
-// A caller's selection for many queries of one sequence (uocr_sparse_attn_seq): sel_ws keeps
-// the slots that name a causal block of a query at a valid position (0 <= j < p / 32 + 1,
-// 0 <= p < seq_len) and -1 elsewhere, flagging UOCR_DEVERR_SEL / UOCR_DEVERR_POS as
-// sparse_attn does; counts[j] += 1 for every kept slot.
-__global__ void __launch_bounds__(kInvThreads)
-prefill_select_count_kernel(const int32_t *__restrict__ sel, const int32_t *__restrict__ q_pos,
-                            const int32_t *__restrict__ seq_len_ptr, int n_entries, int max_blocks,
-                            int32_t *__restrict__ sel_ws, int32_t *counts, int32_t *dev_err) {
-    pdl_wait();
-    const int e = blockIdx.x * kInvThreads + threadIdx.x;
-    if (e >= n_entries) return;
-    const int seq_len = min(__ldg(seq_len_ptr), max_blocks * kBlock);
-    const int p = __ldg(q_pos + e / kSel);
-    int j = __ldg(sel + e);
-    if (p < 0 || p >= seq_len) {
-        if ((e & (kSel - 1)) == 0) flag_error(dev_err, UOCR_DEVERR_POS);
-        j = -1;
-    } else if (j >= p / kBlock + 1) {
-        flag_error(dev_err, UOCR_DEVERR_SEL);
-        j = -1;
-    } else if (j < 0) {
-        j = -1;
-    }
-    sel_ws[e] = j;
-    if (j >= 0) atomicAdd(counts + j, 1);
-}
-
 // The selection inverted in one grid: CTA b places the entries e in [1024 b, 1024 b + 1024) in the
 // per-block lists, grouped by block ({entry = query * 16 + slot, position of the query}), and
 // writes the work items of the blocks j with j % gridDim.x == b: block j with n_j entries gives
@@ -158,7 +131,10 @@ prefill_invert_kernel(const int32_t *counts, const int32_t *__restrict__ bt_row,
                       int4 *__restrict__ items, int32_t *__restrict__ n_items, int2 *__restrict__ list) {
     __shared__ int s_c[kInvTile], s_g[kInvTile];   // exclusive prefixes (entries, items) inside the tile
     __shared__ int s_wc[kInvThreads / 32], s_wg[kInvThreads / 32];
-    pdl_wait();
+    // Launched after the local-window kernel, whose CTAs let this grid start once they are past
+    // their own wait for the classification: the counts and the classified selection are complete
+    // here (read through L2).  The wait at the end makes this grid complete only after the local
+    // kernel, so that the block kernel, which waits for this grid, starts after both.
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     // this thread's entries (kInvEntries, kInvThreads apart), loaded before the scan so that the
     // loads overlap it
@@ -169,7 +145,7 @@ prefill_invert_kernel(const int32_t *counts, const int32_t *__restrict__ bt_row,
         ej[k] = -1;
         ep[k] = 0;
         if (e < n_entries) {   // both loads in flight together
-            ej[k] = sel[e];
+            ej[k] = __ldcg(sel + e);
             ep[k] = __ldg(q_pos + e / kSel);
             if (ej[k] >= max_blocks) ej[k] = -1;
         }
@@ -188,7 +164,7 @@ prefill_invert_kernel(const int32_t *counts, const int32_t *__restrict__ bt_row,
 #pragma unroll
         for (int k = 0; k < kInvPerThread; ++k) {
             const int jb = t0 + kInvPerThread * tid + k;
-            c[k] = jb < max_blocks ? counts[jb] : 0;
+            c[k] = jb < max_blocks ? __ldcg(counts + jb) : 0;
             sc += c[k];
             sg += (c[k] + kItemRows - 1) / kItemRows;
         }
@@ -247,6 +223,7 @@ prefill_invert_kernel(const int32_t *counts, const int32_t *__restrict__ bt_row,
         __syncthreads();   // the next tile reuses s_c, s_g, s_wc, s_wg
     }
     if (blockIdx.x == 0 && tid == 0) *n_items = base_g;
+    pdl_wait();
 }
 
 // One unit of work: (item, head) and the item's record and entries.
@@ -303,6 +280,8 @@ prefill_block_mma_kernel(const uint4 *__restrict__ q, const uint4 *__restrict__ 
 
     const uint64_t pol_kv = l2_evict_first(), pol_part = l2_evict_last();
     pdl_wait();
+    // the merge kernel may start its prologue; it waits for this grid before reading the partials
+    pdl_launch_dependents();
     const int n_work = __ldg(n_items) * H;
     const int stride = gridDim.x * kMmaWarps;
 
@@ -473,58 +452,6 @@ prefill_block_mma_kernel(const uint4 *__restrict__ q, const uint4 *__restrict__ 
     cp_async_wait_all();
 }
 
-// One warp per (query, head): lanes 0..15 hold the 16 slots' (m, l), every lane 4 output dims.
-__global__ void __launch_bounds__(kMergeWarps * 32)
-prefill_merge_kernel(const int32_t *__restrict__ sel, const __nv_bfloat16 *__restrict__ part_o,
-                     const float *__restrict__ part_ml, int n_q, int H, __nv_bfloat16 *__restrict__ out) {
-    const int lane = threadIdx.x & 31;
-    const long long ih = (long long)blockIdx.x * kMergeWarps + (threadIdx.x >> 5);
-    pdl_wait();
-    if (ih >= (long long)n_q * H) return;
-    const long long i = ih / H;
-    const int s = lane & 15;
-    const size_t base = (size_t)ih * kSel;
-    const bool valid = __ldg(sel + i * kSel + s) >= 0;
-    const float m = valid ? __ldcs(part_ml + (base + s) * 2) : -INFINITY;
-    const float l = valid ? __ldcs(part_ml + (base + s) * 2 + 1) : 0.f;
-    const unsigned vmask = __ballot_sync(0xffffffffu, valid);
-    uint2 v[kSel];
-#pragma unroll
-    for (int k = 0; k < kSel; ++k)
-        v[k] = (vmask >> k & 1u) ? __ldcs(reinterpret_cast<const uint2 *>(part_o + (base + k) * kD) + lane)
-                                 : make_uint2(0u, 0u);
-    float M = m;
-#pragma unroll
-    for (int x = 8; x > 0; x >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, x));
-    // partial k holds sum_t 2^(z_t - m_k) v_t and l_k = sum_t 2^(z_t - m_k): rescale both to M
-    const float w = M == -INFINITY ? 0.f : exp2f(m - M);
-    float W = l * w;
-#pragma unroll
-    for (int x = 8; x > 0; x >>= 1) W += __shfl_xor_sync(0xffffffffu, W, x);
-    float A[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-    for (int k = 0; k < kSel; ++k) {
-        const float wk = __shfl_sync(0xffffffffu, w, k);
-        A[0] = fmaf(wk, __uint_as_float(v[k].x << 16), A[0]);
-        A[1] = fmaf(wk, __uint_as_float(v[k].x & 0xffff0000u), A[1]);
-        A[2] = fmaf(wk, __uint_as_float(v[k].y << 16), A[2]);
-        A[3] = fmaf(wk, __uint_as_float(v[k].y & 0xffff0000u), A[3]);
-    }
-    // Every lane has its loads' values: drop this (query, head)'s partial lines from L2 (its 16
-    // x 256 bytes of outputs are 32 lines, one per lane, and its 16 (m, l) pairs one line), so
-    // that they are never written back.  The block kernel writes every slot the merge reads
-    // within the same call, before the merge starts.
-    __syncwarp();
-    l2_discard_line(part_o + base * kD + 64 * lane);
-    if (lane == 0) l2_discard_line(part_ml + base * 2);
-    const float inv = W > 0.f ? 1.f / W : 0.f;
-    float unused = 0.f;
-    uint2 pk;
-    pk.x = pack_bf16(A[0] * inv, A[1] * inv, unused);
-    pk.y = pack_bf16(A[2] * inv, A[3] * inv, unused);
-    reinterpret_cast<uint2 *>(out + (size_t)ih * kD)[lane] = pk;
-}
-
 // ------------------------------------------------------------------ host side
 namespace {
 // Items of 16 entries: at most one partly filled item per block that was selected at all.
@@ -551,51 +478,53 @@ size_t prefill_attn_workspace(int n_q, int H, int max_blocks, PrefillAttnWs *w) 
     off += up(item_bound(n_q, max_blocks) * sizeof(int4));
     l.list_off = off;
     off += up((size_t)n_q * kSel * sizeof(int2));
-    l.sel_off = off;
+    l.sel_off = off;     // the block kernel's entries of the selection (classified)
     off += up((size_t)n_q * kSel * 4);
+    l.loc_off = off;     // per query: the local blocks the tensor-core local kernel attends
+    off += up((size_t)n_q * 4);
+    l.tile_off = off;    // per 128-query tile: its local window {first block, blocks}
+    off += up((size_t)prefill_local_tiles(n_q) * sizeof(int2));
     l.ml_off = off;
     off += up((size_t)n_q * H * kSel * 2 * 4);
     l.o_off = off;
     off += up((size_t)n_q * H * kSel * kD * 2);
+    l.loc_ml_off = off;   // the local window's (m, l) per (query, head)
+    off += up((size_t)n_q * H * sizeof(float2));
+    l.loc_o_off = off;    // the local window's unnormalised output per (query, head), bf16
+    off += up((size_t)n_q * H * kD * 2);
     if (w) *w = l;
     return off;
 }
 
-cudaError_t launch_prefill_select_count(const LaunchCtx &c, const int32_t *sel, const int32_t *q_pos,
-                                       const int32_t *seq_len_ptr, int n_q, int max_blocks, void *ws,
-                                       int32_t *dev_err) {
-    PrefillAttnWs w;
-    prefill_attn_workspace(n_q, 1, max_blocks, &w);   // the regions before the partials do not depend on H
-    char *base = (char *)ws;
-    const int n_entries = n_q * kSel;
-    cudaLaunchAttribute attr[1];
-    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-    attr[0].val.programmaticStreamSerializationAllowed = 1;
-    cudaLaunchConfig_t cfg = {};
-    cfg.stream = c.stream;
-    cfg.attrs = attr;
-    cfg.numAttrs = c.pdl ? 1 : 0;
-    cfg.gridDim = dim3((unsigned)((n_entries + kInvThreads - 1) / kInvThreads));
-    cfg.blockDim = dim3(kInvThreads);
-    return cudaLaunchKernelEx(&cfg, prefill_select_count_kernel, sel, q_pos, seq_len_ptr, n_entries, max_blocks,
-                              (int32_t *)(base + w.sel_off), (int32_t *)(base + w.counts_off), dev_err);
-}
-
 cudaError_t launch_prefill_attn(const LaunchCtx &c, const void *q, const void *k, const void *v,
-                                const int32_t *bt_row, const int32_t *q_pos, const int32_t *sel, int n_q, int H,
-                                int max_blocks, int num_pages, float scale, void *out, void *ws,
-                                int32_t *dev_err) {
+                                const int32_t *bt_row, const int32_t *seq_len_ptr, const int32_t *q_pos,
+                                const int32_t *sel, int n_q, int H, int max_blocks, int num_pages, float scale,
+                                void *out, void *ws, int32_t *dev_err) {
     PrefillAttnWs w;
     prefill_attn_workspace(n_q, H, max_blocks, &w);
     char *base = (char *)ws;
-    const int32_t *counts = (const int32_t *)(base + w.counts_off);
+    int32_t *counts = (int32_t *)(base + w.counts_off);
     int32_t *fill = (int32_t *)(base + w.fill_off);
     int32_t *n_items = (int32_t *)(base + w.n_items_off);
     int4 *items = (int4 *)(base + w.items_off);
     int2 *list = (int2 *)(base + w.list_off);
+    int32_t *sel_ws = (int32_t *)(base + w.sel_off);
+    int32_t *loc = (int32_t *)(base + w.loc_off);
+    int2 *tiles = (int2 *)(base + w.tile_off);
     float *ml = (float *)(base + w.ml_off);
     __nv_bfloat16 *part_o = (__nv_bfloat16 *)(base + w.o_off);
     const int n_entries = n_q * kSel;
+
+    // classify the selection: local-window entries to the tensor-core kernel, the rest to the
+    // block kernel (after a preceding kernel of the same call, or a memset)
+    cudaError_t e = launch_prefill_classify(c, sel, q_pos, seq_len_ptr, n_q, max_blocks, sel_ws, counts, loc, tiles,
+                                            dev_err);
+    if (e != cudaSuccess) return e;
+    // the local windows on tcgen05, beside the inversion that follows
+    void *loc_o = base + w.loc_o_off;
+    float2 *loc_ml = (float2 *)(base + w.loc_ml_off);
+    e = launch_prefill_local(c, q, k, v, bt_row, q_pos, loc, tiles, n_q, H, num_pages, scale, loc_o, loc_ml, dev_err);
+    if (e != cudaSuccess) return e;
 
     cudaLaunchAttribute attr[1];
     attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
@@ -607,8 +536,8 @@ cudaError_t launch_prefill_attn(const LaunchCtx &c, const void *q, const void *k
 
     cfg.gridDim = dim3((unsigned)((n_entries + kInvThreads * kInvEntries - 1) / (kInvThreads * kInvEntries)));
     cfg.blockDim = dim3(kInvThreads);
-    cudaError_t e = cudaLaunchKernelEx(&cfg, prefill_invert_kernel, counts, bt_row, sel, q_pos, n_entries, max_blocks,
-                                       fill, items, n_items, list);
+    e = cudaLaunchKernelEx(&cfg, prefill_invert_kernel, (const int32_t *)counts, bt_row, (const int32_t *)sel_ws,
+                           q_pos, n_entries, max_blocks, fill, items, n_items, list);
     if (e != cudaSuccess) return e;
 
     int per_sm = 0;
@@ -620,12 +549,8 @@ cudaError_t launch_prefill_attn(const LaunchCtx &c, const void *q, const void *k
                            (const int2 *)list, (const int4 *)items, (const int32_t *)n_items, H, num_pages,
                            scale * kLog2e, part_o, ml, dev_err);
     if (e != cudaSuccess) return e;
-    const long long merge_ctas = ((long long)n_q * H + kMergeWarps - 1) / kMergeWarps;
-    if (merge_ctas > 0x7fffffffLL) return cudaErrorInvalidConfiguration;
-    cfg.gridDim = dim3((unsigned)merge_ctas);
-    cfg.blockDim = dim3(kMergeWarps * 32);
-    return cudaLaunchKernelEx(&cfg, prefill_merge_kernel, sel, (const __nv_bfloat16 *)part_o, (const float *)ml, n_q,
-                              H, (__nv_bfloat16 *)out);
+
+    return launch_prefill_merge(c, sel_ws, part_o, ml, loc_o, loc_ml, n_q, H, out);
 }
 
 }  // namespace uocr

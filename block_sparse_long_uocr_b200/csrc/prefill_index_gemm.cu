@@ -91,14 +91,8 @@ struct UnitInfo {
 // two so that a role issues the next unit's position loads (pos_prefetch: predicated loads into
 // registers, nothing consumes them yet) before working on the current unit, and reduces them
 // (unit_info) when it gets there: no role waits on L2 at a unit boundary.
-// A read-only load issued where it stands in the program: the volatile asm keeps the compiler
-// from sinking a prefetch down to its first use (a unit later), which would put the memory
-// latency back on the unit boundary.
-__device__ __forceinline__ int ld_pinned(const int32_t *p) {
-    int v;
-    asm volatile("ld.global.nc.b32 %0, [%1];" : "=r"(v) : "l"(p));
-    return v;
-}
+// (ld_pinned, common.cuh: the prefetches stay where they are issued, so the memory latency is not
+// put back on the unit boundary.)
 
 struct PosPrefetch {
     int raw[kBM * kMT / 32];   // position of row m0 + 32k + lane, -1 past the queries
@@ -284,7 +278,7 @@ prefill_index_gemm_kernel(const __grid_constant__ CUtensorMap map_q, const __gri
         // end marker below completes one more phase of a stage)
         if (lane == 0)
             for (int k = 0; k < kStagesA; ++k)
-                if (a_fills[k] > 0) mbar_wait_timed(&s.a_full[k], (a_fills[k] - 1) & 1, kWaitLimitNs, nullptr);
+                if (a_fills[k] > 0) mbar_drain(&s.a_full[k], (a_fills[k] - 1) & 1, dev_err);
         __syncwarp();
         // end marker for every other role: a stage that holds no unit
         if (!aborted(s)) {
@@ -334,7 +328,7 @@ prefill_index_gemm_kernel(const __grid_constant__ CUtensorMap map_q, const __gri
         }
         if (lane == 0)
             for (int k = 0; k < kStagesB; ++k)
-                if (b_fills[k] > 0) mbar_wait_timed(&s.b_full[k], (b_fills[k] - 1) & 1, kWaitLimitNs, nullptr);
+                if (b_fills[k] > 0) mbar_drain(&s.b_full[k], (b_fills[k] - 1) & 1, dev_err);
     } else if (warp == kMmaWarp || warp == kMmaWarp1) {
         // ------------------------------------------------------------ MMA issuers, one per subtile
         // Two issuing threads: while one waits on a barrier or commits, the other's MMAs keep
@@ -401,7 +395,7 @@ prefill_index_gemm_kernel(const __grid_constant__ CUtensorMap map_q, const __gri
         // drain: every MMA this thread issued has completed before TMEM is freed
         if (lane == 0 && issued) {
             tc::commit(&s.mma_done[m]);
-            mbar_wait_timed(&s.mma_done[m], 0, kWaitLimitNs, nullptr);
+            mbar_drain(&s.mma_done[m], 0, dev_err);
         }
         __syncwarp();
     } else {
@@ -505,13 +499,7 @@ prefill_index_gemm_kernel(const __grid_constant__ CUtensorMap map_q, const __gri
 }
 
 // ---------------------------------------------------------------- host side
-namespace {
-
-typedef CUresult (*EncodeTiledFn)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *, const cuuint64_t *,
-                                  const cuuint64_t *, const cuuint32_t *, const cuuint32_t *, CUtensorMapInterleave,
-                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
-
-EncodeTiledFn get_encode() {
+EncodeTiledFn tensor_map_encoder() {
     void *p = nullptr;
     cudaDriverEntryPointQueryResult q;
     if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) != cudaSuccess ||
@@ -520,9 +508,11 @@ EncodeTiledFn get_encode() {
     return reinterpret_cast<EncodeTiledFn>(p);
 }
 
+namespace {
+
 // 2-D bf16 tensor of `rows` x 128 (row stride 256 B), boxes of 64 x box_rows, 128-byte swizzle.
 bool make_map(CUtensorMap *m, const void *base, uint64_t rows, uint32_t box_rows) {
-    EncodeTiledFn enc = get_encode();
+    EncodeTiledFn enc = tensor_map_encoder();
     if (!enc) return false;
     const cuuint64_t dims[2] = {128, rows};
     const cuuint64_t strides[1] = {256};

@@ -107,6 +107,13 @@ const char *uocr_status_string(uocr_status_t status);
 int uocr_abi_version(void);
 
 /*
+ * The CUDA runtime's description of the error behind the calling thread's
+ * most recent UOCR_ERR_CUDA ("no error" if there was none): which launch or
+ * attribute call failed and why.  Static storage; never NULL.
+ */
+const char *uocr_last_cuda_error(void);
+
+/*
  * Workspace bytes that uocr_sparse_decode and uocr_sparse_prefill need for n_q queries over
  * max_blocks blocks: the fp32 block scores [n_q][max_blocks], rounded up to
  * 256 bytes.  A pure function of the shapes (0 for a non-positive argument);

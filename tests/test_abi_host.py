@@ -56,6 +56,11 @@ def test_status_strings_and_version(pkg):
     assert pkg.lib.uocr_abi_version() == 2
 
 
+def test_last_cuda_error_names_no_error_before_any_failure(pkg):
+    # host-side rejections return before any CUDA call, so they leave no CUDA error behind
+    assert pkg.lib.uocr_last_cuda_error().decode() == "no error"
+
+
 def test_workspace_is_a_pure_function_of_shapes(pkg):
     ws = pkg.workspace_bytes
     assert ws(0, 10, 64) == 0 and ws(4, 0, 64) == 0 and ws(4, 10, 0) == 0

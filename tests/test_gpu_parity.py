@@ -24,11 +24,14 @@ def uocr(cuda_device):
 
 
 def run_decode(uocr, case, layer=0, scores=True):
+    """The decode call on one layer of a valid case; a clean call sets no device error bit."""
     q, qi = case.q_layers[layer]
     kp, vp, ikp = case.layers[layer]
+    err = torch.zeros(1, dtype=torch.int32, device=q.device)
     sc = uocr.index_score(qi, ikp, case.block_table, case.seq_lens) if scores else None
-    out, sel = uocr.sparse_decode(q, kp, vp, qi, ikp, case.block_table, case.seq_lens)
+    out, sel = uocr.sparse_decode(q, kp, vp, qi, ikp, case.block_table, case.seq_lens, dev_err=err)
     torch.cuda.synchronize()
+    assert int(err.item()) == 0
     return out, sel, sc
 
 

@@ -61,10 +61,15 @@ def test_prefill_scores_agree_with_the_scan_kernel(uocr, cuda_device):
 
 
 def test_sparse_prefill_matches_oracle(uocr, cuda_device):
+    """Tiles of consecutive positions (local windows on the tensor-core kernel) and a tile with
+    scattered positions (its local entries on the block kernel); no device error on a clean call
+    (a drain or pipeline wait that ran out would set UOCR_DEVERR_TIMEOUT)."""
     case = _prefill_case(4096, 300, (0, 31, 100, 511, 512, 513), seed=5, device=cuda_device)
+    err = torch.zeros(1, dtype=torch.int32, device=cuda_device)
     out, sel = uocr.sparse_prefill(case.q, case.k_pool, case.v_pool, case.idx_q, case.idx_k_pool, case.block_table,
-                                   case.seq_lens, 0, case.q_pos)
+                                   case.seq_lens, 0, case.q_pos, dev_err=err)
     torch.cuda.synchronize()
+    assert int(err.item()) == 0
     check_queries(case, range(case.n_q), out, sel)
 
 
@@ -177,11 +182,13 @@ def test_sparse_attn_seq_matches_oracle(uocr, cuda_device):
     case = _prefill_case(32 * 90 + 11, 333, (0, 5, 31, 32, 700), seed=31, device=cuda_device)
     sel = _random_selection(case, 31)
     sel_d = torch.from_numpy(sel).to(cuda_device)
+    err = torch.zeros(1, dtype=torch.int32, device=cuda_device)
     out = uocr.sparse_attn_seq(case.q, case.k_pool, case.v_pool, case.block_table, case.seq_lens, 0, case.q_pos,
-                               sel_d)
+                               sel_d, dev_err=err)
     ref_q = uocr.sparse_attn(case.q, case.k_pool, case.v_pool, case.block_table, case.seq_lens, sel_d,
                              case.q_seq, case.q_pos)
     torch.cuda.synchronize()
+    assert int(err.item()) == 0
     got = out.float().cpu().numpy()
     for i in range(case.n_q):
         ref = oracle_attend(case, i, sel[i])
@@ -217,6 +224,24 @@ def test_sparse_attn_seq_reuses_one_workspace(uocr, cuda_device):
             assert d.max() <= OUT_MAX_ATOL and d.mean() <= OUT_MEAN_ATOL, f"query {i}"
 
 
+@pytest.mark.parametrize("heads", [1, 3])
+def test_sparse_attn_seq_odd_head_counts(uocr, cuda_device, heads):
+    """Head counts for which a head-parity split of the block kernel's work would hand consecutive
+    uses of a ring stage to different producers: every output against the oracle, no device error
+    (a pipeline wait that passed on an older phase would show as wrong outputs or a timeout)."""
+    case = _prefill_case(32 * 300, 1200, seed=51 + heads, device=cuda_device, heads=heads)
+    sel = _random_selection(case, 51 + heads, empty_frac=0.0)
+    err = torch.zeros(1, dtype=torch.int32, device=cuda_device)
+    out = uocr.sparse_attn_seq(case.q, case.k_pool, case.v_pool, case.block_table, case.seq_lens, 0, case.q_pos,
+                               torch.from_numpy(sel).to(cuda_device), dev_err=err)
+    torch.cuda.synchronize()
+    assert int(err.item()) == 0
+    got = out.float().cpu().numpy()
+    for i in range(case.n_q):
+        d = np.abs(got[i] - oracle_attend(case, i, sel[i]))
+        assert d.max() <= OUT_MAX_ATOL and d.mean() <= OUT_MEAN_ATOL, f"query {i}"
+
+
 def test_sparse_attn_seq_flags_bad_selections(uocr, cuda_device):
     case = _prefill_case(32 * 40, 64, seed=32, device=cuda_device, heads=3)
     sel = _random_selection(case, 32, empty_frac=0.0)
@@ -228,6 +253,7 @@ def test_sparse_attn_seq_flags_bad_selections(uocr, cuda_device):
                                torch.from_numpy(sel).to(cuda_device), dev_err=err)
     torch.cuda.synchronize()
     assert int(err.item()) & uocr.DEVERR_SEL and int(err.item()) & uocr.DEVERR_POS
+    assert not int(err.item()) & uocr.DEVERR_TIMEOUT
     got = out.float().cpu().numpy()
     assert np.isfinite(got).all() and (got[7] == 0).all()
     s5 = sel[5].copy()
@@ -243,8 +269,10 @@ def test_chunked_prefill_workload_every_query(uocr, cuda_device):
     tensor-core block score, every selection and every output against the oracle."""
     case = workloads.chunked_prefill(device=cuda_device)
     ws = uocr.alloc_prefill_workspace(case.n_q, 10, case.max_blocks, cuda_device)
+    err = torch.zeros(1, dtype=torch.int32, device=cuda_device)
     out, sel = uocr.sparse_prefill(case.q, case.k_pool, case.v_pool, case.idx_q, case.idx_k_pool, case.block_table,
-                                   case.seq_lens, 0, case.q_pos, workspace=ws)
+                                   case.seq_lens, 0, case.q_pos, workspace=ws, dev_err=err)
     torch.cuda.synchronize()
+    assert int(err.item()) == 0
     scores = ws[: case.n_q * case.max_blocks * 4].view(torch.float32).view(case.n_q, case.max_blocks)
     check_all_queries(case, out, sel, scores)
