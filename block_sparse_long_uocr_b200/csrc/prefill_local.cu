@@ -119,6 +119,14 @@ __device__ __forceinline__ void fence_proxy_async_smem() {
     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 }
 
+// 2^x by the hardware's approximate exponential instruction (its error is far below the bf16
+// rounding of the weights that follows; inputs are <= 0 here, and very negative ones give 0).
+__device__ __forceinline__ float ex2_approx(float x) {
+    float y;
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
+
 __device__ __forceinline__ uint32_t pack2_bf16(float lo, float hi, float &sum) {
     const __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
     sum += __low2float(v) + __high2float(v);
@@ -375,7 +383,8 @@ prefill_local_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_con
 #pragma unroll
                 for (int b2 = 0; b2 < kMaxWinBlocks / 2; ++b2)
                     if (__any_sync(0xffffffffu, in_row(2 * b2 + hh))) need |= 1u << b2;
-                // pass 1: the maximum of z = scale * log2(e) * s over the row's visible tokens
+                // pass 1: the maximum of z = scale * log2(e) * s over the row's visible tokens (the
+                // causal test only on the block that holds the row's position)
 #pragma unroll
                 for (int b2 = 0; b2 < kMaxWinBlocks / 2; ++b2) {
                     if (!((need >> b2) & 1)) continue;
@@ -385,9 +394,24 @@ prefill_local_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_con
                     tc::tmem_ld_wait();
                     if (in_row(b)) {
                         const int t0 = (kb0 + b) * kBlock;
+                        float bm = -INFINITY;
+                        if (t0 + kBlock - 1 <= p) {
 #pragma unroll
-                        for (int c = 0; c < 32; ++c)
-                            if (t0 + c <= p) mh = fmaxf(mh, v[c] * scale_log2);
+                            for (int c = 0; c < 32; ++c) bm = fmaxf(bm, v[c]);
+                        } else {
+#pragma unroll
+                            for (int c = 0; c < 32; ++c)
+                                if (t0 + c <= p) bm = fmaxf(bm, v[c]);
+                        }
+                        // scale * log2(e) may be negative (a caller's scale): the extreme of s that
+                        // maximises z
+                        if (scale_log2 < 0.f) {
+                            bm = INFINITY;
+#pragma unroll
+                            for (int c = 0; c < 32; ++c)
+                                if (t0 + c <= p) bm = fminf(bm, v[c]);
+                        }
+                        mh = fmaxf(mh, bm * scale_log2);
                     }
                 }
             }
@@ -409,11 +433,20 @@ prefill_local_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_con
                         tc::tmem_ld_wait();
                         if (in_row(b)) {
                             const int t0 = (kb0 + b) * kBlock;
+                            const float nm = -m;
+                            if (t0 + kBlock - 1 <= p) {
 #pragma unroll
-                            for (int c = 0; c < 16; ++c) {
-                                const float e0 = t0 + 2 * c <= p ? exp2f(v[2 * c] * scale_log2 - m) : 0.f;
-                                const float e1 = t0 + 2 * c + 1 <= p ? exp2f(v[2 * c + 1] * scale_log2 - m) : 0.f;
-                                pk[c] = pack2_bf16(e0, e1, lh);
+                                for (int c = 0; c < 16; ++c)
+                                    pk[c] = pack2_bf16(ex2_approx(fmaf(v[2 * c], scale_log2, nm)),
+                                                       ex2_approx(fmaf(v[2 * c + 1], scale_log2, nm)), lh);
+                            } else {
+#pragma unroll
+                                for (int c = 0; c < 16; ++c) {
+                                    const float e0 = t0 + 2 * c <= p ? ex2_approx(fmaf(v[2 * c], scale_log2, nm)) : 0.f;
+                                    const float e1 =
+                                        t0 + 2 * c + 1 <= p ? ex2_approx(fmaf(v[2 * c + 1], scale_log2, nm)) : 0.f;
+                                    pk[c] = pack2_bf16(e0, e1, lh);
+                                }
                             }
                         }
                     }
