@@ -63,11 +63,11 @@ EncodeTiledFn tensor_map_encoder();
 // the tensor-core local kernel, the rest to the block kernel), the block kernel's entries are
 // inverted per block and attended in items of 16 entries per (block, head), and a merge kernel
 // combines each row's partial states.  Workspace regions, 256-byte aligned.  The first zero_bytes
-// bytes (per-block entry counts, list counters, the scoring GEMM's unit counter) must be zero
-// before the call's first kernel.
+// bytes (per-block entry counts, list counters, the scoring GEMM's and the block kernel's unit
+// counters) must be zero before the call's first kernel.
 struct PrefillAttnWs {
-    size_t counts_off, fill_off, sched_off, n_items_off, items_off, list_off, sel_off, loc_off, tile_off, ml_off,
-        o_off, loc_ml_off, loc_o_off;
+    size_t counts_off, fill_off, sched_off, blk_sched_off, n_items_off, items_off, list_off, sel_off, loc_off,
+        tile_off, ml_off, o_off, loc_ml_off, loc_o_off;
     size_t zero_bytes;
 };
 size_t prefill_attn_workspace(int n_q, int H, int max_blocks, PrefillAttnWs *w);

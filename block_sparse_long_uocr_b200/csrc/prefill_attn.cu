@@ -9,9 +9,9 @@
 // a 2048-query chunk.  Instead:
 //   1. the selection is classified per 128-query tile (prefill_local.cu): the
 //      local-window entries of tiles whose windows fit one 8-block window go
-//      to the tensor-core local kernel, which runs beside the inversion; every
-//      other entry (the 12 remote blocks of a query, and all entries of other
-//      tiles) stays here, counted per block;
+//      to the tensor-core local kernel, which runs on a quarter of the SMs
+//      beside step 3; every other entry (the 12 remote blocks of a query, and
+//      all entries of other tiles) stays here, counted per block;
 //   2. the inversion: per logical block, the list of (query, slot) entries
 //      that selected it (one kernel places the lists by the prefix sums of the
 //      counts, writes them and cuts them into items of 16 entries);
@@ -131,10 +131,11 @@ prefill_invert_kernel(const int32_t *counts, const int32_t *__restrict__ bt_row,
                       int4 *__restrict__ items, int32_t *__restrict__ n_items, int2 *__restrict__ list) {
     __shared__ int s_c[kInvTile], s_g[kInvTile];   // exclusive prefixes (entries, items) inside the tile
     __shared__ int s_wc[kInvThreads / 32], s_wg[kInvThreads / 32];
-    // Launched after the local-window kernel, whose CTAs let this grid start once they are past
-    // their own wait for the classification: the counts and the classified selection are complete
-    // here (read through L2).  The wait at the end makes this grid complete only after the local
-    // kernel, so that the block kernel, which waits for this grid, starts after both.
+    // The counts and the classified selection come from the classification, the preceding kernel.
+    // Once every CTA is past that wait, the local-window kernel may start; it waits for this grid
+    // before anything else.
+    pdl_wait();
+    pdl_launch_dependents();
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     // this thread's entries (kInvEntries, kInvThreads apart), loaded before the scan so that the
     // loads overlap it
@@ -223,7 +224,6 @@ prefill_invert_kernel(const int32_t *counts, const int32_t *__restrict__ bt_row,
         __syncthreads();   // the next tile reuses s_c, s_g, s_wc, s_wg
     }
     if (blockIdx.x == 0 && tid == 0) *n_items = base_g;
-    pdl_wait();
 }
 
 // One unit of work: (item, head) and the item's record and entries.
@@ -242,14 +242,15 @@ __device__ __forceinline__ Unit load_unit(int w, int n_work, int H, const int4 *
         u.ea = u.eb = make_int2(0, 0);
         return u;
     }
-    const int4 rec = __ldg(items + w / H);
+    // written by the inversion earlier in the same call, read through L2
+    const int4 rec = __ldcg(items + w / H);
     u.j = rec.x;
     u.page = rec.y;
     u.rows = rec.w;
     u.h = w % H;
     // rows past the item's end repeat its last entry and store nothing
-    u.ea = __ldg(list + rec.z + min(r, rec.w - 1));
-    u.eb = __ldg(list + rec.z + min(r + 8, rec.w - 1));
+    u.ea = __ldcg(list + rec.z + min(r, rec.w - 1));
+    u.eb = __ldcg(list + rec.z + min(r + 8, rec.w - 1));
     return u;
 }
 
@@ -262,16 +263,25 @@ struct WarpStage {
     uint4 q[kItemRows * kD / 8];
 };
 
-// Persistent: warp w takes units w, w + (warps in the grid), ...; unit = (item, head), heads
-// innermost so that the items of one block run side by side.  Each warp pipelines its units:
-// the next unit's Q and K copies start once this unit's scores are computed, its V copy once
-// this unit's P V is done, so every copy overlaps the math of the unit before it
+// Persistent: each warp takes its units, unit = (item, head), in order from a counter (sched,
+// zero before the call), one unit ahead of the one it computes; heads are innermost so that the
+// items of one block run side by side.  The counter lets the CTAs that start late (beside the
+// local-window kernel, which holds most of a few SMs' shared memory) take fewer units.  Each warp
+// pipelines its units: the next unit's Q and K copies start once this unit's scores are computed,
+// its V copy once this unit's P V is done, so every copy overlaps the math of the unit before it
 // (cp.async groups, waited for with wait_group 1).
+//
+// Launched after the local-window kernel, whose CTAs let this grid start once they are past their
+// own wait for the inversion: the lists and items are complete here (read through L2), and this
+// grid does not wait for the local kernel before its work.  One thread waits for it at the end, so
+// that this grid completes only after the local kernel and the merge, which waits for this grid,
+// reads both kernels' partials.
 __global__ void __launch_bounds__(kMmaWarps * 32)
 prefill_block_mma_kernel(const uint4 *__restrict__ q, const uint4 *__restrict__ kc, const uint4 *__restrict__ vc,
                          const int2 *__restrict__ list, const int4 *__restrict__ items,
-                         const int32_t *__restrict__ n_items, int H, int num_pages, float scale_log2,
-                         __nv_bfloat16 *__restrict__ part_o, float *__restrict__ part_ml, int32_t *dev_err) {
+                         const int32_t *__restrict__ n_items, int32_t *sched, int H, int num_pages,
+                         float scale_log2, __nv_bfloat16 *__restrict__ part_o, float *__restrict__ part_ml,
+                         int32_t *dev_err) {
     __shared__ __align__(128) WarpStage stage[kMmaWarps];
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int r = lane >> 2, t = lane & 3;
@@ -279,11 +289,14 @@ prefill_block_mma_kernel(const uint4 *__restrict__ q, const uint4 *__restrict__ 
     const uint4 *k_s = stage[warp].k, *q_s = stage[warp].q;
 
     const uint64_t pol_kv = l2_evict_first(), pol_part = l2_evict_last();
-    pdl_wait();
     // the merge kernel may start its prologue; it waits for this grid before reading the partials
     pdl_launch_dependents();
-    const int n_work = __ldg(n_items) * H;
-    const int stride = gridDim.x * kMmaWarps;
+    const int n_work = __ldcg(n_items) * H;
+    auto take = [&]() {
+        int w = 0;
+        if (lane == 0) w = atomicAdd(sched, 1);
+        return __shfl_sync(0xffffffffu, w, 0);
+    };
 
     auto page_ok = [&](const Unit &u) { return (unsigned)u.page < (unsigned)num_pages; };
     // Q rows (16) and the K tile of unit u; then its V tile
@@ -321,11 +334,13 @@ prefill_block_mma_kernel(const uint4 *__restrict__ q, const uint4 *__restrict__ 
         cp_async_commit();
     };
 
-    Unit cur = load_unit(blockIdx.x * kMmaWarps + warp, n_work, H, items, list, r);
-    if (cur.w < 0) return;
-    issue_qk(cur);
-    issue_v(cur);
-    Unit nxt = load_unit(cur.w + stride, n_work, H, items, list, r);
+    Unit cur = load_unit(take(), n_work, H, items, list, r);
+    Unit nxt = cur;
+    if (cur.w >= 0) {
+        issue_qk(cur);
+        issue_v(cur);
+        nxt = load_unit(take(), n_work, H, items, list, r);
+    }
 
     while (cur.w >= 0) {
         // ---- S = Q K^T (rows r, r + 8; tokens 8 nt + 2t, 8 nt + 2t + 1) from this unit's Q, K
@@ -447,9 +462,10 @@ prefill_block_mma_kernel(const uint4 *__restrict__ q, const uint4 *__restrict__ 
             if (t == 0) st_f2_pol(part_ml + slot * 2, mb, lb, pol_part);
         }
         cur = nxt;
-        if (cur.w >= 0) nxt = load_unit(cur.w + stride, n_work, H, items, list, r);
+        if (cur.w >= 0) nxt = load_unit(take(), n_work, H, items, list, r);
     }
     cp_async_wait_all();
+    if (blockIdx.x == 0 && threadIdx.x == 0) pdl_wait();   // the local-window kernel is complete
 }
 
 // ------------------------------------------------------------------ host side
@@ -470,6 +486,8 @@ size_t prefill_attn_workspace(int n_q, int H, int max_blocks, PrefillAttnWs *w) 
     l.fill_off = off;
     off += up((size_t)max_blocks * 4);
     l.sched_off = off;   // the scoring GEMM's work-unit counter
+    off += up(4);
+    l.blk_sched_off = off;   // the block kernel's work-unit counter
     off += up(4);
     l.zero_bytes = off;
     l.n_items_off = off;
@@ -520,11 +538,6 @@ cudaError_t launch_prefill_attn(const LaunchCtx &c, const void *q, const void *k
     cudaError_t e = launch_prefill_classify(c, sel, q_pos, seq_len_ptr, n_q, max_blocks, sel_ws, counts, loc, tiles,
                                             dev_err);
     if (e != cudaSuccess) return e;
-    // the local windows on tcgen05, beside the inversion that follows
-    void *loc_o = base + w.loc_o_off;
-    float2 *loc_ml = (float2 *)(base + w.loc_ml_off);
-    e = launch_prefill_local(c, q, k, v, bt_row, q_pos, loc, tiles, n_q, H, num_pages, scale, loc_o, loc_ml, dev_err);
-    if (e != cudaSuccess) return e;
 
     cudaLaunchAttribute attr[1];
     attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
@@ -540,14 +553,20 @@ cudaError_t launch_prefill_attn(const LaunchCtx &c, const void *q, const void *k
                            q_pos, n_entries, max_blocks, fill, items, n_items, list);
     if (e != cudaSuccess) return e;
 
+    // the local windows on tcgen05, on a few SMs beside the block kernel that follows
+    void *loc_o = base + w.loc_o_off;
+    float2 *loc_ml = (float2 *)(base + w.loc_ml_off);
+    e = launch_prefill_local(c, q, k, v, bt_row, q_pos, loc, tiles, n_q, H, num_pages, scale, loc_o, loc_ml, dev_err);
+    if (e != cudaSuccess) return e;
+
     int per_sm = 0;
     e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, prefill_block_mma_kernel, kMmaWarps * 32, 0);
     if (e != cudaSuccess) return e;
     cfg.gridDim = dim3((unsigned)(c.num_sms * (per_sm > 0 ? per_sm : 1)));
     cfg.blockDim = dim3(kMmaWarps * 32);
     e = cudaLaunchKernelEx(&cfg, prefill_block_mma_kernel, (const uint4 *)q, (const uint4 *)k, (const uint4 *)v,
-                           (const int2 *)list, (const int4 *)items, (const int32_t *)n_items, H, num_pages,
-                           scale * kLog2e, part_o, ml, dev_err);
+                           (const int2 *)list, (const int4 *)items, (const int32_t *)n_items,
+                           (int32_t *)(base + w.blk_sched_off), H, num_pages, scale * kLog2e, part_o, ml, dev_err);
     if (e != cudaSuccess) return e;
 
     return launch_prefill_merge(c, sel_ws, part_o, ml, loc_o, loc_ml, n_q, H, out);

@@ -27,16 +27,18 @@
 //       per query and the slot its state goes to, marked -2 in the classified
 //       selection), the rest to the block kernel (block ids in the classified
 //       selection, counted per block for the inversion);
-//   prefill_local_kernel   persistent, one CTA per SM looping over (tile,
-//       head) units, 160 threads: warp 4 allocates 256 TMEM columns, loads Q
-//       (two 64-dim halves, 128-byte swizzle) and the window's K and V tiles
-//       (one 32-token box per block and half; a page outside the pool is loaded
-//       out of bounds, i.e. as zeros, and masked) with TMA, and one of its
-//       threads issues the MMAs; warps 0-3 own TMEM lane quarters (row =
-//       query): they read S back twice (row maximum, then weights), write P as
-//       bf16 into the K tile's shared memory in the 128-byte-swizzled K-major
-//       layout of an MMA operand, and after P V read O back into the row's
-//       partial slot;
+//   prefill_local_kernel   persistent on a quarter of the SMs (one CTA per
+//       SM), each CTA looping over an equal share of the (tile, head) units
+//       while the block kernel runs on the rest, 288 threads: warp 8
+//       allocates 256 TMEM columns, loads Q (two 64-dim halves, 128-byte
+//       swizzle) and the window's K and V tiles (one 32-token box per block and
+//       half; a page outside the pool is loaded out of bounds, i.e. as zeros,
+//       and masked) with TMA, and one of its threads issues the MMAs; warps w
+//       and w + 4 share TMEM lane quarter w % 4 (row = query), each taking
+//       every other window block: they read S back twice (row maximum, then
+//       weights), write P as bf16 into the K tile's shared memory in the
+//       128-byte-swizzled K-major layout of an MMA operand, and after P V read
+//       O back (64 dims each) and store it with TMA into the row's partial;
 //   prefill_merge_kernel   one warp per (query, head): every valid slot's
 //       partial, out = sum_k 2^(m_k - M) acc_k / sum_k 2^(m_k - M) l_k in bf16.
 // P V takes V as an MN-major operand (the V tile is token-major, dims
@@ -154,6 +156,7 @@ prefill_classify_kernel(const int32_t *__restrict__ sel, const int32_t *__restri
                         int2 *__restrict__ tile_info, int32_t *dev_err) {
     __shared__ int s_lo[kTileQ / 32], s_hi[kTileQ / 32];
     pdl_wait();
+    pdl_launch_dependents();   // the inversion waits for this grid before reading its output
     const int t = blockIdx.x, r = threadIdx.x, i = t * kTileQ + r;
     const int warp = r >> 5, lane = r & 31;
     const int seq_len = min(__ldg(seq_len_ptr), max_blocks * kBlock);
@@ -248,11 +251,12 @@ prefill_local_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_con
     __syncthreads();
     tc::fence_after_sync();
     const uint32_t tmem = s.tmem_base;
-    // The classification (tile windows, local masks and slots) is the preceding kernel's output.
+    // The classification (tile windows, local masks and slots) is complete once the preceding
+    // kernel, the inversion, is.
     pdl_wait();
-    // The inversion that follows may start now (it reads only the classification, complete at
-    // this point); it waits for this grid at its end, so the block kernel after it starts once
-    // both are done.
+    // The block kernel that follows may start now (it reads only the inversion, complete at this
+    // point) and runs beside this grid; it waits for this grid at its end, so the merge after it
+    // starts once both are done.
     pdl_launch_dependents();
 
     int it = 0;   // units done by this CTA: each unit completes every barrier once (parity it & 1)
@@ -521,70 +525,86 @@ prefill_local_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_con
     }
 }
 
-// One warp per (query, head): lanes 0..15 hold the 16 slots' (m, l), every lane 4 output dims.  A
-// slot holds a partial when the classified selection names a block there (the block kernel's) or
-// marks it as the local window's slot, and its m is finite.
+// Half a warp per (query, head): lane k of the half holds slot k's (m, l) and output dims 8 k ..
+// 8 k + 7 of every partial.  A slot holds a block partial when the classified selection names a
+// block there; the local window's state, when the query has one, is a seventeenth partial.  Empty
+// states (m = -inf, after a timeout) are skipped.  n_q * H < 2^31 (checked by the launcher).
 __global__ void __launch_bounds__(kMergeWarps * 32)
 prefill_merge_kernel(const int32_t *__restrict__ sel_ws, const __nv_bfloat16 *__restrict__ part_o,
                      const float *__restrict__ part_ml, const __nv_bfloat16 *__restrict__ loc_o,
                      const float2 *__restrict__ loc_ml, int n_q, int H, __nv_bfloat16 *__restrict__ out) {
-    const int lane = threadIdx.x & 31;
-    const long long ih = (long long)blockIdx.x * kMergeWarps + (threadIdx.x >> 5);
+    const int k = threadIdx.x & 15;
+    const unsigned half = 0xffffu << (threadIdx.x & 16);   // this half-warp's lanes
+    const int ih0 = blockIdx.x * (kMergeWarps * 2) + (threadIdx.x >> 4);
+    // a half past the end repeats the last (query, head) and stores nothing, so that every lane
+    // takes part in the warp's shuffles
+    const bool live = ih0 < n_q * H;
+    const int ih = live ? ih0 : n_q * H - 1;
     pdl_wait();
-    if (ih >= (long long)n_q * H) return;
-    const long long i = ih / H;
-    const int sl = lane & 15;
+    const int i = ih / H;
+    const int js = __ldg(sel_ws + (size_t)i * kSel + k);
     const size_t base = (size_t)ih * kSel;
-    const int js = __ldg(sel_ws + i * kSel + sl);
-    // the slot marked for the local window reads the local kernel's state of (query, head)
-    const bool is_loc = js == kLocalSlotMark;
-    const bool named = js >= 0 || is_loc;
-    const float2 mlv = !named ? make_float2(-INFINITY, 0.f)
-                              : (is_loc ? __ldcs(loc_ml + ih) : __ldcs(reinterpret_cast<const float2 *>(part_ml) + base + sl));
-    float m = mlv.x;
-    const float l = mlv.y;
-    const bool valid = named && m != -INFINITY;
-    if (!valid) m = -INFINITY;
-    const unsigned vmask = __ballot_sync(0xffffffffu, valid) & 0xffffu;
-    const unsigned lmask = __ballot_sync(0xffffffffu, is_loc) & 0xffffu;   // at most one slot
-    const int lslot = lmask ? __ffs(lmask) - 1 : -1;
-    uint2 v[kSel];
+    const float2 mlv = js >= 0 ? __ldcs(reinterpret_cast<const float2 *>(part_ml) + base + k)
+                               : make_float2(-INFINITY, 0.f);
+    const bool has_loc = (__ballot_sync(0xffffffffu, js == kLocalSlotMark) & half) != 0u;
+    const float2 mll = has_loc ? __ldcs(loc_ml + ih) : make_float2(-INFINITY, 0.f);
+    const unsigned vmask = (__ballot_sync(0xffffffffu, mlv.x != -INFINITY) & half) >> (threadIdx.x & 16);
+    const bool loc_ok = mll.x != -INFINITY;
+    // every valid partial's 16 bytes of this lane's dims
+    const uint4 *src = reinterpret_cast<const uint4 *>(part_o + base * kD) + k;
+    uint4 v[kSel];
 #pragma unroll
-    for (int k = 0; k < kSel; ++k) {
-        const __nv_bfloat16 *src = k == lslot ? loc_o + (size_t)ih * kD : part_o + (base + k) * kD;
-        v[k] = (vmask >> k & 1u) ? __ldcs(reinterpret_cast<const uint2 *>(src) + lane) : make_uint2(0u, 0u);
+    for (int s = 0; s < kSel; ++s)
+        v[s] = (vmask >> s & 1u) ? __ldcs(src + s * (kD / 8)) : make_uint4(0u, 0u, 0u, 0u);
+    const uint4 vl = loc_ok ? __ldcs(reinterpret_cast<const uint4 *>(loc_o + (size_t)ih * kD) + k)
+                            : make_uint4(0u, 0u, 0u, 0u);
+    float M = fmaxf(mlv.x, mll.x);
+#pragma unroll
+    for (int x = 8; x > 0; x >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, x, 16));
+    // partial s holds sum_t 2^(z_t - m_s) v_t and l_s = sum_t 2^(z_t - m_s): rescale both to M
+    const float w = mlv.x != -INFINITY ? exp2f(mlv.x - M) : 0.f;
+    const float wl = loc_ok ? exp2f(mll.x - M) : 0.f;
+    float W = mlv.y * w;
+#pragma unroll
+    for (int x = 8; x > 0; x >>= 1) W += __shfl_xor_sync(0xffffffffu, W, x, 16);
+    W += mll.y * wl;
+    float A[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+    auto acc = [&](float ws, const uint4 &u) {
+        A[0] = fmaf(ws, __uint_as_float(u.x << 16), A[0]);
+        A[1] = fmaf(ws, __uint_as_float(u.x & 0xffff0000u), A[1]);
+        A[2] = fmaf(ws, __uint_as_float(u.y << 16), A[2]);
+        A[3] = fmaf(ws, __uint_as_float(u.y & 0xffff0000u), A[3]);
+        A[4] = fmaf(ws, __uint_as_float(u.z << 16), A[4]);
+        A[5] = fmaf(ws, __uint_as_float(u.z & 0xffff0000u), A[5]);
+        A[6] = fmaf(ws, __uint_as_float(u.w << 16), A[6]);
+        A[7] = fmaf(ws, __uint_as_float(u.w & 0xffff0000u), A[7]);
+    };
+    acc(wl, vl);
+#pragma unroll
+    for (int s = 0; s < kSel; ++s) {
+        const float ws = __shfl_sync(0xffffffffu, w, s, 16);
+        if (vmask >> s & 1u) acc(ws, v[s]);
     }
-    float M = m;
-#pragma unroll
-    for (int x = 8; x > 0; x >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, x));
-    // partial k holds sum_t 2^(z_t - m_k) v_t and l_k = sum_t 2^(z_t - m_k): rescale both to M
-    const float w = (M == -INFINITY || !valid) ? 0.f : exp2f(m - M);
-    float W = valid ? l * w : 0.f;
-#pragma unroll
-    for (int x = 8; x > 0; x >>= 1) W += __shfl_xor_sync(0xffffffffu, W, x);
-    float A[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-    for (int k = 0; k < kSel; ++k) {
-        const float wk = __shfl_sync(0xffffffffu, w, k);
-        A[0] = fmaf(wk, __uint_as_float(v[k].x << 16), A[0]);
-        A[1] = fmaf(wk, __uint_as_float(v[k].x & 0xffff0000u), A[1]);
-        A[2] = fmaf(wk, __uint_as_float(v[k].y << 16), A[2]);
-        A[3] = fmaf(wk, __uint_as_float(v[k].y & 0xffff0000u), A[3]);
-    }
-    // Every lane has its loads' values: drop this (query, head)'s partial lines from L2 (its 16
-    // x 256 bytes of outputs are 32 lines, one per lane, and its 16 (m, l) pairs one line), so
-    // that they are never written back.  The workspace is 256-byte aligned, so the lines belong to
-    // this (query, head) alone; a slot not written in this call holds nothing that is needed.
+    // Every lane of the half has used its loads' values: drop this (query, head)'s partial lines
+    // from L2 (its 16 x 256 bytes of outputs are 32 lines, two per lane; its 16 (m, l) pairs one
+    // line; its local output two), so that they are never written back.  The workspace is 256-byte
+    // aligned, so the lines belong to this (query, head) alone; a slot not written in this call
+    // holds nothing that is needed.
     __syncwarp();
-    l2_discard_line(part_o + base * kD + 64 * lane);
-    if (lane == 0) l2_discard_line(part_ml + base * 2);
-    if (lslot >= 0 && lane < 2) l2_discard_line(loc_o + (size_t)ih * kD + 64 * lane);
+    if (!live) return;
+    const char *po = reinterpret_cast<const char *>(part_o + base * kD);
+    l2_discard_line(po + 256 * k);
+    l2_discard_line(po + 256 * k + 128);
+    if (k == 0) l2_discard_line(part_ml + base * 2);
+    if (has_loc && k < 2) l2_discard_line(reinterpret_cast<const char *>(loc_o + (size_t)ih * kD) + 128 * k);
     const float inv = W > 0.f ? 1.f / W : 0.f;
     float unused = 0.f;
-    uint2 pk;
+    uint4 pk;
     pk.x = pack2_bf16(A[0] * inv, A[1] * inv, unused);
     pk.y = pack2_bf16(A[2] * inv, A[3] * inv, unused);
-    reinterpret_cast<uint2 *>(out + (size_t)ih * kD)[lane] = pk;
+    pk.z = pack2_bf16(A[4] * inv, A[5] * inv, unused);
+    pk.w = pack2_bf16(A[6] * inv, A[7] * inv, unused);
+    reinterpret_cast<uint4 *>(out + (size_t)ih * kD)[k] = pk;
 }
 
 // ---------------------------------------------------------------- host side
@@ -651,7 +671,12 @@ cudaError_t launch_prefill_local(const LaunchCtx &c, const void *q, const void *
     attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3((unsigned)(units < c.num_sms ? units : c.num_sms));
+    // A quarter of the SMs (one CTA each: the kernel holds most of an SM's shared memory), each
+    // taking the same number of units; the block kernel launched after this one fills the rest.
+    const long long share = c.num_sms / 4 > 0 ? c.num_sms / 4 : 1;
+    const long long per_cta = (units + share - 1) / share;
+    const long long ctas = per_cta > 0 ? (units + per_cta - 1) / per_cta : 0;
+    cfg.gridDim = dim3((unsigned)(ctas > 0 ? ctas : 1));
     cfg.blockDim = dim3(kLocThreads);
     cfg.dynamicSmemBytes = smem;
     cfg.stream = c.stream;
@@ -663,8 +688,8 @@ cudaError_t launch_prefill_local(const LaunchCtx &c, const void *q, const void *
 
 cudaError_t launch_prefill_merge(const LaunchCtx &c, const int32_t *sel_ws, const void *part_o, const float *part_ml,
                                  const void *loc_o, const float2 *loc_ml, int n_q, int H, void *out) {
-    const long long merge_ctas = ((long long)n_q * H + kMergeWarps - 1) / kMergeWarps;
-    if (merge_ctas > 0x7fffffffLL) return cudaErrorInvalidConfiguration;
+    if ((long long)n_q * H > 0x7fffffffLL) return cudaErrorInvalidConfiguration;
+    const long long merge_ctas = ((long long)n_q * H + 2 * kMergeWarps - 1) / (2 * kMergeWarps);
     cudaLaunchAttribute attr[1];
     attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
     attr[0].val.programmaticStreamSerializationAllowed = 1;
