@@ -528,83 +528,112 @@ prefill_local_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_con
 // Half a warp per (query, head): lane k of the half holds slot k's (m, l) and output dims 8 k ..
 // 8 k + 7 of every partial.  A slot holds a block partial when the classified selection names a
 // block there; the local window's state, when the query has one, is a seventeenth partial.  Empty
-// states (m = -inf, after a timeout) are skipped.  n_q * H < 2^31 (checked by the launcher).
+// states (m = -inf, after a timeout) are skipped.  Persistent: warp w of the grid takes the pairs
+// of (query, head)s 2 w, 2 w + 1, then 2 (w + warps), ..., and loads the next pair's entries and
+// (m, l) while the current pair's partials are on their way.  n_q * H < 2^31 (checked by the
+// launcher).
 __global__ void __launch_bounds__(kMergeWarps * 32)
 prefill_merge_kernel(const int32_t *__restrict__ sel_ws, const __nv_bfloat16 *__restrict__ part_o,
                      const float *__restrict__ part_ml, const __nv_bfloat16 *__restrict__ loc_o,
                      const float2 *__restrict__ loc_ml, int n_q, int H, __nv_bfloat16 *__restrict__ out) {
     const int k = threadIdx.x & 15;
     const unsigned half = 0xffffu << (threadIdx.x & 16);   // this half-warp's lanes
-    const int ih0 = blockIdx.x * (kMergeWarps * 2) + (threadIdx.x >> 4);
-    // a half past the end repeats the last (query, head) and stores nothing, so that every lane
-    // takes part in the warp's shuffles
-    const bool live = ih0 < n_q * H;
-    const int ih = live ? ih0 : n_q * H - 1;
-    pdl_wait();
-    const int i = ih / H;
-    const int js = __ldg(sel_ws + (size_t)i * kSel + k);
-    const size_t base = (size_t)ih * kSel;
-    const float2 mlv = js >= 0 ? __ldcs(reinterpret_cast<const float2 *>(part_ml) + base + k)
-                               : make_float2(-INFINITY, 0.f);
-    const bool has_loc = (__ballot_sync(0xffffffffu, js == kLocalSlotMark) & half) != 0u;
-    const float2 mll = has_loc ? __ldcs(loc_ml + ih) : make_float2(-INFINITY, 0.f);
-    const unsigned vmask = (__ballot_sync(0xffffffffu, mlv.x != -INFINITY) & half) >> (threadIdx.x & 16);
-    const bool loc_ok = mll.x != -INFINITY;
-    // every valid partial's 16 bytes of this lane's dims
-    const uint4 *src = reinterpret_cast<const uint4 *>(part_o + base * kD) + k;
-    uint4 v[kSel];
-#pragma unroll
-    for (int s = 0; s < kSel; ++s)
-        v[s] = (vmask >> s & 1u) ? __ldcs(src + s * (kD / 8)) : make_uint4(0u, 0u, 0u, 0u);
-    const uint4 vl = loc_ok ? __ldcs(reinterpret_cast<const uint4 *>(loc_o + (size_t)ih * kD) + k)
-                            : make_uint4(0u, 0u, 0u, 0u);
-    float M = fmaxf(mlv.x, mll.x);
-#pragma unroll
-    for (int x = 8; x > 0; x >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, x, 16));
-    // partial s holds sum_t 2^(z_t - m_s) v_t and l_s = sum_t 2^(z_t - m_s): rescale both to M
-    const float w = mlv.x != -INFINITY ? exp2f(mlv.x - M) : 0.f;
-    const float wl = loc_ok ? exp2f(mll.x - M) : 0.f;
-    float W = mlv.y * w;
-#pragma unroll
-    for (int x = 8; x > 0; x >>= 1) W += __shfl_xor_sync(0xffffffffu, W, x, 16);
-    W += mll.y * wl;
-    float A[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-    auto acc = [&](float ws, const uint4 &u) {
-        A[0] = fmaf(ws, __uint_as_float(u.x << 16), A[0]);
-        A[1] = fmaf(ws, __uint_as_float(u.x & 0xffff0000u), A[1]);
-        A[2] = fmaf(ws, __uint_as_float(u.y << 16), A[2]);
-        A[3] = fmaf(ws, __uint_as_float(u.y & 0xffff0000u), A[3]);
-        A[4] = fmaf(ws, __uint_as_float(u.z << 16), A[4]);
-        A[5] = fmaf(ws, __uint_as_float(u.z & 0xffff0000u), A[5]);
-        A[6] = fmaf(ws, __uint_as_float(u.w << 16), A[6]);
-        A[7] = fmaf(ws, __uint_as_float(u.w & 0xffff0000u), A[7]);
+    const int n = n_q * H;
+    const int stride = 2 * gridDim.x * kMergeWarps;
+    // A half past the end repeats the last (query, head) and stores nothing, so that every lane
+    // takes part in the warp's shuffles and both halves run the same iterations.
+    auto clamp = [&](int ih) { return ih < n ? ih : n - 1; };
+    // the first round of a (query, head)'s loads: the slot's entry, its (m, l) and the local
+    // state's (m, l) (the (m, l) line of a (query, head) is read whole either way; an unnamed
+    // slot's value is not used)
+    struct First {
+        int js;
+        float2 ml, mll;
     };
-    acc(wl, vl);
+    auto first = [&](int ih) {
+        First f;
+        f.js = __ldg(sel_ws + (size_t)(ih / H) * kSel + k);
+        f.ml = __ldcs(reinterpret_cast<const float2 *>(part_ml) + (size_t)ih * kSel + k);
+        f.mll = __ldcs(loc_ml + ih);
+        return f;
+    };
+    int pair = blockIdx.x * (2 * kMergeWarps) + (threadIdx.x >> 5) * 2;   // even (query, head) of the warp
+    pdl_wait();
+    if (pair >= n) return;   // uniform over the warp
+    int ih = clamp(pair + ((threadIdx.x >> 4) & 1));
+    First cur = first(ih);
+    for (; pair < n; pair += stride) {
+        const bool live = pair + ((threadIdx.x >> 4) & 1) < n;
+        const size_t base = (size_t)ih * kSel;
+        const bool has_loc = (__ballot_sync(0xffffffffu, cur.js == kLocalSlotMark) & half) != 0u;
+        const unsigned named = (__ballot_sync(0xffffffffu, cur.js >= 0) & half) >> (threadIdx.x & 16);
+        const uint4 *src = reinterpret_cast<const uint4 *>(part_o + base * kD) + k;
+        uint4 v[kSel];
 #pragma unroll
-    for (int s = 0; s < kSel; ++s) {
-        const float ws = __shfl_sync(0xffffffffu, w, s, 16);
-        if (vmask >> s & 1u) acc(ws, v[s]);
+        for (int s = 0; s < kSel; ++s)
+            v[s] = (named >> s & 1u) ? __ldcs(src + s * (kD / 8)) : make_uint4(0u, 0u, 0u, 0u);
+        const uint4 vl = has_loc ? __ldcs(reinterpret_cast<const uint4 *>(loc_o + (size_t)ih * kD) + k)
+                                 : make_uint4(0u, 0u, 0u, 0u);
+        // the next pair's first round, in flight beside this pair's partials
+        const int ih_next = clamp(pair + stride + ((threadIdx.x >> 4) & 1));
+        const First nxt = pair + stride < n ? first(ih_next) : cur;
+        // a named slot with m = -inf (an empty state) and a missing local state are skipped
+        const float2 mlv = cur.js >= 0 ? cur.ml : make_float2(-INFINITY, 0.f);
+        const float2 mll = has_loc ? cur.mll : make_float2(-INFINITY, 0.f);
+        const unsigned vmask = (__ballot_sync(0xffffffffu, mlv.x != -INFINITY) & half) >> (threadIdx.x & 16);
+        const bool loc_ok = mll.x != -INFINITY;
+        float M = fmaxf(mlv.x, mll.x);
+#pragma unroll
+        for (int x = 8; x > 0; x >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, x, 16));
+        // partial s holds sum_t 2^(z_t - m_s) v_t and l_s = sum_t 2^(z_t - m_s): rescale both to M
+        const float w = mlv.x != -INFINITY ? exp2f(mlv.x - M) : 0.f;
+        const float wl = loc_ok ? exp2f(mll.x - M) : 0.f;
+        float W = mlv.y * w;
+#pragma unroll
+        for (int x = 8; x > 0; x >>= 1) W += __shfl_xor_sync(0xffffffffu, W, x, 16);
+        W += mll.y * wl;
+        float A[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+        auto acc = [&](float ws, const uint4 &u) {
+            A[0] = fmaf(ws, __uint_as_float(u.x << 16), A[0]);
+            A[1] = fmaf(ws, __uint_as_float(u.x & 0xffff0000u), A[1]);
+            A[2] = fmaf(ws, __uint_as_float(u.y << 16), A[2]);
+            A[3] = fmaf(ws, __uint_as_float(u.y & 0xffff0000u), A[3]);
+            A[4] = fmaf(ws, __uint_as_float(u.z << 16), A[4]);
+            A[5] = fmaf(ws, __uint_as_float(u.z & 0xffff0000u), A[5]);
+            A[6] = fmaf(ws, __uint_as_float(u.w << 16), A[6]);
+            A[7] = fmaf(ws, __uint_as_float(u.w & 0xffff0000u), A[7]);
+        };
+        if (loc_ok) acc(wl, vl);   // (an empty local state's output is not read: it may be anything)
+#pragma unroll
+        for (int s = 0; s < kSel; ++s) {
+            const float ws = __shfl_sync(0xffffffffu, w, s, 16);
+            if (vmask >> s & 1u) acc(ws, v[s]);
+        }
+        // Every lane of the warp has used its loads' values: drop this (query, head)'s partial
+        // lines from L2 (its 16 x 256 bytes of outputs are 32 lines, two per lane; its 16 (m, l)
+        // pairs one line; its local output two), so that they are never written back.  The
+        // workspace is 256-byte aligned, so the lines belong to this (query, head) alone; a slot
+        // not written in this call holds nothing that is needed.
+        __syncwarp();
+        if (live) {
+            const char *po = reinterpret_cast<const char *>(part_o + base * kD);
+            l2_discard_line(po + 256 * k);
+            l2_discard_line(po + 256 * k + 128);
+            if (k == 0) l2_discard_line(part_ml + base * 2);
+            if (has_loc && k < 2)
+                l2_discard_line(reinterpret_cast<const char *>(loc_o + (size_t)ih * kD) + 128 * k);
+            const float inv = W > 0.f ? 1.f / W : 0.f;
+            float unused = 0.f;
+            uint4 pk;
+            pk.x = pack2_bf16(A[0] * inv, A[1] * inv, unused);
+            pk.y = pack2_bf16(A[2] * inv, A[3] * inv, unused);
+            pk.z = pack2_bf16(A[4] * inv, A[5] * inv, unused);
+            pk.w = pack2_bf16(A[6] * inv, A[7] * inv, unused);
+            reinterpret_cast<uint4 *>(out + (size_t)ih * kD)[k] = pk;
+        }
+        ih = ih_next;
+        cur = nxt;
     }
-    // Every lane of the half has used its loads' values: drop this (query, head)'s partial lines
-    // from L2 (its 16 x 256 bytes of outputs are 32 lines, two per lane; its 16 (m, l) pairs one
-    // line; its local output two), so that they are never written back.  The workspace is 256-byte
-    // aligned, so the lines belong to this (query, head) alone; a slot not written in this call
-    // holds nothing that is needed.
-    __syncwarp();
-    if (!live) return;
-    const char *po = reinterpret_cast<const char *>(part_o + base * kD);
-    l2_discard_line(po + 256 * k);
-    l2_discard_line(po + 256 * k + 128);
-    if (k == 0) l2_discard_line(part_ml + base * 2);
-    if (has_loc && k < 2) l2_discard_line(reinterpret_cast<const char *>(loc_o + (size_t)ih * kD) + 128 * k);
-    const float inv = W > 0.f ? 1.f / W : 0.f;
-    float unused = 0.f;
-    uint4 pk;
-    pk.x = pack2_bf16(A[0] * inv, A[1] * inv, unused);
-    pk.y = pack2_bf16(A[2] * inv, A[3] * inv, unused);
-    pk.z = pack2_bf16(A[4] * inv, A[5] * inv, unused);
-    pk.w = pack2_bf16(A[6] * inv, A[7] * inv, unused);
-    reinterpret_cast<uint4 *>(out + (size_t)ih * kD)[k] = pk;
 }
 
 // ---------------------------------------------------------------- host side
@@ -688,8 +717,14 @@ cudaError_t launch_prefill_local(const LaunchCtx &c, const void *q, const void *
 
 cudaError_t launch_prefill_merge(const LaunchCtx &c, const int32_t *sel_ws, const void *part_o, const float *part_ml,
                                  const void *loc_o, const float2 *loc_ml, int n_q, int H, void *out) {
-    if ((long long)n_q * H > 0x7fffffffLL) return cudaErrorInvalidConfiguration;
-    const long long merge_ctas = ((long long)n_q * H + 2 * kMergeWarps - 1) / (2 * kMergeWarps);
+    if ((long long)n_q * H > 0x7fffffffLL / 2) return cudaErrorInvalidConfiguration;
+    int per_sm = 0;
+    cudaError_t e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, prefill_merge_kernel, kMergeWarps * 32, 0);
+    if (e != cudaSuccess) return e;
+    // persistent: as many CTAs as fit at once, fewer when there are fewer pairs
+    const long long need = ((long long)n_q * H + 2 * kMergeWarps - 1) / (2 * kMergeWarps);
+    const long long fit = (long long)c.num_sms * (per_sm > 0 ? per_sm : 1);
+    const long long merge_ctas = need < fit ? need : fit;
     cudaLaunchAttribute attr[1];
     attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
     attr[0].val.programmaticStreamSerializationAllowed = 1;
