@@ -308,8 +308,12 @@ prefill_block_mma_kernel(const uint4 *__restrict__ q, const uint4 *__restrict__ 
                 const int src = (row & 7) * 4;
                 const int ea = __shfl_sync(0xffffffffu, u.ea.x, src), eb = __shfl_sync(0xffffffffu, u.eb.x, src);
                 const int ent = row < 8 ? ea : eb;
-                cp_async16(sq + (uint32_t)((row * 16 + (c ^ ((row & 1) << 2))) * 16),
-                           q + ((size_t)(ent >> 4) * H + u.h) * (kD / 8) + c);
+                // rows past the item's end are not copied: their scores and outputs are computed
+                // from whatever the buffer holds and never stored (each row of an MMA's result
+                // depends on its own row of A alone)
+                if (row < u.rows)
+                    cp_async16(sq + (uint32_t)((row * 16 + (c ^ ((row & 1) << 2))) * 16),
+                               q + ((size_t)(ent >> 4) * H + u.h) * (kD / 8) + c);
             }
             if (page_ok(u)) {
                 const uint4 *src = kc + ((size_t)u.page * H + u.h) * (kPageElems / 8);
