@@ -72,7 +72,9 @@ block_topk_warp_kernel(const float *__restrict__ scores, const int32_t *__restri
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int i = blockIdx.x * kTopkWarpRows + warp;
     pdl_wait();
-    pdl_launch_dependents();
+    // No early trigger: this grid holds nearly every SM's registers while it runs, so a dependent
+    // grid launched early would crowd its CTAs onto the few SMs left free.  Each warp lets the
+    // dependents start once its row is done (the grid triggers when every warp has, or exited).
     if (i >= n_q) return;
     int32_t *out = sel + (size_t)i * kSel;
     QueryRef r;
@@ -86,6 +88,7 @@ block_topk_warp_kernel(const float *__restrict__ scores, const int32_t *__restri
         __syncwarp();
         if (lane < kSel) count_selected(out, lane, counts);
     }
+    pdl_launch_dependents();
 }
 
 cudaError_t launch_block_topk(const LaunchCtx &c, const float *scores, const int32_t *seq_lens,
