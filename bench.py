@@ -248,24 +248,17 @@ def run_uocr(args):
         if flush:
             flush_l2()
         step()
-    step_graph = capture_step(step, stream) if flush else None
+    timed = TimedSteps(step, flush_l2, stream, args.steps) if flush else None
+    if timed is not None:
+        timed.warm()
     torch.cuda.synchronize()
     barrier()
     torch.cuda.synchronize()
 
     clk.mark_start()
     if flush:
-        # L2 flushed between steps; each step (one graph replay) timed on its own
-        times = []
-        for _ in range(args.steps):
-            flush_l2()
-            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-            e0.record(stream)
-            step_graph.replay()
-            e1.record(stream)
-            times.append((e0, e1))
-        torch.cuda.synchronize()
-        elapsed_ms = sum(a.elapsed_time(b) for a, b in times)
+        # L2 flushed between steps, every step timed between its own events inside one graph
+        elapsed_ms = timed.run()
     else:
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         e0.record(stream)
@@ -413,8 +406,8 @@ def run_uocr(args):
         "config": {"workload": case.name, "batch_per_gpu": B, "context": int(case.seq_lens.max().item()),
                    "layers": n_layers, "heads": H, "head_dim": 128, "block": 32, "local_blocks": 4,
                    "remote_blocks": 12, "max_blocks": mb,
-                   "l2": L2_FLUSH_NOTE if flush else "inputs larger than L2 (no flush)",
-                   "launch": "one CUDA-graph replay per step" if flush else "stream launches queued ahead",
+                   "l2": L2_FLUSH_NOTE if flush else "inputs larger than L2 (no flush)", "launch": STEPS_IN_ONE_GRAPH,
+                   "launch": STEPS_IN_ONE_GRAPH if flush else "stream launches queued ahead",
                    "parallelism": f"dp{world} (independent sequence shards)"},
         "roofline": {"bound": "hbm", "kernel": "index_scan_kernel", "achieved": round(scan_gbs, 1),
                      "peak": peak, "unit": "GB/s", "frac": round(scan_gbs / peak, 4), "traffic": traffic,
@@ -438,7 +431,7 @@ def run_uocr(args):
         result["cpu_baseline"] = cpu_baseline(case, budget_s=args.cpu_budget)
     if world == 1 and args.workload == "long_decode" and not args.no_configs:
         # the other workloads, each measured on its own after the headline's caches are freed
-        del case, ws, outs, sels, scores, step_graph, flush_l2, step
+        del case, ws, outs, sels, scores, timed, flush_l2, step
         import gc
         gc.collect()
         torch.cuda.empty_cache()
@@ -497,20 +490,43 @@ class L2Flush:
         torch.sum(self.r, dim=0, out=self.acc)
 
 
-def capture_step(fn, stream):
-    """One call of fn(stream) captured in a CUDA graph (after one eager call on a side stream, so
-    that lazily created resources exist).  The timed loops of the L2-flushed workloads replay it,
-    so that a step's launches reach the GPU back to back: the work is the same, the host's
-    launch gaps are not timed."""
-    side = torch.cuda.Stream()
-    side.wait_stream(stream)
-    with torch.cuda.stream(side):
-        fn(side)
-    side.synchronize()
-    g = torch.cuda.CUDAGraph()
-    with torch.cuda.graph(g, stream=side):
-        fn(side)
-    return g
+STEPS_IN_ONE_GRAPH = ("all timed steps in one CUDA graph, each step timed between its own event-record "
+                      "nodes (no host launch inside a step)")
+
+
+class TimedSteps:
+    """`steps` steps of fn(stream), each after an L2 flush when one is given, captured in one CUDA
+    graph with an event-record node right before and right after every step.  A replay runs them
+    back to back on the device; each step is timed between its own two events, so neither a flush
+    nor a host-side launch falls inside a step's time.  `run()` replays once to warm up, then once
+    timed, and returns the sum of the steps' device ms."""
+
+    def __init__(self, fn, flush_l2, stream, steps):
+        self.ev = [(torch.cuda.Event(enable_timing=True, external=True),
+                    torch.cuda.Event(enable_timing=True, external=True)) for _ in range(steps)]
+        side = torch.cuda.Stream()
+        side.wait_stream(stream)
+        with torch.cuda.stream(side):
+            fn(side)
+        side.synchronize()
+        self.g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(self.g, stream=side):
+            for e0, e1 in self.ev:
+                if flush_l2 is not None:
+                    flush_l2()
+                e0.record(side)
+                fn(side)
+                e1.record(side)
+        torch.cuda.synchronize()
+
+    def warm(self):
+        self.g.replay()
+        torch.cuda.synchronize()
+
+    def run(self):
+        self.g.replay()
+        torch.cuda.synchronize()
+        return sum(a.elapsed_time(b) for a, b in self.ev)
 
 
 def graph_time_fn(fn, stream, n_rep, flush_l2=None):
@@ -594,23 +610,15 @@ def prefill_measure(args, uocr, dev, rank, local_rank, world, steps, extras):
     for _ in range(args.warmup):
         flush_l2()
         step()
-    step_graph = capture_step(step, stream)
+    timed = TimedSteps(step, flush_l2, stream, steps)
+    timed.warm()
     torch.cuda.synchronize()
     barrier()
     torch.cuda.synchronize()
     clk.mark_start()
-    times = []
-    for _ in range(steps):
-        flush_l2()
-        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        e0.record(stream)
-        step_graph.replay()
-        e1.record(stream)
-        times.append((e0, e1))
-    torch.cuda.synchronize()
+    elapsed_ms = timed.run()
     clk.mark_end()
     clk.stop()
-    elapsed_ms = sum(a.elapsed_time(b) for a, b in times)
     barrier()
     max_ms = udist.max_over_ranks(elapsed_ms, dev)
     ms_per_step = max_ms / steps
@@ -652,7 +660,7 @@ def prefill_measure(args, uocr, dev, rank, local_rank, world, steps, extras):
         "warmup": args.warmup, "ms_per_step": round(ms_per_step, 4), "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
         "config": {"workload": case.name, "queries": n_q, "context": int(case.seq_lens[0]), "heads": H,
-                   "max_blocks": mb, "l2": L2_FLUSH_NOTE, "launch": "one CUDA-graph replay per step",
+                   "max_blocks": mb, "l2": L2_FLUSH_NOTE, "launch": STEPS_IN_ONE_GRAPH,
                    "parallelism": f"dp{world}"},
         "roofline": {"bound": "tensor", "kernel": "prefill_index_gemm_kernel", "achieved": round(gemm_tflops, 1),
                      "peak": tc_peak, "unit": "TFLOP/s", "frac": round(gemm_tflops / tc_peak, 4), "traffic": gemm_traffic,
@@ -688,9 +696,10 @@ PREFILL_LAUNCHES = 7
 
 def decode_config_record(name, args, uocr, dev, steps):
     """One decode workload measured on its own for the `configs` record of the default run:
-    `steps` timed decode calls (each replaying one captured call, L2 flushed before it when the
-    call's bytes would otherwise stay in L2), the scan kernel and the whole call from CUDA-graph
-    replays, the HBM fractions on the algorithmic bytes, and the clocks of its timed region."""
+    `steps` timed decode calls (all captured in one CUDA graph, each timed between its own event
+    nodes, L2 flushed before each when the call's bytes would otherwise stay in L2), the scan
+    kernel and the whole call from CUDA-graph replays, the HBM fractions on the algorithmic bytes,
+    and the clocks of its timed region."""
     case = build_workload(name, dev, args.seed)
     B, H, mb = case.n_q, case.q.shape[1], case.max_blocks
     bytes_call, scan_bytes = algorithmic_bytes(case)
@@ -711,23 +720,13 @@ def decode_config_record(name, args, uocr, dev, steps):
         if flush:
             flush_l2()
         call()
-    g = capture_step(call, stream)
-    torch.cuda.synchronize()
+    timed = TimedSteps(call, flush_l2, stream, steps)
+    timed.warm()
     clk = ClockSampler(physical_gpu(torch.cuda.current_device())).start()
     clk.mark_start()
-    times = []
-    for _ in range(steps):
-        if flush:
-            flush_l2()
-        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        e0.record(stream)
-        g.replay()
-        e1.record(stream)
-        times.append((e0, e1))
-    torch.cuda.synchronize()
+    call_ms = timed.run() / steps
     clk.mark_end()
     clk.stop()
-    call_ms = sum(a.elapsed_time(b) for a, b in times) / steps
     n_rep = 20
     scan_ms = graph_time_fn(lambda st: uocr.index_score(case.idx_q, case.idx_k_pool, case.block_table, case.seq_lens,
                                                         scores=scores, stream=st), stream, n_rep, flush_l2)
@@ -740,14 +739,14 @@ def decode_config_record(name, args, uocr, dev, steps):
     rec = {"workload": case.name, "queries_per_call": B,
            "value": round(B / (call_ms / 1e3), 1), "unit": "queries/s per layer",
            "ms_per_call": round(call_ms, 5), "steps": steps,
-           "l2": L2_FLUSH_NOTE if flush else "inputs larger than L2 (no flush)",
+           "l2": L2_FLUSH_NOTE if flush else "inputs larger than L2 (no flush)", "launch": STEPS_IN_ONE_GRAPH,
            "roofline": {"bound": "hbm", "achieved": round(gbs, 1), "peak": peak, "unit": "GB/s",
                         "frac": round(gbs / peak, 4), "frac_of_8tbs": round(gbs / NOMINAL_HBM_GBS, 4),
                         "bytes_per_call": bytes_call, "peak_kind": f"{peak_kind} hbm copy"},
            "scan": {"kernel": "index_scan_kernel", "achieved": round(scan_gbs, 1), "frac": round(scan_gbs / peak, 4),
                     "bytes_per_launch": scan_bytes, "avg_launch_ms": round(scan_ms, 5), "traffic": traffic},
            "gpu_launches": steps * 3, "clocks": clk.summary()}
-    del case, ws, out, sel, scores, g, flush_l2
+    del case, ws, out, sel, scores, timed, flush_l2
     torch.cuda.empty_cache()
     return rec
 
