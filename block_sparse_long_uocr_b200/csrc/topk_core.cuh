@@ -505,16 +505,35 @@ __device__ void topk_warp_select(const float *row, int nb, const uint32_t *mask,
         if (keep && slot < kWarpSurvivorCap) sm.surv[slot] = composite(k, j);
         n += __popc(m);
     };
-    // every lane runs the same number of iterations (the ballots need the whole warp)
     if (in_regs) {
+        // each lane counts its survivors, takes its place in the list from a prefix sum over the
+        // lanes and writes them there: no warp-wide step per candidate (the list's order does not
+        // matter, the ranking below orders it)
+        int mine = 0;
+#pragma unroll
+        for (int q = 0; q < kRegQuads; ++q)
+#pragma unroll
+            for (int e = 0; e < 4; ++e) mine += (128 * q + 4 * lane + e < nc && kr[q][e] >= thr) ? 1 : 0;
+        int incl = mine;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const int v = __shfl_up_sync(0xffffffffu, incl, o);
+            if (lane >= o) incl += v;
+        }
+        int slot = incl - mine;
+        n = __shfl_sync(0xffffffffu, incl, 31);
 #pragma unroll
         for (int q = 0; q < kRegQuads; ++q)
 #pragma unroll
             for (int e = 0; e < 4; ++e) {
                 const int j = 128 * q + 4 * lane + e;
-                append(j < nc && kr[q][e] >= thr, kr[q][e], j);
+                if (j < nc && kr[q][e] >= thr) {
+                    if (slot < kWarpSurvivorCap) sm.surv[slot] = composite(kr[q][e], j);
+                    ++slot;
+                }
             }
     } else {
+        // every lane runs the same number of iterations (the ballots need the whole warp)
 #pragma unroll 4
         for (int j0 = 0; j0 < n_vec; j0 += 128) {
             const int j = j0 + 4 * lane;
