@@ -39,8 +39,9 @@
 //       weights), write P as bf16 into the K tile's shared memory in the
 //       128-byte-swizzled K-major layout of an MMA operand, and after P V read
 //       O back (64 dims each) and store it with TMA into the row's partial;
-//   prefill_merge_kernel   one warp per (query, head): every valid slot's
-//       partial, out = sum_k 2^(m_k - M) acc_k / sum_k 2^(m_k - M) l_k in bf16.
+//   prefill_merge_kernel   persistent, half a warp per (query, head): every
+//       valid slot's partial and the local window's state, out = sum_k
+//       2^(m_k - M) acc_k / sum_k 2^(m_k - M) l_k in bf16.
 // P V takes V as an MN-major operand (the V tile is token-major, dims
 // contiguous), so no transpose is needed.  Weights are rounded to bf16 for the
 // tensor cores and l sums the rounded weights (the output moves by at most
