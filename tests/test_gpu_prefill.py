@@ -276,3 +276,19 @@ def test_chunked_prefill_workload_every_query(uocr, cuda_device):
     assert int(err.item()) == 0
     scores = ws[: case.n_q * case.max_blocks * 4].view(torch.float32).view(case.n_q, case.max_blocks)
     check_all_queries(case, out, sel, scores)
+
+
+@pytest.mark.slow
+def test_long_chunk_twelve_heads_every_query(uocr, cuda_device):
+    """A 4096-query chunk starting 7 tokens into a block, 12 heads, shuffled pages: 32 local-window
+    tiles of 8-block windows x 12 heads = 384 units for the local kernel's CTAs (about 11 each), the
+    block kernel's units from its counter beside them, and 49152 (query, head) merges; every
+    selection and every output against the oracle, no device error."""
+    total = 32 * 400 + 7
+    case = _prefill_case(total, 4096, seed=61, device=cuda_device, heads=12)
+    err = torch.zeros(1, dtype=torch.int32, device=cuda_device)
+    out, sel = uocr.sparse_prefill(case.q, case.k_pool, case.v_pool, case.idx_q, case.idx_k_pool, case.block_table,
+                                   case.seq_lens, 0, case.q_pos, dev_err=err)
+    torch.cuda.synchronize()
+    assert int(err.item()) == 0
+    check_all_queries(case, out, sel)
