@@ -210,7 +210,8 @@ uocr_status_t uocr_prefill_index_score(const void *idx_q, const void *idx_k_cach
  * [0, seq_len) gets a zero output and sets UOCR_DEVERR_POS; a block whose page
  * is outside the pool contributes nothing and sets UOCR_DEVERR_PAGE.  The
  * per-slot partial outputs are rounded to bf16 before the merge (at most
- * 2^-9 max|v| on an output).  Workspace: uocr_sparse_attn_seq_workspace_bytes
+ * 2^-9 max|v| on an output), and the tensor-core products take the softmax
+ * weights in bf16.  Workspace: uocr_sparse_attn_seq_workspace_bytes
  * bytes, 256-byte aligned, owned by the caller, a pure function of the shapes.
  * After the call its partial region holds undefined bytes: the merge drops the
  * partials' L2 lines once it has read them, without writing them back.
@@ -232,12 +233,16 @@ uocr_status_t uocr_sparse_attn_seq(const void *q, const void *k_cache, const voi
  * keeps its own 4 local + 12 remote blocks over its causal prefix), and exact
  * attention over the selected blocks with scale = 1/sqrt(128) (the result of
  * uocr_sparse_attn).  out [n_q][H][128] bf16, sel_out [n_q][16] int32.
- * The attention is block-centric: the selection is inverted per block, every
+ * The local windows of a tile of 128 consecutive queries share one window of
+ * at most 8 blocks and are attended per (tile, head) on the tensor cores
+ * (tcgen05, one partial per query and head); the other selected blocks are
+ * attended block-centrically: the selection is inverted per block, every
  * selected (block, head) K/V tile is read once for all the queries that chose
  * it, and each (query, slot, head) partial -- the row maximum and weight sum in
- * fp32, the unnormalised partial output in bf16 -- is merged per (query, head);
- * the bf16 partial adds at most 2^-9 max|v| to an output, the size of the
- * output's own bf16 rounding.  Workspace: uocr_prefill_workspace_bytes(n_q, H,
+ * fp32, the unnormalised partial output in bf16 -- is merged per (query, head).
+ * The softmax weights are rounded to bf16 for the tensor-core products (the
+ * weight sums add the rounded weights), and the bf16 partials add at most
+ * 2^-9 max|v| to an output, the size of the output's own bf16 rounding.  Workspace: uocr_prefill_workspace_bytes(n_q, H,
  * max_blocks) bytes, 256-byte aligned (the block scores first, then the
  * inverted index and the partials; after the call the block scores are
  * readable and the partial region holds undefined bytes, dropped from L2 by
