@@ -438,22 +438,32 @@ __device__ void topk_warp_select(const float *row, int nb, const uint32_t *mask,
 #pragma unroll
         for (int q = 0; q < kRegQuads; ++q) {
             const int j = 128 * q + 4 * lane;
+            const float f[4] = {v[q].x, v[q].y, v[q].z, v[q].w};
+            if (!mask && 128 * q + 127 < nc) {
+                // every lane's quad is whole and unmasked (the same for the warp): keys only
+#pragma unroll
+                for (int e = 0; e < 4; ++e) kr[q][e] = order_key(f[e]);
+                continue;
+            }
             if (j < nc && j + 3 >= nc) {   // the quad that holds the row's end: scalar reads
                 v[q].x = __ldcg(row + j);
                 v[q].y = j + 1 < nc ? __ldcg(row + j + 1) : 0.f;
                 v[q].z = j + 2 < nc ? __ldcg(row + j + 2) : 0.f;
             }
-            const float f[4] = {v[q].x, v[q].y, v[q].z, v[q].w};
+            const float g[4] = {v[q].x, v[q].y, v[q].z, v[q].w};
 #pragma unroll
-            for (int e = 0; e < 4; ++e) kr[q][e] = (j + e < nc && ((mw[q] >> e) & 1u)) ? order_key(f[e]) : 0u;
+            for (int e = 0; e < 4; ++e) kr[q][e] = (j + e < nc && ((mw[q] >> e) & 1u)) ? order_key(g[e]) : 0u;
         }
 #pragma unroll
         for (int q = 0; q < kRegQuads; ++q)
 #pragma unroll
-            for (int e = 0; e < 4; ++e) {
-                tmax = kr[q][e] > tmax ? kr[q][e] : tmax;
-                allowed += kr[q][e] != 0u;
-            }
+            for (int e = 0; e < 4; ++e) tmax = kr[q][e] > tmax ? kr[q][e] : tmax;
+        if (mask) {   // (the count of allowed candidates matters only with a mask)
+#pragma unroll
+            for (int q = 0; q < kRegQuads; ++q)
+#pragma unroll
+                for (int e = 0; e < 4; ++e) allowed += kr[q][e] != 0u;
+        }
     } else {
 #pragma unroll 4
         for (int j = 4 * lane; j < n_vec; j += 128) {
